@@ -1,0 +1,191 @@
+"""Python binding of ``libfp8w8a8.so`` (the C ABI in ``include/fp8w8a8.h``).
+
+Argument marshalling only: every step of the W8A8 path runs in the library's
+CUDA kernels. PyTorch provides device memory and the current stream. Importing
+this package fails loudly if the compiled library is missing; there is no CPU
+fallback.
+
+Functions mirror the C entry points:
+
+* :func:`repack_qat` - QAT q4_0 grid -> per-channel E4M3 weight + scales.
+* :func:`convert_fnuz` - E4M3FNUZ-stored weight -> E4M3 weight + scales.
+* :func:`quant_act` - per-token E4M3 activation quantization.
+* :func:`rowwise_linear` - ``y = (x8 . w8^T) * s_tok * s_ch`` in bf16.
+* :func:`linear` - bf16 activations in, bf16 out (quantizer + GEMM).
+* :func:`cast_e4m3` - the element-wise encoder.
+* :func:`device_status` - read and clear the device status word.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libfp8w8a8.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(
+        f"{LIB_PATH} is missing: build it with `python -m fp8_w8a8_linear_b200.build` "
+        "(the FP8 W8A8 path has no fallback)")
+
+_lib = ctypes.CDLL(LIB_PATH)
+
+_P = ctypes.c_void_p
+_I64 = ctypes.c_int64
+_SIGS = {
+    "fp8_version": ([], ctypes.c_int),
+    "fp8_status_string": ([ctypes.c_int], ctypes.c_char_p),
+    "fp8_device_supported": ([ctypes.c_int], ctypes.c_int),
+    "fp8_get_device_status": ([ctypes.POINTER(ctypes.c_uint)], ctypes.c_int),
+    "fp8_repack_qat": ([_P, _P, _I64, _I64, _P, _P, _P], ctypes.c_int),
+    "fp8_convert_fnuz": ([_P, _P, _I64, _I64, _P, _P, _P], ctypes.c_int),
+    "fp8_quant_act": ([_P, _I64, _I64, _I64, _P, _P, _P], ctypes.c_int),
+    "fp8_rowwise_linear": ([_P, _P, _P, _P, _I64, _I64, _I64, _P, _P], ctypes.c_int),
+    "fp8_linear_bf16": ([_P, _P, _P, _I64, _I64, _I64, _P, _P, _P, _P], ctypes.c_int),
+    "fp8_cast_e4m3": ([_P, _I64, _P, _P], ctypes.c_int),
+}
+for _name, (_args, _ret) in _SIGS.items():
+    _f = getattr(_lib, _name)
+    _f.argtypes = _args
+    _f.restype = _ret
+
+raw = _lib  # the C entry points themselves (plain pointers and sizes)
+
+FP8_OK = 0
+DEV_NONFINITE = 0x1
+DEV_NAN_CODE = 0x2
+DEV_INEXACT = 0x4
+DEV_TIMEOUT = 0x8
+
+
+class Fp8Error(RuntimeError):
+    def __init__(self, status: int, where: str):
+        super().__init__(f"{where}: {_lib.fp8_status_string(status).decode()} ({status})")
+        self.status = status
+
+
+def _check(status: int, where: str):
+    if status != FP8_OK:
+        raise Fp8Error(status, where)
+
+
+def _stream() -> int:
+    return torch.cuda.current_stream().cuda_stream
+
+
+def _dev(t: torch.Tensor, dtype, name: str, shape=None):
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    return t.data_ptr()
+
+
+def version() -> int:
+    return _lib.fp8_version()
+
+
+def device_supported(device: int = 0) -> bool:
+    return bool(_lib.fp8_device_supported(device))
+
+
+def device_status() -> int:
+    """Synchronize the current device, return its status bits and clear them."""
+    v = ctypes.c_uint(0)
+    _check(_lib.fp8_get_device_status(ctypes.byref(v)), "fp8_get_device_status")
+    return v.value
+
+
+def repack_qat(q4: torch.Tensor, d: torch.Tensor, w8: torch.Tensor | None = None,
+               s_ch: torch.Tensor | None = None):
+    """q4 uint8 [N, K/2] (packed int4) and d float32 [N, K/32] -> (w8 uint8 [N, K], s_ch float32 [N])."""
+    N, K2 = q4.shape
+    K = 2 * K2
+    w8 = torch.empty((N, K), dtype=torch.uint8, device=q4.device) if w8 is None else w8
+    s_ch = torch.empty((N,), dtype=torch.float32, device=q4.device) if s_ch is None else s_ch
+    _check(_lib.fp8_repack_qat(_dev(q4, torch.uint8, "q4"), _dev(d, torch.float32, "d", (N, K // 32)),
+                               N, K, _dev(w8, torch.uint8, "w8", (N, K)),
+                               _dev(s_ch, torch.float32, "s_ch", (N,)), _stream()), "fp8_repack_qat")
+    return w8, s_ch
+
+
+def convert_fnuz(w8_fnuz: torch.Tensor, s_fnuz: torch.Tensor, w8: torch.Tensor | None = None,
+                 s_ch: torch.Tensor | None = None):
+    """E4M3FNUZ codes [N, K] + scales [N] -> E4M3 codes + scales (in place if outputs alias)."""
+    N, K = w8_fnuz.shape
+    w8 = torch.empty_like(w8_fnuz) if w8 is None else w8
+    s_ch = torch.empty_like(s_fnuz) if s_ch is None else s_ch
+    _check(_lib.fp8_convert_fnuz(_dev(w8_fnuz, torch.uint8, "w8_fnuz"),
+                                 _dev(s_fnuz, torch.float32, "s_fnuz", (N,)), N, K,
+                                 _dev(w8, torch.uint8, "w8", (N, K)),
+                                 _dev(s_ch, torch.float32, "s_ch", (N,)), _stream()),
+           "fp8_convert_fnuz")
+    return w8, s_ch
+
+
+def quant_act(x: torch.Tensor, x8: torch.Tensor | None = None, s_tok: torch.Tensor | None = None):
+    """x bf16 [M, K] -> (x8 uint8 [M, K], s_tok float32 [M])."""
+    if x.dtype != torch.bfloat16 or x.dim() != 2 or x.stride(1) != 1:
+        raise ValueError("x must be a bf16 [M, K] tensor with unit inner stride")
+    M, K = x.shape
+    x8 = torch.empty((M, K), dtype=torch.uint8, device=x.device) if x8 is None else x8
+    s_tok = torch.empty((M,), dtype=torch.float32, device=x.device) if s_tok is None else s_tok
+    if not x.is_cuda:
+        raise ValueError("x must be a CUDA tensor")
+    _check(_lib.fp8_quant_act(x.data_ptr(), M, K, x.stride(0), _dev(x8, torch.uint8, "x8", (M, K)),
+                              _dev(s_tok, torch.float32, "s_tok", (M,)), _stream()), "fp8_quant_act")
+    return x8, s_tok
+
+
+def rowwise_linear(x8: torch.Tensor, s_tok: torch.Tensor, w8: torch.Tensor, s_ch: torch.Tensor,
+                   y: torch.Tensor | None = None):
+    """y bf16 [M, N] = (x8 . w8^T) * s_tok[:, None] * s_ch[None, :]."""
+    M, K = x8.shape
+    N = w8.shape[0]
+    y = torch.empty((M, N), dtype=torch.bfloat16, device=x8.device) if y is None else y
+    _check(_lib.fp8_rowwise_linear(_dev(x8, torch.uint8, "x8"), _dev(s_tok, torch.float32, "s_tok", (M,)),
+                                   _dev(w8, torch.uint8, "w8", (N, K)),
+                                   _dev(s_ch, torch.float32, "s_ch", (N,)), M, N, K,
+                                   _dev(y, torch.bfloat16, "y", (M, N)), _stream()),
+           "fp8_rowwise_linear")
+    return y
+
+
+def linear(x: torch.Tensor, w8: torch.Tensor, s_ch: torch.Tensor, y: torch.Tensor | None = None,
+           x8: torch.Tensor | None = None, s_tok: torch.Tensor | None = None):
+    """The W8A8 linear from bf16 activations: quantize per token, then GEMM."""
+    M, K = x.shape
+    N = w8.shape[0]
+    dev = x.device
+    y = torch.empty((M, N), dtype=torch.bfloat16, device=dev) if y is None else y
+    x8 = torch.empty((M, K), dtype=torch.uint8, device=dev) if x8 is None else x8
+    s_tok = torch.empty((M,), dtype=torch.float32, device=dev) if s_tok is None else s_tok
+    _check(_lib.fp8_linear_bf16(_dev(x, torch.bfloat16, "x"), _dev(w8, torch.uint8, "w8", (N, K)),
+                                _dev(s_ch, torch.float32, "s_ch", (N,)), M, N, K,
+                                _dev(x8, torch.uint8, "x8", (M, K)),
+                                _dev(s_tok, torch.float32, "s_tok", (M,)),
+                                _dev(y, torch.bfloat16, "y", (M, N)), _stream()), "fp8_linear_bf16")
+    return y
+
+
+def cast_e4m3(x: torch.Tensor, out: torch.Tensor | None = None):
+    """Element-wise fp32 -> E4M3 codes with the library's encoder."""
+    n = x.numel()
+    out = torch.empty(x.shape, dtype=torch.uint8, device=x.device) if out is None else out
+    _check(_lib.fp8_cast_e4m3(_dev(x, torch.float32, "x"), n, _dev(out, torch.uint8, "out"), _stream()),
+           "fp8_cast_e4m3")
+    return out
+
+
+__all__ = [
+    "Fp8Error", "raw", "version", "device_supported", "device_status", "repack_qat",
+    "convert_fnuz", "quant_act", "rowwise_linear", "linear", "cast_e4m3",
+    "DEV_NONFINITE", "DEV_NAN_CODE", "DEV_INEXACT", "DEV_TIMEOUT", "LIB_PATH",
+]

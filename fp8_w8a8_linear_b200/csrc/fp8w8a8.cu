@@ -1,0 +1,369 @@
+// fp8w8a8.cu - the C ABI (include/fp8w8a8.h): argument checks, TMA tensor
+// maps, kernel selection and launches. Every kernel of the library lives in
+// this translation unit (quant.cuh, gemm.cuh), so the device status word is
+// a single __device__ variable per device.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/fp8w8a8.h"
+#include "gemm.cuh"
+#include "ptx.cuh"
+#include "quant.cuh"
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
+
+struct DeviceInfo {
+  int sm_count = 0;
+  bool supported = false;
+  bool attrs_set = false;
+};
+
+DeviceInfo g_dev[kMaxDevices];
+std::mutex g_dev_mu;
+
+// Current device's info; sets the kernels' shared-memory attributes once.
+fp8_status device_info(DeviceInfo** out);
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// Row-major uint8 matrix [rows, cols] (pitch = cols bytes), 128-byte-wide
+// boxes of box_rows rows, 128B swizzle, out-of-bounds elements read as 0.
+bool make_tmap_u8(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols,
+                  uint32_t box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols};
+  cuuint32_t box[2] = {128, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  std::memset(m, 0, sizeof(*m));
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+fp8_status last_launch() {
+  return cudaGetLastError() == cudaSuccess ? FP8_OK : FP8_ERR_CUDA;
+}
+
+// ----------------------------------------------------------------- GEMM plans
+using namespace fp8k;
+
+template <int BN, int STAGES>
+fp8_status set_prefill_attr() {
+  return cudaFuncSetAttribute(gemm_prefill_kernel<BN, STAGES>,
+                              cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              static_cast<int>(PrefillCfg<BN, STAGES>::kSmem)) == cudaSuccess
+             ? FP8_OK
+             : FP8_ERR_CUDA;
+}
+
+template <int BNT, int STAGES>
+fp8_status set_decode_attr() {
+  return cudaFuncSetAttribute(gemm_decode_kernel<BNT, STAGES>,
+                              cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              static_cast<int>(DecodeCfg<BNT, STAGES>::kSmem)) == cudaSuccess
+             ? FP8_OK
+             : FP8_ERR_CUDA;
+}
+
+constexpr int kPrefillBN = 256;
+constexpr int kPrefillStages = 4;
+
+fp8_status device_info(DeviceInfo** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return FP8_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_dev_mu);
+  DeviceInfo& d = g_dev[dev];
+  if (!d.attrs_set) {
+    cudaDeviceProp prop;
+    if (cudaGetDeviceProperties(&prop, dev) != cudaSuccess) return FP8_ERR_CUDA;
+    d.sm_count = prop.multiProcessorCount;
+    d.supported = prop.major == 10 && prop.minor == 0;
+    if (!d.supported) return FP8_ERR_UNSUPPORTED;
+    fp8_status st = FP8_OK;
+    st = st != FP8_OK ? st : set_prefill_attr<kPrefillBN, kPrefillStages>();
+    st = st != FP8_OK ? st : set_decode_attr<16, 6>();
+    st = st != FP8_OK ? st : set_decode_attr<32, 5>();
+    st = st != FP8_OK ? st : set_decode_attr<64, 4>();
+    st = st != FP8_OK ? st : set_decode_attr<128, 3>();
+    if (st != FP8_OK) return st;
+    d.attrs_set = true;
+  }
+  if (!d.supported) return FP8_ERR_UNSUPPORTED;
+  *out = &d;
+  return FP8_OK;
+}
+
+void set_pdl(cudaLaunchAttribute* a, int& n, bool pdl) {
+  if (!pdl) return;
+  a[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  a[n].val.programmaticStreamSerializationAllowed = 1;
+  ++n;
+}
+
+fp8_status launch_prefill(const DeviceInfo& dev, const uint8_t* x8, const float* s_tok,
+                          const uint8_t* w8, const float* s_ch, int M, int N, int K, uint16_t* y,
+                          cudaStream_t stream, bool pdl) {
+  constexpr int BN = kPrefillBN, ST = kPrefillStages;
+  CUtensorMap tmA, tmB;
+  if (!make_tmap_u8(&tmA, x8, M, K, kBM) || !make_tmap_u8(&tmB, w8, N, K, BN)) return FP8_ERR_CUDA;
+  const int tiles_m = (M + kBM - 1) / kBM;
+  const int tiles_n = (N + BN - 1) / BN;
+  const int num_tiles = tiles_m * tiles_n;
+  const int group_m = std::min(tiles_m, 16);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(std::min(num_tiles, dev.sm_count));
+  cfg.blockDim = dim3(192);
+  cfg.dynamicSmemBytes = PrefillCfg<BN, ST>::kSmem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attrs[1];
+  int na = 0;
+  set_pdl(attrs, na, pdl);
+  cfg.attrs = attrs;
+  cfg.numAttrs = na;
+  if (cudaLaunchKernelEx(&cfg, gemm_prefill_kernel<BN, ST>, tmA, tmB, s_tok, s_ch, y, M, N, K,
+                         tiles_m, tiles_n, group_m) != cudaSuccess)
+    return FP8_ERR_CUDA;
+  return FP8_OK;
+}
+
+template <int BNT, int ST>
+fp8_status launch_decode_t(const DeviceInfo& dev, const uint8_t* x8, const float* s_tok,
+                           const uint8_t* w8, const float* s_ch, int M, int N, int K, uint16_t* y,
+                           cudaStream_t stream, bool pdl) {
+  CUtensorMap tmW, tmX;
+  if (!make_tmap_u8(&tmW, w8, N, K, kBM) || !make_tmap_u8(&tmX, x8, M, K, BNT))
+    return FP8_ERR_CUDA;
+  const int tiles = (N + kBM - 1) / kBM;
+  const int num_kb = (K + kBK - 1) / kBK;
+  // Split K so that about two CTAs per SM stream weights; splits divide 128.
+  int splits = 1;
+  while (splits < 8 && tiles * splits * 2 <= 2 * dev.sm_count && splits * 2 <= num_kb) splits *= 2;
+  const int kb_per_split = (num_kb + splits - 1) / splits;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(tiles * splits);
+  cfg.blockDim = dim3(192);
+  cfg.dynamicSmemBytes = DecodeCfg<BNT, ST>::kSmem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attrs[2];
+  int na = 0;
+  attrs[na].id = cudaLaunchAttributeClusterDimension;
+  attrs[na].val.clusterDim.x = splits;
+  attrs[na].val.clusterDim.y = 1;
+  attrs[na].val.clusterDim.z = 1;
+  ++na;
+  set_pdl(attrs, na, pdl);
+  cfg.attrs = attrs;
+  cfg.numAttrs = na;
+  if (cudaLaunchKernelEx(&cfg, gemm_decode_kernel<BNT, ST>, tmW, tmX, s_tok, s_ch, y, M, N, K,
+                         splits, kb_per_split) != cudaSuccess)
+    return FP8_ERR_CUDA;
+  return FP8_OK;
+}
+
+fp8_status launch_linear(const DeviceInfo& dev, const uint8_t* x8, const float* s_tok,
+                         const uint8_t* w8, const float* s_ch, int M, int N, int K, uint16_t* y,
+                         cudaStream_t stream, bool pdl) {
+  if (M <= 16) return launch_decode_t<16, 6>(dev, x8, s_tok, w8, s_ch, M, N, K, y, stream, pdl);
+  if (M <= 32) return launch_decode_t<32, 5>(dev, x8, s_tok, w8, s_ch, M, N, K, y, stream, pdl);
+  if (M <= 64) return launch_decode_t<64, 4>(dev, x8, s_tok, w8, s_ch, M, N, K, y, stream, pdl);
+  if (M <= 128) return launch_decode_t<128, 3>(dev, x8, s_tok, w8, s_ch, M, N, K, y, stream, pdl);
+  return launch_prefill(dev, x8, s_tok, w8, s_ch, M, N, K, y, stream, pdl);
+}
+
+// ----------------------------------------------------------------- quant plans
+fp8_status launch_quant_act(const uint16_t* x, int64_t M, int64_t K, int64_t ldx, uint8_t* x8,
+                            float* s_tok, cudaStream_t stream) {
+  const int64_t nvec = K / 8;
+  if (M <= 1024) {
+    // Few tokens: a whole 256-thread block per token row.
+    const dim3 grid(static_cast<unsigned>(M));
+    if (nvec <= 4 * 256)
+      quant_act_kernel<256, 4><<<grid, 256, 0, stream>>>(x, M, K, ldx, x8, s_tok);
+    else
+      quant_act_kernel<256, 0><<<grid, 256, 0, stream>>>(x, M, K, ldx, x8, s_tok);
+  } else {
+    const dim3 grid(static_cast<unsigned>((M + 7) / 8));
+    if (nvec <= 24 * 32)
+      quant_act_kernel<32, 24><<<grid, 256, 0, stream>>>(x, M, K, ldx, x8, s_tok);
+    else
+      quant_act_kernel<32, 0><<<grid, 256, 0, stream>>>(x, M, K, ldx, x8, s_tok);
+  }
+  return last_launch();
+}
+
+bool dims_ok(int64_t v, int64_t lim) { return v >= 0 && v <= lim; }
+
+constexpr int64_t kMaxRows = (int64_t(1) << 31) - 1;
+
+}  // namespace
+
+// =================================================================== C ABI
+extern "C" {
+
+int fp8_version(void) { return 100; }
+
+const char* fp8_status_string(fp8_status s) {
+  switch (s) {
+    case FP8_OK: return "FP8_OK";
+    case FP8_ERR_INVALID_ARG: return "FP8_ERR_INVALID_ARG";
+    case FP8_ERR_ALIGNMENT: return "FP8_ERR_ALIGNMENT";
+    case FP8_ERR_SHAPE: return "FP8_ERR_SHAPE";
+    case FP8_ERR_CUDA: return "FP8_ERR_CUDA";
+    case FP8_ERR_UNSUPPORTED: return "FP8_ERR_UNSUPPORTED";
+  }
+  return "FP8_ERR_UNKNOWN";
+}
+
+int fp8_device_supported(int device) {
+  cudaDeviceProp prop;
+  if (cudaGetDeviceProperties(&prop, device) != cudaSuccess) return 0;
+  return prop.major == 10 && prop.minor == 0;
+}
+
+fp8_status fp8_get_device_status(unsigned int* out) {
+  if (!out) return FP8_ERR_INVALID_ARG;
+  if (cudaDeviceSynchronize() != cudaSuccess) return FP8_ERR_CUDA;
+  unsigned int v = 0, zero = 0;
+  if (cudaMemcpyFromSymbol(&v, fp8k::g_dev_status, sizeof(v)) != cudaSuccess) return FP8_ERR_CUDA;
+  if (cudaMemcpyToSymbol(fp8k::g_dev_status, &zero, sizeof(zero)) != cudaSuccess) return FP8_ERR_CUDA;
+  *out = v;
+  return FP8_OK;
+}
+
+fp8_status fp8_repack_qat(const uint8_t* q4, const float* d, int64_t N, int64_t K, uint8_t* w8,
+                          float* s_ch, void* stream) {
+  if (!dims_ok(N, kMaxRows) || !dims_ok(K, int64_t(1) << 24)) return FP8_ERR_INVALID_ARG;
+  if (K % 32 != 0) return FP8_ERR_SHAPE;
+  if (N == 0) return FP8_OK;
+  if (!q4 || !d || !w8 || !s_ch) return FP8_ERR_INVALID_ARG;
+  if (!aligned16(q4) || !aligned16(w8) || !aligned4(d) || !aligned4(s_ch)) return FP8_ERR_ALIGNMENT;
+  DeviceInfo* dev;
+  if (fp8_status st = device_info(&dev)) return st;
+  const dim3 grid(static_cast<unsigned>((N + 7) / 8));
+  if (K / 32 <= 6 * 32)
+    repack_qat_kernel<32, 6><<<grid, 256, 0, as_stream(stream)>>>(q4, d, N, K, w8, s_ch);
+  else
+    repack_qat_kernel<32, 0><<<grid, 256, 0, as_stream(stream)>>>(q4, d, N, K, w8, s_ch);
+  return last_launch();
+}
+
+fp8_status fp8_convert_fnuz(const uint8_t* w8_fnuz, const float* s_fnuz, int64_t N, int64_t K,
+                            uint8_t* w8, float* s_ch, void* stream) {
+  if (!dims_ok(N, kMaxRows) || !dims_ok(K, int64_t(1) << 24)) return FP8_ERR_INVALID_ARG;
+  if (K % 16 != 0) return FP8_ERR_SHAPE;
+  if (N == 0) return FP8_OK;
+  if (!w8_fnuz || !s_fnuz || !w8 || !s_ch) return FP8_ERR_INVALID_ARG;
+  if (!aligned16(w8_fnuz) || !aligned16(w8) || !aligned4(s_fnuz) || !aligned4(s_ch))
+    return FP8_ERR_ALIGNMENT;
+  DeviceInfo* dev;
+  if (fp8_status st = device_info(&dev)) return st;
+  const dim3 grid(static_cast<unsigned>((N + 7) / 8));
+  convert_fnuz_kernel<32><<<grid, 256, 0, as_stream(stream)>>>(w8_fnuz, s_fnuz, N, K, w8, s_ch);
+  return last_launch();
+}
+
+fp8_status fp8_quant_act(const uint16_t* x, int64_t M, int64_t K, int64_t ldx, uint8_t* x8,
+                         float* s_tok, void* stream) {
+  if (!dims_ok(M, kMaxRows) || !dims_ok(K, int64_t(1) << 24) || ldx < K) return FP8_ERR_INVALID_ARG;
+  if (K % 16 != 0 || ldx % 8 != 0) return FP8_ERR_SHAPE;
+  if (M == 0 || K == 0) return FP8_OK;
+  if (!x || !x8 || !s_tok) return FP8_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(x8) || !aligned4(s_tok)) return FP8_ERR_ALIGNMENT;
+  DeviceInfo* dev;
+  if (fp8_status st = device_info(&dev)) return st;
+  return launch_quant_act(x, M, K, ldx, x8, s_tok, as_stream(stream));
+}
+
+static fp8_status check_linear(const void* x, const float* s_tok, const uint8_t* w8,
+                               const float* s_ch, int64_t M, int64_t N, int64_t K,
+                               const uint16_t* y) {
+  if (!dims_ok(M, kMaxRows) || !dims_ok(N, kMaxRows) || !dims_ok(K, 65536))
+    return FP8_ERR_INVALID_ARG;
+  if (K % 16 != 0) return FP8_ERR_SHAPE;
+  if (M == 0 || N == 0) return FP8_OK;
+  if (!x || !s_tok || !w8 || !s_ch || !y) return FP8_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(w8) || !aligned16(y) || !aligned4(s_tok) || !aligned4(s_ch))
+    return FP8_ERR_ALIGNMENT;
+  return FP8_OK;
+}
+
+fp8_status fp8_rowwise_linear(const uint8_t* x8, const float* s_tok, const uint8_t* w8,
+                              const float* s_ch, int64_t M, int64_t N, int64_t K, uint16_t* y,
+                              void* stream) {
+  if (fp8_status st = check_linear(x8, s_tok, w8, s_ch, M, N, K, y)) return st;
+  if (M == 0 || N == 0) return FP8_OK;
+  DeviceInfo* dev;
+  if (fp8_status st = device_info(&dev)) return st;
+  if (K == 0) {
+    if (cudaMemsetAsync(y, 0, static_cast<size_t>(M) * N * 2, as_stream(stream)) != cudaSuccess)
+      return FP8_ERR_CUDA;
+    return FP8_OK;
+  }
+  return launch_linear(*dev, x8, s_tok, w8, s_ch, static_cast<int>(M), static_cast<int>(N),
+                       static_cast<int>(K), y, as_stream(stream), false);
+}
+
+fp8_status fp8_linear_bf16(const uint16_t* x, const uint8_t* w8, const float* s_ch, int64_t M,
+                           int64_t N, int64_t K, uint8_t* x8, float* s_tok, uint16_t* y,
+                           void* stream) {
+  if (fp8_status st = check_linear(x, s_tok, w8, s_ch, M, N, K, y)) return st;
+  if (M == 0 || N == 0) return FP8_OK;
+  if (!x8) return FP8_ERR_INVALID_ARG;
+  if (!aligned16(x8)) return FP8_ERR_ALIGNMENT;
+  DeviceInfo* dev;
+  if (fp8_status st = device_info(&dev)) return st;
+  if (K == 0) {
+    if (cudaMemsetAsync(y, 0, static_cast<size_t>(M) * N * 2, as_stream(stream)) != cudaSuccess)
+      return FP8_ERR_CUDA;
+    return FP8_OK;
+  }
+  if (fp8_status st = launch_quant_act(x, M, K, K, x8, s_tok, as_stream(stream))) return st;
+  return launch_linear(*dev, x8, s_tok, w8, s_ch, static_cast<int>(M), static_cast<int>(N),
+                       static_cast<int>(K), y, as_stream(stream), true);
+}
+
+fp8_status fp8_cast_e4m3(const float* x, int64_t n, uint8_t* out, void* stream) {
+  if (n < 0 || n > (int64_t(1) << 40)) return FP8_ERR_INVALID_ARG;
+  if (n == 0) return FP8_OK;
+  if (!x || !out) return FP8_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(out)) return FP8_ERR_ALIGNMENT;
+  DeviceInfo* dev;
+  if (fp8_status st = device_info(&dev)) return st;
+  const int64_t threads = (n + 3) / 4;
+  const dim3 grid(static_cast<unsigned>((threads + 255) / 256));
+  cast_e4m3_kernel<<<grid, 256, 0, as_stream(stream)>>>(x, n, out);
+  return last_launch();
+}
+
+}  // extern "C"

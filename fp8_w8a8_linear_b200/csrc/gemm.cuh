@@ -1,0 +1,412 @@
+// gemm.cuh - row-wise scaled FP8 GEMM on sm_100a tensor cores.
+//
+//   y[m, n] = bf16_rn( fp32( acc[m, n] * s_tok[m] ) * s_ch[n] ),
+//   acc[m, n] = sum_k e4m3(x8[m, k]) * e4m3(w8[n, k])   (fp32, in TMEM)
+//
+// The row-wise scaled FP8 GEMM of the W8A8 scheme (E2B MI300X article, step 3
+// boot log and the E4M3/E4M3FNUZ tip: RowWiseTorchFP8ScaledMMLinearKernel for
+// CompressedTensorsW8A8Fp8; 31B model card header: per-output-channel fp32
+// weight scales, per-token activation scales, bf16 output).
+//
+// Two kernels share one pipeline design:
+//
+// * gemm_prefill_kernel (M > 128): persistent, one CTA per SM, warp
+//   specialised. Warp 0 lane 0 streams 128x128-byte A tiles (activations)
+//   and BNx128-byte B tiles (weights) with TMA into a STAGES-deep ring of
+//   128B-swizzled shared-memory buffers; warp 1 lane 0 issues
+//   tcgen05.mma.kind::f8f6f4 (M=128, N=BN, K=32 per instruction) into one of
+//   two TMEM accumulators; warps 2-5 drain the other accumulator (tcgen05.ld),
+//   apply both scales and store bf16, so the epilogue of tile i overlaps the
+//   main loop of tile i+1. Tiles are walked in groups of `group_m` row tiles
+//   so that a wave of CTAs shares A and B tiles in L2.
+//
+// * gemm_decode_kernel (M <= 128): swap-AB. The weight tile is the MMA's A
+//   operand (128 output channels per CTA) and the tokens are its N (16..128),
+//   so a single token does not waste the 128-row MMA. K is split across the
+//   CTAs of a thread-block cluster (splits = cluster size, 1..8); each CTA
+//   writes its fp32 partial tile to its own shared memory, and after a cluster
+//   barrier each CTA sums one slice of rows over all CTAs' partials through
+//   distributed shared memory, in rank order, so the result is deterministic
+//   and needs no global workspace and no spin-waits. The weight stream uses an
+//   L2 evict-first policy, the (tiny) activation tile evict-last.
+//
+// Every mbarrier wait is bounded (ptx.cuh); the only unbounded waits are the
+// hardware cluster barriers, which every thread reaches on every path.
+#pragma once
+
+#include <cuda_bf16.h>
+
+#include <cstdint>
+
+#include "ptx.cuh"
+
+namespace fp8k {
+
+constexpr int kBM = 128;  // MMA M (rows of operand A)
+constexpr int kBK = 128;  // K bytes per pipeline stage (= one 128B swizzle row)
+
+__host__ __device__ constexpr int tmem_cols_for(int cols) {
+  return cols <= 32 ? 32 : cols <= 64 ? 64 : cols <= 128 ? 128 : cols <= 256 ? 256 : 512;
+}
+
+__device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
+  return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
+}
+
+__device__ __forceinline__ uint16_t f32_to_bf16_rn(float f) {
+  return __bfloat16_as_ushort(__float2bfloat16_rn(f));
+}
+
+// Two fp32 -> bf16 (round to nearest even), `lo` in bits [0,16).
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+// Tile order: groups of `group_m` row tiles; inside a group, row tiles vary
+// fastest, then column tiles.
+__device__ __forceinline__ void tile_coords(int tile, int tiles_m, int tiles_n, int group_m,
+                                            int& tm, int& tn) {
+  const int per_group = group_m * tiles_n;
+  const int g = tile / per_group;
+  const int first_m = g * group_m;
+  const int gm = min(tiles_m - first_m, group_m);
+  const int local = tile - g * per_group;
+  tm = first_m + local % gm;
+  tn = local / gm;
+}
+
+// ============================================================== prefill
+template <int BN, int STAGES>
+struct PrefillCfg {
+  static constexpr int kABytes = kBM * kBK;
+  static constexpr int kBBytes = BN * kBK;
+  static constexpr int kStageBytes = kABytes + kBBytes;
+  static constexpr int kTmemCols = tmem_cols_for(2 * BN);
+  static constexpr int kBarBytes = 8 * (2 * STAGES + 4) + 16;
+  static constexpr size_t kSmem = 1024 + static_cast<size_t>(STAGES) * kStageBytes + kBarBytes;
+  static_assert(BN % 32 == 0 && BN >= 32 && BN <= 256, "BN");
+};
+
+template <int BN, int STAGES>
+__global__ void __launch_bounds__(192, 1)
+    gemm_prefill_kernel(const __grid_constant__ CUtensorMap tmA,
+                        const __grid_constant__ CUtensorMap tmB, const float* __restrict__ s_a,
+                        const float* __restrict__ s_b, uint16_t* __restrict__ y, int M, int N,
+                        int K, int tiles_m, int tiles_n, int group_m) {
+  using C = PrefillCfg<BN, STAGES>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align1024(smem_raw);
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + STAGES * C::kABytes;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sB + STAGES * C::kBBytes);
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 4);
+  const uint32_t full0 = smem_u32(bars);
+  const uint32_t empty0 = smem_u32(bars + STAGES);
+  const uint32_t tfull0 = smem_u32(bars + 2 * STAGES);
+  const uint32_t tempty0 = smem_u32(bars + 2 * STAGES + 2);
+
+  const int warp = warp_id(), lane = lane_id();
+  const int num_kb = (K + kBK - 1) / kBK;
+  const int num_tiles = tiles_m * tiles_n;
+
+  if (warp == 0 && lane == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(full0 + 8 * s, 1);
+      mbar_init(empty0 + 8 * s, 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(tfull0 + 8 * b, 1);
+      mbar_init(tempty0 + 8 * b, 4);
+    }
+    fence_barrier_init();
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_holder), C::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_holder;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      pdl_wait();  // activations may come from a preceding quantizer grid
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
+        int tm, tn;
+        tile_coords(tile, tiles_m, tiles_n, group_m, tm, tn);
+        for (int kb = 0; kb < num_kb; ++kb) {
+          if (!mbar_wait(empty0 + 8 * stage, phase ^ 1)) { ok = false; break; }
+          const uint32_t fb = full0 + 8 * stage;
+          mbar_arrive_expect_tx(fb, C::kStageBytes);
+          tma_load_2d(smem_u32(sA + stage * C::kABytes), &tmA, fb, kb * kBK, tm * kBM, 0ull);
+          tma_load_2d(smem_u32(sB + stage * C::kBBytes), &tmB, fb, kb * kBK, tn * BN, 0ull);
+          if (++stage == STAGES) { stage = 0; phase ^= 1; }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_e4m3_f32(kBM, BN);
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
+        if (!mbar_wait(tempty0 + 8 * acc, acc_phase ^ 1)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + acc * BN;
+        for (int kb = 0; kb < num_kb; ++kb) {
+          if (!mbar_wait(full0 + 8 * stage, phase)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t a0 = smem_u32(sA + stage * C::kABytes);
+          const uint32_t b0 = smem_u32(sB + stage * C::kBBytes);
+#pragma unroll
+          for (int k = 0; k < kBK / 32; ++k) {
+            umma_f8(d_tmem, sw128_kmajor_desc(a0 + 32 * k), sw128_kmajor_desc(b0 + 32 * k), idesc,
+                    (kb | k) != 0);
+          }
+          umma_commit(empty0 + 8 * stage);
+          if (++stage == STAGES) { stage = 0; phase ^= 1; }
+        }
+        umma_commit(tfull0 + 8 * acc);
+        if (++acc == 2) { acc = 0; acc_phase ^= 1; }
+      }
+    }
+  } else {
+    // Epilogue warps 2..5; a warp may only touch TMEM lanes 32*(warp%4)..+31.
+    const int quad = warp & 3;
+    const bool vec_ok = (N % 8) == 0;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    bool waited = false;
+    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
+      int tm, tn;
+      tile_coords(tile, tiles_m, tiles_n, group_m, tm, tn);
+      if (!mbar_wait(tfull0 + 8 * acc, acc_phase)) break;
+      tc_fence_after();
+      if (!waited) { pdl_wait(); waited = true; }
+      const int row = tm * kBM + quad * 32 + lane;
+      const float sa = row < M ? __ldg(s_a + row) : 0.0f;
+      uint16_t* yrow = y + static_cast<int64_t>(row) * N;
+      const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + acc * BN;
+#pragma unroll 1
+      for (int c = 0; c < BN / 32; ++c) {
+        uint32_t r[32];
+        tmem_ld32(t_row + c * 32, r);
+        tmem_ld_wait();
+        const int n0 = tn * BN + c * 32;
+        if (row < M && n0 < N) {
+          if (vec_ok && n0 + 32 <= N) {
+            const float4* sb4 = reinterpret_cast<const float4*>(s_b + n0);
+            uint4* dst = reinterpret_cast<uint4*>(yrow + n0);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              const float4 b0 = __ldg(sb4 + 2 * q), b1 = __ldg(sb4 + 2 * q + 1);
+              const float sb[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+              float v[8];
+#pragma unroll
+              for (int i = 0; i < 8; ++i)
+                v[i] = __fmul_rn(__fmul_rn(__uint_as_float(r[8 * q + i]), sa), sb[i]);
+              dst[q] = make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]),
+                                  pack_bf16x2(v[4], v[5]), pack_bf16x2(v[6], v[7]));
+            }
+          } else {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              if (n0 + j < N) {
+                const float v = __fmul_rn(__fmul_rn(__uint_as_float(r[j]), sa), __ldg(s_b + n0 + j));
+                yrow[n0 + j] = f32_to_bf16_rn(v);
+              }
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(tempty0 + 8 * acc);
+      if (++acc == 2) { acc = 0; acc_phase ^= 1; }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem_base, C::kTmemCols);
+  }
+}
+
+// ============================================================== decode
+template <int BNT, int STAGES>
+struct DecodeCfg {
+  static constexpr int kWBytes = kBM * kBK;   // weight tile: 128 channels x 128 K bytes
+  static constexpr int kXBytes = BNT * kBK;   // token tile
+  static constexpr int kStageBytes = kWBytes + kXBytes;
+  static constexpr int kTmemCols = tmem_cols_for(BNT);
+  static constexpr int kRedBytes = BNT * kBM * 4;  // fp32 partial tile [token][channel]
+  static constexpr int kBarBytes = 8 * (2 * STAGES + 1) + 16;
+  static constexpr int kPipeBytes = STAGES * kStageBytes;
+  static constexpr size_t kSmem =
+      1024 + static_cast<size_t>(kPipeBytes > kRedBytes ? kPipeBytes : kRedBytes) + kBarBytes;
+  static_assert(BNT % 16 == 0 && BNT >= 16 && BNT <= 256, "BNT");
+  static_assert(kXBytes % 1024 == 0, "token tile must keep 1024-byte alignment");
+};
+
+template <int BNT, int STAGES>
+__global__ void __launch_bounds__(192)
+    gemm_decode_kernel(const __grid_constant__ CUtensorMap tmW,
+                       const __grid_constant__ CUtensorMap tmX, const float* __restrict__ s_tok,
+                       const float* __restrict__ s_ch, uint16_t* __restrict__ y, int M, int N,
+                       int K, int splits, int kb_per_split) {
+  using C = DecodeCfg<BNT, STAGES>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align1024(smem_raw);
+  uint8_t* sW = smem;
+  uint8_t* sX = smem + STAGES * C::kWBytes;
+  constexpr int kRegion = C::kPipeBytes > C::kRedBytes ? C::kPipeBytes : C::kRedBytes;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kRegion);
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 1);
+  float* red = reinterpret_cast<float*>(smem);  // reuses the pipeline buffers after the MMAs
+  const uint32_t full0 = smem_u32(bars);
+  const uint32_t empty0 = smem_u32(bars + STAGES);
+  const uint32_t tfull = smem_u32(bars + 2 * STAGES);
+
+  const int warp = warp_id(), lane = lane_id();
+  const int tile_n = blockIdx.x / splits;
+  const int rank = blockIdx.x % splits;  // == %cluster_ctarank for cluster dims (splits,1,1)
+  const int num_kb = (K + kBK - 1) / kBK;
+  const int kb0 = rank * kb_per_split;
+  const int kb1 = min(num_kb, kb0 + kb_per_split);
+
+  if (warp == 0 && lane == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(full0 + 8 * s, 1);
+      mbar_init(empty0 + 8 * s, 1);
+    }
+    mbar_init(tfull, 1);
+    fence_barrier_init();
+    tma_prefetch_desc(&tmW);
+    tma_prefetch_desc(&tmX);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_holder), C::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_holder;
+  bool have_acc = kb1 > kb0;
+
+  if (warp == 0) {
+    if (lane == 0 && have_acc) {
+      const uint64_t pol_w = l2_policy_evict_first();
+      const uint64_t pol_x = l2_policy_evict_last();
+      // The weight stream does not depend on a preceding quantizer grid: issue
+      // the first ring's weight tiles, then wait for the activations.
+      const int pre = min(STAGES, kb1 - kb0);
+      for (int i = 0; i < pre; ++i) {
+        const uint32_t fb = full0 + 8 * i;
+        mbar_arrive_expect_tx(fb, C::kStageBytes);
+        tma_load_2d(smem_u32(sW + i * C::kWBytes), &tmW, fb, (kb0 + i) * kBK, tile_n * kBM, pol_w);
+      }
+      pdl_wait();
+      for (int i = 0; i < pre; ++i)
+        tma_load_2d(smem_u32(sX + i * C::kXBytes), &tmX, full0 + 8 * i, (kb0 + i) * kBK, 0, pol_x);
+      int stage = pre % STAGES;
+      uint32_t phase = pre == STAGES ? 1u : 0u;
+      for (int kb = kb0 + pre; kb < kb1; ++kb) {
+        if (!mbar_wait(empty0 + 8 * stage, phase ^ 1)) break;
+        const uint32_t fb = full0 + 8 * stage;
+        mbar_arrive_expect_tx(fb, C::kStageBytes);
+        tma_load_2d(smem_u32(sW + stage * C::kWBytes), &tmW, fb, kb * kBK, tile_n * kBM, pol_w);
+        tma_load_2d(smem_u32(sX + stage * C::kXBytes), &tmX, fb, kb * kBK, 0, pol_x);
+        if (++stage == STAGES) { stage = 0; phase ^= 1; }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0 && have_acc) {
+      constexpr uint32_t idesc = idesc_e4m3_f32(kBM, BNT);
+      int stage = 0;
+      uint32_t phase = 0;
+      for (int kb = kb0; kb < kb1; ++kb) {
+        if (!mbar_wait(full0 + 8 * stage, phase)) break;
+        tc_fence_after();
+        const uint32_t a0 = smem_u32(sW + stage * C::kWBytes);
+        const uint32_t b0 = smem_u32(sX + stage * C::kXBytes);
+#pragma unroll
+        for (int k = 0; k < kBK / 32; ++k) {
+          umma_f8(tmem_base, sw128_kmajor_desc(a0 + 32 * k), sw128_kmajor_desc(b0 + 32 * k), idesc,
+                  (kb != kb0) || (k != 0));
+        }
+        umma_commit(empty0 + 8 * stage);
+        if (++stage == STAGES) { stage = 0; phase ^= 1; }
+      }
+      umma_commit(tfull);
+    }
+  } else {
+    const int quad = warp & 3;
+    const int ch = quad * 32 + lane;                 // channel within the tile (TMEM lane)
+    const int n = tile_n * kBM + ch;
+    if (have_acc && !mbar_wait(tfull, 0)) have_acc = false;
+    tc_fence_after();
+    pdl_wait();
+    const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quad * 32) << 16);
+    const float sc = n < N ? __ldg(s_ch + n) : 0.0f;
+#pragma unroll 1
+    for (int c = 0; c < BNT / 16; ++c) {
+      uint32_t r[16];
+      tmem_ld16(t_row + c * 16, r);
+      tmem_ld_wait();
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        const int tok = c * 16 + j;
+        const float acc = have_acc ? __uint_as_float(r[j]) : 0.0f;
+        if (splits == 1) {
+          if (tok < M && n < N)
+            y[static_cast<int64_t>(tok) * N + n] = f32_to_bf16_rn(__fmul_rn(__fmul_rn(acc, __ldg(s_tok + tok)), sc));
+        } else {
+          red[tok * kBM + ch] = acc;
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem_base, C::kTmemCols);
+  }
+  if (splits > 1) {
+    cluster_sync();  // every CTA's partial tile is in its shared memory
+    if (warp >= 2) {
+      const int et = threadIdx.x - 64;
+      const int rows = kBM / splits;
+      const uint32_t red_base = smem_u32(red);
+      for (int e = et; e < rows * BNT; e += 128) {
+        const int tok = e / rows;
+        const int ch = rank * rows + e % rows;
+        const int n = tile_n * kBM + ch;
+        if (tok >= M || n >= N) continue;
+        const uint32_t off = red_base + static_cast<uint32_t>((tok * kBM + ch) * 4);
+        float sum = 0.0f;
+        for (int j = 0; j < splits; ++j) sum = __fadd_rn(sum, ld_shared_cluster_f32(mapa_shared(off, j)));
+        y[static_cast<int64_t>(tok) * N + n] =
+            f32_to_bf16_rn(__fmul_rn(__fmul_rn(sum, __ldg(s_tok + tok)), __ldg(s_ch + n)));
+      }
+    }
+    cluster_sync();  // keep every CTA's shared memory alive until all reads are done
+  }
+}
+
+}  // namespace fp8k

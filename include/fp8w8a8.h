@@ -1,0 +1,176 @@
+/*
+ * fp8w8a8.h - C ABI of the B200 (sm_100a) FP8 W8A8 row-wise linear library.
+ *
+ * The method (pages cited by title and section):
+ *   - "Gemma 4 31B-it QAT, FP8 E4M3 W8A8, text only (unofficial)", header
+ *     paragraph: every Linear weight is FP8 E4M3 with one float32 scale per
+ *     output channel; activations are quantized to FP8 per token at run
+ *     time; other tensors stay bf16.
+ *   - Same card, "QAT trained the weights onto a 4-bit grid with one scale
+ *     per group of 32 values ... this build rounds the QAT weights again".
+ *   - "MI300X 上跑 Gemma 4 E2B：fp8 最快，却离原始权重最远", tip
+ *     "E4M3 还是 E4M3FNUZ，都能用": E4M3FNUZ (max 240, no negative zero)
+ *     checkpoints are converted at load and serve like the E4M3 build.
+ *   - Same article, step 3 boot log: the linear runs as a row-wise scaled
+ *     FP8 GEMM (RowWiseTorchFP8ScaledMMLinearKernel on the MI300X).
+ *
+ * Conventions shared by every entry point:
+ *   - All pointers are DEVICE pointers of the current CUDA device unless a
+ *     parameter says otherwise. The caller allocates and owns every buffer;
+ *     the library allocates no device memory. It keeps one device status word
+ *     per device (read with fp8_get_device_status) and a cached driver entry
+ *     point for tensor-map encoding.
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream). Every call
+ *     is asynchronous on that stream and returns after enqueueing work.
+ *   - Row-major layouts. bf16 values are passed as uint16_t bit patterns.
+ *     E4M3 / E4M3FNUZ values are uint8_t codes.
+ *   - Host-checkable errors (null pointers, sizes, alignment) return a
+ *     non-zero fp8_status BEFORE anything is enqueued. Conditions only the
+ *     GPU can see (non-finite inputs, FNUZ NaN codes, inexact FNUZ rows, a
+ *     wait that timed out) set bits of the device status word; the call
+ *     itself still returns FP8_OK, and the affected rows' outputs are
+ *     unspecified.
+ *   - Shapes are int64_t; all must be >= 0. A zero-sized problem enqueues
+ *     nothing and returns FP8_OK.
+ *
+ * Quantization arithmetic (bit-exact contract, the same in every kernel):
+ *   per row r of fp32 values v:  amax = max_k |v[k]|,
+ *   s[r] = fp32(amax / 448) (IEEE division, round to nearest even),
+ *   code[k] = E4M3_RNE_SATFINITE(fp32(v[k] / s[r])) with a zero result always
+ *   encoded as +0 (0x00). A row with amax == 0 gets s = 0 and all-zero codes.
+ */
+#ifndef FP8W8A8_H
+#define FP8W8A8_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum fp8_status {
+  FP8_OK = 0,
+  FP8_ERR_INVALID_ARG = 1, /* null pointer, negative size, ldx < K        */
+  FP8_ERR_ALIGNMENT = 2,   /* a pointer or row pitch is not 16-byte aligned */
+  FP8_ERR_SHAPE = 3,       /* K not a multiple of 16 (32 for q4_0), or a
+                              dimension beyond the library's limits        */
+  FP8_ERR_CUDA = 4,        /* a CUDA runtime/driver call failed            */
+  FP8_ERR_UNSUPPORTED = 5  /* the current device is not sm_100             */
+} fp8_status;
+
+/* Bits of the device status word. */
+#define FP8_DEV_NONFINITE 0x1u /* a row held NaN/Inf (amax not finite)        */
+#define FP8_DEV_NAN_CODE 0x2u  /* FNUZ input held code 0x80 (its NaN)          */
+#define FP8_DEV_INEXACT 0x4u   /* FNUZ row not exactly representable in E4M3  */
+#define FP8_DEV_TIMEOUT 0x8u   /* a bounded in-kernel wait gave up            */
+
+/* Library version: major * 10000 + minor * 100 + patch. */
+int fp8_version(void);
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* fp8_status_string(fp8_status status);
+
+/* Returns 1 when `device` is an sm_100 GPU this library was built for. */
+int fp8_device_supported(int device);
+
+/*
+ * Reads and clears the current device's status word. Synchronizes the
+ * current device first, so every previously enqueued call is covered.
+ * `out` is a HOST pointer.
+ */
+fp8_status fp8_get_device_status(unsigned int* out);
+
+/*
+ * fp8_repack_qat: QAT q4_0-grid weights -> per-output-channel E4M3.
+ * Source: model card above, "QAT trained the weights onto a 4-bit grid with
+ * one scale per group of 32 values"; header paragraph (one float32 scale per
+ * output channel).
+ *   q4   [N, K/2] uint8: packed int4, element 2j in the low nibble and 2j+1 in
+ *        the high nibble, 4-bit two's complement (values -8..7).
+ *   d    [N, K/32] float32: one scale per group of 32 values along K.
+ *   w8   [N, K] uint8 out: E4M3 codes of w = fp32(d[n, k/32] * q[n, k])
+ *        quantized per row with the contract above.
+ *   s_ch [N] float32 out: per-output-channel scales.
+ * Requires K % 32 == 0; q4, d, w8 16-byte aligned; s_ch 4-byte aligned.
+ * Device status: FP8_DEV_NONFINITE when a row's d*q is not finite.
+ */
+fp8_status fp8_repack_qat(const uint8_t* q4, const float* d, int64_t N, int64_t K,
+                          uint8_t* w8, float* s_ch, void* stream);
+
+/*
+ * fp8_convert_fnuz: load-time conversion of an E4M3FNUZ-stored weight to the
+ * E4M3 format the GEMM consumes. Source: E2B article, tip "E4M3 还是
+ * E4M3FNUZ，都能用" (converted at load; FNUZ max 240, no negative zero).
+ *   w8_fnuz [N, K] uint8, s_fnuz [N] float32: the FNUZ weight and scales.
+ *   w8 [N, K] uint8 out, s_ch [N] float32 out: E4M3 codes and scales with
+ *   dec_e4m3(w8) * s_ch == dec_fnuz(w8_fnuz) * s_fnuz for every element.
+ * Per row: with no +-240 code (0x7F / 0xFF) and an exactly halvable scale the
+ * bytes are copied and the scale halved; otherwise each value is re-encoded
+ * in E4M3 at the same scale (round to nearest even), which is exact except
+ * for FNUZ codes with exponent field <= 1 and an odd mantissa; such rows set
+ * FP8_DEV_INEXACT. Code 0x80 sets FP8_DEV_NAN_CODE; a non-finite scale sets
+ * FP8_DEV_NONFINITE. Requires K % 16 == 0 and 16-byte aligned byte arrays.
+ * w8 may alias w8_fnuz and s_ch may alias s_fnuz (in-place conversion).
+ */
+fp8_status fp8_convert_fnuz(const uint8_t* w8_fnuz, const float* s_fnuz, int64_t N,
+                            int64_t K, uint8_t* w8, float* s_ch, void* stream);
+
+/*
+ * fp8_quant_act: per-token dynamic activation quantization. Source: model
+ * card header paragraph ("activations quantized to FP8 per token at run
+ * time"); sizes article, format table (fp8 = FP8 activations per token).
+ *   x    [M, ldx] bf16 (uint16 bit patterns), row pitch ldx >= K elements.
+ *   x8   [M, K] uint8 out: E4M3 codes (dense, pitch K).
+ *   s_tok [M] float32 out: per-token scales amax/448.
+ * Requires K % 16 == 0, ldx % 8 == 0, x and x8 16-byte aligned.
+ * Device status: FP8_DEV_NONFINITE when a token row holds NaN/Inf.
+ */
+fp8_status fp8_quant_act(const uint16_t* x, int64_t M, int64_t K, int64_t ldx, uint8_t* x8,
+                         float* s_tok, void* stream);
+
+/*
+ * fp8_rowwise_linear: y = (x8 . w8^T) * s_tok * s_ch in bf16. Source: E2B
+ * article step 3 and model card ("vLLM picked
+ * RowWiseTorchFP8ScaledMMLinearKernel"), row-wise scaled FP8 GEMM.
+ *   x8 [M, K] uint8 E4M3, s_tok [M] float32 (per token).
+ *   w8 [N, K] uint8 E4M3, s_ch  [N] float32 (per output channel).
+ *   y  [M, N] bf16 out (uint16 bit patterns), pitch N.
+ * y[m, n] = bf16_rn(fp32(acc[m, n] * s_tok[m]) * s_ch[n]) where acc is the
+ * fp32 tensor-core sum over k of dec(x8[m,k]) * dec(w8[n,k]). The sum order
+ * is fixed per shape, so results are bit-reproducible run to run.
+ * Requires K % 16 == 0 and K <= 65536; x8, w8, y 16-byte aligned.
+ * Runs on tcgen05 tensor cores with TMA-staged tiles and a TMEM accumulator;
+ * M <= 64 selects a swap-AB split-K variant bound by the weight stream.
+ */
+fp8_status fp8_rowwise_linear(const uint8_t* x8, const float* s_tok, const uint8_t* w8,
+                              const float* s_ch, int64_t M, int64_t N, int64_t K,
+                              uint16_t* y, void* stream);
+
+/*
+ * fp8_linear_bf16: the whole W8A8 linear from bf16 activations: per-token
+ * quantization of x (exactly fp8_quant_act) followed by the row-wise GEMM
+ * (exactly fp8_rowwise_linear). The GEMM is launched as a programmatic
+ * dependent of the quantizer, so its prologue and weight stream start while
+ * the quantizer runs.
+ *   x [M, K] bf16 (pitch K); x8 [M, K] uint8 and s_tok [M] float32 are
+ *   caller-provided scratch that also receive the quantized activations;
+ *   w8, s_ch, y as in fp8_rowwise_linear.
+ */
+fp8_status fp8_linear_bf16(const uint16_t* x, const uint8_t* w8, const float* s_ch, int64_t M,
+                           int64_t N, int64_t K, uint8_t* x8, float* s_tok, uint16_t* y,
+                           void* stream);
+
+/*
+ * fp8_cast_e4m3: element-wise fp32 -> E4M3 with the library's encoder
+ * (round to nearest even, saturating to +-448, NaN -> 0x7F, zero -> 0x00).
+ * The encoding step the quantizers use, exposed for exhaustive testing.
+ *   x [n] float32, out [n] uint8. Requires 16-byte aligned x and out.
+ */
+fp8_status fp8_cast_e4m3(const float* x, int64_t n, uint8_t* out, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FP8W8A8_H */

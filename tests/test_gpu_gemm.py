@@ -1,0 +1,175 @@
+"""GPU parity of the row-wise scaled FP8 GEMM against the exact fp64 oracle:
+|y - y_ref| <= 4e-3 * s_tok * s_ch * sum_k |x8*w8| + 1 bf16 ulp, element by
+element (the whole output at moderate sizes, sampled rows at full size),
+plus bit-exact identities the kernels must keep (determinism, the one-call
+quantize+GEMM path, the FNUZ-converted weights, one-hot rows)."""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from oracle import formats as F
+from tests.gpu_util import bf16_to_np_bits, bf16_values, f32, same_bits_f32, to_dev, u8
+from workloads import activations_bf16, q4_weights
+
+pytestmark = pytest.mark.gpu
+
+
+def _operands(M, N, K, seed, outl=0.01):
+    q4, d = q4_weights(N, K, seed=seed)
+    xb = activations_bf16(M, K, seed=seed, outlier_frac=outl)
+    w = oracle.repack_qat(q4, d)
+    a = oracle.quant_act(xb)
+    return xb, a, w
+
+
+def _check(y_gpu, a, w, rows=None):
+    x8, st = (a.codes, a.scales) if rows is None else (a.codes[rows], a.scales[rows])
+    y_ref, abs_s = oracle.rowwise_linear_ref(x8, st, w.codes, w.scales, return_abs=True)
+    got = bf16_values(y_gpu) if rows is None else bf16_values(y_gpu)[rows]
+    ok, worst = oracle.check_linear(got, y_ref, abs_s)
+    assert ok, f"worst error / tolerance = {worst}"
+    return worst
+
+
+GEMM_SHAPES = [
+    # (M, N, K): decode (swap-AB, split-K) and prefill (persistent) kernels,
+    # ragged M / N / K tails, K shorter than one 128-byte stage.
+    (4, 128, 256),
+    (1, 128, 16),
+    (3, 200, 48),
+    (17, 1000, 272),
+    (33, 130, 4096),
+    (64, 8190, 512),
+    (100, 384, 1024),
+    (128, 520, 1040),
+    (129, 520, 1040),
+    (255, 256, 128),
+    (1000, 1000, 2000),
+    (2048, 2304, 4096),
+    (300, 4096, 5376),
+]
+
+
+@pytest.mark.parametrize("M,N,K", GEMM_SHAPES)
+def test_gemm_within_bound(lib, M, N, K):
+    xb, a, w = _operands(M, N, K, seed=M + N + K)
+    y = lib.rowwise_linear(to_dev(a.codes), to_dev(a.scales), to_dev(w.codes), to_dev(w.scales))
+    _check(y, a, w)
+    assert lib.device_status() == 0
+
+
+@pytest.mark.parametrize("M", [1, 8, 64])
+def test_decode_sweep_shapes(lib, M):
+    """Decode GEMM sweep: K=2048, N=8192, activations with 1% outlier channels."""
+    xb, a, w = _operands(M, 8192, 2048, seed=1)
+    x8, s = lib.quant_act(to_dev(xb))
+    assert np.array_equal(u8(x8), a.codes) and same_bits_f32(f32(s), a.scales)
+    wd, sw = lib.repack_qat(*[to_dev(t) for t in q4_weights(8192, 2048, seed=1)])
+    assert np.array_equal(u8(wd), w.codes) and same_bits_f32(f32(sw), w.scales)
+    y = lib.rowwise_linear(x8, s, wd, sw)
+    _check(y, a, w)
+
+
+def test_deterministic_and_one_call_path(lib):
+    for M, N, K in [(8, 4096, 2048), (64, 1024, 4096), (512, 2048, 1024)]:
+        xb, a, w = _operands(M, N, K, seed=21)
+        x8d, sd = to_dev(a.codes), to_dev(a.scales)
+        wd, swd = to_dev(w.codes), to_dev(w.scales)
+        y1 = bf16_to_np_bits(lib.rowwise_linear(x8d, sd, wd, swd))
+        y2 = bf16_to_np_bits(lib.rowwise_linear(x8d, sd, wd, swd))
+        assert np.array_equal(y1, y2)
+        y3 = bf16_to_np_bits(lib.linear(to_dev(xb), wd, swd))
+        assert np.array_equal(y1, y3)
+
+
+def test_one_hot_rows_are_exact(lib):
+    K, N = 256, 384
+    rng = np.random.default_rng(4)
+    w = oracle.repack_qat(*q4_weights(N, K, seed=4))
+    M = 200
+    ks = rng.integers(0, K, M)
+    x8 = np.zeros((M, K), np.uint8)
+    x8[np.arange(M), ks] = 0x38                       # 1.0
+    st = np.full(M, 0.5, np.float32)
+    y = bf16_values(lib.rowwise_linear(to_dev(x8), to_dev(st), to_dev(w.codes), to_dev(w.scales)))
+    # a single product: the fp32 path is exact up to the final bf16 rounding
+    prod = (F.dec_e4m3(w.codes[:, ks].T) * 0.5).astype(np.float32) * w.scales[None, :]
+    expect = bf16_values(torch.from_numpy(prod.astype(np.float32)).to(torch.bfloat16))
+    assert np.array_equal(y, expect)
+
+
+def test_negated_activations_negate_output(lib):
+    M, N, K = 96, 512, 768
+    xb, a, w = _operands(M, N, K, seed=8)
+    args = (to_dev(w.codes), to_dev(w.scales))
+    y = bf16_values(lib.rowwise_linear(to_dev(a.codes), to_dev(a.scales), *args))
+    neg = np.where(a.codes != 0, a.codes ^ 0x80, 0).astype(np.uint8)
+    yn = bf16_values(lib.rowwise_linear(to_dev(neg), to_dev(a.scales), *args))
+    assert np.array_equal(yn, -y)
+
+
+@pytest.fixture(scope="module")
+def prefill_weights():
+    q4, d = q4_weights(14336, 4096, seed=2)
+    return q4, d, oracle.repack_qat(q4, d)
+
+
+def test_prefill_with_fnuz_weights_matches_e4m3_path(lib, prefill_weights):
+    """Prefill GEMM (K=4096, N=14336) from an E4M3FNUZ-stored copy of the
+    weights, converted at load, gives the same bits as from the E4M3 repack."""
+    q4, d, w = prefill_weights
+    wd, sw = lib.repack_qat(to_dev(q4), to_dev(d))
+    assert np.array_equal(u8(wd), w.codes) and same_bits_f32(f32(sw), w.scales)
+    cn, sn = oracle.fnuz_copy_of_e4m3(w.codes, w.scales)
+    wf, sf = lib.convert_fnuz(to_dev(cn), to_dev(sn))
+    assert np.array_equal(u8(wf), w.codes) and same_bits_f32(f32(sf), w.scales)
+    for M in (128, 1024):
+        xb = activations_bf16(M, 4096, seed=2, outlier_frac=0.01)
+        x8, s = lib.quant_act(to_dev(xb))
+        y1 = bf16_to_np_bits(lib.rowwise_linear(x8, s, wd, sw))
+        y2 = bf16_to_np_bits(lib.rowwise_linear(x8, s, wf, sf))
+        assert np.array_equal(y1, y2)
+    assert lib.device_status() == 0
+
+
+@pytest.mark.parametrize("M", [128, 1024, 8192])
+def test_prefill_shapes_sampled(lib, prefill_weights, M):
+    """Prefill GEMM, K=4096, N=14336: every output of 64 sampled rows (all of
+    them at M=128) against the oracle."""
+    q4, d, w = prefill_weights
+    xb = activations_bf16(M, 4096, seed=2, outlier_frac=0.01)
+    x8, s = lib.quant_act(to_dev(xb))
+    y = lib.rowwise_linear(x8, s, to_dev(w.codes), to_dev(w.scales))
+    rows = np.arange(M) if M <= 128 else np.sort(np.random.default_rng(M).choice(M, 64, replace=False))
+    a = oracle.quant_act(xb[rows])
+    assert np.array_equal(u8(x8)[rows], a.codes)
+    y_ref, abs_s = oracle.rowwise_linear_ref(a.codes, a.scales, w.codes, w.scales, return_abs=True)
+    ok, worst = oracle.check_linear(bf16_values(y)[rows], y_ref, abs_s)
+    assert ok, worst
+
+
+@pytest.mark.parametrize("M", [1, 64, 65536])
+def test_large_layer_sampled(lib, M):
+    """Large dense layer K=5376, N=21504 from the GPU repack of its q4_0 grid:
+    512 sampled weight rows bit-exact against the oracle repack, and the
+    outputs of sampled token rows on those channels within the bound, at the
+    sizes the benchmark runs."""
+    N, K = 21504, 5376
+    q4, d = q4_weights(N, K, seed=3)
+    wd, sw = lib.repack_qat(to_dev(q4), to_dev(d))
+    cols = np.sort(np.random.default_rng(1).choice(N, 512, replace=False))
+    w = oracle.repack_qat(q4[cols], d[cols])
+    assert np.array_equal(u8(wd)[cols], w.codes) and same_bits_f32(f32(sw)[cols], w.scales)
+    xb = activations_bf16(M, K, seed=3, outlier_frac=0.01)
+    x8 = torch.empty((M, K), dtype=torch.uint8, device="cuda")
+    st = torch.empty((M,), dtype=torch.float32, device="cuda")
+    y = lib.linear(to_dev(xb), wd, sw, x8=x8, s_tok=st)
+    rows = np.arange(M) if M <= 64 else np.sort(np.random.default_rng(M).choice(M, 32, replace=False))
+    a = oracle.quant_act(xb[rows])
+    assert np.array_equal(u8(x8)[rows], a.codes) and same_bits_f32(f32(st)[rows], a.scales)
+    y_ref, abs_s = oracle.rowwise_linear_ref(a.codes, a.scales, w.codes, w.scales, return_abs=True)
+    ok, worst = oracle.check_linear(bf16_values(y)[rows][:, cols], y_ref, abs_s)
+    assert ok, worst
+    assert lib.device_status() == 0
