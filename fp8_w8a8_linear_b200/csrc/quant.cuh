@@ -145,9 +145,10 @@ __device__ __forceinline__ GroupLUT group_lut(float d, float s) {
   for (int q = 1; q <= 8; ++q) f[q - 1] = __fdiv_rn(__fmul_rn(d, static_cast<float>(q)), s);
   const uint32_t p0 = pack4_e4m3(f[0], f[1], f[2], f[3]);  // codes of q = 1..4
   const uint32_t p1 = pack4_e4m3(f[4], f[5], f[6], f[7]);  // codes of q = 5..8
-  // Negation flips bit 7 of every nonzero code.
-  const uint32_t n0 = p0 | (0x80808080u & ~__vcmpeq4(p0, 0u));
-  const uint32_t n1 = p1 | (0x80808080u & ~__vcmpeq4(p1, 0u));
+  // Negation flips bit 7 of every nonzero code (d may be negative, so the
+  // codes of q = 1..8 can carry either sign).
+  const uint32_t n0 = p0 ^ (0x80808080u & ~__vcmpeq4(p0, 0u));
+  const uint32_t n1 = p1 ^ (0x80808080u & ~__vcmpeq4(p1, 0u));
   GroupLUT L;
   // nibble 0..7 -> q = 0..7: [0, c1, c2, c3 | c4, c5, c6, c7]
   L.t0 = (p0 << 8);

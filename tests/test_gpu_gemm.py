@@ -17,9 +17,15 @@ pytestmark = pytest.mark.gpu
 
 
 def _operands(M, N, K, seed, outl=0.01):
-    q4, d = q4_weights(N, K, seed=seed)
+    """Oracle-quantized operands. For K that is not a whole number of q4_0
+    groups the weight is the first K columns of a wider repacked weight (still
+    a valid E4M3 weight with per-channel scales)."""
+    K32 = -(-K // 32) * 32
+    q4, d = q4_weights(N, K32, seed=seed)
     xb = activations_bf16(M, K, seed=seed, outlier_frac=outl)
     w = oracle.repack_qat(q4, d)
+    if K32 != K:
+        w = oracle.QuantResult(np.ascontiguousarray(w.codes[:, :K]), w.scales, w.bad_rows)
     a = oracle.quant_act(xb)
     return xb, a, w
 
