@@ -1,0 +1,463 @@
+"""Benchmark of the FP8 W8A8 row-wise linear path on B200.
+
+One step is one pass of the whole path over one batch of synthetic input. For
+the default workload (the large dense layer K=5376, N=21504, the only one that
+spans the metric's M = 1..65536) a step is:
+
+  1. the QAT q4_0 -> per-channel E4M3 repack of the 21504x5376 weight,
+  2. the load-time conversion of an E4M3FNUZ-stored copy of that weight,
+  3. the per-token activation quantization and the row-wise FP8 GEMM at
+     M = 65536 (64 requests x 1,024 tokens), M = 1 and M = 64,
+
+with every input resident in HBM. The L2 is flushed (a 256 MiB write) before
+each decode-sized GEMM so its weights stream from HBM; the flushes are not
+counted in the step time. Other workloads (``--workload tiny|decode|prefill``)
+measure the other configurations.
+
+Output: one JSON line (rank 0). ``value`` is GEMM TFLOP/s of the whole step
+(all ranks' FLOPs / max-over-ranks device time); ``kernels`` breaks the step
+into ops with their own time, TFLOP/s, GB/s of algorithmic bytes and roofline
+fraction; ``roofline`` is the dominant kernel's; ``e2e`` repeats the step
+through the public API from pinned host buffers with the copies in the timed
+region; ``cpu_baseline`` times the CPU oracle on a bounded sample.
+
+``--impl reference`` times the CPU oracle itself (rank 0 only) on a bounded
+sample of the same workload and prints the same JSON line with
+``"impl": "reference"``.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "FP8 W8A8 row-wise linear TFLOP/s and GB/s, % of roofline, M=1..65536"
+UNIT = "TFLOP/s"
+
+# Fallback denominators (used only if MEASURED_PEAKS.json is absent).
+FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+FALLBACK_BF16_TFLOPS_SUSTAINED = 1400.0
+FP8_PER_BF16 = 2.0  # nominal dense ratio, 4.5 PF fp8 / 2.25 PF bf16
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return {"hbm_gbs": d["hbm_gbs"], "bf16": d["bf16_tflops"],
+                "bf16_sustained": d["bf16_tflops_sustained"], "source": "measured"}
+    return {"hbm_gbs": FALLBACK_HBM_GBS, "bf16": FALLBACK_BF16_TFLOPS,
+            "bf16_sustained": FALLBACK_BF16_TFLOPS_SUSTAINED, "source": "fallback"}
+
+
+# --------------------------------------------------------------------- workloads
+WORKLOADS = {
+    "large": dict(K=5376, N=21504, Ms=(65536, 1, 64), seed=3, outl=0.01, repack=True, fnuz=True,
+                  desc="large dense layer K=5376 N=21504, M in {65536,1,64}, QAT repack + FNUZ load conversion"),
+    "decode": dict(K=2048, N=8192, Ms=(1, 8, 64), seed=1, outl=0.01, repack=False, fnuz=False,
+                   desc="decode GEMM sweep K=2048 N=8192, M in {1,8,64}"),
+    "prefill": dict(K=4096, N=14336, Ms=(8192, 1024, 128), seed=2, outl=0.01, repack=False, fnuz=True,
+                    desc="prefill GEMM K=4096 N=14336, M in {8192,1024,128}, FNUZ load conversion"),
+    "tiny": dict(K=256, N=128, Ms=(4,), seed=0, outl=0.0, repack=True, fnuz=False,
+                 desc="tiny W8A8 linear M=4 K=256 N=128"),
+}
+
+
+def gemm_flops(M, N, K):
+    return 2.0 * M * N * K
+
+
+def linear_bytes(M, N, K):
+    """Algorithmic HBM bytes of quantize + GEMM (quantizer separate, so x8 and
+    s_tok are written and read back once)."""
+    quant = 2 * M * K + M * K + 4 * M
+    gemm = M * K + N * K + 4 * M + 4 * N + 2 * M * N
+    return quant, gemm
+
+
+# --------------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.gpu_id = gpu_id
+        self.proc = None
+        self.lines = []
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.gpu_id, f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.thread.join(timeout=5)
+        sm, smax, power, reasons = [], [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 7:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                smax.append(float(parts[1]))
+                power.append(float(parts[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[3:7]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax),
+                "power_w_max": max(power), "samples": len(sm), "reasons": sorted(reasons)}
+
+
+# --------------------------------------------------------------------- our arm
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+
+    import fp8_w8a8_linear_b200 as f
+    from workloads import activations_bf16, q4_weights
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    wl = WORKLOADS[args.workload]
+    K, N, Ms = wl["K"], wl["N"], wl["Ms"]
+    seed = wl["seed"] + 1000 * rank  # each rank has its own batch (weak scaling)
+    stream = torch.cuda.current_stream()
+
+    # ---- host inputs (pinned) and their device copies
+    def pinned(a):
+        a = np.ascontiguousarray(a)
+        t = torch.from_numpy(a.view(np.int16) if a.dtype == np.uint16 else a)
+        return t.pin_memory()
+
+    q4, d = q4_weights(N, K, seed=seed)
+    h = {"q4": pinned(q4), "d": pinned(d)}
+    for M in Ms:
+        h[f"x{M}"] = pinned(activations_bf16(M, K, seed=seed + M, outlier_frac=wl["outl"]))
+    D = {k: v.to(dev) for k, v in h.items()}
+    for M in Ms:
+        D[f"x{M}"] = D[f"x{M}"].view(torch.bfloat16)
+    w8, s_ch = f.repack_qat(D["q4"], D["d"])
+    if wl["fnuz"]:
+        # The E4M3FNUZ-stored copy of the same weights: identical bytes, doubled
+        # scales (every E4M3 code the repack emits means half as much in FNUZ).
+        D["wf"] = w8.clone()
+        D["sf"] = s_ch * 2
+        h["wf"] = D["wf"].cpu().pin_memory()
+        h["sf"] = D["sf"].cpu().pin_memory()
+    w8c = torch.empty_like(w8)
+    s_c = torch.empty_like(s_ch)
+    bufs = {}
+    for M in Ms:
+        bufs[M] = (torch.empty((M, K), dtype=torch.uint8, device=dev),
+                   torch.empty((M,), dtype=torch.float32, device=dev),
+                   torch.empty((M, N), dtype=torch.bfloat16, device=dev))
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+
+    # ---- one step: list of (name, fn, flops, bytes, bound)
+    def ops():
+        L = []
+        if wl["repack"]:
+            L.append(("repack_qat", lambda: f.repack_qat(D["q4"], D["d"], w8, s_ch), 0.0,
+                      N * K * 1.625 + 4 * N, "hbm", None))
+        if wl["fnuz"]:
+            L.append(("convert_fnuz", lambda: f.convert_fnuz(D["wf"], D["sf"], w8c, s_c), 0.0,
+                      2.0 * N * K + 8 * N, "hbm", None))
+        wsrc = (w8c, s_c) if wl["fnuz"] else (w8, s_ch)
+        for M in Ms:
+            x8, st, y = bufs[M]
+            qb, gb = linear_bytes(M, N, K)
+            fl = gemm_flops(M, N, K)
+            if M > 128:
+                L.append((f"quant_act[M={M}]", lambda x=D[f"x{M}"], x8=x8, st=st: f.quant_act(x, x8, st),
+                          0.0, qb, "hbm", None))
+                L.append((f"gemm_prefill[M={M}]",
+                          lambda x8=x8, st=st, y=y: f.rowwise_linear(x8, st, wsrc[0], wsrc[1], y),
+                          fl, gb, "tensor", None))
+            else:
+                L.append((f"linear_decode[M={M}]",
+                          lambda x=D[f"x{M}"], x8=x8, st=st, y=y: f.linear(x, wsrc[0], wsrc[1], y, x8, st),
+                          fl, qb + gb, "hbm", "flush"))
+        return L
+
+    step_ops = ops()
+    n_launch_per_step = sum(2 if n.startswith("linear") else 1 for n, *_ in step_ops)
+
+    def run_step(record):
+        evs = []
+        for name, fn, fl, by, bound, pre in step_ops:
+            if pre == "flush":
+                flush.zero_()
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            fn()
+            e1.record(stream)
+            evs.append((e0, e1))
+        return evs
+
+    for _ in range(args.warmup):
+        run_step(False)
+    torch.cuda.synchronize()
+    assert f.device_status() == 0, "device status set during warm-up"
+
+    gpu_uuid = str(torch.cuda.get_device_properties(dev).uuid)
+    sampler = ClockSampler(gpu_uuid if gpu_uuid.startswith("GPU-") else f"GPU-{gpu_uuid}")
+    sampler.start()
+    time.sleep(0.3)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    t_all0 = torch.cuda.Event(enable_timing=True)
+    t_all1 = torch.cuda.Event(enable_timing=True)
+    t_all0.record(stream)
+    all_evs = [run_step(True) for _ in range(args.steps)]
+    t_all1.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clocks = sampler.stop()
+    status = f.device_status()
+
+    per_op = np.zeros((args.steps, len(step_ops)))
+    for s, evs in enumerate(all_evs):
+        for i, (e0, e1) in enumerate(evs):
+            per_op[s, i] = e0.elapsed_time(e1)
+    op_ms = per_op.mean(axis=0)
+    step_ms = float(per_op.sum(axis=1).mean())
+    total_ms = float(per_op.sum())
+    if world > 1:
+        t = torch.tensor([total_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+        step_ms = total_ms / args.steps
+    flops_step = sum(o[2] for o in step_ops)
+    value = world * flops_step * args.steps / (total_ms * 1e-3) / 1e12
+
+    peaks = load_peaks()
+    fp8_sus = peaks["bf16_sustained"] * FP8_PER_BF16
+    kernels = []
+    for (name, fn, fl, by, bound, pre), ms in zip(step_ops, op_ms):
+        k = {"op": name, "us": round(ms * 1e3, 2), "gbs": round(by / (ms * 1e-3) / 1e9, 1),
+             "tflops": round(fl / (ms * 1e-3) / 1e12, 1), "bound": bound}
+        k["frac"] = round((k["tflops"] / fp8_sus) if bound == "tensor" else (k["gbs"] / peaks["hbm_gbs"]), 3)
+        kernels.append(k)
+    dom = max(range(len(step_ops)), key=lambda i: op_ms[i])
+    dname, _, dfl, dby, dbound, _ = step_ops[dom]
+    dms = op_ms[dom]
+    if dbound == "tensor":
+        roof = {"kernel": dname, "bound": "tensor", "achieved": round(dfl / (dms * 1e-3) / 1e12, 1),
+                "peak": round(fp8_sus, 1), "unit": "TFLOP/s",
+                "peak_note": f"fp8 dense = 2 x {peaks['source']} sustained bf16 cuBLAS ({peaks['bf16_sustained']})"}
+    else:
+        roof = {"kernel": dname, "bound": "hbm", "achieved": round(dby / (dms * 1e-3) / 1e9, 1),
+                "peak": peaks["hbm_gbs"], "unit": "GB/s", "peak_note": f"{peaks['source']} HBM copy"}
+    roof["frac"] = round(roof["achieved"] / roof["peak"], 3)
+    roof["traffic"] = TRAFFIC.get((args.workload, dname))
+
+    # ---- end to end through the public API, from pinned host buffers
+    e2e_steps = max(1, min(args.steps, 3))
+    outs_host = {M: torch.empty((M, N), dtype=torch.bfloat16).pin_memory() for M in Ms}
+    h2d = sum(t.numel() * t.element_size() for k, t in h.items())
+    d2h = sum(o.numel() * 2 for o in outs_host.values())
+
+    def e2e_step():
+        for k in h:
+            D[k].view(h[k].dtype).copy_(h[k], non_blocking=True)
+        for name, fn, *_ in step_ops:
+            fn()
+        for M in Ms:
+            outs_host[M].copy_(bufs[M][2], non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    ea, eb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ea.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    eb.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = ea.elapsed_time(eb)
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    e2e_val = world * flops_step * e2e_steps / (e2e_ms * 1e-3) / 1e12
+    status |= f.device_status()
+
+    out = None
+    if rank == 0:
+        out = {
+            "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(step_ms, 4),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "e4m3",
+            "data": "synthetic (seeded q4_0-grid weights, bf16 N(0,1) activations with 1% x20 outlier channels)",
+            "config": {"workload": args.workload, "desc": wl["desc"], "K": K, "N": N, "M": list(Ms),
+                       "parallelism": f"replicas x{world} (independent batches, no collective on the data path)",
+                       "l2": "inputs > L2 for the prefill GEMM; 256 MiB L2 flush before each decode GEMM (not timed)"},
+            "kernels": kernels,
+            "roofline": roof,
+            "gpu_launches": n_launch_per_step * args.steps,
+            "clocks": clocks,
+            "device_status": status,
+            "e2e": {"value": round(e2e_val, 3), "unit": UNIT, "steps": e2e_steps,
+                    "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)},
+        }
+    return out
+
+
+# Measured DRAM traffic per launch (dram__bytes_read.sum + dram__bytes_write.sum)
+# for the dominant kernel, from the ncu summaries under profiles/, keyed by
+# (workload, op). Kept null until a capture of the current kernel exists.
+TRAFFIC = {}
+
+
+# --------------------------------------------------------------------- oracle arm
+def oracle_sample(workload: str, rank: int = 0):
+    """The CPU oracle on a bounded sample of one step: the repack and FNUZ
+    conversion of 2048 weight rows, the activation quant of min(M, 2048) token
+    rows per M, and the exact GEMM of those tokens against those 2048 weight
+    rows. Returns (seconds, GEMM FLOPs, description)."""
+    import oracle
+    from workloads import activations_bf16, q4_weights
+
+    wl = WORKLOADS[workload]
+    K, N = wl["K"], wl["N"]
+    ns = min(N, 2048)
+    seed = wl["seed"] + 1000 * rank
+    q4, d = q4_weights(N, K, seed=seed, rows=slice(0, ns))
+    xs = {M: activations_bf16(M, K, seed=seed + M, outlier_frac=wl["outl"], rows=slice(0, min(M, 2048)))
+          for M in wl["Ms"]}
+    t0 = time.perf_counter()
+    w = oracle.repack_qat(q4, d)
+    if wl["fnuz"]:
+        cn, sn = oracle.fnuz_copy_of_e4m3(w.codes, w.scales)
+        oracle.convert_fnuz_to_e4m3(cn, sn)
+    flops = 0.0
+    for M, xb in xs.items():
+        a = oracle.quant_act(xb)
+        oracle.rowwise_linear_ref(a.codes, a.scales, w.codes, w.scales)
+        flops += gemm_flops(xb.shape[0], ns, K)
+    dt = time.perf_counter() - t0
+    desc = (f"{ns} of {N} weight rows (repack{', FNUZ conversion' if wl['fnuz'] else ''}), "
+            f"min(M,2048) token rows per M in {list(wl['Ms'])} (quant + exact fp64 GEMM vs those rows), K={K}")
+    return dt, flops, desc
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+
+        n = [i.get("num_threads", 0) for i in threadpool_info()]
+        return max(n) if n else os.cpu_count()
+    except Exception:
+        return os.cpu_count()
+
+
+def run_reference(args):
+    steps = []
+    for i in range(args.warmup + args.steps):
+        dt, fl, desc = oracle_sample(args.workload)
+        if i >= args.warmup:
+            steps.append((dt, fl))
+    tot = sum(s[0] for s in steps)
+    value = sum(s[1] for s in steps) / tot / 1e12
+    wl = WORKLOADS[args.workload]
+    cores = blas_threads()
+    return {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": 0,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(1e3 * tot / len(steps), 1),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": {"workload": args.workload, "desc": wl["desc"]},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": desc},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+# --------------------------------------------------------------------- main
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="large", choices=sorted(WORKLOADS))
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "ours":
+        ap.error("--warmup must be >= 3")
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args)), flush=True)
+        return
+
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        out = run_ours(args, rank, world, local_rank)
+        if rank == 0:
+            if world == 1 and not args.no_cpu_baseline:
+                dt, fl, desc = oracle_sample(args.workload)
+                out["cpu_baseline"] = {"value": fl / dt / 1e12, "unit": UNIT, "cores": blas_threads(),
+                                       "kind": "oracle", "sample": desc, "seconds": round(dt, 2)}
+            print(json.dumps(out), flush=True)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()
