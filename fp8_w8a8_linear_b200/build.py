@@ -1,7 +1,9 @@
 """Builds ``libfp8w8a8.so`` in-tree with nvcc for sm_100a.
 
-Usage: ``python -m fp8_w8a8_linear_b200.build [--verbose-ptxas]``. nvcc
-cross-compiles, so this runs without a GPU.
+Usage: ``python fp8_w8a8_linear_b200/build.py [--verbose-ptxas]``. nvcc
+cross-compiles, so this runs without a GPU. The script is self-contained and
+is loaded by file path, never through the package, whose
+``__init__`` needs the compiled library to exist already.
 """
 
 from __future__ import annotations

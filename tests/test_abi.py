@@ -13,10 +13,13 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 @pytest.fixture(scope="module")
 def clib():
-    from fp8_w8a8_linear_b200 import build
+    import importlib.util
 
-    path = build.build()
-    return ctypes.CDLL(path)
+    spec = importlib.util.spec_from_file_location(
+        "fp8w8a8_build", os.path.join(ROOT, "fp8_w8a8_linear_b200", "build.py"))
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    return ctypes.CDLL(mod.build())
 
 
 def _declared():
