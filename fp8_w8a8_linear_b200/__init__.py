@@ -28,7 +28,7 @@ LIB_PATH = os.path.join(_HERE, "libfp8w8a8.so")
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(
-        f"{LIB_PATH} is missing: build it with `python -m fp8_w8a8_linear_b200.build` "
+        f"{LIB_PATH} is missing: build it with `python fp8_w8a8_linear_b200/build.py` "
         "(the FP8 W8A8 path has no fallback)")
 
 _lib = ctypes.CDLL(LIB_PATH)
@@ -46,6 +46,7 @@ _SIGS = {
     "fp8_rowwise_linear": ([_P, _P, _P, _P, _I64, _I64, _I64, _P, _P], ctypes.c_int),
     "fp8_linear_bf16": ([_P, _P, _P, _I64, _I64, _I64, _P, _P, _P, _P], ctypes.c_int),
     "fp8_cast_e4m3": ([_P, _I64, _P, _P], ctypes.c_int),
+    "fp8_linear_bf16_noalloc": ([_P, _P, _P, _I64, _I64, _I64, _P, _P], ctypes.c_int),
 }
 for _name, (_args, _ret) in _SIGS.items():
     _f = getattr(_lib, _name)
@@ -175,6 +176,27 @@ def linear(x: torch.Tensor, w8: torch.Tensor, s_ch: torch.Tensor, y: torch.Tenso
     return y
 
 
+NOALLOC_SCRATCH_BYTES = 4 << 20
+
+
+def linear_noalloc(x: torch.Tensor, w8: torch.Tensor, s_ch: torch.Tensor,
+                   y: torch.Tensor | None = None):
+    """Same result as :func:`linear`, with the quantized activations kept in
+    the library's fixed device scratch array instead of caller buffers (for
+    callers that cannot allocate device memory). Problems needing more than
+    ``NOALLOC_SCRATCH_BYTES`` of scratch raise ``Fp8Error``. Calls that can
+    overlap on the GPU share that scratch and must be serialized."""
+    M, K = x.shape
+    N = w8.shape[0]
+    if y is None:
+        raise ValueError("pass a preallocated y: this entry point is for callers that do not allocate")
+    _check(_lib.fp8_linear_bf16_noalloc(_dev(x, torch.bfloat16, "x"), _dev(w8, torch.uint8, "w8", (N, K)),
+                                        _dev(s_ch, torch.float32, "s_ch", (N,)), M, N, K,
+                                        _dev(y, torch.bfloat16, "y", (M, N)), _stream()),
+           "fp8_linear_bf16_noalloc")
+    return y
+
+
 def cast_e4m3(x: torch.Tensor, out: torch.Tensor | None = None):
     """Element-wise fp32 -> E4M3 codes with the library's encoder."""
     n = x.numel()
@@ -186,6 +208,6 @@ def cast_e4m3(x: torch.Tensor, out: torch.Tensor | None = None):
 
 __all__ = [
     "Fp8Error", "raw", "version", "device_supported", "device_status", "repack_qat",
-    "convert_fnuz", "quant_act", "rowwise_linear", "linear", "cast_e4m3",
+    "convert_fnuz", "quant_act", "rowwise_linear", "linear", "linear_noalloc", "cast_e4m3",
     "DEV_NONFINITE", "DEV_NAN_CODE", "DEV_INEXACT", "DEV_TIMEOUT", "LIB_PATH",
 ]

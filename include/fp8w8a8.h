@@ -56,7 +56,9 @@ typedef enum fp8_status {
   FP8_ERR_SHAPE = 3,       /* K not a multiple of 16 (32 for q4_0), or a
                               dimension beyond the library's limits        */
   FP8_ERR_CUDA = 4,        /* a CUDA runtime/driver call failed            */
-  FP8_ERR_UNSUPPORTED = 5  /* the current device is not sm_100             */
+  FP8_ERR_UNSUPPORTED = 5, /* the current device is not sm_100             */
+  FP8_ERR_SCRATCH_LIMIT = 6 /* the problem needs more scratch than the
+                               library's fixed scratch array holds            */
 } fp8_status;
 
 /* Bits of the device status word. */
@@ -168,6 +170,40 @@ fp8_status fp8_linear_bf16(const uint16_t* x, const uint8_t* w8, const float* s_
  *   x [n] float32, out [n] uint8. Requires 16-byte aligned x and out.
  */
 fp8_status fp8_cast_e4m3(const float* x, int64_t n, uint8_t* out, void* stream);
+
+/*
+ * fp8_linear_bf16_noalloc: the same computation as fp8_linear_bf16 (per-token
+ * quantization of x, then the row-wise FP8 GEMM, with bit-identical results),
+ * for callers that cannot provide the quantized-activation scratch buffers.
+ * The pages have no counterpart to this entry point; it exists for callers
+ * that must not allocate device memory at all, for example a plugin that a
+ * host framework hands nothing but fixed input and output buffers because
+ * that framework owns all of device memory, or a latency-critical serving
+ * loop that cannot afford cudaMalloc's implicit device-wide synchronization.
+ *
+ *   x [M, K] bf16 (pitch K), w8 [N, K] E4M3, s_ch [N] fp32, y [M, N] bf16 out:
+ *   as in fp8_linear_bf16.
+ *
+ * Scratch: the quantized activations (M*K bytes, rounded up to 256) and the
+ * per-token scales (4*M bytes) live in one file-scope device array of
+ * FP8_NOALLOC_SCRATCH_BYTES bytes that every GPU which loads this library
+ * holds until the process exits. Larger problems return
+ * FP8_ERR_SCRATCH_LIMIT before anything is enqueued. The call allocates
+ * nothing: no cudaMalloc, no cudaFree, no allocating library routine.
+ *
+ * All calls share that one array and it keeps the last call's contents
+ * (nothing in it needs to start at zero: each call writes the scratch it
+ * reads). Calls that can overlap on the GPU - on different streams, or on
+ * different host threads without ordering - race on the array and must be
+ * serialized by the caller.
+ *
+ * The first call on each device looks up that device's address of the array
+ * (cudaGetSymbolAddress, with that device current) and caches it; make that
+ * first call before any stream capture begins.
+ */
+#define FP8_NOALLOC_SCRATCH_BYTES (4u << 20)
+fp8_status fp8_linear_bf16_noalloc(const uint16_t* x, const uint8_t* w8, const float* s_ch,
+                                   int64_t M, int64_t N, int64_t K, uint16_t* y, void* stream);
 
 #ifdef __cplusplus
 }
