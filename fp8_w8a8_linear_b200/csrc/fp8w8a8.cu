@@ -97,6 +97,8 @@ fp8_status set_decode_attr() {
 }
 
 constexpr int kPrefillBN = 256;
+// Shared memory the staged quantizer may use per block (one block per SM).
+constexpr int kStagedSmemBudget = 200 * 1024;
 constexpr int kPrefillStages = 4;
 
 fp8_status device_info(DeviceInfo** out) {
@@ -116,6 +118,10 @@ fp8_status device_info(DeviceInfo** out) {
     st = st != FP8_OK ? st : set_decode_attr<32, 5>();
     st = st != FP8_OK ? st : set_decode_attr<64, 4>();
     st = st != FP8_OK ? st : set_decode_attr<128, 3>();
+    if (st == FP8_OK &&
+        cudaFuncSetAttribute(quant_act_staged_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             kStagedSmemBudget + 1024) != cudaSuccess)
+      st = FP8_ERR_CUDA;
     if (st != FP8_OK) return st;
     d.attrs_set = true;
   }
@@ -202,9 +208,20 @@ fp8_status launch_linear(const DeviceInfo& dev, const uint8_t* x8, const float* 
 }
 
 // ----------------------------------------------------------------- quant plans
-fp8_status launch_quant_act(const uint16_t* x, int64_t M, int64_t K, int64_t ldx, uint8_t* x8,
-                            float* s_tok, cudaStream_t stream) {
+fp8_status launch_quant_act(const DeviceInfo& dev, const uint16_t* x, int64_t M, int64_t K,
+                            int64_t ldx, uint8_t* x8, float* s_tok, cudaStream_t stream) {
   const int64_t nvec = K / 8;
+  const uint32_t row_pad = static_cast<uint32_t>((2 * K + 127) / 128 * 128);
+  const int64_t staged_warps = std::min<int64_t>(8, kStagedSmemBudget / (2 * int64_t(row_pad) + 16));
+  if (M > 1024 && staged_warps >= 2) {
+    // Large M: warp-per-row pipeline through shared memory, one block per SM.
+    const int warps = static_cast<int>(staged_warps);
+    const size_t smem = static_cast<size_t>(warps) * 2 * row_pad + 16 * warps;
+    const int64_t blocks = std::min<int64_t>(dev.sm_count, (M + warps - 1) / warps);
+    quant_act_staged_kernel<<<static_cast<unsigned>(blocks), 32 * warps, smem, stream>>>(
+        x, M, K, ldx, x8, s_tok, row_pad);
+    return last_launch();
+  }
   if (M <= 1024) {
     // Few tokens: a whole 256-thread block per token row.
     const dim3 grid(static_cast<unsigned>(M));
@@ -303,7 +320,7 @@ fp8_status fp8_quant_act(const uint16_t* x, int64_t M, int64_t K, int64_t ldx, u
   if (!aligned16(x) || !aligned16(x8) || !aligned4(s_tok)) return FP8_ERR_ALIGNMENT;
   DeviceInfo* dev;
   if (fp8_status st = device_info(&dev)) return st;
-  return launch_quant_act(x, M, K, ldx, x8, s_tok, as_stream(stream));
+  return launch_quant_act(*dev, x, M, K, ldx, x8, s_tok, as_stream(stream));
 }
 
 static fp8_status check_linear(const void* x, const float* s_tok, const uint8_t* w8,
@@ -349,7 +366,7 @@ fp8_status fp8_linear_bf16(const uint16_t* x, const uint8_t* w8, const float* s_
       return FP8_ERR_CUDA;
     return FP8_OK;
   }
-  if (fp8_status st = launch_quant_act(x, M, K, K, x8, s_tok, as_stream(stream))) return st;
+  if (fp8_status st = launch_quant_act(*dev, x, M, K, K, x8, s_tok, as_stream(stream))) return st;
   return launch_linear(*dev, x8, s_tok, w8, s_ch, static_cast<int>(M), static_cast<int>(N),
                        static_cast<int>(K), y, as_stream(stream), true);
 }
@@ -417,7 +434,7 @@ extern "C" fp8_status fp8_linear_bf16_noalloc(const uint16_t* x, const uint8_t* 
       return FP8_ERR_CUDA;
     return FP8_OK;
   }
-  if (fp8_status st = launch_quant_act(x, M, K, K, x8, s_tok, as_stream(stream))) return st;
+  if (fp8_status st = launch_quant_act(*dev, x, M, K, K, x8, s_tok, as_stream(stream))) return st;
   return launch_linear(*dev, x8, s_tok, w8, s_ch, static_cast<int>(M), static_cast<int>(N),
                        static_cast<int>(K), y, as_stream(stream), true);
 }

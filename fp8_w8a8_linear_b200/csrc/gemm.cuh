@@ -399,8 +399,14 @@ __global__ void __launch_bounds__(192)
         const int n = tile_n * kBM + ch;
         if (tok >= M || n >= N) continue;
         const uint32_t off = red_base + static_cast<uint32_t>((tok * kBM + ch) * 4);
-        float sum = 0.0f;
-        for (int j = 0; j < splits; ++j) sum = __fadd_rn(sum, ld_shared_cluster_f32(mapa_shared(off, j)));
+        // Issue every rank's load before summing (in rank order).
+        float part[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) part[j] = j < splits ? ld_shared_cluster_f32(mapa_shared(off, j)) : 0.0f;
+        float sum = part[0];
+#pragma unroll
+        for (int j = 1; j < 8; ++j)
+          if (j < splits) sum = __fadd_rn(sum, part[j]);
         y[static_cast<int64_t>(tok) * N + n] =
             f32_to_bf16_rn(__fmul_rn(__fmul_rn(sum, __ldg(s_tok + tok)), __ldg(s_ch + n)));
       }

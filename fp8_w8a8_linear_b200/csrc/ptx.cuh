@@ -88,6 +88,23 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map
       : "memory");
 }
 
+// 1-D bulk copy global -> shared (no tensor map): both addresses 16-byte
+// aligned, size a multiple of 16. Completion is signalled on `bar`.
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes,
+                                          uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          dst),
+      "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar)
+      : "memory");
+}
+
+// Orders this thread's earlier generic-proxy shared-memory accesses before
+// later async-proxy (bulk copy / TMA) accesses of the same memory.
+__device__ __forceinline__ void fence_proxy_async_shared() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
 __device__ __forceinline__ uint64_t l2_policy_evict_first() {
   uint64_t p;
   asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
@@ -210,9 +227,12 @@ __device__ __forceinline__ uint32_t mapa_shared(uint32_t addr, uint32_t rank) {
   asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
   return r;
 }
+// Distributed shared-memory load. Not volatile and no memory clobber, so
+// independent loads overlap; ordering against the producers' writes comes
+// from the cluster barrier that precedes every use.
 __device__ __forceinline__ float ld_shared_cluster_f32(uint32_t addr) {
   float v;
-  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
+  asm("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr));
   return v;
 }
 
@@ -231,11 +251,23 @@ __device__ __forceinline__ uint32_t cvt_e4m3x2(float hi, float lo) {
   return r;
 }
 
+// Four E4M3 codes with every zero-magnitude byte forced to +0: a byte keeps
+// its sign bit only if its low 7 bits are nonzero (t + 0x7F sets bit 7 of a
+// byte exactly when t's byte is nonzero; no carries cross bytes).
+__device__ __forceinline__ uint32_t canon_zero4(uint32_t w) {
+  const uint32_t t = w & 0x7F7F7F7Fu;
+  const uint32_t nz = t + 0x7F7F7F7Fu;
+  return w & (nz | 0x7F7F7F7Fu);
+}
+
 // Four codes packed little-endian (value a in byte 0), zeros forced to +0.
 __device__ __forceinline__ uint32_t pack4_e4m3(float a, float b, float c, float d) {
-  uint32_t w = cvt_e4m3x2(b, a) | (cvt_e4m3x2(d, c) << 16);
-  const uint32_t zero = __vcmpeq4(w & 0x7F7F7F7Fu, 0u);  // 0xFF where magnitude is 0
-  return w & ~zero;
+  return canon_zero4(cvt_e4m3x2(b, a) | (cvt_e4m3x2(d, c) << 16));
+}
+
+// True when some byte of v is zero (exact as a yes/no test).
+__device__ __forceinline__ bool has_zero_byte(uint32_t v) {
+  return ((v - 0x01010101u) & ~v & 0x80808080u) != 0u;
 }
 
 }  // namespace fp8k

@@ -29,6 +29,39 @@ namespace fp8k {
 
 constexpr float kE4M3Max = 448.0f;
 
+// Correctly rounded v / s for a fixed divisor s (one row's scale). With
+// r = RN(1/s) computed once (__frcp_rn), q0 = RN(v * r) is within 1.5 ulp of
+// v/s; one correction q1 = RN(q0 + RN(v - q0 s) r) brings it within one ulp,
+// and a second correction then returns RN(v/s) exactly: that is Markstein's
+// theorem for the correction step (P. Markstein, "Computation of elementary
+// functions on the IBM RISC System/6000 processor", IBM J. Res. Dev. 34(1),
+// 1990), whose premises are r within half an ulp of 1/s, q within one ulp of
+// v/s and no underflow in the residual v - q s (which the FMA then computes
+// exactly). The no-underflow premise holds for every quotient that can reach
+// a nonzero E4M3 code when the row's amax >= 2^-80; rows below that use
+// __fdiv_rn. Either way the result equals IEEE division bit for bit.
+struct RowDivisor {
+  float s, r;
+  bool fast;
+};
+
+__device__ __forceinline__ RowDivisor make_divisor(float s, float amax) {
+  RowDivisor d;
+  d.s = s;
+  d.fast = amax >= 0x1p-80f && isfinite(amax);
+  d.r = d.fast ? __frcp_rn(s) : 0.0f;
+  return d;
+}
+
+__device__ __forceinline__ float div_rn(const RowDivisor& d, float v) {
+  if (!d.fast) return __fdiv_rn(v, d.s);
+  float q = __fmul_rn(v, d.r);
+  float e = __fmaf_rn(-q, d.s, v);
+  q = __fmaf_rn(e, d.r, q);
+  e = __fmaf_rn(-q, d.s, v);
+  return __fmaf_rn(e, d.r, q);
+}
+
 // Reduction of a 32-bit unsigned max across the TPR threads of one row.
 // TPR is 32 (one warp per row) or a multiple of 32 up to the block size (a
 // whole block per row); `red` holds one word per warp of the block.
@@ -102,6 +135,7 @@ __global__ void __launch_bounds__(256) quant_act_kernel(const uint16_t* __restri
   const float s = __fdiv_rn(amax, kE4M3Max);
   if (t == 0) s_tok[row] = s;
   uint2* dst = reinterpret_cast<uint2*>(x8 + row * K);
+  const RowDivisor dv = make_divisor(s, amax);
 
   auto quant8 = [&](const uint4& u) -> uint2 {
     if (s == 0.0f) return make_uint2(0, 0);
@@ -109,8 +143,8 @@ __global__ void __launch_bounds__(256) quant_act_kernel(const uint16_t* __restri
     float f[8];
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      f[2 * i] = __fdiv_rn(__uint_as_float(w[i] << 16), s);
-      f[2 * i + 1] = __fdiv_rn(__uint_as_float(w[i] & 0xFFFF0000u), s);
+      f[2 * i] = div_rn(dv, __uint_as_float(w[i] << 16));
+      f[2 * i + 1] = div_rn(dv, __uint_as_float(w[i] & 0xFFFF0000u));
     }
     return make_uint2(pack4_e4m3(f[0], f[1], f[2], f[3]), pack4_e4m3(f[4], f[5], f[6], f[7]));
   };
@@ -126,6 +160,102 @@ __global__ void __launch_bounds__(256) quant_act_kernel(const uint16_t* __restri
   }
 }
 
+// Large-M activation quantization, one warp per token row, rows staged in
+// shared memory by 1-D bulk async copies (cp.async.bulk) with two buffers per
+// warp: while a warp quantizes row i from shared memory, row i+1 is already
+// in flight. Few registers, so many warps per SM; the row is read from HBM
+// exactly once and from shared memory twice (amax pass, quantize pass).
+// Dynamic shared memory: warps * 2 * row_bytes_padded, then 2 barriers per warp.
+__global__ void __launch_bounds__(256) quant_act_staged_kernel(const uint16_t* __restrict__ x,
+                                                                int64_t M, int64_t K, int64_t ldx,
+                                                                uint8_t* __restrict__ x8,
+                                                                float* __restrict__ s_tok,
+                                                                uint32_t row_bytes_padded) {
+  pdl_launch_dependents();
+  extern __shared__ __align__(128) uint8_t qsm[];
+  const int warps = blockDim.x >> 5;
+  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  uint8_t* buf0 = qsm + static_cast<size_t>(w) * 2 * row_bytes_padded;
+  uint64_t* bars =
+      reinterpret_cast<uint64_t*>(qsm + static_cast<size_t>(warps) * 2 * row_bytes_padded);
+  const uint32_t bar0 = smem_u32(bars + 2 * w);
+  const uint32_t row_bytes = static_cast<uint32_t>(K) * 2;
+  const int64_t nvec = K / 8;
+  const int64_t gw = static_cast<int64_t>(blockIdx.x) * warps + w;
+  const int64_t nw = static_cast<int64_t>(gridDim.x) * warps;
+  if (lane == 0) {
+    mbar_init(bar0, 1);
+    mbar_init(bar0 + 8, 1);
+    fence_barrier_init();
+  }
+  __syncwarp();
+  auto issue = [&](int64_t row, int b) {
+    if (lane == 0) {
+      fence_proxy_async_shared();
+      mbar_arrive_expect_tx(bar0 + 8 * b, row_bytes);
+      bulk_load(smem_u32(buf0 + b * row_bytes_padded), x + row * ldx, row_bytes, bar0 + 8 * b);
+    }
+  };
+  if (gw < M) issue(gw, 0);
+  if (gw + nw < M) issue(gw + nw, 1);
+  uint32_t phases = 0u;  // bit b: parity to wait for on buffer b
+  int b = 0;
+  for (int64_t row = gw; row < M; row += nw, b ^= 1) {
+    if (!mbar_wait(bar0 + 8 * b, (phases >> b) & 1u)) return;
+    phases ^= 1u << b;
+    const uint4* src = reinterpret_cast<const uint4*>(buf0 + b * row_bytes_padded);
+    uint32_t mx = 0;
+#pragma unroll 4
+    for (int64_t j = lane; j < nvec; j += 32) {
+      const uint4 u = src[j];
+      mx = __vmaxu2(mx, u.x & 0x7FFF7FFFu);
+      mx = __vmaxu2(mx, u.y & 0x7FFF7FFFu);
+      mx = __vmaxu2(mx, u.z & 0x7FFF7FFFu);
+      mx = __vmaxu2(mx, u.w & 0x7FFF7FFFu);
+    }
+    mx = max(mx & 0xFFFFu, mx >> 16);
+    const uint32_t amax_bits = __reduce_max_sync(0xFFFFFFFFu, mx);
+    if (amax_bits >= 0x7F80u && lane == 0) report(FP8_DEV_NONFINITE);
+    const float amax = __uint_as_float(amax_bits << 16);
+    const float s = __fdiv_rn(amax, kE4M3Max);
+    if (lane == 0) s_tok[row] = s;
+    const RowDivisor dv = make_divisor(s, amax);
+    uint2* dst = reinterpret_cast<uint2*>(x8 + row * K);
+    if (s == 0.0f) {
+      for (int64_t j = lane; j < nvec; j += 32) dst[j] = make_uint2(0, 0);
+    } else if (dv.fast) {
+#pragma unroll 2
+      for (int64_t j = lane; j < nvec; j += 32) {
+        const uint4 u = src[j];
+        const uint32_t wv[4] = {u.x, u.y, u.z, u.w};
+        float f[8];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          f[2 * i] = div_rn(dv, __uint_as_float(wv[i] << 16));
+          f[2 * i + 1] = div_rn(dv, __uint_as_float(wv[i] & 0xFFFF0000u));
+        }
+        dst[j] = make_uint2(canon_zero4(cvt_e4m3x2(f[1], f[0]) | (cvt_e4m3x2(f[3], f[2]) << 16)),
+                            canon_zero4(cvt_e4m3x2(f[5], f[4]) | (cvt_e4m3x2(f[7], f[6]) << 16)));
+      }
+    } else {
+      for (int64_t j = lane; j < nvec; j += 32) {
+        const uint4 u = src[j];
+        const uint32_t wv[4] = {u.x, u.y, u.z, u.w};
+        float f[8];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          f[2 * i] = __fdiv_rn(__uint_as_float(wv[i] << 16), s);
+          f[2 * i + 1] = __fdiv_rn(__uint_as_float(wv[i] & 0xFFFF0000u), s);
+        }
+        dst[j] = make_uint2(canon_zero4(cvt_e4m3x2(f[1], f[0]) | (cvt_e4m3x2(f[3], f[2]) << 16)),
+                            canon_zero4(cvt_e4m3x2(f[5], f[4]) | (cvt_e4m3x2(f[7], f[6]) << 16)));
+      }
+    }
+    __syncwarp();  // every lane is done reading this buffer before it is refilled
+    if (row + 2 * nw < M) issue(row + 2 * nw, b);
+  }
+}
+
 // ----------------------------------------------------------- QAT repack
 // One q4_0 group = 32 values = one 16-byte vector of packed nibbles + one
 // fp32 scale. Because every value in a group is d * q with q in [-8, 7], the
@@ -138,17 +268,20 @@ struct GroupLUT {
   uint32_t t0, t1, t2, t3;  // table bytes for nibbles 0..15
 };
 
-__device__ __forceinline__ GroupLUT group_lut(float d, float s) {
+__device__ __forceinline__ GroupLUT group_lut(float d, const RowDivisor& dv) {
   // c[q] = code(fp32(fp32(d*q) / s)) for q = 1..8; code(0) = 0.
   float f[8];
 #pragma unroll
-  for (int q = 1; q <= 8; ++q) f[q - 1] = __fdiv_rn(__fmul_rn(d, static_cast<float>(q)), s);
-  const uint32_t p0 = pack4_e4m3(f[0], f[1], f[2], f[3]);  // codes of q = 1..4
-  const uint32_t p1 = pack4_e4m3(f[4], f[5], f[6], f[7]);  // codes of q = 5..8
+  for (int q = 1; q <= 8; ++q) f[q - 1] = div_rn(dv, __fmul_rn(d, static_cast<float>(q)));
+  const uint32_t p0 = canon_zero4(cvt_e4m3x2(f[1], f[0]) | (cvt_e4m3x2(f[3], f[2]) << 16));
+  const uint32_t p1 = canon_zero4(cvt_e4m3x2(f[5], f[4]) | (cvt_e4m3x2(f[7], f[6]) << 16));
   // Negation flips bit 7 of every nonzero code (d may be negative, so the
-  // codes of q = 1..8 can carry either sign).
-  const uint32_t n0 = p0 ^ (0x80808080u & ~__vcmpeq4(p0, 0u));
-  const uint32_t n1 = p1 ^ (0x80808080u & ~__vcmpeq4(p1, 0u));
+  // codes of q = 1..8 can carry either sign); a code is zero only as 0x00.
+  auto negate4 = [](uint32_t p) {
+    return p ^ ((((p & 0x7F7F7F7Fu) + 0x7F7F7F7Fu) | p) & 0x80808080u);
+  };
+  const uint32_t n0 = negate4(p0);
+  const uint32_t n1 = negate4(p1);
   GroupLUT L;
   // nibble 0..7 -> q = 0..7: [0, c1, c2, c3 | c4, c5, c6, c7]
   L.t0 = (p0 << 8);
@@ -159,22 +292,36 @@ __device__ __forceinline__ GroupLUT group_lut(float d, float s) {
   return L;
 }
 
-// Four nibbles (the low 16 bits of `chunk`, nibble i -> output byte i).
+// Four nibbles (the low 16 bits of `chunk`, nibble i -> output byte i): look
+// each up in both 8-entry halves of the table, then pick per byte by the
+// nibble's top bit (selector i or i + 4).
 __device__ __forceinline__ uint32_t lut4(const GroupLUT& L, uint32_t chunk) {
   const uint32_t idx = chunk & 0x7777u;
   const uint32_t lo = __byte_perm(L.t0, L.t1, idx);
   const uint32_t hi = __byte_perm(L.t2, L.t3, idx);
-  const uint32_t sel = __byte_perm(0x0000FF00u, 0u, (chunk >> 3) & 0x1111u);  // 0xFF if nibble >= 8
-  return lo ^ ((lo ^ hi) & sel);
+  return __byte_perm(lo, hi, 0x3210u | ((chunk >> 1) & 0x4444u));
 }
 
-// Largest |q| over the 8 nibbles of a word, as a byte-wise running max.
-__device__ __forceinline__ uint32_t nib_absmax(uint32_t w, uint32_t acc) {
-  const uint32_t a = w & 0x0F0F0F0Fu;
-  const uint32_t b = (w >> 4) & 0x0F0F0F0Fu;
-  acc = __vmaxu4(acc, __vminu4(a, __vsub4(0x10101010u, a)));
-  acc = __vmaxu4(acc, __vminu4(b, __vsub4(0x10101010u, b)));
-  return acc;
+// max |q| over the 32 nibbles of one q4_0 group (4-bit two's complement).
+// Per nibble |q| = (n ^ 15s) + s with s the nibble's sign bit, computed for
+// eight nibbles at once without carries (|q| <= 8 fits a nibble). If no
+// |q| is 8, bit 3 of every nibble is free, and adding 8 - t to each nibble
+// sets bit 3 exactly where |q| >= t, so three threshold tests find the max.
+__device__ __forceinline__ uint32_t group_maxabs(const uint4& u) {
+  auto nabs = [](uint32_t w) {
+    const uint32_t s = (w >> 3) & 0x11111111u;
+    return (w ^ (s * 15u)) + s;
+  };
+  const uint32_t a0 = nabs(u.x), a1 = nabs(u.y), a2 = nabs(u.z), a3 = nabs(u.w);
+  if ((a0 | a1 | a2 | a3) & 0x88888888u) return 8u;
+  auto any_ge = [&](uint32_t t) {
+    const uint32_t c = (8u - t) * 0x11111111u;
+    return (((a0 + c) | (a1 + c) | (a2 + c) | (a3 + c)) & 0x88888888u) != 0u;
+  };
+  uint32_t m = any_ge(4) ? 4u : 0u;
+  m += any_ge(m + 2) ? 2u : 0u;
+  m += any_ge(m + 1) ? 1u : 0u;
+  return m;
 }
 
 template <int TPR, int V>
@@ -196,14 +343,7 @@ __global__ void __launch_bounds__(256) repack_qat_kernel(const uint8_t* __restri
   float dc[V > 0 ? V : 1];
   uint32_t mbits = 0;  // max over groups of the bit pattern of fp32(|d| * max|q|)
   auto group_amax = [&](const uint4& u, float dg) {
-    uint32_t acc = 0;
-    acc = nib_absmax(u.x, acc);
-    acc = nib_absmax(u.y, acc);
-    acc = nib_absmax(u.z, acc);
-    acc = nib_absmax(u.w, acc);
-    acc = __vmaxu4(acc, acc >> 16);
-    acc = __vmaxu4(acc, acc >> 8);
-    const float qmax = static_cast<float>(acc & 0xFFu);
+    const float qmax = static_cast<float>(group_maxabs(u));
     // max_k |fp32(d*q_k)| = fp32(|d| * max_k |q_k|): rounding is monotone.
     return __float_as_uint(__fmul_rn(fabsf(dg), qmax));
   };
@@ -233,6 +373,7 @@ __global__ void __launch_bounds__(256) repack_qat_kernel(const uint8_t* __restri
   const float s = __fdiv_rn(amax, kE4M3Max);
   if (t == 0) s_ch[row] = s;
   uint4* dst = reinterpret_cast<uint4*>(w8 + row * K);
+  const RowDivisor dv = make_divisor(s, amax);
 
   auto emit = [&](int64_t g, const uint4& u, float dg) {
     uint4 o0, o1;
@@ -240,7 +381,7 @@ __global__ void __launch_bounds__(256) repack_qat_kernel(const uint8_t* __restri
       o0 = make_uint4(0, 0, 0, 0);
       o1 = o0;
     } else {
-      const GroupLUT L = group_lut(dg, s);
+      const GroupLUT L = group_lut(dg, dv);
       o0.x = lut4(L, u.x);
       o0.y = lut4(L, u.x >> 16);
       o0.z = lut4(L, u.y);
@@ -302,8 +443,8 @@ __global__ void __launch_bounds__(256) convert_fnuz_kernel(const uint8_t* src,
     const uint32_t w[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      if (__vcmpeq4(w[i], 0x80808080u)) flags |= 1u;
-      if (__vcmpeq4(w[i] & 0x7F7F7F7Fu, 0x7F7F7F7Fu)) flags |= 2u;
+      if (has_zero_byte(w[i] ^ 0x80808080u)) flags |= 1u;
+      if (has_zero_byte((w[i] & 0x7F7F7F7Fu) ^ 0x7F7F7F7Fu)) flags |= 2u;
     }
   }
   flags = row_max_u32<TPR>(__reduce_or_sync(0xFFFFFFFFu, flags), red);

@@ -102,6 +102,36 @@ def test_quant_act_special_rows(lib):
     assert lib.device_status() == 0
 
 
+def test_quant_act_quotients_near_e4m3_midpoints(lib):
+    """Rows whose values sit on or next to s * (E4M3 midpoint): the division
+    must round exactly like IEEE fp32 division for the codes to match."""
+    rng = np.random.default_rng(17)
+    mags = F.DEC_E4M3[:0x7F]
+    mids = (mags[:-1] + mags[1:]) / 2
+    M, K = 4096, 512
+    amax = (rng.uniform(0.5, 2.0, M) * 2.0 ** rng.integers(-60, 60, M)).astype(np.float32)
+    amax = f32_to_bf16_bits(amax)
+    amax_f = (amax.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    mu = rng.choice(mids, size=(M, K)) * rng.choice([-1.0, 1.0], size=(M, K))
+    v = (mu * amax_f[:, None] / 448.0).astype(np.float32)
+    xb = f32_to_bf16_bits(v)
+    xb += rng.integers(-1, 2, size=(M, K)).astype(np.uint16)   # +-1 bf16 ulp around it
+    xb[:, 0] = amax                                               # the row maximum
+    ref = oracle.quant_act(xb)
+    x8, s = lib.quant_act(to_dev(xb))
+    assert np.array_equal(u8(x8), ref.codes)
+    assert same_bits_f32(f32(s), ref.scales)
+
+
+def test_quant_act_large_full_compare(lib):
+    M, K = 16384, 5376
+    xb = activations_bf16(M, K, seed=3, outlier_frac=0.01)
+    ref = oracle.quant_act(xb)
+    x8, s = lib.quant_act(to_dev(xb))
+    assert np.array_equal(u8(x8), ref.codes)
+    assert same_bits_f32(f32(s), ref.scales)
+
+
 def test_quant_act_pitched_input(lib):
     M, K, ldx = 37, 1024, 1040
     xb = activations_bf16(M, ldx, seed=12)
