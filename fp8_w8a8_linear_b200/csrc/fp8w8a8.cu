@@ -71,6 +71,23 @@ bool make_tmap_u8(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Row-major bf16 matrix [rows, cols] (pitch = cols elements), boxes of
+// box_cols x box_rows, no swizzle; out-of-range parts of a stored box are
+// not written. Requires cols % 8 == 0 (16-byte pitch).
+bool make_tmap_bf16_store(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols,
+                          uint32_t box_cols, uint32_t box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * 2};
+  cuuint32_t box[2] = {box_cols, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  std::memset(m, 0, sizeof(*m));
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+            CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 fp8_status last_launch() {
   return cudaGetLastError() == cudaSuccess ? FP8_OK : FP8_ERR_CUDA;
 }
@@ -87,11 +104,12 @@ fp8_status set_prefill_attr() {
              : FP8_ERR_CUDA;
 }
 
-template <int BNT, int STAGES>
+template <int BNT, int STAGES, int KBS>
 fp8_status set_decode_attr() {
-  return cudaFuncSetAttribute(gemm_decode_kernel<BNT, STAGES>,
+  return cudaFuncSetAttribute(gemm_decode_kernel<BNT, STAGES, KBS>,
                               cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              static_cast<int>(DecodeCfg<BNT, STAGES>::kSmem)) == cudaSuccess
+                              static_cast<int>(DecodeCfg<BNT, STAGES, KBS>::kSmemSplit)) ==
+                 cudaSuccess
              ? FP8_OK
              : FP8_ERR_CUDA;
 }
@@ -114,13 +132,20 @@ fp8_status device_info(DeviceInfo** out) {
     if (!d.supported) return FP8_ERR_UNSUPPORTED;
     fp8_status st = FP8_OK;
     st = st != FP8_OK ? st : set_prefill_attr<kPrefillBN, kPrefillStages>();
-    st = st != FP8_OK ? st : set_decode_attr<16, 6>();
-    st = st != FP8_OK ? st : set_decode_attr<32, 5>();
-    st = st != FP8_OK ? st : set_decode_attr<64, 4>();
-    st = st != FP8_OK ? st : set_decode_attr<128, 3>();
+    st = st != FP8_OK ? st : set_decode_attr<16, 3, 2>();
+    st = st != FP8_OK ? st : set_decode_attr<32, 4, 1>();
+    st = st != FP8_OK ? st : set_decode_attr<32, 3, 2>();
+    st = st != FP8_OK ? st : set_decode_attr<64, 4, 1>();
+    st = st != FP8_OK ? st : set_decode_attr<64, 4, 2>();
+    st = st != FP8_OK ? st : set_decode_attr<128, 2, 1>();
+    st = st != FP8_OK ? st : set_decode_attr<128, 4, 1>();
     if (st == FP8_OK &&
         cudaFuncSetAttribute(quant_act_staged_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              kStagedSmemBudget + 1024) != cudaSuccess)
+      st = FP8_ERR_CUDA;
+    if (st == FP8_OK &&
+        cudaFuncSetAttribute(repack_qat_staged_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             110 * 1024) != cudaSuccess)
       st = FP8_ERR_CUDA;
     if (st != FP8_OK) return st;
     d.attrs_set = true;
@@ -163,23 +188,33 @@ fp8_status launch_prefill(const DeviceInfo& dev, const uint8_t* x8, const float*
   return FP8_OK;
 }
 
-template <int BNT, int ST>
+template <int BNT, int ST, int KBS>
 fp8_status launch_decode_t(const DeviceInfo& dev, const uint8_t* x8, const float* s_tok,
                            const uint8_t* w8, const float* s_ch, int M, int N, int K, uint16_t* y,
-                           cudaStream_t stream, bool pdl) {
+                           cudaStream_t stream, bool pdl, int force_splits = 0) {
+  using C = DecodeCfg<BNT, ST, KBS>;
   CUtensorMap tmW, tmX;
   if (!make_tmap_u8(&tmW, w8, N, K, kBM) || !make_tmap_u8(&tmX, x8, M, K, BNT))
     return FP8_ERR_CUDA;
   const int tiles = (N + kBM - 1) / kBM;
-  const int num_kb = (K + kBK - 1) / kBK;
-  // Split K so that about two CTAs per SM stream weights; splits divide 128.
+  const int num_steps = (K + kBK * KBS - 1) / (kBK * KBS);
+  // K is split over a cluster only when there are too few 128-channel tiles to
+  // keep the SMs streaming (measured on B200: with >= SMs/4 tiles the cluster
+  // reduction costs more than the extra streams bring). Splits divide 128 and
+  // keep at least two pipeline steps each.
   int splits = 1;
-  while (splits < 8 && tiles * splits * 2 <= 2 * dev.sm_count && splits * 2 <= num_kb) splits *= 2;
-  const int kb_per_split = (num_kb + splits - 1) / splits;
+  if (4 * tiles < dev.sm_count)
+    while (splits < 8 && tiles * splits * 2 <= dev.sm_count && splits * 4 <= num_steps) splits *= 2;
+  if (force_splits > 0) splits = force_splits;
+  const int steps_per_split = (num_steps + splits - 1) / splits;
+  CUtensorMap tmY;
+  std::memset(&tmY, 0, sizeof(tmY));
+  const int use_tma_store =
+      (N % 8 == 0) && make_tmap_bf16_store(&tmY, y, M, N, kBM / splits, BNT) ? 1 : 0;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(tiles * splits);
   cfg.blockDim = dim3(192);
-  cfg.dynamicSmemBytes = DecodeCfg<BNT, ST>::kSmem;
+  cfg.dynamicSmemBytes = splits > 1 ? C::kSmemSplit : C::kSmemSingle;
   cfg.stream = stream;
   cudaLaunchAttribute attrs[2];
   int na = 0;
@@ -191,8 +226,8 @@ fp8_status launch_decode_t(const DeviceInfo& dev, const uint8_t* x8, const float
   set_pdl(attrs, na, pdl);
   cfg.attrs = attrs;
   cfg.numAttrs = na;
-  if (cudaLaunchKernelEx(&cfg, gemm_decode_kernel<BNT, ST>, tmW, tmX, s_tok, s_ch, y, M, N, K,
-                         splits, kb_per_split) != cudaSuccess)
+  if (cudaLaunchKernelEx(&cfg, gemm_decode_kernel<BNT, ST, KBS>, tmW, tmX, tmY, s_tok, s_ch, y, M,
+                         N, K, splits, steps_per_split, use_tma_store) != cudaSuccess)
     return FP8_ERR_CUDA;
   return FP8_OK;
 }
@@ -200,10 +235,20 @@ fp8_status launch_decode_t(const DeviceInfo& dev, const uint8_t* x8, const float
 fp8_status launch_linear(const DeviceInfo& dev, const uint8_t* x8, const float* s_tok,
                          const uint8_t* w8, const float* s_ch, int M, int N, int K, uint16_t* y,
                          cudaStream_t stream, bool pdl) {
-  if (M <= 16) return launch_decode_t<16, 6>(dev, x8, s_tok, w8, s_ch, M, N, K, y, stream, pdl);
-  if (M <= 32) return launch_decode_t<32, 5>(dev, x8, s_tok, w8, s_ch, M, N, K, y, stream, pdl);
-  if (M <= 64) return launch_decode_t<64, 4>(dev, x8, s_tok, w8, s_ch, M, N, K, y, stream, pdl);
-  if (M <= 128) return launch_decode_t<128, 3>(dev, x8, s_tok, w8, s_ch, M, N, K, y, stream, pdl);
+  // Decode-sized M: swap-AB kernel. Pipeline depth is chosen so that every
+  // CTA is resident at once: with more 128-channel tiles than SMs, two CTAs
+  // share an SM (<= ~110 KB of stages each), otherwise one CTA gets ~200 KB.
+  const bool one_per_sm = (N + kBM - 1) / kBM <= dev.sm_count;
+  if (M <= 16) return launch_decode_t<16, 3, 2>(dev, x8, s_tok, w8, s_ch, M, N, K, y, stream, pdl);
+  if (M <= 32)
+    return one_per_sm ? launch_decode_t<32, 3, 2>(dev, x8, s_tok, w8, s_ch, M, N, K, y, stream, pdl)
+                      : launch_decode_t<32, 4, 1>(dev, x8, s_tok, w8, s_ch, M, N, K, y, stream, pdl);
+  if (M <= 64)
+    return one_per_sm ? launch_decode_t<64, 4, 2>(dev, x8, s_tok, w8, s_ch, M, N, K, y, stream, pdl)
+                      : launch_decode_t<64, 4, 1>(dev, x8, s_tok, w8, s_ch, M, N, K, y, stream, pdl);
+  if (M <= 128)
+    return one_per_sm ? launch_decode_t<128, 4, 1>(dev, x8, s_tok, w8, s_ch, M, N, K, y, stream, pdl)
+                      : launch_decode_t<128, 2, 1>(dev, x8, s_tok, w8, s_ch, M, N, K, y, stream, pdl);
   return launch_prefill(dev, x8, s_tok, w8, s_ch, M, N, K, y, stream, pdl);
 }
 
@@ -288,6 +333,17 @@ fp8_status fp8_repack_qat(const uint8_t* q4, const float* d, int64_t N, int64_t 
   if (!aligned16(q4) || !aligned16(w8) || !aligned4(d) || !aligned4(s_ch)) return FP8_ERR_ALIGNMENT;
   DeviceInfo* dev;
   if (fp8_status st = device_info(&dev)) return st;
+  const uint32_t rbuf = static_cast<uint32_t>((K / 2 + K / 8 + 127) / 128 * 128);
+  const size_t rsmem = size_t(8) * kRepackBufs * rbuf + 8 * 8 * kRepackBufs;
+  if (K % 128 == 0 && N >= 4 * dev->sm_count && rsmem <= 110 * 1024) {
+    // Rows staged through shared memory, two blocks of 8 warps per SM.
+    const uint32_t buf = rbuf;
+    const size_t smem = rsmem;
+    const int64_t blocks = std::min<int64_t>(2 * dev->sm_count, (N + 7) / 8);
+    repack_qat_staged_kernel<<<static_cast<unsigned>(blocks), 256, smem, as_stream(stream)>>>(
+        q4, d, N, K, w8, s_ch, buf);
+    return last_launch();
+  }
   const dim3 grid(static_cast<unsigned>((N + 7) / 8));
   if (K / 32 <= 6 * 32)
     repack_qat_kernel<32, 6><<<grid, 256, 0, as_stream(stream)>>>(q4, d, N, K, w8, s_ch);

@@ -23,12 +23,13 @@
 // * gemm_decode_kernel (M <= 128): swap-AB. The weight tile is the MMA's A
 //   operand (128 output channels per CTA) and the tokens are its N (16..128),
 //   so a single token does not waste the 128-row MMA. K is split across the
-//   CTAs of a thread-block cluster (splits = cluster size, 1..8); each CTA
-//   writes its fp32 partial tile to its own shared memory, and after a cluster
-//   barrier each CTA sums one slice of rows over all CTAs' partials through
-//   distributed shared memory, in rank order, so the result is deterministic
-//   and needs no global workspace and no spin-waits. The weight stream uses an
-//   L2 evict-first policy, the (tiny) activation tile evict-last.
+//   CTAs of a thread-block cluster (splits = cluster size, 1..8). Each CTA
+//   owns one slice of the 128 output rows; every CTA stores its fp32 partials
+//   for each slice straight into the owner's shared memory (distributed
+//   shared memory), and after one cluster barrier each owner sums its slice
+//   in rank order - deterministic, no global workspace, no spin-waits. The
+//   weight stream uses an L2 evict-first policy, the activation tile
+//   evict-last.
 //
 // Every mbarrier wait is bounded (ptx.cuh); the only unbounded waits are the
 // hardware cluster barriers, which every thread reaches on every path.
@@ -246,36 +247,47 @@ __global__ void __launch_bounds__(192, 1)
 }
 
 // ============================================================== decode
-template <int BNT, int STAGES>
+// KBS 128-byte k-blocks per pipeline stage (one TMA box each per operand).
+template <int BNT, int STAGES, int KBS>
 struct DecodeCfg {
-  static constexpr int kWBytes = kBM * kBK;   // weight tile: 128 channels x 128 K bytes
-  static constexpr int kXBytes = BNT * kBK;   // token tile
-  static constexpr int kStageBytes = kWBytes + kXBytes;
+  static constexpr int kWBytes = kBM * kBK;   // one weight box: 128 channels x 128 K bytes
+  static constexpr int kXBytes = BNT * kBK;   // one token box
+  static constexpr int kStageBytes = KBS * (kWBytes + kXBytes);
   static constexpr int kTmemCols = tmem_cols_for(BNT);
-  static constexpr int kRedBytes = BNT * kBM * 4;  // fp32 partial tile [token][channel]
-  static constexpr int kBarBytes = 8 * (2 * STAGES + 1) + 16;
   static constexpr int kPipeBytes = STAGES * kStageBytes;
-  static constexpr size_t kSmem =
-      1024 + static_cast<size_t>(kPipeBytes > kRedBytes ? kPipeBytes : kRedBytes) + kBarBytes;
+  static constexpr int kYBytes = BNT * kBM * 2;    // bf16 output tile, reuses the pipeline
+  static constexpr int kBarBytes = 8 * (2 * STAGES + 1) + 16;
+  static constexpr int kScaleBytes = (kBM + BNT) * 4;  // s_ch of the tile, s_tok
+  static constexpr int kRedBytes = BNT * kBM * 4;  // fp32 partials [rank][token][row in slice]
+  static constexpr int kFixed = kPipeBytes + kBarBytes + kScaleBytes;
+  // Shared memory without (single) and with (split) the reduction buffer.
+  static constexpr size_t kSmemSingle = 1024 + static_cast<size_t>(kFixed);
+  static constexpr size_t kSmemSplit = kSmemSingle + kRedBytes;
   static_assert(BNT % 16 == 0 && BNT >= 16 && BNT <= 256, "BNT");
   static_assert(kXBytes % 1024 == 0, "token tile must keep 1024-byte alignment");
+  static_assert(kYBytes <= kPipeBytes, "output tile must fit in the pipeline buffers");
 };
 
-template <int BNT, int STAGES>
+// y is written either by one TMA store per output tile (tmY valid, N % 8 == 0;
+// its box is {rows written per CTA, BNT}) or element by element.
+template <int BNT, int STAGES, int KBS>
 __global__ void __launch_bounds__(192)
     gemm_decode_kernel(const __grid_constant__ CUtensorMap tmW,
-                       const __grid_constant__ CUtensorMap tmX, const float* __restrict__ s_tok,
+                       const __grid_constant__ CUtensorMap tmX,
+                       const __grid_constant__ CUtensorMap tmY, const float* __restrict__ s_tok,
                        const float* __restrict__ s_ch, uint16_t* __restrict__ y, int M, int N,
-                       int K, int splits, int kb_per_split) {
-  using C = DecodeCfg<BNT, STAGES>;
+                       int K, int splits, int kb_per_split, int use_tma_store) {
+  using C = DecodeCfg<BNT, STAGES, KBS>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
-  uint8_t* sW = smem;
-  uint8_t* sX = smem + STAGES * C::kWBytes;
-  constexpr int kRegion = C::kPipeBytes > C::kRedBytes ? C::kPipeBytes : C::kRedBytes;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kRegion);
+  uint8_t* sW = smem;                                   // STAGES x KBS weight boxes
+  uint8_t* sX = smem + STAGES * KBS * C::kWBytes;       // STAGES x KBS token boxes
+  uint16_t* ytile = reinterpret_cast<uint16_t*>(smem);  // after the MMAs: bf16 [token][row]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kPipeBytes);
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 1);
-  float* red = reinterpret_cast<float*>(smem);  // reuses the pipeline buffers after the MMAs
+  float* sch_s = reinterpret_cast<float*>(smem + C::kPipeBytes + C::kBarBytes);
+  float* stok_s = sch_s + kBM;
+  float* red = reinterpret_cast<float*>(smem + C::kFixed);  // split only
   const uint32_t full0 = smem_u32(bars);
   const uint32_t empty0 = smem_u32(bars + STAGES);
   const uint32_t tfull = smem_u32(bars + 2 * STAGES);
@@ -284,9 +296,15 @@ __global__ void __launch_bounds__(192)
   const int tile_n = blockIdx.x / splits;
   const int rank = blockIdx.x % splits;  // == %cluster_ctarank for cluster dims (splits,1,1)
   const int num_kb = (K + kBK - 1) / kBK;
-  const int kb0 = rank * kb_per_split;
-  const int kb1 = min(num_kb, kb0 + kb_per_split);
+  const int num_steps = (num_kb + KBS - 1) / KBS;       // pipeline steps over all of K
+  const int st0 = rank * kb_per_split;                  // kb_per_split counts steps
+  const int st1 = min(num_steps, st0 + kb_per_split);
+  const bool split = splits > 1;
+  const int rows = kBM / splits;                        // output rows each rank writes
+  bool have_acc = st1 > st0;
+  const int pre = have_acc ? min(STAGES, st1 - st0) : 0;
 
+  if (split) cluster_arrive_relaxed();  // this CTA has started (waited on before any DSMEM store)
   if (warp == 0 && lane == 0) {
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(full0 + 8 * s, 1);
@@ -296,6 +314,17 @@ __global__ void __launch_bounds__(192)
     fence_barrier_init();
     tma_prefetch_desc(&tmW);
     tma_prefetch_desc(&tmX);
+    // The weight stream depends neither on the TMEM allocation nor on a
+    // preceding quantizer grid: start the first ring of weight boxes now.
+    const uint64_t pol_w = l2_policy_evict_first();
+    for (int i = 0; i < pre; ++i) {
+      const uint32_t fb = full0 + 8 * i;
+      mbar_arrive_expect_tx(fb, C::kStageBytes);
+#pragma unroll
+      for (int j = 0; j < KBS; ++j)
+        tma_load_2d(smem_u32(sW + (i * KBS + j) * C::kWBytes), &tmW, fb,
+                    ((st0 + i) * KBS + j) * kBK, tile_n * kBM, pol_w);
+    }
   }
   if (warp == 1) {
     tmem_alloc(smem_u32(tmem_holder), C::kTmemCols);
@@ -305,31 +334,30 @@ __global__ void __launch_bounds__(192)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
-  bool have_acc = kb1 > kb0;
 
   if (warp == 0) {
     if (lane == 0 && have_acc) {
       const uint64_t pol_w = l2_policy_evict_first();
       const uint64_t pol_x = l2_policy_evict_last();
-      // The weight stream does not depend on a preceding quantizer grid: issue
-      // the first ring's weight tiles, then wait for the activations.
-      const int pre = min(STAGES, kb1 - kb0);
-      for (int i = 0; i < pre; ++i) {
-        const uint32_t fb = full0 + 8 * i;
-        mbar_arrive_expect_tx(fb, C::kStageBytes);
-        tma_load_2d(smem_u32(sW + i * C::kWBytes), &tmW, fb, (kb0 + i) * kBK, tile_n * kBM, pol_w);
-      }
-      pdl_wait();
+      pdl_wait();  // activations come from a preceding quantizer grid
       for (int i = 0; i < pre; ++i)
-        tma_load_2d(smem_u32(sX + i * C::kXBytes), &tmX, full0 + 8 * i, (kb0 + i) * kBK, 0, pol_x);
+#pragma unroll
+        for (int j = 0; j < KBS; ++j)
+          tma_load_2d(smem_u32(sX + (i * KBS + j) * C::kXBytes), &tmX, full0 + 8 * i,
+                      ((st0 + i) * KBS + j) * kBK, 0, pol_x);
       int stage = pre % STAGES;
       uint32_t phase = pre == STAGES ? 1u : 0u;
-      for (int kb = kb0 + pre; kb < kb1; ++kb) {
+      for (int st = st0 + pre; st < st1; ++st) {
         if (!mbar_wait(empty0 + 8 * stage, phase ^ 1)) break;
         const uint32_t fb = full0 + 8 * stage;
         mbar_arrive_expect_tx(fb, C::kStageBytes);
-        tma_load_2d(smem_u32(sW + stage * C::kWBytes), &tmW, fb, kb * kBK, tile_n * kBM, pol_w);
-        tma_load_2d(smem_u32(sX + stage * C::kXBytes), &tmX, fb, kb * kBK, 0, pol_x);
+#pragma unroll
+        for (int j = 0; j < KBS; ++j) {
+          tma_load_2d(smem_u32(sW + (stage * KBS + j) * C::kWBytes), &tmW, fb, (st * KBS + j) * kBK,
+                      tile_n * kBM, pol_w);
+          tma_load_2d(smem_u32(sX + (stage * KBS + j) * C::kXBytes), &tmX, fb, (st * KBS + j) * kBK,
+                      0, pol_x);
+        }
         if (++stage == STAGES) { stage = 0; phase ^= 1; }
       }
     }
@@ -338,15 +366,18 @@ __global__ void __launch_bounds__(192)
       constexpr uint32_t idesc = idesc_e4m3_f32(kBM, BNT);
       int stage = 0;
       uint32_t phase = 0;
-      for (int kb = kb0; kb < kb1; ++kb) {
+      for (int st = st0; st < st1; ++st) {
         if (!mbar_wait(full0 + 8 * stage, phase)) break;
         tc_fence_after();
-        const uint32_t a0 = smem_u32(sW + stage * C::kWBytes);
-        const uint32_t b0 = smem_u32(sX + stage * C::kXBytes);
 #pragma unroll
-        for (int k = 0; k < kBK / 32; ++k) {
-          umma_f8(tmem_base, sw128_kmajor_desc(a0 + 32 * k), sw128_kmajor_desc(b0 + 32 * k), idesc,
-                  (kb != kb0) || (k != 0));
+        for (int j = 0; j < KBS; ++j) {
+          const uint32_t a0 = smem_u32(sW + (stage * KBS + j) * C::kWBytes);
+          const uint32_t b0 = smem_u32(sX + (stage * KBS + j) * C::kXBytes);
+#pragma unroll
+          for (int k = 0; k < kBK / 32; ++k) {
+            umma_f8(tmem_base, sw128_kmajor_desc(a0 + 32 * k), sw128_kmajor_desc(b0 + 32 * k),
+                    idesc, (st != st0) || (j != 0) || (k != 0));
+          }
         }
         umma_commit(empty0 + 8 * stage);
         if (++stage == STAGES) { stage = 0; phase ^= 1; }
@@ -354,14 +385,28 @@ __global__ void __launch_bounds__(192)
       umma_commit(tfull);
     }
   } else {
+    const int et = threadIdx.x - 64;                 // 0..127
     const int quad = warp & 3;
     const int ch = quad * 32 + lane;                 // channel within the tile (TMEM lane)
-    const int n = tile_n * kBM + ch;
+    // Stage both scale vectors while the main loop runs.
+    {
+      const int n = tile_n * kBM + et;
+      sch_s[et] = n < N ? __ldg(s_ch + n) : 0.0f;
+      pdl_wait();  // per-token scales come from a preceding quantizer grid
+      if (et < BNT) stok_s[et] = et < M ? s_tok[et] : 0.0f;
+      named_bar_sync(1, 128);
+    }
     if (have_acc && !mbar_wait(tfull, 0)) have_acc = false;
+    __syncwarp();
     tc_fence_after();
-    pdl_wait();
     const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quad * 32) << 16);
-    const float sc = n < N ? __ldg(s_ch + n) : 0.0f;
+    uint32_t dst = 0;
+    if (split) {
+      cluster_wait_acquire();  // every CTA of the cluster has started
+      dst = mapa_shared(smem_u32(red) + static_cast<uint32_t>((rank * BNT * rows + ch % rows) * 4),
+                        ch / rows);
+    }
+    const float sc = sch_s[ch];
 #pragma unroll 1
     for (int c = 0; c < BNT / 16; ++c) {
       uint32_t r[16];
@@ -371,11 +416,11 @@ __global__ void __launch_bounds__(192)
       for (int j = 0; j < 16; ++j) {
         const int tok = c * 16 + j;
         const float acc = have_acc ? __uint_as_float(r[j]) : 0.0f;
-        if (splits == 1) {
-          if (tok < M && n < N)
-            y[static_cast<int64_t>(tok) * N + n] = f32_to_bf16_rn(__fmul_rn(__fmul_rn(acc, __ldg(s_tok + tok)), sc));
-        } else {
-          red[tok * kBM + ch] = acc;
+        if (!split) {
+          ytile[tok * kBM + ch] = f32_to_bf16_rn(__fmul_rn(__fmul_rn(acc, stok_s[tok]), sc));
+        } else if (tok < M) {
+          // owner's buffer [rank][token][row in slice]: lanes write consecutive words
+          st_shared_cluster_f32(dst + static_cast<uint32_t>(tok * rows * 4), acc);
         }
       }
     }
@@ -387,31 +432,42 @@ __global__ void __launch_bounds__(192)
     tc_fence_after();
     tmem_dealloc(tmem_base, C::kTmemCols);
   }
-  if (splits > 1) {
-    cluster_sync();  // every CTA's partial tile is in its shared memory
+  if (split) {
+    if (warp < 2) cluster_wait_acquire();  // the first barrier phase, for the non-epilogue warps
+    cluster_arrive_release();              // this CTA's partials are in their owners' buffers
+    cluster_wait_acquire();
     if (warp >= 2) {
       const int et = threadIdx.x - 64;
-      const int rows = kBM / splits;
-      const uint32_t red_base = smem_u32(red);
       for (int e = et; e < rows * BNT; e += 128) {
         const int tok = e / rows;
-        const int ch = rank * rows + e % rows;
-        const int n = tile_n * kBM + ch;
-        if (tok >= M || n >= N) continue;
-        const uint32_t off = red_base + static_cast<uint32_t>((tok * kBM + ch) * 4);
-        // Issue every rank's load before summing (in rank order).
-        float part[8];
-#pragma unroll
-        for (int j = 0; j < 8; ++j) part[j] = j < splits ? ld_shared_cluster_f32(mapa_shared(off, j)) : 0.0f;
-        float sum = part[0];
-#pragma unroll
-        for (int j = 1; j < 8; ++j)
-          if (j < splits) sum = __fadd_rn(sum, part[j]);
-        y[static_cast<int64_t>(tok) * N + n] =
-            f32_to_bf16_rn(__fmul_rn(__fmul_rn(sum, __ldg(s_tok + tok)), __ldg(s_ch + n)));
+        const int rl = e % rows;
+        float sum = red[tok * rows + rl];
+        for (int j = 1; j < splits; ++j) sum = __fadd_rn(sum, red[(j * BNT + tok) * rows + rl]);
+        ytile[tok * rows + rl] =
+            f32_to_bf16_rn(__fmul_rn(__fmul_rn(sum, stok_s[tok]), sch_s[rank * rows + rl]));
       }
     }
-    cluster_sync();  // keep every CTA's shared memory alive until all reads are done
+  }
+  // Write the tile (or this rank's slice of it): [BNT tokens][rows_out channels].
+  const int rows_out = split ? rows : kBM;
+  const int n0 = tile_n * kBM + (split ? rank * rows : 0);
+  if (use_tma_store) {
+    if (warp >= 2) {
+      fence_proxy_async_shared();  // generic writes of the tile -> visible to the TMA store
+      named_bar_sync(1, 128);
+      if (threadIdx.x == 64) {
+        tma_store_2d(&tmY, smem_u32(ytile), n0, 0);
+        bulk_commit_group();
+        bulk_wait_group_all();
+      }
+    }
+  } else if (warp >= 2) {
+    named_bar_sync(1, 128);
+    const int et = threadIdx.x - 64;
+    for (int e = et; e < rows_out * BNT; e += 128) {
+      const int tok = e / rows_out, rl = e % rows_out;
+      if (tok < M && n0 + rl < N) y[static_cast<int64_t>(tok) * N + n0 + rl] = ytile[tok * rows_out + rl];
+    }
   }
 }
 

@@ -268,11 +268,9 @@ struct GroupLUT {
   uint32_t t0, t1, t2, t3;  // table bytes for nibbles 0..15
 };
 
-__device__ __forceinline__ GroupLUT group_lut(float d, const RowDivisor& dv) {
-  // c[q] = code(fp32(fp32(d*q) / s)) for q = 1..8; code(0) = 0.
-  float f[8];
-#pragma unroll
-  for (int q = 1; q <= 8; ++q) f[q - 1] = div_rn(dv, __fmul_rn(d, static_cast<float>(q)));
+// Codes of q = 1..8 from their fp32 quotients f[q-1] (canonical zeros), and
+// the table built from them.
+__device__ __forceinline__ GroupLUT group_lut_from(const float (&f)[8]) {
   const uint32_t p0 = canon_zero4(cvt_e4m3x2(f[1], f[0]) | (cvt_e4m3x2(f[3], f[2]) << 16));
   const uint32_t p1 = canon_zero4(cvt_e4m3x2(f[5], f[4]) | (cvt_e4m3x2(f[7], f[6]) << 16));
   // Negation flips bit 7 of every nonzero code (d may be negative, so the
@@ -290,6 +288,33 @@ __device__ __forceinline__ GroupLUT group_lut(float d, const RowDivisor& dv) {
   L.t2 = __byte_perm(n1, 0, 0x0123);
   L.t3 = __byte_perm(n0, 0, 0x0123);
   return L;
+}
+
+// Table of one group from its scale d, for rows on the fast division path:
+// only q = 1, 3, 5, 7 need a division. In this path every quotient that can
+// reach a nonzero code is a normal fp32 number, and scaling a normal number
+// by 2 is exact, so fp32(d*2q) = 2 fp32(d*q) and fp32(2w/s) = 2 fp32(w/s);
+// the even q's quotients are therefore doublings, bit for bit. (Quotients
+// too small to be normal encode to 0 either way.)
+__device__ __forceinline__ GroupLUT group_lut_fast(float d, const RowDivisor& dv) {
+  float f[8];
+  f[0] = div_rn(dv, d);
+  f[2] = div_rn(dv, __fmul_rn(d, 3.0f));
+  f[4] = div_rn(dv, __fmul_rn(d, 5.0f));
+  f[6] = div_rn(dv, __fmul_rn(d, 7.0f));
+  f[1] = __fmul_rn(f[0], 2.0f);
+  f[3] = __fmul_rn(f[1], 2.0f);
+  f[5] = __fmul_rn(f[2], 2.0f);
+  f[7] = __fmul_rn(f[3], 2.0f);
+  return group_lut_from(f);
+}
+
+// Same table with IEEE division for each q (rows with tiny amax).
+__device__ __forceinline__ GroupLUT group_lut_slow(float d, float s) {
+  float f[8];
+#pragma unroll
+  for (int q = 1; q <= 8; ++q) f[q - 1] = __fdiv_rn(__fmul_rn(d, static_cast<float>(q)), s);
+  return group_lut_from(f);
 }
 
 // Four nibbles (the low 16 bits of `chunk`, nibble i -> output byte i): look
@@ -381,7 +406,7 @@ __global__ void __launch_bounds__(256) repack_qat_kernel(const uint8_t* __restri
       o0 = make_uint4(0, 0, 0, 0);
       o1 = o0;
     } else {
-      const GroupLUT L = group_lut(dg, dv);
+      const GroupLUT L = dv.fast ? group_lut_fast(dg, dv) : group_lut_slow(dg, s);
       o0.x = lut4(L, u.x);
       o0.y = lut4(L, u.x >> 16);
       o0.z = lut4(L, u.y);
@@ -402,6 +427,95 @@ __global__ void __launch_bounds__(256) repack_qat_kernel(const uint8_t* __restri
     }
   } else {
     for (int64_t g = t; g < ng; g += TPR) emit(g, __ldg(qsrc + g), __ldg(dsrc + g));
+  }
+}
+
+// Emits the 32 codes of one group (two 16-byte stores).
+__device__ __forceinline__ void emit_group(uint4* dst, const uint4& u, const GroupLUT& L) {
+  uint4 o0, o1;
+  o0.x = lut4(L, u.x);
+  o0.y = lut4(L, u.x >> 16);
+  o0.z = lut4(L, u.y);
+  o0.w = lut4(L, u.y >> 16);
+  o1.x = lut4(L, u.z);
+  o1.y = lut4(L, u.z >> 16);
+  o1.z = lut4(L, u.w);
+  o1.w = lut4(L, u.w >> 16);
+  dst[0] = o0;
+  dst[1] = o1;
+}
+
+// Repack with rows staged in shared memory (K % 128 == 0, so both the q4 row,
+// K/2 bytes, and the scale row, K/8 bytes, are 16-byte multiples): one warp
+// per output row, NBUF row buffers per warp filled by 1-D bulk async copies,
+// so several rows per warp are in flight while one is encoded.
+constexpr int kRepackBufs = 3;
+
+__global__ void __launch_bounds__(256) repack_qat_staged_kernel(const uint8_t* __restrict__ q4,
+                                                                 const float* __restrict__ d,
+                                                                 int64_t N, int64_t K,
+                                                                 uint8_t* __restrict__ w8,
+                                                                 float* __restrict__ s_ch,
+                                                                 uint32_t buf_bytes) {
+  extern __shared__ __align__(128) uint8_t rsm[];
+  const int warps = blockDim.x >> 5;
+  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  uint8_t* bufs = rsm + static_cast<size_t>(w) * kRepackBufs * buf_bytes;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(rsm + static_cast<size_t>(warps) * kRepackBufs * buf_bytes);
+  const uint32_t bar0 = smem_u32(bars + kRepackBufs * w);
+  const uint32_t qbytes = static_cast<uint32_t>(K / 2), dbytes = static_cast<uint32_t>(K / 8);
+  const int64_t ng = K / 32;
+  const int64_t gw = static_cast<int64_t>(blockIdx.x) * warps + w;
+  const int64_t nw = static_cast<int64_t>(gridDim.x) * warps;
+  if (lane == 0) {
+    for (int b = 0; b < kRepackBufs; ++b) mbar_init(bar0 + 8 * b, 1);
+    fence_barrier_init();
+  }
+  __syncwarp();
+  auto issue = [&](int64_t row, int b) {
+    if (lane == 0) {
+      fence_proxy_async_shared();
+      const uint32_t dst = smem_u32(bufs + b * buf_bytes);
+      mbar_arrive_expect_tx(bar0 + 8 * b, qbytes + dbytes);
+      bulk_load(dst, q4 + row * qbytes, qbytes, bar0 + 8 * b);
+      bulk_load(dst + qbytes, d + row * ng, dbytes, bar0 + 8 * b);
+    }
+  };
+  for (int b = 0; b < kRepackBufs; ++b)
+    if (gw + b * nw < N) issue(gw + b * nw, b);
+  uint32_t phases = 0u;
+  int b = 0;
+  for (int64_t row = gw; row < N; row += nw) {
+    if (!mbar_wait(bar0 + 8 * b, (phases >> b) & 1u)) return;
+    phases ^= 1u << b;
+    const uint4* qs = reinterpret_cast<const uint4*>(bufs + b * buf_bytes);
+    const float* ds = reinterpret_cast<const float*>(bufs + b * buf_bytes + qbytes);
+    uint32_t mbits = 0;
+    for (int64_t g = lane; g < ng; g += 32) {
+      const float qmax = static_cast<float>(group_maxabs(qs[g]));
+      mbits = max(mbits, __float_as_uint(__fmul_rn(fabsf(ds[g]), qmax)));
+    }
+    const uint32_t amax_bits = __reduce_max_sync(0xFFFFFFFFu, mbits);
+    if (amax_bits >= 0x7F800000u && lane == 0) report(FP8_DEV_NONFINITE);
+    const float amax = __uint_as_float(amax_bits);
+    const float s = __fdiv_rn(amax, kE4M3Max);
+    if (lane == 0) s_ch[row] = s;
+    const RowDivisor dv = make_divisor(s, amax);
+    uint4* dst = reinterpret_cast<uint4*>(w8 + row * K);
+    if (s == 0.0f) {
+      for (int64_t g = lane; g < ng; g += 32) {
+        dst[2 * g] = make_uint4(0, 0, 0, 0);
+        dst[2 * g + 1] = make_uint4(0, 0, 0, 0);
+      }
+    } else if (dv.fast) {
+#pragma unroll 2
+      for (int64_t g = lane; g < ng; g += 32) emit_group(dst + 2 * g, qs[g], group_lut_fast(ds[g], dv));
+    } else {
+      for (int64_t g = lane; g < ng; g += 32) emit_group(dst + 2 * g, qs[g], group_lut_slow(ds[g], s));
+    }
+    __syncwarp();
+    if (row + kRepackBufs * nw < N) issue(row + kRepackBufs * nw, b);
+    if (++b == kRepackBufs) b = 0;
   }
 }
 
