@@ -46,10 +46,11 @@ from .quantize import (
     qat_values,
 )
 from .gemm import rowwise_linear_ref, rowwise_linear_tolerance, check_linear, bf16_ulp
+from . import moe
 
 __all__ = [
     "E4M3_MAX", "E4M3FNUZ_MAX", "dec_e4m3", "dec_e4m3fnuz", "enc_e4m3", "enc_e4m3fnuz",
     "QuantResult", "convert_fnuz_to_e4m3", "fnuz_copy_of_e4m3", "quant_act",
     "quantize_rows", "quantize_rows_fnuz", "repack_qat", "unpack_q4", "qat_values",
-    "rowwise_linear_ref", "rowwise_linear_tolerance", "check_linear", "bf16_ulp",
+    "rowwise_linear_ref", "rowwise_linear_tolerance", "check_linear", "bf16_ulp", "moe",
 ]
