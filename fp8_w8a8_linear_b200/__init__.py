@@ -13,6 +13,8 @@ Functions mirror the C entry points:
 * :func:`rowwise_linear` - ``y = (x8 . w8^T) * s_tok * s_ch`` in bf16.
 * :func:`linear` - bf16 activations in, bf16 out (quantizer + GEMM).
 * :func:`cast_e4m3` - the element-wise encoder.
+* :func:`moe_route`, :func:`moe_gather`, :func:`grouped_linear`,
+  :func:`moe_geglu_quant`, :func:`moe_combine` - the mixture-of-experts layer.
 * :func:`device_status` - read and clear the device status word.
 """
 
@@ -47,6 +49,12 @@ _SIGS = {
     "fp8_linear_bf16": ([_P, _P, _P, _I64, _I64, _I64, _P, _P, _P, _P], ctypes.c_int),
     "fp8_cast_e4m3": ([_P, _I64, _P, _P], ctypes.c_int),
     "fp8_linear_bf16_noalloc": ([_P, _P, _P, _I64, _I64, _I64, _P, _P], ctypes.c_int),
+    "fp8_moe_route": ([_P, _I64, ctypes.c_int32, ctypes.c_int32, _P, _P, _P, _P], ctypes.c_int),
+    "fp8_moe_gather": ([_P, _P, _P, _I64, _I64, ctypes.c_int32, _P, _P, _P], ctypes.c_int),
+    "fp8_grouped_linear": ([_P, _P, _P, ctypes.c_int32, _I64, _P, _P, _I64, _I64, _P, _P],
+                           ctypes.c_int),
+    "fp8_moe_geglu_quant": ([_P, _I64, _I64, _P, _P, _P, _P], ctypes.c_int),
+    "fp8_moe_combine": ([_P, _P, _I64, ctypes.c_int32, _I64, _P, _P, _P], ctypes.c_int),
 }
 for _name, (_args, _ret) in _SIGS.items():
     _f = getattr(_lib, _name)
@@ -60,6 +68,7 @@ DEV_NONFINITE = 0x1
 DEV_NAN_CODE = 0x2
 DEV_INEXACT = 0x4
 DEV_TIMEOUT = 0x8
+DEV_BAD_INDEX = 0x10
 
 
 class Fp8Error(RuntimeError):
@@ -176,6 +185,73 @@ def linear(x: torch.Tensor, w8: torch.Tensor, s_ch: torch.Tensor, y: torch.Tenso
     return y
 
 
+# ------------------------------------------------------------------ MoE
+def moe_route(topk_ids: torch.Tensor, num_experts: int):
+    """topk_ids int32 [T, k] -> (perm [T*k], inv [T*k], offsets [E+1]) int32."""
+    T, k = topk_ids.shape
+    dev = topk_ids.device
+    perm = torch.empty(T * k, dtype=torch.int32, device=dev)
+    inv = torch.empty(T * k, dtype=torch.int32, device=dev)
+    offsets = torch.empty(num_experts + 1, dtype=torch.int32, device=dev)
+    _check(_lib.fp8_moe_route(_dev(topk_ids, torch.int32, "topk_ids"), T, k, num_experts,
+                              perm.data_ptr(), inv.data_ptr(), offsets.data_ptr(), _stream()),
+           "fp8_moe_route")
+    return perm, inv, offsets
+
+
+def moe_gather(x8: torch.Tensor, s_tok: torch.Tensor, perm: torch.Tensor, top_k: int,
+               x8_rows: torch.Tensor | None = None, s_rows: torch.Tensor | None = None):
+    rows = perm.numel()
+    K = x8.shape[1]
+    x8_rows = torch.empty((rows, K), dtype=torch.uint8, device=x8.device) if x8_rows is None else x8_rows
+    s_rows = torch.empty((rows,), dtype=torch.float32, device=x8.device) if s_rows is None else s_rows
+    _check(_lib.fp8_moe_gather(_dev(x8, torch.uint8, "x8"), _dev(s_tok, torch.float32, "s_tok"),
+                               _dev(perm, torch.int32, "perm"), rows, K, top_k,
+                               _dev(x8_rows, torch.uint8, "x8_rows", (rows, K)),
+                               _dev(s_rows, torch.float32, "s_rows", (rows,)), _stream()),
+           "fp8_moe_gather")
+    return x8_rows, s_rows
+
+
+def grouped_linear(x8_rows: torch.Tensor, s_rows: torch.Tensor, offsets: torch.Tensor,
+                   w8: torch.Tensor, s_ch: torch.Tensor, y: torch.Tensor | None = None):
+    """Per-expert GEMM: w8 [E, N, K] (or stacked [E*N, K]), s_ch [E, N] or [E*N]."""
+    M, K = x8_rows.shape
+    E = offsets.numel() - 1
+    N = w8.numel() // (E * K)
+    y = torch.empty((M, N), dtype=torch.bfloat16, device=x8_rows.device) if y is None else y
+    _check(_lib.fp8_grouped_linear(_dev(x8_rows, torch.uint8, "x8_rows"),
+                                   _dev(s_rows, torch.float32, "s_rows", (M,)),
+                                   _dev(offsets, torch.int32, "offsets"), E, M,
+                                   _dev(w8, torch.uint8, "w8"), _dev(s_ch, torch.float32, "s_ch"),
+                                   N, K, _dev(y, torch.bfloat16, "y", (M, N)), _stream()),
+           "fp8_grouped_linear")
+    return y
+
+
+def moe_geglu_quant(gate_up: torch.Tensor, inter: int, h8=None, s_h=None, h_out=None):
+    M = gate_up.shape[0]
+    dev = gate_up.device
+    h8 = torch.empty((M, inter), dtype=torch.uint8, device=dev) if h8 is None else h8
+    s_h = torch.empty((M,), dtype=torch.float32, device=dev) if s_h is None else s_h
+    _check(_lib.fp8_moe_geglu_quant(_dev(gate_up, torch.bfloat16, "gate_up", (M, 2 * inter)), M, inter,
+                                    _dev(h8, torch.uint8, "h8", (M, inter)),
+                                    _dev(s_h, torch.float32, "s_h", (M,)),
+                                    None if h_out is None else _dev(h_out, torch.bfloat16, "h_out", (M, inter)),
+                                    _stream()), "fp8_moe_geglu_quant")
+    return h8, s_h
+
+
+def moe_combine(rows: torch.Tensor, inv: torch.Tensor, tokens: int, top_k: int,
+                weights: torch.Tensor | None = None, out: torch.Tensor | None = None):
+    H = rows.shape[1]
+    out = torch.empty((tokens, H), dtype=torch.bfloat16, device=rows.device) if out is None else out
+    _check(_lib.fp8_moe_combine(_dev(rows, torch.bfloat16, "rows"), _dev(inv, torch.int32, "inv"), tokens,
+                                top_k, H, None if weights is None else _dev(weights, torch.float32, "weights"),
+                                _dev(out, torch.bfloat16, "out", (tokens, H)), _stream()), "fp8_moe_combine")
+    return out
+
+
 NOALLOC_SCRATCH_BYTES = 4 << 20
 
 
@@ -209,5 +285,6 @@ def cast_e4m3(x: torch.Tensor, out: torch.Tensor | None = None):
 __all__ = [
     "Fp8Error", "raw", "version", "device_supported", "device_status", "repack_qat",
     "convert_fnuz", "quant_act", "rowwise_linear", "linear", "linear_noalloc", "cast_e4m3",
+    "moe_route", "moe_gather", "grouped_linear", "moe_geglu_quant", "moe_combine",
     "DEV_NONFINITE", "DEV_NAN_CODE", "DEV_INEXACT", "DEV_TIMEOUT", "LIB_PATH",
 ]

@@ -12,6 +12,7 @@
 
 #include "../../include/fp8w8a8.h"
 #include "gemm.cuh"
+#include "moe.cuh"
 #include "ptx.cuh"
 #include "quant.cuh"
 
@@ -95,11 +96,12 @@ fp8_status last_launch() {
 // ----------------------------------------------------------------- GEMM plans
 using namespace fp8k;
 
-template <int BN, int STAGES>
+template <int BN, int STAGES, bool GROUPED>
 fp8_status set_prefill_attr() {
-  return cudaFuncSetAttribute(gemm_prefill_kernel<BN, STAGES>,
+  const size_t smem = PrefillCfg<BN, STAGES>::kSmem + (GROUPED ? 4 * (kMaxExperts + 1) : 0);
+  return cudaFuncSetAttribute(gemm_prefill_kernel<BN, STAGES, GROUPED>,
                               cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              static_cast<int>(PrefillCfg<BN, STAGES>::kSmem)) == cudaSuccess
+                              static_cast<int>(smem)) == cudaSuccess
              ? FP8_OK
              : FP8_ERR_CUDA;
 }
@@ -131,7 +133,9 @@ fp8_status device_info(DeviceInfo** out) {
     d.supported = prop.major == 10 && prop.minor == 0;
     if (!d.supported) return FP8_ERR_UNSUPPORTED;
     fp8_status st = FP8_OK;
-    st = st != FP8_OK ? st : set_prefill_attr<kPrefillBN, kPrefillStages>();
+    st = st != FP8_OK ? st : set_prefill_attr<kPrefillBN, kPrefillStages, false>();
+    st = st != FP8_OK ? st : set_prefill_attr<256, kPrefillStages, true>();
+    st = st != FP8_OK ? st : set_prefill_attr<128, 6, true>();
     st = st != FP8_OK ? st : set_decode_attr<16, 3, 2>();
     st = st != FP8_OK ? st : set_decode_attr<32, 4, 1>();
     st = st != FP8_OK ? st : set_decode_attr<32, 3, 2>();
@@ -182,10 +186,71 @@ fp8_status launch_prefill(const DeviceInfo& dev, const uint8_t* x8, const float*
   set_pdl(attrs, na, pdl);
   cfg.attrs = attrs;
   cfg.numAttrs = na;
-  if (cudaLaunchKernelEx(&cfg, gemm_prefill_kernel<BN, ST>, tmA, tmB, s_tok, s_ch, y, M, N, K,
-                         tiles_m, tiles_n, group_m) != cudaSuccess)
+  GemmArgs g = {};
+  g.s_a = s_tok;
+  g.s_b = s_ch;
+  g.y = y;
+  g.M = M;
+  g.N = N;
+  g.K = K;
+  g.tiles_m = tiles_m;
+  g.tiles_n = tiles_n;
+  g.group_m = group_m;
+  if (cudaLaunchKernelEx(&cfg, gemm_prefill_kernel<BN, ST, false>, tmA, tmB, g) != cudaSuccess)
     return FP8_ERR_CUDA;
   return FP8_OK;
+}
+
+// Per-expert GEMM: persistent grid, tiles decoded on the GPU from offsets.
+template <int BN, int ST>
+fp8_status launch_grouped(const DeviceInfo& dev, const uint8_t* x8, const float* s_rows,
+                          const int32_t* offsets, int E, int M_total, const uint8_t* w8,
+                          const float* s_ch, int N, int K, uint16_t* y, cudaStream_t stream) {
+  CUtensorMap tmA, tmB;
+  if (!make_tmap_u8(&tmA, x8, M_total, K, kBM) ||
+      !make_tmap_u8(&tmB, w8, static_cast<uint64_t>(E) * N, K, BN))
+    return FP8_ERR_CUDA;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(dev.sm_count);
+  cfg.blockDim = dim3(192);
+  cfg.dynamicSmemBytes = PrefillCfg<BN, ST>::kSmem + 4 * (E + 1);
+  cfg.stream = stream;
+  cudaLaunchAttribute attrs[1];
+  int na = 0;
+  set_pdl(attrs, na, true);
+  cfg.attrs = attrs;
+  cfg.numAttrs = na;
+  GemmArgs g = {};
+  g.s_a = s_rows;
+  g.s_b = s_ch;
+  g.y = y;
+  g.M = M_total;
+  g.N = N;
+  g.K = K;
+  g.tiles_n = (N + BN - 1) / BN;
+  g.offsets = offsets;
+  g.num_experts = E;
+  if (cudaLaunchKernelEx(&cfg, gemm_prefill_kernel<BN, ST, true>, tmA, tmB, g) != cudaSuccess)
+    return FP8_ERR_CUDA;
+  return FP8_OK;
+}
+
+// Launch of a plain kernel as a programmatic dependent of the previous work
+// in the stream (its prologue may overlap that work; the kernel itself calls
+// griddepcontrol.wait before reading what the previous grid wrote).
+template <typename... KArgs, typename... Args>
+fp8_status launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, cudaStream_t stream,
+                      Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.stream = stream;
+  cudaLaunchAttribute attrs[1];
+  int na = 0;
+  set_pdl(attrs, na, true);
+  cfg.attrs = attrs;
+  cfg.numAttrs = na;
+  return cudaLaunchKernelEx(&cfg, kernel, args...) == cudaSuccess ? FP8_OK : FP8_ERR_CUDA;
 }
 
 template <int BNT, int ST, int KBS>
@@ -438,6 +503,101 @@ fp8_status fp8_cast_e4m3(const float* x, int64_t n, uint8_t* out, void* stream) 
   const dim3 grid(static_cast<unsigned>((threads + 255) / 256));
   cast_e4m3_kernel<<<grid, 256, 0, as_stream(stream)>>>(x, n, out);
   return last_launch();
+}
+
+fp8_status fp8_moe_route(const int32_t* topk_ids, int64_t tokens, int32_t top_k,
+                         int32_t num_experts, int32_t* perm, int32_t* inv, int32_t* offsets,
+                         void* stream) {
+  if (tokens < 0 || top_k < 1 || num_experts < 1 || num_experts > kMaxExperts)
+    return FP8_ERR_INVALID_ARG;
+  const int64_t n = tokens * top_k;
+  if (n >= (int64_t(1) << 31)) return FP8_ERR_SHAPE;
+  if (!offsets || (n > 0 && (!topk_ids || !perm || !inv))) return FP8_ERR_INVALID_ARG;
+  if (!aligned4(topk_ids) || !aligned4(perm) || !aligned4(inv) || !aligned4(offsets))
+    return FP8_ERR_ALIGNMENT;
+  DeviceInfo* dev;
+  if (fp8_status st = device_info(&dev)) return st;
+  cudaStream_t s = as_stream(stream);
+  moe_count_kernel<<<num_experts, 256, 0, s>>>(topk_ids, n, offsets);
+  if (fp8_status st = last_launch()) return st;
+  if (fp8_status st = launch_pdl(moe_scatter_kernel, dim3(num_experts), dim3(256), s, topk_ids, n,
+                                 static_cast<const int32_t*>(offsets + 1), perm, inv))
+    return st;
+  return launch_pdl(moe_offsets_kernel, dim3(1), dim3(32), s, offsets, static_cast<int>(num_experts));
+}
+
+fp8_status fp8_moe_gather(const uint8_t* x8, const float* s_tok, const int32_t* perm,
+                          int64_t rows, int64_t K, int32_t top_k, uint8_t* x8_rows,
+                          float* s_rows, void* stream) {
+  if (rows < 0 || K < 0 || top_k < 1) return FP8_ERR_INVALID_ARG;
+  if (K % 16 != 0) return FP8_ERR_SHAPE;
+  if (rows == 0 || K == 0) return FP8_OK;
+  if (!x8 || !s_tok || !perm || !x8_rows || !s_rows) return FP8_ERR_INVALID_ARG;
+  if (!aligned16(x8) || !aligned16(x8_rows) || !aligned4(s_tok) || !aligned4(perm) ||
+      !aligned4(s_rows))
+    return FP8_ERR_ALIGNMENT;
+  DeviceInfo* dev;
+  if (fp8_status st = device_info(&dev)) return st;
+  return launch_pdl(moe_gather_kernel, dim3(static_cast<unsigned>((rows + 7) / 8)), dim3(256),
+                    as_stream(stream), x8, s_tok, perm, rows, K, static_cast<int>(top_k), x8_rows,
+                    s_rows);
+}
+
+fp8_status fp8_grouped_linear(const uint8_t* x8_rows, const float* s_rows, const int32_t* offsets,
+                              int32_t num_experts, int64_t M_total, const uint8_t* w8,
+                              const float* s_ch, int64_t N, int64_t K, uint16_t* y, void* stream) {
+  if (num_experts < 1 || num_experts > kMaxExperts) return FP8_ERR_INVALID_ARG;
+  if (fp8_status st = check_linear(x8_rows, s_rows, w8, s_ch, M_total, N, K, y)) return st;
+  if (M_total == 0 || N == 0) return FP8_OK;
+  if (!offsets) return FP8_ERR_INVALID_ARG;
+  if (!aligned4(offsets)) return FP8_ERR_ALIGNMENT;
+  if (static_cast<int64_t>(num_experts) * N >= (int64_t(1) << 31)) return FP8_ERR_SHAPE;
+  DeviceInfo* dev;
+  if (fp8_status st = device_info(&dev)) return st;
+  if (K == 0) {
+    if (cudaMemsetAsync(y, 0, static_cast<size_t>(M_total) * N * 2, as_stream(stream)) != cudaSuccess)
+      return FP8_ERR_CUDA;
+    return FP8_OK;
+  }
+  // Column tiles of 256 when they divide N evenly, else 128 (less waste on
+  // the last tile, e.g. N = 1408 = 11 x 128).
+  if (N % 256 == 0)
+    return launch_grouped<256, kPrefillStages>(*dev, x8_rows, s_rows, offsets, num_experts,
+                                               static_cast<int>(M_total), w8, s_ch,
+                                               static_cast<int>(N), static_cast<int>(K), y,
+                                               as_stream(stream));
+  return launch_grouped<128, 6>(*dev, x8_rows, s_rows, offsets, num_experts,
+                                static_cast<int>(M_total), w8, s_ch, static_cast<int>(N),
+                                static_cast<int>(K), y, as_stream(stream));
+}
+
+fp8_status fp8_moe_geglu_quant(const uint16_t* gate_up, int64_t M, int64_t inter, uint8_t* h8,
+                               float* s_h, uint16_t* h_out, void* stream) {
+  if (M < 0 || inter < 0) return FP8_ERR_INVALID_ARG;
+  if (inter % 16 != 0) return FP8_ERR_SHAPE;
+  if (M == 0 || inter == 0) return FP8_OK;
+  if (!gate_up || !h8 || !s_h) return FP8_ERR_INVALID_ARG;
+  if (!aligned16(gate_up) || !aligned16(h8) || !aligned4(s_h) || (h_out && !aligned16(h_out)))
+    return FP8_ERR_ALIGNMENT;
+  DeviceInfo* dev;
+  if (fp8_status st = device_info(&dev)) return st;
+  return launch_pdl(moe_geglu_quant_kernel, dim3(static_cast<unsigned>((M + 7) / 8)), dim3(256),
+                    as_stream(stream), gate_up, M, inter, h8, s_h, h_out);
+}
+
+fp8_status fp8_moe_combine(const uint16_t* rows, const int32_t* inv, int64_t tokens,
+                           int32_t top_k, int64_t H, const float* weights, uint16_t* out,
+                           void* stream) {
+  if (tokens < 0 || top_k < 1 || H < 0) return FP8_ERR_INVALID_ARG;
+  if (H % 8 != 0) return FP8_ERR_SHAPE;
+  if (tokens == 0 || H == 0) return FP8_OK;
+  if (!rows || !inv || !out) return FP8_ERR_INVALID_ARG;
+  if (!aligned16(rows) || !aligned16(out) || !aligned4(inv) || (weights && !aligned4(weights)))
+    return FP8_ERR_ALIGNMENT;
+  DeviceInfo* dev;
+  if (fp8_status st = device_info(&dev)) return st;
+  return launch_pdl(moe_combine_kernel, dim3(static_cast<unsigned>((tokens + 7) / 8)), dim3(256),
+                    as_stream(stream), rows, inv, tokens, static_cast<int>(top_k), H, weights, out);
 }
 
 }  // extern "C"

@@ -90,12 +90,67 @@ struct PrefillCfg {
   static_assert(BN % 32 == 0 && BN >= 32 && BN <= 256, "BN");
 };
 
-template <int BN, int STAGES>
+// Largest number of experts the grouped GEMM handles (its m-tile prefix
+// lives in shared memory).
+constexpr int kMaxExperts = 1024;
+
+// Arguments shared by the dense and the grouped (per-expert) GEMM.
+//  dense:   A rows [0, M), B rows [0, N); tiles walked in groups of group_m.
+//  grouped: expert e owns A rows offsets[e]..offsets[e+1] and B rows
+//           e*N..e*N+N (weights stacked [E*N, K], scales [E*N]).
+struct GemmArgs {
+  const float* s_a;
+  const float* s_b;
+  uint16_t* y;
+  int M, N, K;
+  int tiles_m, tiles_n, group_m;
+  const int* offsets;  // grouped only
+  int num_experts;     // grouped only
+};
+
+struct Tile {
+  int a_row;    // first A row (TMA coordinate)
+  int row_end;  // rows >= row_end belong to another expert / are out of range
+  int b_row;    // first B row (TMA coordinate)
+  int col0;     // first output column
+  int sb_off;   // offset of this tile's expert in s_b
+};
+
+// Tile t of the grouped problem: m-tiles are numbered expert by expert
+// (mt_off[e] = first m-tile of expert e), n-tiles vary fastest.
+__device__ __forceinline__ Tile grouped_tile(const GemmArgs& g, const int* mt_off, int t, int BN) {
+  const int gmt = t / g.tiles_n, tn = t - (t / g.tiles_n) * g.tiles_n;
+  int lo = 0, hi = g.num_experts;  // find e with mt_off[e] <= gmt < mt_off[e+1]
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (mt_off[mid] <= gmt) lo = mid; else hi = mid;
+  }
+  const int e = lo;
+  Tile T;
+  T.a_row = g.offsets[e] + (gmt - mt_off[e]) * kBM;
+  T.row_end = g.offsets[e + 1];
+  T.b_row = e * g.N + tn * BN;
+  T.col0 = tn * BN;
+  T.sb_off = e * g.N;
+  return T;
+}
+
+__device__ __forceinline__ Tile dense_tile(const GemmArgs& g, int t, int BN) {
+  int tm, tn;
+  tile_coords(t, g.tiles_m, g.tiles_n, g.group_m, tm, tn);
+  Tile T;
+  T.a_row = tm * kBM;
+  T.row_end = g.M;
+  T.b_row = tn * BN;
+  T.col0 = tn * BN;
+  T.sb_off = 0;
+  return T;
+}
+
+template <int BN, int STAGES, bool GROUPED>
 __global__ void __launch_bounds__(192, 1)
     gemm_prefill_kernel(const __grid_constant__ CUtensorMap tmA,
-                        const __grid_constant__ CUtensorMap tmB, const float* __restrict__ s_a,
-                        const float* __restrict__ s_b, uint16_t* __restrict__ y, int M, int N,
-                        int K, int tiles_m, int tiles_n, int group_m) {
+                        const __grid_constant__ CUtensorMap tmB, const GemmArgs g) {
   using C = PrefillCfg<BN, STAGES>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
@@ -103,14 +158,16 @@ __global__ void __launch_bounds__(192, 1)
   uint8_t* sB = smem + STAGES * C::kABytes;
   uint64_t* bars = reinterpret_cast<uint64_t*>(sB + STAGES * C::kBBytes);
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 4);
+  // grouped: E+1 ints after the barriers and the TMEM holder (the launch adds
+  // 4 * (E + 1) bytes of dynamic shared memory for them)
+  int* mt_off = reinterpret_cast<int*>(reinterpret_cast<uint8_t*>(bars) + C::kBarBytes);
   const uint32_t full0 = smem_u32(bars);
   const uint32_t empty0 = smem_u32(bars + STAGES);
   const uint32_t tfull0 = smem_u32(bars + 2 * STAGES);
   const uint32_t tempty0 = smem_u32(bars + 2 * STAGES + 2);
 
   const int warp = warp_id(), lane = lane_id();
-  const int num_kb = (K + kBK - 1) / kBK;
-  const int num_tiles = tiles_m * tiles_n;
+  const int num_kb = (g.K + kBK - 1) / kBK;
 
   if (warp == 0 && lane == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -129,10 +186,41 @@ __global__ void __launch_bounds__(192, 1)
     tmem_alloc(smem_u32(tmem_holder), C::kTmemCols);
     tmem_relinquish();
   }
+  if constexpr (GROUPED) {
+    // m-tile prefix over experts: warp 2 scans ceil(rows_e / 128); the row
+    // offsets may come from a preceding routing grid.
+    if (warp == 2) {
+      pdl_wait();
+      const int E = g.num_experts;
+      const int per = (E + 31) / 32;
+      int sum = 0;
+      for (int i = 0; i < per; ++i) {
+        const int e = lane * per + i;
+        if (e < E) sum += (g.offsets[e + 1] - g.offsets[e] + kBM - 1) / kBM;
+      }
+      int incl = sum;
+#pragma unroll
+      for (int d = 1; d < 32; d <<= 1) {
+        const int v = __shfl_up_sync(0xFFFFFFFFu, incl, d);
+        if (lane >= d) incl += v;
+      }
+      int run = incl - sum;
+      for (int i = 0; i < per; ++i) {
+        const int e = lane * per + i;
+        if (e < E) {
+          mt_off[e] = run;
+          run += (g.offsets[e + 1] - g.offsets[e] + kBM - 1) / kBM;
+        }
+      }
+      if (lane == 31) mt_off[E] = incl;
+    }
+  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
+  const int num_tiles = GROUPED ? mt_off[g.num_experts] * g.tiles_n : g.tiles_m * g.tiles_n;
+  auto tile_of = [&](int t) { return GROUPED ? grouped_tile(g, mt_off, t, BN) : dense_tile(g, t, BN); };
 
   if (warp == 0) {
     if (lane == 0) {
@@ -141,14 +229,13 @@ __global__ void __launch_bounds__(192, 1)
       uint32_t phase = 0;
       bool ok = true;
       for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
-        int tm, tn;
-        tile_coords(tile, tiles_m, tiles_n, group_m, tm, tn);
+        const Tile T = tile_of(tile);
         for (int kb = 0; kb < num_kb; ++kb) {
           if (!mbar_wait(empty0 + 8 * stage, phase ^ 1)) { ok = false; break; }
           const uint32_t fb = full0 + 8 * stage;
           mbar_arrive_expect_tx(fb, C::kStageBytes);
-          tma_load_2d(smem_u32(sA + stage * C::kABytes), &tmA, fb, kb * kBK, tm * kBM, 0ull);
-          tma_load_2d(smem_u32(sB + stage * C::kBBytes), &tmB, fb, kb * kBK, tn * BN, 0ull);
+          tma_load_2d(smem_u32(sA + stage * C::kABytes), &tmA, fb, kb * kBK, T.a_row, 0ull);
+          tma_load_2d(smem_u32(sB + stage * C::kBBytes), &tmB, fb, kb * kBK, T.b_row, 0ull);
           if (++stage == STAGES) { stage = 0; phase ^= 1; }
         }
       }
@@ -185,29 +272,31 @@ __global__ void __launch_bounds__(192, 1)
   } else {
     // Epilogue warps 2..5; a warp may only touch TMEM lanes 32*(warp%4)..+31.
     const int quad = warp & 3;
+    const int N = g.N;
     const bool vec_ok = (N % 8) == 0;
     int acc = 0;
     uint32_t acc_phase = 0;
     bool waited = false;
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
-      int tm, tn;
-      tile_coords(tile, tiles_m, tiles_n, group_m, tm, tn);
+      const Tile T = tile_of(tile);
       if (!mbar_wait(tfull0 + 8 * acc, acc_phase)) break;
       tc_fence_after();
       if (!waited) { pdl_wait(); waited = true; }
-      const int row = tm * kBM + quad * 32 + lane;
-      const float sa = row < M ? __ldg(s_a + row) : 0.0f;
-      uint16_t* yrow = y + static_cast<int64_t>(row) * N;
+      const int row = T.a_row + quad * 32 + lane;
+      const bool row_ok = row < T.row_end;
+      const float sa = row_ok ? __ldg(g.s_a + row) : 0.0f;
+      uint16_t* yrow = g.y + static_cast<int64_t>(row) * N;
+      const float* sb_base = g.s_b + T.sb_off;
       const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + acc * BN;
 #pragma unroll 1
       for (int c = 0; c < BN / 32; ++c) {
         uint32_t r[32];
         tmem_ld32(t_row + c * 32, r);
         tmem_ld_wait();
-        const int n0 = tn * BN + c * 32;
-        if (row < M && n0 < N) {
+        const int n0 = T.col0 + c * 32;
+        if (row_ok && n0 < N) {
           if (vec_ok && n0 + 32 <= N) {
-            const float4* sb4 = reinterpret_cast<const float4*>(s_b + n0);
+            const float4* sb4 = reinterpret_cast<const float4*>(sb_base + n0);
             uint4* dst = reinterpret_cast<uint4*>(yrow + n0);
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
@@ -224,7 +313,7 @@ __global__ void __launch_bounds__(192, 1)
 #pragma unroll
             for (int j = 0; j < 32; ++j) {
               if (n0 + j < N) {
-                const float v = __fmul_rn(__fmul_rn(__uint_as_float(r[j]), sa), __ldg(s_b + n0 + j));
+                const float v = __fmul_rn(__fmul_rn(__uint_as_float(r[j]), sa), __ldg(sb_base + n0 + j));
                 yrow[n0 + j] = f32_to_bf16_rn(v);
               }
             }

@@ -66,6 +66,7 @@ typedef enum fp8_status {
 #define FP8_DEV_NAN_CODE 0x2u  /* FNUZ input held code 0x80 (its NaN)          */
 #define FP8_DEV_INEXACT 0x4u   /* FNUZ row not exactly representable in E4M3  */
 #define FP8_DEV_TIMEOUT 0x8u   /* a bounded in-kernel wait gave up            */
+#define FP8_DEV_BAD_INDEX 0x10u /* an expert id outside [0, num_experts)       */
 
 /* Library version: major * 10000 + minor * 100 + patch. */
 int fp8_version(void);
@@ -170,6 +171,74 @@ fp8_status fp8_linear_bf16(const uint16_t* x, const uint8_t* w8, const float* s_
  *   x [n] float32, out [n] uint8. Requires 16-byte aligned x and out.
  */
 fp8_status fp8_cast_e4m3(const float* x, int64_t n, uint8_t* out, void* stream);
+
+/* ------------------------------------------------------------------------
+ * Mixture-of-experts layer. Source: dev.to "Gemma 4 From E2B to 31B on an AMD
+ * MI300X", section "Step 1 - Build the Larger Repacks" (128 experts per layer,
+ * fused expert banks split into one gate/up/down FP8 linear per expert, bf16
+ * router) and section "Why the Mixture-of-Experts Model Sits Lower" (the
+ * fp8_w8a8 fused-MoE expert GEMM, E=128, N=704). Routing decisions are inputs;
+ * the library groups, gathers, multiplies, activates and combines.
+ * ------------------------------------------------------------------------ */
+
+/*
+ * fp8_moe_route: group the (token, slot) pairs by expert.
+ *   topk_ids [tokens, top_k] int32: expert of each slot, in [0, num_experts).
+ *   perm [tokens*top_k] int32 out: flat index token*top_k + slot of each row of
+ *     the expert-sorted order; inside one expert rows ascend by flat index.
+ *   inv [tokens*top_k] int32 out: inverse of perm.
+ *   offsets [num_experts + 1] int32 out: expert e owns rows offsets[e] ..
+ *     offsets[e+1] - 1.
+ * Deterministic (no atomics decide positions). 1 <= num_experts <= 1024.
+ * Ids out of range set FP8_DEV_BAD_INDEX (their rows are missing).
+ */
+fp8_status fp8_moe_route(const int32_t* topk_ids, int64_t tokens, int32_t top_k,
+                         int32_t num_experts, int32_t* perm, int32_t* inv, int32_t* offsets,
+                         void* stream);
+
+/*
+ * fp8_moe_gather: rows of per-token quantized activations in expert order:
+ *   x8_rows[i] = x8[perm[i] / top_k], s_rows[i] = s_tok[perm[i] / top_k].
+ *   x8 [tokens, K] uint8, s_tok [tokens] fp32 (from fp8_quant_act); rows =
+ *   tokens * top_k. Requires K % 16 == 0, 16-byte aligned x8 / x8_rows.
+ */
+fp8_status fp8_moe_gather(const uint8_t* x8, const float* s_tok, const int32_t* perm,
+                          int64_t rows, int64_t K, int32_t top_k, uint8_t* x8_rows,
+                          float* s_rows, void* stream);
+
+/*
+ * fp8_grouped_linear: per-expert row-wise scaled FP8 GEMM. For each expert e,
+ * rows offsets[e] .. offsets[e+1]-1 of x8_rows [M_total, K] (scales s_rows)
+ * are multiplied by w8[e] (stacked [num_experts * N, K], K-major, scales
+ * s_ch [num_experts * N]) into y [M_total, N] bf16, with the same arithmetic
+ * and bound as fp8_rowwise_linear. One persistent tcgen05 kernel walks
+ * (expert, 128-row tile, column tile) work items derived on the GPU from
+ * offsets. Requires K % 16 == 0, num_experts <= 1024, offsets[num_experts]
+ * <= M_total.
+ */
+fp8_status fp8_grouped_linear(const uint8_t* x8_rows, const float* s_rows, const int32_t* offsets,
+                              int32_t num_experts, int64_t M_total, const uint8_t* w8,
+                              const float* s_ch, int64_t N, int64_t K, uint16_t* y, void* stream);
+
+/*
+ * fp8_moe_geglu_quant: h = bf16(gelu_tanh(gate) * up) per element of
+ * gate_up [M, 2*inter] bf16 (gate in columns 0..inter-1, up after it; fp32
+ * arithmetic, one rounding to bf16), then per-row E4M3 quantization of h with
+ * the contract above: h8 [M, inter] uint8, s_h [M] fp32. h_out [M, inter]
+ * bf16 receives h when not NULL. Requires inter % 16 == 0.
+ */
+fp8_status fp8_moe_geglu_quant(const uint16_t* gate_up, int64_t M, int64_t inter, uint8_t* h8,
+                               float* s_h, uint16_t* h_out, void* stream);
+
+/*
+ * fp8_moe_combine: out[t] = sum_{j<top_k} w[t,j] * rows[inv[t*top_k + j]]
+ * (fp32 products and sums in slot order, one rounding to bf16); rows
+ * [tokens*top_k, H] bf16 in expert order, weights [tokens, top_k] fp32 or
+ * NULL for 1/top_k. Requires H % 8 == 0.
+ */
+fp8_status fp8_moe_combine(const uint16_t* rows, const int32_t* inv, int64_t tokens,
+                           int32_t top_k, int64_t H, const float* weights, uint16_t* out,
+                           void* stream);
 
 /*
  * fp8_linear_bf16_noalloc: the same computation as fp8_linear_bf16 (per-token
