@@ -73,6 +73,8 @@ WORKLOADS = {
                     desc="prefill GEMM K=4096 N=14336, M in {8192,1024,128}, FNUZ load conversion"),
     "tiny": dict(K=256, N=128, Ms=(4,), seed=0, outl=0.0, repack=True, fnuz=False,
                  desc="tiny W8A8 linear M=4 K=256 N=128"),
+    "moe": dict(moe=True, tokens=8192, hidden=2048, inter=704, experts=128, top_k=8, seed=4, outl=0.01,
+                desc="MoE layer: 128 experts (gate/up/down, hidden 2048, inter 704), 8192 tokens top-8"),
 }
 
 
@@ -147,30 +149,21 @@ class ClockSampler:
 
 
 # --------------------------------------------------------------------- our arm
-def run_ours(args, rank, world, local_rank):
-    import torch
-    import torch.distributed as dist
+def _pinned(torch, a):
+    a = np.ascontiguousarray(a)
+    t = torch.from_numpy(a.view(np.int16) if a.dtype == np.uint16 else a)
+    return t.pin_memory()
 
-    import fp8_w8a8_linear_b200 as f
+
+def setup_dense(torch, f, wl, seed, dev, flushable):
+    """Inputs and ops of a dense-layer workload. Returns (ops, h, D, outs)."""
     from workloads import activations_bf16, q4_weights
 
-    torch.cuda.set_device(local_rank)
-    dev = torch.device("cuda", local_rank)
-    wl = WORKLOADS[args.workload]
     K, N, Ms = wl["K"], wl["N"], wl["Ms"]
-    seed = wl["seed"] + 1000 * rank  # each rank has its own batch (weak scaling)
-    stream = torch.cuda.current_stream()
-
-    # ---- host inputs (pinned) and their device copies
-    def pinned(a):
-        a = np.ascontiguousarray(a)
-        t = torch.from_numpy(a.view(np.int16) if a.dtype == np.uint16 else a)
-        return t.pin_memory()
-
     q4, d = q4_weights(N, K, seed=seed)
-    h = {"q4": pinned(q4), "d": pinned(d)}
+    h = {"q4": _pinned(torch, q4), "d": _pinned(torch, d)}
     for M in Ms:
-        h[f"x{M}"] = pinned(activations_bf16(M, K, seed=seed + M, outlier_frac=wl["outl"]))
+        h[f"x{M}"] = _pinned(torch, activations_bf16(M, K, seed=seed + M, outlier_frac=wl["outl"]))
     D = {k: v.to(dev) for k, v in h.items()}
     for M in Ms:
         D[f"x{M}"] = D[f"x{M}"].view(torch.bfloat16)
@@ -189,6 +182,103 @@ def run_ours(args, rank, world, local_rank):
         bufs[M] = (torch.empty((M, K), dtype=torch.uint8, device=dev),
                    torch.empty((M,), dtype=torch.float32, device=dev),
                    torch.empty((M, N), dtype=torch.bfloat16, device=dev))
+    # Decode-sized GEMMs stream their weights from HBM: in the step each one
+    # follows an L2 flush; timed alone, they rotate over weight copies that
+    # together exceed 2.5x the L2.
+    wsrc = (w8c, s_c) if wl["fnuz"] else (w8, s_ch)
+    ncopies = max(2, -(-int(2.5 * 126e6) // (N * K)))
+    wcopies = [wsrc[0]] + [wsrc[0].clone() for _ in range(ncopies - 1)]
+
+    L = []  # (name, fn(rotation), flops, bytes, bound, flushed_before, launches)
+    if wl["repack"]:
+        L.append(("repack_qat", lambda i: f.repack_qat(D["q4"], D["d"], w8, s_ch), 0.0,
+                  N * K * 1.625 + 4 * N, "hbm", False, 1))
+    if wl["fnuz"]:
+        L.append(("convert_fnuz", lambda i: f.convert_fnuz(D["wf"], D["sf"], w8c, s_c), 0.0,
+                  2.0 * N * K + 8 * N, "hbm", False, 1))
+    for M in Ms:
+        x8, st, y = bufs[M]
+        qb, gb = linear_bytes(M, N, K)
+        fl = gemm_flops(M, N, K)
+        if M > 128:
+            L.append((f"quant_act[M={M}]", lambda i, x=D[f"x{M}"], x8=x8, st=st: f.quant_act(x, x8, st),
+                      0.0, qb, "hbm", False, 1))
+            L.append((f"gemm_prefill[M={M}]",
+                      lambda i, x8=x8, st=st, y=y: f.rowwise_linear(x8, st, wsrc[0], wsrc[1], y),
+                      fl, gb, "tensor", False, 1))
+        else:
+            L.append((f"linear_decode[M={M}]",
+                      lambda i, x=D[f"x{M}"], x8=x8, st=st, y=y: f.linear(
+                          x, wcopies[i % ncopies], wsrc[1], y, x8, st),
+                      fl, qb + gb, "hbm", flushable, 2))
+    outs = [bufs[M][2] for M in Ms]
+    cfg = {"K": K, "N": N, "M": list(Ms)}
+    return L, h, D, outs, cfg
+
+
+def setup_moe(torch, f, wl, seed, dev):
+    """The MoE layer: route, quantize, gather, gate/up GEMM, GeGLU + quant,
+    down GEMM, combine. Expert weights are resident (repacked at setup)."""
+    from workloads import activations_bf16, moe_routing, q4_weights
+
+    T, Hd, I, E, k = wl["tokens"], wl["hidden"], wl["inter"], wl["experts"], wl["top_k"]
+    R = T * k
+    h = {"x": _pinned(torch, activations_bf16(T, Hd, seed=seed, outlier_frac=wl["outl"])),
+         "ids": _pinned(torch, moe_routing(T, E, k, seed=seed))}
+    D = {key: v.to(dev) for key, v in h.items()}
+    D["x"] = D["x"].view(torch.bfloat16)
+    wgu, sgu = f.repack_qat(*[torch.from_numpy(a).to(dev) for a in q4_weights(E * 2 * I, Hd, seed=seed + 1)])
+    wdn, sdn = f.repack_qat(*[torch.from_numpy(a).to(dev) for a in q4_weights(E * Hd, I, seed=seed + 2)])
+    perm = torch.empty(R, dtype=torch.int32, device=dev)
+    inv = torch.empty(R, dtype=torch.int32, device=dev)
+    off = torch.empty(E + 1, dtype=torch.int32, device=dev)
+    x8 = torch.empty((T, Hd), dtype=torch.uint8, device=dev)
+    st = torch.empty((T,), dtype=torch.float32, device=dev)
+    xr = torch.empty((R, Hd), dtype=torch.uint8, device=dev)
+    sr = torch.empty((R,), dtype=torch.float32, device=dev)
+    gu = torch.empty((R, 2 * I), dtype=torch.bfloat16, device=dev)
+    h8 = torch.empty((R, I), dtype=torch.uint8, device=dev)
+    sh = torch.empty((R,), dtype=torch.float32, device=dev)
+    dn = torch.empty((R, Hd), dtype=torch.bfloat16, device=dev)
+    out = torch.empty((T, Hd), dtype=torch.bfloat16, device=dev)
+    ids = D["ids"]
+
+    def route(i):
+        f.raw.fp8_moe_route(ids.data_ptr(), T, k, E, perm.data_ptr(), inv.data_ptr(), off.data_ptr(),
+                            torch.cuda.current_stream().cuda_stream)
+
+    fl_gu = gemm_flops(R, 2 * I, Hd)
+    fl_dn = gemm_flops(R, Hd, I)
+    L = [
+        ("moe_route", route, 0.0, 4.0 * R * 3 + 4 * (E + 1), "latency", False, 3),
+        ("quant_act", lambda i: f.quant_act(D["x"], x8, st), 0.0, 3.0 * T * Hd + 4 * T, "hbm", False, 1),
+        ("moe_gather", lambda i: f.moe_gather(x8, st, perm, k, xr, sr), 0.0,
+         1.0 * T * Hd + 1.0 * R * Hd + 8 * R, "hbm", False, 1),
+        ("grouped_gate_up", lambda i: f.grouped_linear(xr, sr, off, wgu, sgu, gu), fl_gu,
+         1.0 * R * Hd + E * 2 * I * Hd + 2.0 * R * 2 * I, "tensor", False, 1),
+        ("geglu_quant", lambda i: f.moe_geglu_quant(gu, I, h8, sh), 0.0,
+         2.0 * R * 2 * I + 1.0 * R * I + 4 * R, "hbm", False, 1),
+        ("grouped_down", lambda i: f.grouped_linear(h8, sh, off, wdn, sdn, dn), fl_dn,
+         1.0 * R * I + E * Hd * I + 2.0 * R * Hd, "tensor", False, 1),
+        ("moe_combine", lambda i: f.moe_combine(dn, inv, T, k, out=out), 0.0,
+         2.0 * R * Hd + 2.0 * T * Hd + 4 * R, "hbm", False, 1),
+    ]
+    cfg = {"tokens": T, "hidden": Hd, "inter": I, "experts": E, "top_k": k}
+    return L, h, D, [out], cfg
+
+
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+
+    import fp8_w8a8_linear_b200 as f
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    wl = WORKLOADS[args.workload]
+    seed = wl["seed"] + 1000 * rank  # each rank has its own batch (weak scaling)
+    stream = torch.cuda.current_stream()
+
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     flush_rd = torch.ones(64 << 20, dtype=torch.float32, device=dev)   # 256 MiB
     flush_sum = torch.empty((), dtype=torch.float32, device=dev)
@@ -199,42 +289,11 @@ def run_ours(args, rank, world, local_rank):
         flush.zero_()
         torch.sum(flush_rd, dim=0, out=flush_sum)
 
-    # Decode-sized GEMMs stream their weights from HBM: in the step each one
-    # follows an L2 flush; timed alone, they rotate over weight copies that
-    # together exceed 2.5x the L2.
-    wsrc = (w8c, s_c) if wl["fnuz"] else (w8, s_ch)
-    wbytes = N * K
-    ncopies = max(2, -(-int(2.5 * 126e6) // wbytes))
-    wcopies = [wsrc[0]] + [wsrc[0].clone() for _ in range(ncopies - 1)]
-
-    # ---- one step: list of (name, fn(rotation), flops, bytes, bound, flushed_before)
-    def ops():
-        L = []
-        if wl["repack"]:
-            L.append(("repack_qat", lambda i: f.repack_qat(D["q4"], D["d"], w8, s_ch), 0.0,
-                      N * K * 1.625 + 4 * N, "hbm", False))
-        if wl["fnuz"]:
-            L.append(("convert_fnuz", lambda i: f.convert_fnuz(D["wf"], D["sf"], w8c, s_c), 0.0,
-                      2.0 * N * K + 8 * N, "hbm", False))
-        for M in Ms:
-            x8, st, y = bufs[M]
-            qb, gb = linear_bytes(M, N, K)
-            fl = gemm_flops(M, N, K)
-            if M > 128:
-                L.append((f"quant_act[M={M}]", lambda i, x=D[f"x{M}"], x8=x8, st=st: f.quant_act(x, x8, st),
-                          0.0, qb, "hbm", False))
-                L.append((f"gemm_prefill[M={M}]",
-                          lambda i, x8=x8, st=st, y=y: f.rowwise_linear(x8, st, wsrc[0], wsrc[1], y),
-                          fl, gb, "tensor", False))
-            else:
-                L.append((f"linear_decode[M={M}]",
-                          lambda i, x=D[f"x{M}"], x8=x8, st=st, y=y: f.linear(
-                              x, wcopies[i % ncopies], wsrc[1], y, x8, st),
-                          fl, qb + gb, "hbm", True))
-        return L
-
-    step_ops = ops()
-    n_launch_per_step = sum(2 if n.startswith("linear") else 1 for n, *_ in step_ops)
+    if wl.get("moe"):
+        step_ops, h, D, outs, cfg = setup_moe(torch, f, wl, seed, dev)
+    else:
+        step_ops, h, D, outs, cfg = setup_dense(torch, f, wl, seed, dev, True)
+    n_launch_per_step = sum(o[6] for o in step_ops)
 
     for _ in range(args.warmup):
         for name, fn, *_rest in step_ops:
@@ -262,7 +321,7 @@ def run_ours(args, rank, world, local_rank):
         return a.elapsed_time(b) / reps
 
     alone_ms = []
-    for name, fn, fl, by, bound, flushed in step_ops:
+    for name, fn, fl, by, bound, flushed, nl in step_ops:
         reps = 40 if flushed else 5
         alone_ms.append(time_alone(fn, reps))
 
@@ -282,7 +341,7 @@ def run_ours(args, rank, world, local_rank):
             e0, e1 = ev(), ev()
             fl_pairs, op_pairs = [], {}
             e0.record()
-            for i, (name, fn, fl, by, bound, flushed) in enumerate(step_ops):
+            for i, (name, fn, fl, by, bound, flushed, nl) in enumerate(step_ops):
                 if flushed:
                     a, b = ev(), ev()
                     a.record()
@@ -344,14 +403,17 @@ def run_ours(args, rank, world, local_rank):
     peaks = load_peaks()
     fp8_sus = peaks["bf16_sustained"] * FP8_PER_BF16
     kernels = []
-    for i, ((name, fn, fl, by, bound, pre), ms) in enumerate(zip(step_ops, op_ms)):
+    for i, ((name, fn, fl, by, bound, pre, nl), ms) in enumerate(zip(step_ops, op_ms)):
         k = {"op": name, "us": round(ms * 1e3, 2), "gbs": round(by / (ms * 1e-3) / 1e9, 1),
              "tflops": round(fl / (ms * 1e-3) / 1e12, 1), "bound": bound,
              "timed": "in step" if long_op[i] else "alone, back to back"}
-        k["frac"] = round((k["tflops"] / fp8_sus) if bound == "tensor" else (k["gbs"] / peaks["hbm_gbs"]), 3)
+        if bound == "tensor":
+            k["frac"] = round(k["tflops"] / fp8_sus, 3)
+        elif bound == "hbm":
+            k["frac"] = round(k["gbs"] / peaks["hbm_gbs"], 3)
         kernels.append(k)
     dom = max(range(len(step_ops)), key=lambda i: op_ms[i])  # the longest op of the step
-    dname, _, dfl, dby, dbound, _ = step_ops[dom]
+    dname, _, dfl, dby, dbound, _, _ = step_ops[dom]
     dms = op_ms[dom]
     if dbound == "tensor":
         roof = {"kernel": dname, "bound": "tensor", "achieved": round(dfl / (dms * 1e-3) / 1e12, 1),
@@ -363,19 +425,20 @@ def run_ours(args, rank, world, local_rank):
     roof["frac"] = round(roof["achieved"] / roof["peak"], 3)
     roof["traffic"] = TRAFFIC.get((args.workload, dname))
 
-    # ---- end to end through the public API, from pinned host buffers
+    # ---- end to end through the public API, from pinned host buffers: the
+    # step's inputs are copied in and its results read back every step.
     e2e_steps = max(1, min(args.steps, 3))
-    outs_host = {M: torch.empty((M, N), dtype=torch.bfloat16).pin_memory() for M in Ms}
-    h2d = sum(t.numel() * t.element_size() for k, t in h.items())
-    d2h = sum(o.numel() * 2 for o in outs_host.values())
+    outs_host = [torch.empty(o.shape, dtype=o.dtype).pin_memory() for o in outs]
+    h2d = sum(t.numel() * t.element_size() for t in h.values())
+    d2h = sum(o.numel() * o.element_size() for o in outs_host)
 
     def e2e_step():
-        for k in h:
-            D[k].view(h[k].dtype).copy_(h[k], non_blocking=True)
+        for key in h:
+            D[key].view(h[key].dtype).copy_(h[key], non_blocking=True)
         for name, fn, *_ in step_ops:
             fn(0)
-        for M in Ms:
-            outs_host[M].copy_(bufs[M][2], non_blocking=True)
+        for oh, od in zip(outs_host, outs):
+            oh.copy_(od, non_blocking=True)
 
     e2e_step()
     torch.cuda.synchronize()
@@ -397,6 +460,10 @@ def run_ours(args, rank, world, local_rank):
 
     out = None
     if rank == 0:
+        config = {"workload": args.workload, "desc": wl["desc"], **cfg,
+                  "parallelism": f"replicas x{world} (independent batches, no collective on the data path)",
+                  "l2": ("inputs > L2 for the long ops; before each decode GEMM a 256 MiB write then a "
+                         "256 MiB read flush L2 (not timed)")}
         out = {
             "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(step_ms, 4),
@@ -406,9 +473,7 @@ def run_ours(args, rank, world, local_rank):
                                  "from a back-to-back graph of that op alone",
                        "graph_ms_incl_flushes": round(graph_ms, 3)},
             "data": "synthetic (seeded q4_0-grid weights, bf16 N(0,1) activations with 1% x20 outlier channels)",
-            "config": {"workload": args.workload, "desc": wl["desc"], "K": K, "N": N, "M": list(Ms),
-                       "parallelism": f"replicas x{world} (independent batches, no collective on the data path)",
-                       "l2": "inputs > L2 for the prefill GEMM; before each decode GEMM a 256 MiB write then a 256 MiB read flush L2 (not timed)"},
+            "config": config,
             "kernels": kernels,
             "roofline": roof,
             "gpu_launches": n_launch_per_step * args.steps,
@@ -427,6 +492,42 @@ TRAFFIC = {}
 
 
 # --------------------------------------------------------------------- oracle arm
+def oracle_sample_moe(wl, rank: int = 0):
+    """The CPU oracle on a bounded sample of one MoE step: the routing sort of
+    all tokens, the activation quant of all tokens, and for the first two
+    experts the repack of their weights, the gather, gate/up GEMM, GeGLU,
+    quant and down GEMM of their rows."""
+    import oracle
+    from oracle import moe
+    from workloads import activations_bf16, moe_routing, q4_weights
+
+    T, Hd, I, E, k = wl["tokens"], wl["hidden"], wl["inter"], wl["experts"], wl["top_k"]
+    seed = wl["seed"] + 1000 * rank
+    xb = activations_bf16(T, Hd, seed=seed, outlier_frac=wl["outl"])
+    ids = moe_routing(T, E, k, seed=seed)
+    ne = 2
+    q_gu = q4_weights(E * 2 * I, Hd, seed=seed + 1, rows=slice(0, ne * 2 * I))
+    q_dn = q4_weights(E * Hd, I, seed=seed + 2, rows=slice(0, ne * Hd))
+    t0 = time.perf_counter()
+    perm, inv, off = moe.route_sort(ids, E)
+    a = oracle.quant_act(xb)
+    xs, ss = moe.gather_rows(a.codes, a.scales, perm[:off[ne]], k)
+    wgu = oracle.repack_qat(*q_gu)
+    wdn = oracle.repack_qat(*q_dn)
+    off_s = off[:ne + 1]
+    gu = moe.grouped_linear_ref(xs, ss, off_s, wgu.codes.reshape(ne, 2 * I, Hd), wgu.scales.reshape(ne, 2 * I))
+    gu_b = (np.asarray(gu, np.float32).view(np.uint32) >> 16).astype(np.uint16)
+    h = moe.geglu_bf16(gu_b, I)
+    hq = oracle.quant_act(h)
+    moe.grouped_linear_ref(hq.codes, hq.scales, off_s, wdn.codes.reshape(ne, Hd, I), wdn.scales.reshape(ne, Hd))
+    dt = time.perf_counter() - t0
+    rows = int(off[ne])
+    flops = gemm_flops(rows, 2 * I, Hd) + gemm_flops(rows, Hd, I)
+    desc = (f"routing sort and activation quant of all {T} tokens; weights repack, gather, gate/up GEMM, "
+            f"GeGLU, quant and down GEMM for experts 0..{ne - 1} ({rows} rows)")
+    return dt, flops, desc
+
+
 def oracle_sample(workload: str, rank: int = 0):
     """The CPU oracle on a bounded sample of one step: the repack and FNUZ
     conversion of 2048 weight rows, the activation quant of min(M, 2048) token
@@ -436,6 +537,8 @@ def oracle_sample(workload: str, rank: int = 0):
     from workloads import activations_bf16, q4_weights
 
     wl = WORKLOADS[workload]
+    if wl.get("moe"):
+        return oracle_sample_moe(wl, rank)
     K, N = wl["K"], wl["N"]
     ns = min(N, 2048)
     seed = wl["seed"] + 1000 * rank
