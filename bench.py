@@ -67,6 +67,8 @@ def load_peaks():
 WORKLOADS = {
     "large": dict(K=5376, N=21504, Ms=(65536, 1, 64), seed=3, outl=0.01, repack=True, fnuz=True,
                   desc="large dense layer K=5376 N=21504, M in {65536,1,64}, QAT repack + FNUZ load conversion"),
+    "large8k": dict(K=5376, N=21504, Ms=(8192, 1, 64), seed=3, outl=0.01, repack=True, fnuz=True,
+                    desc="large dense layer K=5376 N=21504 at M in {8192,1,64} (profiling size), repack + FNUZ"),
     "decode": dict(K=2048, N=8192, Ms=(1, 8, 64), seed=1, outl=0.01, repack=False, fnuz=False,
                    desc="decode GEMM sweep K=2048 N=8192, M in {1,8,64}"),
     "prefill": dict(K=4096, N=14336, Ms=(8192, 1024, 128), seed=2, outl=0.01, repack=False, fnuz=True,
@@ -486,9 +488,15 @@ def run_ours(args, rank, world, local_rank):
 
 
 # Measured DRAM traffic per launch (dram__bytes_read.sum + dram__bytes_write.sum)
-# for the dominant kernel, from the ncu summaries under profiles/, keyed by
-# (workload, op). Kept null until a capture of the current kernel exists.
-TRAFFIC = {}
+# of the dominant kernel, from the ncu summaries under profiles/, keyed by
+# (workload, op); reset to absent whenever that kernel changes. The M=65536
+# figure is the M=8192 capture of the same K and N scaled by 8 (x8, y and
+# the number of weight re-reads all grow in proportion to M).
+TRAFFIC = {
+    ("large8k", "gemm_prefill[M=8192]"): 825.25e6,
+    ("large", "gemm_prefill[M=65536]"): 8 * 825.25e6,
+    ("moe", "grouped_gate_up"): 671.35e6,
+}
 
 
 # --------------------------------------------------------------------- oracle arm
