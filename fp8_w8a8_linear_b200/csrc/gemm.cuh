@@ -147,8 +147,13 @@ __device__ __forceinline__ Tile dense_tile(const GemmArgs& g, int t, int BN) {
   return T;
 }
 
+// Warps: 0 = TMA producer, 1 = MMA issuer + TMEM owner, 2..9 = epilogue (two
+// warps per TMEM lane quadrant, each draining half of the tile's columns).
+constexpr int kEpiWarps = 8;
+constexpr int kPrefillThreads = 64 + 32 * kEpiWarps;
+
 template <int BN, int STAGES, bool GROUPED>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(kPrefillThreads, 1)
     gemm_prefill_kernel(const __grid_constant__ CUtensorMap tmA,
                         const __grid_constant__ CUtensorMap tmB, const GemmArgs g) {
   using C = PrefillCfg<BN, STAGES>;
@@ -176,7 +181,7 @@ __global__ void __launch_bounds__(192, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(tfull0 + 8 * b, 1);
-      mbar_init(tempty0 + 8 * b, 4);
+      mbar_init(tempty0 + 8 * b, kEpiWarps);
     }
     fence_barrier_init();
     tma_prefetch_desc(&tmA);
@@ -270,8 +275,10 @@ __global__ void __launch_bounds__(192, 1)
       }
     }
   } else {
-    // Epilogue warps 2..5; a warp may only touch TMEM lanes 32*(warp%4)..+31.
+    // Epilogue warps 2..9; a warp may only touch TMEM lanes 32*(warp%4)..+31,
+    // and warps w and w+4 share a quadrant, splitting its column chunks.
     const int quad = warp & 3;
+    const int half = (warp - 2) >> 2;
     const int N = g.N;
     const bool vec_ok = (N % 8) == 0;
     int acc = 0;
@@ -289,7 +296,7 @@ __global__ void __launch_bounds__(192, 1)
       const float* sb_base = g.s_b + T.sb_off;
       const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + acc * BN;
 #pragma unroll 1
-      for (int c = 0; c < BN / 32; ++c) {
+      for (int c = half * (BN / 64); c < (half + 1) * (BN / 64); ++c) {
         uint32_t r[32];
         tmem_ld32(t_row + c * 32, r);
         tmem_ld_wait();
