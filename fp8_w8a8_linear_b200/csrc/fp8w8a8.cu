@@ -27,6 +27,7 @@ bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0
 
 struct DeviceInfo {
   int sm_count = 0;
+  int pair_clusters = 0;  // co-resident 2-CTA clusters of the pair GEMM
   bool supported = false;
   bool attrs_set = false;
 };
@@ -116,6 +117,15 @@ fp8_status set_decode_attr() {
              : FP8_ERR_CUDA;
 }
 
+template <int STAGES>
+fp8_status set_pair_attr() {
+  return cudaFuncSetAttribute(gemm_pair_kernel<STAGES>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              static_cast<int>(PairCfg<STAGES>::kSmem)) == cudaSuccess
+             ? FP8_OK
+             : FP8_ERR_CUDA;
+}
+
+constexpr int kPairStages = 6;
 constexpr int kPrefillBN = 256;
 // Shared memory the staged quantizer may use per block (one block per SM).
 constexpr int kStagedSmemBudget = 200 * 1024;
@@ -135,6 +145,26 @@ fp8_status device_info(DeviceInfo** out) {
     fp8_status st = FP8_OK;
     st = st != FP8_OK ? st : set_prefill_attr<kPrefillBN, kPrefillStages, false>();
     st = st != FP8_OK ? st : set_prefill_attr<256, kPrefillStages, true>();
+    st = st != FP8_OK ? st : set_pair_attr<kPairStages>();
+    if (st == FP8_OK) {
+      // A persistent grid must fit at once: count the 2-CTA clusters that can
+      // be resident together (an SM left over in a GPC cannot host a pair).
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3(2 * (d.sm_count / 2));
+      cfg.blockDim = dim3(kPrefillThreads);
+      cfg.dynamicSmemBytes = PairCfg<kPairStages>::kSmem;
+      cudaLaunchAttribute a;
+      a.id = cudaLaunchAttributeClusterDimension;
+      a.val.clusterDim.x = 2;
+      a.val.clusterDim.y = 1;
+      a.val.clusterDim.z = 1;
+      cfg.attrs = &a;
+      cfg.numAttrs = 1;
+      int n = 0;
+      if (cudaOccupancyMaxActiveClusters(&n, gemm_pair_kernel<kPairStages>, &cfg) != cudaSuccess)
+        st = FP8_ERR_CUDA;
+      d.pair_clusters = n;
+    }
     st = st != FP8_OK ? st : set_decode_attr<16, 3, 2>();
     st = st != FP8_OK ? st : set_decode_attr<32, 4, 1>();
     st = st != FP8_OK ? st : set_decode_attr<32, 3, 2>();
@@ -196,6 +226,46 @@ fp8_status launch_prefill(const DeviceInfo& dev, const uint8_t* x8, const float*
   g.tiles_n = tiles_n;
   g.group_m = group_m;
   if (cudaLaunchKernelEx(&cfg, gemm_prefill_kernel<BN, ST, false>, tmA, tmB, g) != cudaSuccess)
+    return FP8_ERR_CUDA;
+  return FP8_OK;
+}
+
+// Dense GEMM on 256 x 256 tiles per CTA pair (clusters of 2, persistent).
+fp8_status launch_pair(const DeviceInfo& dev, const uint8_t* x8, const float* s_tok,
+                       const uint8_t* w8, const float* s_ch, int M, int N, int K, uint16_t* y,
+                       cudaStream_t stream, bool pdl) {
+  CUtensorMap tmA, tmB;
+  if (!make_tmap_u8(&tmA, x8, M, K, 128) || !make_tmap_u8(&tmB, w8, N, K, 128)) return FP8_ERR_CUDA;
+  const int tiles_m = (M + 255) / 256;
+  const int tiles_n = (N + 255) / 256;
+  const int num_tiles = tiles_m * tiles_n;
+  const int pairs = std::min(num_tiles, dev.pair_clusters);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * pairs);
+  cfg.blockDim = dim3(kPrefillThreads);
+  cfg.dynamicSmemBytes = PairCfg<kPairStages>::kSmem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attrs[2];
+  int na = 0;
+  attrs[na].id = cudaLaunchAttributeClusterDimension;
+  attrs[na].val.clusterDim.x = 2;
+  attrs[na].val.clusterDim.y = 1;
+  attrs[na].val.clusterDim.z = 1;
+  ++na;
+  set_pdl(attrs, na, pdl);
+  cfg.attrs = attrs;
+  cfg.numAttrs = na;
+  GemmArgs g = {};
+  g.s_a = s_tok;
+  g.s_b = s_ch;
+  g.y = y;
+  g.M = M;
+  g.N = N;
+  g.K = K;
+  g.tiles_m = tiles_m;
+  g.tiles_n = tiles_n;
+  g.group_m = std::min(tiles_m, 8);
+  if (cudaLaunchKernelEx(&cfg, gemm_pair_kernel<kPairStages>, tmA, tmB, g) != cudaSuccess)
     return FP8_ERR_CUDA;
   return FP8_OK;
 }
@@ -313,6 +383,10 @@ fp8_status launch_linear(const DeviceInfo& dev, const uint8_t* x8, const float* 
   if (M <= 128)
     return one_per_sm ? launch_decode_t<128, 4, 1>(dev, x8, s_tok, w8, s_ch, M, N, K, y, stream, pdl)
                       : launch_decode_t<128, 2, 1>(dev, x8, s_tok, w8, s_ch, M, N, K, y, stream, pdl);
+  // Prefill: 256 x 256 tiles on CTA pairs when there are at least two row
+  // tiles of 256, single-SM 128 x 256 tiles below that.
+  if (M >= 512 && dev.pair_clusters > 0)
+    return launch_pair(dev, x8, s_tok, w8, s_ch, M, N, K, y, stream, pdl);
   return launch_prefill(dev, x8, s_tok, w8, s_ch, M, N, K, y, stream, pdl);
 }
 

@@ -342,6 +342,194 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
   }
 }
 
+// ============================================================== prefill, CTA pair
+// Dense GEMM on 256 x 256 output tiles computed by a cluster of two CTAs on
+// two SMs with tcgen05.mma.cta_group::2: each CTA stages 128 rows of A (its
+// half of the tile's rows) and 128 rows of B (its half of the tile's
+// columns), so every SM moves 32 KB per 128-deep k-block for a 256 x 256 x
+// 128 product - two thirds of the operand traffic of a 128 x 256 single-SM
+// tile per unit of work. The even CTA's MMA thread issues the pair MMAs; both
+// CTAs' TMA loads complete on the even CTA's full barrier; each MMA commit is
+// multicast to the stage's empty barrier (or the accumulator's full barrier)
+// in both CTAs; each CTA drains its own 128 TMEM lanes (its 128 rows), and the
+// even CTA's accumulator-empty barrier counts the epilogue warps of both.
+template <int STAGES>
+struct PairCfg {
+  static constexpr int kHalf = 128;                  // rows of A and of B per CTA
+  static constexpr int kBN = 256;                    // tile columns
+  static constexpr int kABytes = kHalf * kBK;
+  static constexpr int kBBytes = kHalf * kBK;
+  static constexpr int kStageBytes = kABytes + kBBytes;
+  static constexpr int kTmemCols = 512;              // two 256-column accumulators
+  static constexpr int kBarBytes = 8 * (2 * STAGES + 4) + 16;
+  static constexpr size_t kSmem = 1024 + static_cast<size_t>(STAGES) * kStageBytes + kBarBytes;
+};
+
+template <int STAGES>
+__global__ void __launch_bounds__(kPrefillThreads, 1)
+    gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                     const GemmArgs g) {
+  using C = PairCfg<STAGES>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align1024(smem_raw);
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + STAGES * C::kABytes;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sB + STAGES * C::kBBytes);
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 4);
+  const uint32_t full0 = smem_u32(bars);
+  const uint32_t empty0 = smem_u32(bars + STAGES);
+  const uint32_t tfull0 = smem_u32(bars + 2 * STAGES);
+  const uint32_t tempty0 = smem_u32(bars + 2 * STAGES + 2);
+
+  const int warp = warp_id(), lane = lane_id();
+  const uint32_t rank = cluster_ctarank();        // 0 = leader (issues the MMAs)
+  const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
+  const int num_kb = (g.K + kBK - 1) / kBK;
+  const int num_tiles = g.tiles_m * g.tiles_n;    // tiles of 256 x 256
+
+  if (warp == 0 && lane == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(full0 + 8 * s, 1);
+      mbar_init(empty0 + 8 * s, 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(tfull0 + 8 * b, 1);
+      mbar_init(tempty0 + 8 * b, 2 * kEpiWarps);
+    }
+    fence_barrier_init();
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(smem_u32(tmem_holder), C::kTmemCols);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  cluster_sync();  // both CTAs' barriers exist before any cross-CTA arrive or load
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_holder;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      pdl_wait();
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int tile = pair; ok && tile < num_tiles; tile += npairs) {
+        int tm, tn;
+        tile_coords(tile, g.tiles_m, g.tiles_n, g.group_m, tm, tn);
+        const int a_row = tm * 256 + rank * C::kHalf;
+        const int b_row = tn * C::kBN + rank * C::kHalf;
+        for (int kb = 0; kb < num_kb; ++kb) {
+          if (!mbar_wait(empty0 + 8 * stage, phase ^ 1)) { ok = false; break; }
+          const uint32_t fb_local = full0 + 8 * stage;
+          const uint32_t fb_leader = mapa_shared(fb_local, 0);
+          // Both CTAs' bytes complete on the leader's full barrier.
+          if (rank == 0) mbar_arrive_expect_tx(fb_local, 2 * C::kStageBytes);
+          tma_load_2d_pair(smem_u32(sA + stage * C::kABytes), &tmA, fb_leader, kb * kBK, a_row);
+          tma_load_2d_pair(smem_u32(sB + stage * C::kBBytes), &tmB, fb_leader, kb * kBK, b_row);
+          if (++stage == STAGES) { stage = 0; phase ^= 1; }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0 && rank == 0) {
+      constexpr uint32_t idesc = idesc_e4m3_f32(256, C::kBN);
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      bool ok = true;
+      for (int tile = pair; ok && tile < num_tiles; tile += npairs) {
+        if (!mbar_wait(tempty0 + 8 * acc, acc_phase ^ 1)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + acc * C::kBN;
+        for (int kb = 0; kb < num_kb; ++kb) {
+          if (!mbar_wait(full0 + 8 * stage, phase)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t a0 = smem_u32(sA + stage * C::kABytes);
+          const uint32_t b0 = smem_u32(sB + stage * C::kBBytes);
+#pragma unroll
+          for (int k = 0; k < kBK / 32; ++k) {
+            umma_f8_pair(d_tmem, sw128_kmajor_desc(a0 + 32 * k), sw128_kmajor_desc(b0 + 32 * k), idesc,
+                         (kb | k) != 0);
+          }
+          umma_commit_pair(empty0 + 8 * stage, 0x3);
+          if (++stage == STAGES) { stage = 0; phase ^= 1; }
+        }
+        umma_commit_pair(tfull0 + 8 * acc, 0x3);
+        if (++acc == 2) { acc = 0; acc_phase ^= 1; }
+      }
+    }
+  } else {
+    // Epilogue warps 2..9 of each CTA drain that CTA's 128 TMEM lanes.
+    const int quad = warp & 3;
+    const int half = (warp - 2) >> 2;
+    const int N = g.N;
+    const bool vec_ok = (N % 8) == 0;
+    const uint32_t tempty_leader0 = mapa_shared(tempty0, 0);
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    bool waited = false;
+    for (int tile = pair; tile < num_tiles; tile += npairs) {
+      int tm, tn;
+      tile_coords(tile, g.tiles_m, g.tiles_n, g.group_m, tm, tn);
+      if (!mbar_wait(tfull0 + 8 * acc, acc_phase)) break;
+      tc_fence_after();
+      if (!waited) { pdl_wait(); waited = true; }
+      const int row = tm * 256 + rank * C::kHalf + quad * 32 + lane;
+      const bool row_ok = row < g.M;
+      const float sa = row_ok ? __ldg(g.s_a + row) : 0.0f;
+      uint16_t* yrow = g.y + static_cast<int64_t>(row) * N;
+      const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + acc * C::kBN;
+#pragma unroll 1
+      for (int c = half * 4; c < half * 4 + 4; ++c) {
+        uint32_t r[32];
+        tmem_ld32(t_row + c * 32, r);
+        tmem_ld_wait();
+        const int n0 = tn * C::kBN + c * 32;
+        if (row_ok && n0 < N) {
+          if (vec_ok && n0 + 32 <= N) {
+            const float4* sb4 = reinterpret_cast<const float4*>(g.s_b + n0);
+            uint4* dst = reinterpret_cast<uint4*>(yrow + n0);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              const float4 b0 = __ldg(sb4 + 2 * q), b1 = __ldg(sb4 + 2 * q + 1);
+              const float sb[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+              float v[8];
+#pragma unroll
+              for (int i = 0; i < 8; ++i)
+                v[i] = __fmul_rn(__fmul_rn(__uint_as_float(r[8 * q + i]), sa), sb[i]);
+              dst[q] = make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]),
+                                  pack_bf16x2(v[4], v[5]), pack_bf16x2(v[6], v[7]));
+            }
+          } else {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              if (n0 + j < N) {
+                const float v = __fmul_rn(__fmul_rn(__uint_as_float(r[j]), sa), __ldg(g.s_b + n0 + j));
+                yrow[n0 + j] = f32_to_bf16_rn(v);
+              }
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(tempty_leader0 + 8 * acc);
+      if (++acc == 2) { acc = 0; acc_phase ^= 1; }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();  // the pair's MMAs have read both CTAs' shared memory; remote arrives are done
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_base, C::kTmemCols);
+  }
+}
+
 // ============================================================== decode
 // KBS 128-byte k-blocks per pipeline stage (one TMA box each per operand).
 template <int BNT, int STAGES, int KBS>
