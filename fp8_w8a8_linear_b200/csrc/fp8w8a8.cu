@@ -107,11 +107,12 @@ fp8_status set_prefill_attr() {
              : FP8_ERR_CUDA;
 }
 
-template <int BNT, int STAGES, int KBS>
+template <int BNT, int STAGES, int KBS, bool FUSED = false>
 fp8_status set_decode_attr() {
-  return cudaFuncSetAttribute(gemm_decode_kernel<BNT, STAGES, KBS>,
+  using C = DecodeCfg<BNT, STAGES, KBS>;
+  return cudaFuncSetAttribute(gemm_decode_kernel<BNT, STAGES, KBS, FUSED>,
                               cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              static_cast<int>(DecodeCfg<BNT, STAGES, KBS>::kSmemSplit)) ==
+                              static_cast<int>(FUSED ? C::kSmemFused : C::kSmemSplit)) ==
                  cudaSuccess
              ? FP8_OK
              : FP8_ERR_CUDA;
@@ -166,6 +167,7 @@ fp8_status device_info(DeviceInfo** out) {
       d.pair_clusters = n;
     }
     st = st != FP8_OK ? st : set_decode_attr<16, 3, 2>();
+    st = st != FP8_OK ? st : set_decode_attr<16, 3, 2, true>();
     st = st != FP8_OK ? st : set_decode_attr<32, 4, 1>();
     st = st != FP8_OK ? st : set_decode_attr<32, 3, 2>();
     st = st != FP8_OK ? st : set_decode_attr<64, 4, 1>();
@@ -322,16 +324,10 @@ fp8_status launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, cudaStrea
   return cudaLaunchKernelEx(&cfg, kernel, args...) == cudaSuccess ? FP8_OK : FP8_ERR_CUDA;
 }
 
-template <int BNT, int ST, int KBS>
-fp8_status launch_decode_t(const DeviceInfo& dev, const uint8_t* x8, const float* s_tok,
-                           const uint8_t* w8, const float* s_ch, int M, int N, int K, uint16_t* y,
-                           cudaStream_t stream, bool pdl, int force_splits = 0) {
-  using C = DecodeCfg<BNT, ST, KBS>;
-  CUtensorMap tmW, tmX;
-  if (!make_tmap_u8(&tmW, w8, N, K, kBM) || !make_tmap_u8(&tmX, x8, M, K, BNT))
-    return FP8_ERR_CUDA;
+// Number of K splits the decode GEMM uses for N output channels.
+int decode_splits(const DeviceInfo& dev, int N, int K, int kbs) {
   const int tiles = (N + kBM - 1) / kBM;
-  const int num_steps = (K + kBK * KBS - 1) / (kBK * KBS);
+  const int num_steps = (K + kBK * kbs - 1) / (kBK * kbs);
   // K is split over a cluster only when there are too few 128-channel tiles to
   // keep the SMs streaming (measured on B200: with >= SMs/4 tiles the cluster
   // reduction costs more than the extra streams bring). Splits divide 128 and
@@ -339,7 +335,28 @@ fp8_status launch_decode_t(const DeviceInfo& dev, const uint8_t* x8, const float
   int splits = 1;
   if (4 * tiles < dev.sm_count)
     while (splits < 8 && tiles * splits * 2 <= dev.sm_count && splits * 4 <= num_steps) splits *= 2;
+  return splits;
+}
+
+template <int BNT, int ST, int KBS, bool FUSED = false>
+fp8_status launch_decode_t(const DeviceInfo& dev, const uint8_t* x8, const float* s_tok,
+                           const uint8_t* w8, const float* s_ch, int M, int N, int K, uint16_t* y,
+                           cudaStream_t stream, bool pdl, int force_splits = 0,
+                           FusedX fx = FusedX{}) {
+  using C = DecodeCfg<BNT, ST, KBS>;
+  CUtensorMap tmW, tmX;
+  if (!make_tmap_u8(&tmW, w8, N, K, kBM)) return FP8_ERR_CUDA;
+  if (FUSED) {
+    tmX = tmW;  // unused: the kernel quantizes the tokens itself
+  } else if (!make_tmap_u8(&tmX, x8, M, K, BNT)) {
+    return FP8_ERR_CUDA;
+  }
+  const int tiles = (N + kBM - 1) / kBM;
+  const int num_steps = (K + kBK * KBS - 1) / (kBK * KBS);
+  int splits = decode_splits(dev, N, K, KBS);
   if (force_splits > 0) splits = force_splits;
+  if (FUSED && (splits != 1 || int64_t(M) * K * 2 > kFusedXBytes || M > BNT))
+    return FP8_ERR_INVALID_ARG;
   const int steps_per_split = (num_steps + splits - 1) / splits;
   CUtensorMap tmY;
   std::memset(&tmY, 0, sizeof(tmY));
@@ -348,7 +365,7 @@ fp8_status launch_decode_t(const DeviceInfo& dev, const uint8_t* x8, const float
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(tiles * splits);
   cfg.blockDim = dim3(192);
-  cfg.dynamicSmemBytes = splits > 1 ? C::kSmemSplit : C::kSmemSingle;
+  cfg.dynamicSmemBytes = FUSED ? C::kSmemFused : splits > 1 ? C::kSmemSplit : C::kSmemSingle;
   cfg.stream = stream;
   cudaLaunchAttribute attrs[2];
   int na = 0;
@@ -360,8 +377,8 @@ fp8_status launch_decode_t(const DeviceInfo& dev, const uint8_t* x8, const float
   set_pdl(attrs, na, pdl);
   cfg.attrs = attrs;
   cfg.numAttrs = na;
-  if (cudaLaunchKernelEx(&cfg, gemm_decode_kernel<BNT, ST, KBS>, tmW, tmX, tmY, s_tok, s_ch, y, M,
-                         N, K, splits, steps_per_split, use_tma_store) != cudaSuccess)
+  if (cudaLaunchKernelEx(&cfg, gemm_decode_kernel<BNT, ST, KBS, FUSED>, tmW, tmX, tmY, s_tok, s_ch,
+                         y, M, N, K, splits, steps_per_split, use_tma_store, fx) != cudaSuccess)
     return FP8_ERR_CUDA;
   return FP8_OK;
 }
@@ -406,12 +423,13 @@ fp8_status launch_quant_act(const DeviceInfo& dev, const uint16_t* x, int64_t M,
     return last_launch();
   }
   if (M <= 1024) {
-    // Few tokens: a whole 256-thread block per token row.
+    // Few tokens: a whole block per token row, sized so that the row sits in
+    // registers (one memory round trip for the amax, none for the quantize).
     const dim3 grid(static_cast<unsigned>(M));
     if (nvec <= 4 * 256)
       quant_act_kernel<256, 4><<<grid, 256, 0, stream>>>(x, M, K, ldx, x8, s_tok);
     else
-      quant_act_kernel<256, 0><<<grid, 256, 0, stream>>>(x, M, K, ldx, x8, s_tok);
+      quant_act_kernel<1024, 8, 1024><<<grid, 1024, 0, stream>>>(x, M, K, ldx, x8, s_tok);
   } else {
     const dim3 grid(static_cast<unsigned>((M + 7) / 8));
     if (nvec <= 24 * 32)
@@ -559,6 +577,17 @@ fp8_status fp8_linear_bf16(const uint16_t* x, const uint8_t* w8, const float* s_
     if (cudaMemsetAsync(y, 0, static_cast<size_t>(M) * N * 2, as_stream(stream)) != cudaSuccess)
       return FP8_ERR_CUDA;
     return FP8_OK;
+  }
+  if (M <= 16 && M * K * 2 <= kFusedXBytes &&
+      decode_splits(*dev, static_cast<int>(N), static_cast<int>(K), 2) == 1) {
+    // A handful of short tokens: quantize them inside the decode GEMM (one launch).
+    FusedX fx;
+    fx.x = x;
+    fx.x8_out = x8;
+    fx.stok_out = s_tok;
+    return launch_decode_t<16, 3, 2, true>(*dev, nullptr, s_tok, w8, s_ch, static_cast<int>(M),
+                                           static_cast<int>(N), static_cast<int>(K), y,
+                                           as_stream(stream), true, 0, fx);
   }
   if (fp8_status st = launch_quant_act(*dev, x, M, K, K, x8, s_tok, as_stream(stream))) return st;
   return launch_linear(*dev, x8, s_tok, w8, s_ch, static_cast<int>(M), static_cast<int>(N),

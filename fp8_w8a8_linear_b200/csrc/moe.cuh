@@ -191,15 +191,28 @@ __global__ void __launch_bounds__(256) moe_geglu_quant_kernel(const uint16_t* __
   const uint4* g = reinterpret_cast<const uint4*>(gu + row * 2 * I);
   const uint4* u = reinterpret_cast<const uint4*>(gu + row * 2 * I + I);
   const int64_t nvec = I / 8;
+  // h of up to kCache vectors per lane stays in registers between the amax
+  // pass and the quantize pass; longer rows recompute it (same arithmetic,
+  // same values).
+  constexpr int kCache = 4;
+  uint4 hc[kCache];
   uint32_t mx = 0;
-  for (int64_t j = lane; j < nvec; j += 32) {
-    const uint4 h = geglu8(__ldg(g + j), __ldg(u + j));
+  auto amax_of = [&](const uint4& h, int64_t j) {
     if (h_out) reinterpret_cast<uint4*>(h_out + row * I)[j] = h;
     mx = __vmaxu2(mx, h.x & 0x7FFF7FFFu);
     mx = __vmaxu2(mx, h.y & 0x7FFF7FFFu);
     mx = __vmaxu2(mx, h.z & 0x7FFF7FFFu);
     mx = __vmaxu2(mx, h.w & 0x7FFF7FFFu);
+  };
+#pragma unroll
+  for (int i = 0; i < kCache; ++i) {
+    const int64_t j = lane + 32 * i;
+    if (j < nvec) {
+      hc[i] = geglu8(__ldg(g + j), __ldg(u + j));
+      amax_of(hc[i], j);
+    }
   }
+  for (int64_t j = lane + 32 * kCache; j < nvec; j += 32) amax_of(geglu8(__ldg(g + j), __ldg(u + j)), j);
   mx = max(mx & 0xFFFFu, mx >> 16);
   const uint32_t amax_bits = __reduce_max_sync(0xFFFFFFFFu, mx);
   if (amax_bits >= 0x7F80u && lane == 0) report(FP8_DEV_NONFINITE);
@@ -208,21 +221,23 @@ __global__ void __launch_bounds__(256) moe_geglu_quant_kernel(const uint16_t* __
   if (lane == 0) s_h[row] = s;
   const RowDivisor dv = make_divisor(s, amax);
   uint2* dst = reinterpret_cast<uint2*>(h8 + row * I);
-  for (int64_t j = lane; j < nvec; j += 32) {
-    if (s == 0.0f) {
-      dst[j] = make_uint2(0, 0);
-      continue;
-    }
-    const uint4 h = geglu8(__ldg(g + j), __ldg(u + j));
+  auto quant = [&](const uint4& h) -> uint2 {
+    if (s == 0.0f) return make_uint2(0, 0);
     const uint32_t wv[4] = {h.x, h.y, h.z, h.w};
     float f[8];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      f[2 * i] = div_rn(dv, __uint_as_float(wv[i] << 16));
-      f[2 * i + 1] = div_rn(dv, __uint_as_float(wv[i] & 0xFFFF0000u));
+    for (int q = 0; q < 4; ++q) {
+      f[2 * q] = div_rn(dv, __uint_as_float(wv[q] << 16));
+      f[2 * q + 1] = div_rn(dv, __uint_as_float(wv[q] & 0xFFFF0000u));
     }
-    dst[j] = make_uint2(pack4_e4m3(f[0], f[1], f[2], f[3]), pack4_e4m3(f[4], f[5], f[6], f[7]));
+    return make_uint2(pack4_e4m3(f[0], f[1], f[2], f[3]), pack4_e4m3(f[4], f[5], f[6], f[7]));
+  };
+#pragma unroll
+  for (int i = 0; i < kCache; ++i) {
+    const int64_t j = lane + 32 * i;
+    if (j < nvec) dst[j] = quant(hc[i]);
   }
+  for (int64_t j = lane + 32 * kCache; j < nvec; j += 32) dst[j] = quant(geglu8(__ldg(g + j), __ldg(u + j)));
 }
 
 // ------------------------------------------------------------------ combine

@@ -86,14 +86,16 @@ __device__ __forceinline__ uint32_t row_max_u32(uint32_t v, uint32_t* red) {
 
 // ----------------------------------------------------------- activation quant
 // x: [M, ldx] bf16, K % 8 == 0 (16-byte vectors of 8 values).
-template <int TPR, int V>
-__global__ void __launch_bounds__(256) quant_act_kernel(const uint16_t* __restrict__ x, int64_t M,
-                                                         int64_t K, int64_t ldx,
-                                                         uint8_t* __restrict__ x8,
-                                                         float* __restrict__ s_tok) {
+// BLOCK threads per block, TPR threads per row, V cached 16-byte vectors per
+// thread (the row is read from memory once when K / 8 <= V * TPR).
+template <int TPR, int V, int BLOCK = 256>
+__global__ void __launch_bounds__(BLOCK) quant_act_kernel(const uint16_t* __restrict__ x, int64_t M,
+                                                           int64_t K, int64_t ldx,
+                                                           uint8_t* __restrict__ x8,
+                                                           float* __restrict__ s_tok) {
   pdl_launch_dependents();
-  __shared__ uint32_t red[8];
-  constexpr int RPB = 256 / TPR;  // rows per block
+  __shared__ uint32_t red[BLOCK / 32];
+  constexpr int RPB = BLOCK / TPR;  // rows per block
   const int64_t row = static_cast<int64_t>(blockIdx.x) * RPB + threadIdx.x / TPR;
   const int t = threadIdx.x % TPR;
   const bool active = row < M;

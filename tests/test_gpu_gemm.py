@@ -179,3 +179,24 @@ def test_large_layer_sampled(lib, M):
     ok, worst = oracle.check_linear(bf16_values(y)[rows][:, cols], y_ref, abs_s)
     assert ok, worst
     assert lib.device_status() == 0
+
+
+@pytest.mark.parametrize("M,N,K", [(1, 8192, 2048), (3, 8192, 2064), (8, 8192, 2048),
+                                   (16, 6144, 1024), (1, 21504, 5376), (16, 8192, 2048),
+                                   (4, 8192, 8176), (5, 8192, 8176)])
+def test_fused_quant_decode_is_bit_identical(lib, M, N, K):
+    """fp8_linear_bf16 quantizes a handful of short tokens (up to 64 KB of
+    bf16) inside the decode GEMM: its codes and scales equal the oracle's, and
+    y equals the two-kernel path (quantizer, then GEMM) bit for bit. The last
+    case is just over that size and takes the two-kernel path itself."""
+    xb, a, w = _operands(M, N, K, seed=40 + M)
+    wd, sd = to_dev(w.codes), to_dev(w.scales)
+    x8 = torch.full((M, K), 0x7F, dtype=torch.uint8, device="cuda")
+    st = torch.full((M,), -1.0, dtype=torch.float32, device="cuda")
+    y_fused = lib.linear(to_dev(xb), wd, sd, x8=x8, s_tok=st)
+    assert np.array_equal(u8(x8), a.codes) and same_bits_f32(f32(st), a.scales)
+    x8b, stb = lib.quant_act(to_dev(xb))
+    y_two = lib.rowwise_linear(x8b, stb, wd, sd)
+    assert np.array_equal(bf16_to_np_bits(y_fused), bf16_to_np_bits(y_two))
+    _check(y_fused, a, w)
+    assert lib.device_status() == 0

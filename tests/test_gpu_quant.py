@@ -65,7 +65,8 @@ ACT_SHAPES = [
     (3, 48, 5, 0.0),
     (1025, 5376, 3, 0.01),   # warp-per-row path, row held in registers
     (2000, 16, 7, 0.0),
-    (5, 9008, 8, 0.01),      # block-per-row path, re-read from cache
+    (5, 9008, 8, 0.01),      # 1024-thread block per row, row held in registers
+    (2, 21504, 11, 0.01),
     (1100, 6160, 9, 0.01),   # warp-per-row path, re-read from cache
     (7, 65536, 10, 0.01),
 ]
