@@ -107,12 +107,11 @@ fp8_status set_prefill_attr() {
              : FP8_ERR_CUDA;
 }
 
-template <int BNT, int STAGES, int KBS, bool FUSED = false>
+template <int BNT, int STAGES, int KBS>
 fp8_status set_decode_attr() {
-  using C = DecodeCfg<BNT, STAGES, KBS>;
-  return cudaFuncSetAttribute(gemm_decode_kernel<BNT, STAGES, KBS, FUSED>,
+  return cudaFuncSetAttribute(gemm_decode_kernel<BNT, STAGES, KBS>,
                               cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              static_cast<int>(FUSED ? C::kSmemFused : C::kSmemSplit)) ==
+                              static_cast<int>(DecodeCfg<BNT, STAGES, KBS>::kSmemSplit)) ==
                  cudaSuccess
              ? FP8_OK
              : FP8_ERR_CUDA;
@@ -167,7 +166,6 @@ fp8_status device_info(DeviceInfo** out) {
       d.pair_clusters = n;
     }
     st = st != FP8_OK ? st : set_decode_attr<16, 3, 2>();
-    st = st != FP8_OK ? st : set_decode_attr<16, 3, 2, true>();
     st = st != FP8_OK ? st : set_decode_attr<32, 4, 1>();
     st = st != FP8_OK ? st : set_decode_attr<32, 3, 2>();
     st = st != FP8_OK ? st : set_decode_attr<64, 4, 1>();
@@ -338,25 +336,18 @@ int decode_splits(const DeviceInfo& dev, int N, int K, int kbs) {
   return splits;
 }
 
-template <int BNT, int ST, int KBS, bool FUSED = false>
+template <int BNT, int ST, int KBS>
 fp8_status launch_decode_t(const DeviceInfo& dev, const uint8_t* x8, const float* s_tok,
                            const uint8_t* w8, const float* s_ch, int M, int N, int K, uint16_t* y,
-                           cudaStream_t stream, bool pdl, int force_splits = 0,
-                           FusedX fx = FusedX{}) {
+                           cudaStream_t stream, bool pdl, int force_splits = 0) {
   using C = DecodeCfg<BNT, ST, KBS>;
   CUtensorMap tmW, tmX;
-  if (!make_tmap_u8(&tmW, w8, N, K, kBM)) return FP8_ERR_CUDA;
-  if (FUSED) {
-    tmX = tmW;  // unused: the kernel quantizes the tokens itself
-  } else if (!make_tmap_u8(&tmX, x8, M, K, BNT)) {
+  if (!make_tmap_u8(&tmW, w8, N, K, kBM) || !make_tmap_u8(&tmX, x8, M, K, BNT))
     return FP8_ERR_CUDA;
-  }
   const int tiles = (N + kBM - 1) / kBM;
   const int num_steps = (K + kBK * KBS - 1) / (kBK * KBS);
   int splits = decode_splits(dev, N, K, KBS);
   if (force_splits > 0) splits = force_splits;
-  if (FUSED && (splits != 1 || int64_t(M) * K * 2 > kFusedXBytes || M > BNT))
-    return FP8_ERR_INVALID_ARG;
   const int steps_per_split = (num_steps + splits - 1) / splits;
   CUtensorMap tmY;
   std::memset(&tmY, 0, sizeof(tmY));
@@ -365,7 +356,7 @@ fp8_status launch_decode_t(const DeviceInfo& dev, const uint8_t* x8, const float
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(tiles * splits);
   cfg.blockDim = dim3(192);
-  cfg.dynamicSmemBytes = FUSED ? C::kSmemFused : splits > 1 ? C::kSmemSplit : C::kSmemSingle;
+  cfg.dynamicSmemBytes = splits > 1 ? C::kSmemSplit : C::kSmemSingle;
   cfg.stream = stream;
   cudaLaunchAttribute attrs[2];
   int na = 0;
@@ -377,8 +368,8 @@ fp8_status launch_decode_t(const DeviceInfo& dev, const uint8_t* x8, const float
   set_pdl(attrs, na, pdl);
   cfg.attrs = attrs;
   cfg.numAttrs = na;
-  if (cudaLaunchKernelEx(&cfg, gemm_decode_kernel<BNT, ST, KBS, FUSED>, tmW, tmX, tmY, s_tok, s_ch,
-                         y, M, N, K, splits, steps_per_split, use_tma_store, fx) != cudaSuccess)
+  if (cudaLaunchKernelEx(&cfg, gemm_decode_kernel<BNT, ST, KBS>, tmW, tmX, tmY, s_tok, s_ch, y, M,
+                         N, K, splits, steps_per_split, use_tma_store) != cudaSuccess)
     return FP8_ERR_CUDA;
   return FP8_OK;
 }
@@ -578,17 +569,10 @@ fp8_status fp8_linear_bf16(const uint16_t* x, const uint8_t* w8, const float* s_
       return FP8_ERR_CUDA;
     return FP8_OK;
   }
-  if (M <= 16 && M * K * 2 <= kFusedXBytes &&
-      decode_splits(*dev, static_cast<int>(N), static_cast<int>(K), 2) == 1) {
-    // A handful of short tokens: quantize them inside the decode GEMM (one launch).
-    FusedX fx;
-    fx.x = x;
-    fx.x8_out = x8;
-    fx.stok_out = s_tok;
-    return launch_decode_t<16, 3, 2, true>(*dev, nullptr, s_tok, w8, s_ch, static_cast<int>(M),
-                                           static_cast<int>(N), static_cast<int>(K), y,
-                                           as_stream(stream), true, 0, fx);
-  }
+  // Two launches: the GEMM is a programmatic dependent of the quantizer, so
+  // its weight stream starts while the quantizer runs. (Quantizing inside the
+  // decode GEMM was measured slower on B200: every CTA must quantize the whole
+  // token block, and staging it costs the second CTA per SM.)
   if (fp8_status st = launch_quant_act(*dev, x, M, K, K, x8, s_tok, as_stream(stream))) return st;
   return launch_linear(*dev, x8, s_tok, w8, s_ch, static_cast<int>(M), static_cast<int>(N),
                        static_cast<int>(K), y, as_stream(stream), true);

@@ -40,7 +40,6 @@
 #include <cstdint>
 
 #include "ptx.cuh"
-#include "quant.cuh"
 
 namespace fp8k {
 
@@ -532,10 +531,6 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
 }
 
 // ============================================================== decode
-// Largest bf16 token block [M, K] (bytes) the fused-quantization decode GEMM
-// stages in shared memory.
-constexpr int kFusedXBytes = 64 * 1024;
-
 // KBS 128-byte k-blocks per pipeline stage (one TMA box each per operand).
 template <int BNT, int STAGES, int KBS>
 struct DecodeCfg {
@@ -545,46 +540,27 @@ struct DecodeCfg {
   static constexpr int kTmemCols = tmem_cols_for(BNT);
   static constexpr int kPipeBytes = STAGES * kStageBytes;
   static constexpr int kYBytes = BNT * kBM * 2;    // bf16 output tile, reuses the pipeline
-  static constexpr int kBarBytes = 8 * (2 * STAGES + 2) + 16;  // full, empty, tfull, xfull; TMEM base
-  static constexpr int kScaleBytes = (kBM + BNT) * 4 + BNT * 16;  // s_ch, s_tok, token divisors
+  static constexpr int kBarBytes = 8 * (2 * STAGES + 1) + 16;
+  static constexpr int kScaleBytes = (kBM + BNT) * 4;  // s_ch of the tile, s_tok
   static constexpr int kRedBytes = BNT * kBM * 4;  // fp32 partials [rank][token][row in slice]
   static constexpr int kFixed = kPipeBytes + kBarBytes + kScaleBytes;
   // Shared memory without (single) and with (split) the reduction buffer.
   static constexpr size_t kSmemSingle = 1024 + static_cast<size_t>(kFixed);
   static constexpr size_t kSmemSplit = kSmemSingle + kRedBytes;
-  // Fused prologue: the raw bf16 tokens sit after the fixed layout.
-  static constexpr size_t kSmemFused = kSmemSingle + kFusedXBytes;
-  static_assert(kFixed % 16 == 0, "bulk-copy destination alignment");
   static_assert(BNT % 16 == 0 && BNT >= 16 && BNT <= 256, "BNT");
   static_assert(kXBytes % 1024 == 0, "token tile must keep 1024-byte alignment");
   static_assert(kYBytes <= kPipeBytes, "output tile must fit in the pipeline buffers");
 };
 
-// Activation-quantization prologue fused into the decode GEMM (FUSED, no K
-// split): the four epilogue warps, idle during the main loop, quantize the
-// bf16 tokens themselves. They first take each token row's amax (the same
-// integer max of |bf16| patterns, scale and row divisor as the activation
-// quantizer, so the codes are bit-identical), then for every pipeline stage
-// write that stage's token tile - 16-byte chunks of codes at their 128-byte
-// swizzle positions, rows >= M left zero - and arrive on the stage's full
-// barrier next to the weight TMA. Block 0 also stores the codes and scales to
-// x8_out / stok_out, which then hold exactly what the separate quantizer
-// would have written.
-struct FusedX {
-  const uint16_t* x;   // [M, K] bf16
-  uint8_t* x8_out;     // [M, K] codes (written by block 0)
-  float* stok_out;     // [M] scales (written by block 0)
-};
-
 // y is written either by one TMA store per output tile (tmY valid, N % 8 == 0;
 // its box is {rows written per CTA, BNT}) or element by element.
-template <int BNT, int STAGES, int KBS, bool FUSED = false>
+template <int BNT, int STAGES, int KBS>
 __global__ void __launch_bounds__(192)
     gemm_decode_kernel(const __grid_constant__ CUtensorMap tmW,
                        const __grid_constant__ CUtensorMap tmX,
                        const __grid_constant__ CUtensorMap tmY, const float* __restrict__ s_tok,
                        const float* __restrict__ s_ch, uint16_t* __restrict__ y, int M, int N,
-                       int K, int splits, int kb_per_split, int use_tma_store, const FusedX fx) {
+                       int K, int splits, int kb_per_split, int use_tma_store) {
   using C = DecodeCfg<BNT, STAGES, KBS>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
@@ -592,15 +568,13 @@ __global__ void __launch_bounds__(192)
   uint8_t* sX = smem + STAGES * KBS * C::kWBytes;       // STAGES x KBS token boxes
   uint16_t* ytile = reinterpret_cast<uint16_t*>(smem);  // after the MMAs: bf16 [token][row]
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kPipeBytes);
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 2);
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 1);
   float* sch_s = reinterpret_cast<float*>(smem + C::kPipeBytes + C::kBarBytes);
   float* stok_s = sch_s + kBM;
   float* red = reinterpret_cast<float*>(smem + C::kFixed);  // split only
-  const uint8_t* xraw = smem + C::kFixed;                   // fused only: bf16 [M, K]
   const uint32_t full0 = smem_u32(bars);
   const uint32_t empty0 = smem_u32(bars + STAGES);
   const uint32_t tfull = smem_u32(bars + 2 * STAGES);
-  const uint32_t xfull = smem_u32(bars + 2 * STAGES + 1);
 
   const int warp = warp_id(), lane = lane_id();
   const int tile_n = blockIdx.x / splits;
@@ -614,27 +588,22 @@ __global__ void __launch_bounds__(192)
   bool have_acc = st1 > st0;
   const int pre = have_acc ? min(STAGES, st1 - st0) : 0;
 
-  // Fused: the full barrier also waits for the four token-writer warps, and
-  // only the weight boxes arrive by TMA.
-  constexpr uint32_t kFullCount = FUSED ? 5u : 1u;
-  constexpr uint32_t kTmaBytes = FUSED ? KBS * C::kWBytes : C::kStageBytes;
   if (split) cluster_arrive_relaxed();  // this CTA has started (waited on before any DSMEM store)
   if (warp == 0 && lane == 0) {
     for (int s = 0; s < STAGES; ++s) {
-      mbar_init(full0 + 8 * s, kFullCount);
+      mbar_init(full0 + 8 * s, 1);
       mbar_init(empty0 + 8 * s, 1);
     }
     mbar_init(tfull, 1);
-    mbar_init(xfull, 1);
     fence_barrier_init();
     tma_prefetch_desc(&tmW);
-    if (!FUSED) tma_prefetch_desc(&tmX);
+    tma_prefetch_desc(&tmX);
     // The weight stream depends neither on the TMEM allocation nor on a
     // preceding quantizer grid: start the first ring of weight boxes now.
     const uint64_t pol_w = l2_policy_evict_first();
     for (int i = 0; i < pre; ++i) {
       const uint32_t fb = full0 + 8 * i;
-      mbar_arrive_expect_tx(fb, kTmaBytes);
+      mbar_arrive_expect_tx(fb, C::kStageBytes);
 #pragma unroll
       for (int j = 0; j < KBS; ++j)
         tma_load_2d(smem_u32(sW + (i * KBS + j) * C::kWBytes), &tmW, fb,
@@ -651,39 +620,27 @@ __global__ void __launch_bounds__(192)
   const uint32_t tmem_base = *tmem_holder;
 
   if (warp == 0) {
-    if (FUSED && lane == 0) {
-      // The whole token block in one bulk stream (its size is a multiple of 32 bytes).
-      pdl_wait();  // x may come from a preceding grid
-      const uint32_t xbytes = static_cast<uint32_t>(M) * static_cast<uint32_t>(K) * 2u;
-      mbar_arrive_expect_tx(xfull, xbytes);
-      for (uint32_t off = 0; off < xbytes; off += 16384u)
-        bulk_load(smem_u32(xraw + off), reinterpret_cast<const uint8_t*>(fx.x) + off,
-                  min(16384u, xbytes - off), xfull);
-    }
     if (lane == 0 && have_acc) {
       const uint64_t pol_w = l2_policy_evict_first();
       const uint64_t pol_x = l2_policy_evict_last();
-      if (!FUSED) {
-        pdl_wait();  // activations come from a preceding quantizer grid
-        for (int i = 0; i < pre; ++i)
+      pdl_wait();  // activations come from a preceding quantizer grid
+      for (int i = 0; i < pre; ++i)
 #pragma unroll
-          for (int j = 0; j < KBS; ++j)
-            tma_load_2d(smem_u32(sX + (i * KBS + j) * C::kXBytes), &tmX, full0 + 8 * i,
-                        ((st0 + i) * KBS + j) * kBK, 0, pol_x);
-      }
+        for (int j = 0; j < KBS; ++j)
+          tma_load_2d(smem_u32(sX + (i * KBS + j) * C::kXBytes), &tmX, full0 + 8 * i,
+                      ((st0 + i) * KBS + j) * kBK, 0, pol_x);
       int stage = pre % STAGES;
       uint32_t phase = pre == STAGES ? 1u : 0u;
       for (int st = st0 + pre; st < st1; ++st) {
         if (!mbar_wait(empty0 + 8 * stage, phase ^ 1)) break;
         const uint32_t fb = full0 + 8 * stage;
-        mbar_arrive_expect_tx(fb, kTmaBytes);
+        mbar_arrive_expect_tx(fb, C::kStageBytes);
 #pragma unroll
         for (int j = 0; j < KBS; ++j) {
           tma_load_2d(smem_u32(sW + (stage * KBS + j) * C::kWBytes), &tmW, fb, (st * KBS + j) * kBK,
                       tile_n * kBM, pol_w);
-          if (!FUSED)
-            tma_load_2d(smem_u32(sX + (stage * KBS + j) * C::kXBytes), &tmX, fb,
-                        (st * KBS + j) * kBK, 0, pol_x);
+          tma_load_2d(smem_u32(sX + (stage * KBS + j) * C::kXBytes), &tmX, fb, (st * KBS + j) * kBK,
+                      0, pol_x);
         }
         if (++stage == STAGES) { stage = 0; phase ^= 1; }
       }
@@ -715,120 +672,12 @@ __global__ void __launch_bounds__(192)
     const int et = threadIdx.x - 64;                 // 0..127
     const int quad = warp & 3;
     const int ch = quad * 32 + lane;                 // channel within the tile (TMEM lane)
-    if constexpr (FUSED) {
-      // ---- token-tile producer (see FusedX) --------------------------------
-      pdl_wait();  // x8_out / stok_out may still be read by a preceding grid
-      // Rows >= M of every stage's token tile stay zero for the whole kernel.
-      for (int i = et; i < STAGES * KBS * C::kXBytes / 16; i += 128) {
-        const int rr = (i * 16 % C::kXBytes) / kBK;
-        if (rr >= M) reinterpret_cast<uint4*>(sX)[i] = make_uint4(0, 0, 0, 0);
-      }
-      uint32_t* smax = reinterpret_cast<uint32_t*>(stok_s);  // amax bits, then scales
-      RowDivisor* dv_s = reinterpret_cast<RowDivisor*>(stok_s + BNT);
-      if (et < BNT) smax[et] = 0u;
-      named_bar_sync(1, 128);
-      const bool have_x = mbar_wait(xfull, 0);
-      if (have_x) {
-        // Row amax over the staged [M, K] (K % 16 == 0): a thread's 16-byte
-        // vectors grow in index, so its row changes rarely and each run of one
-        // row is folded into the row's shared max with one atomic.
-        const uint32_t nvec = static_cast<uint32_t>(K) / 8u;
-        const uint32_t total = static_cast<uint32_t>(M) * nvec;
-        const uint4* xv = reinterpret_cast<const uint4*>(xraw);
-        int cur_r = -1;
-        uint32_t cur = 0;
-#pragma unroll 4
-        for (uint32_t idx = et; idx < total; idx += 128u) {
-          const uint4 u = xv[idx];
-          const int r = static_cast<int>(idx / nvec);
-          if (r != cur_r) {
-            if (cur_r >= 0) atomicMax(smax + cur_r, cur);
-            cur_r = r;
-            cur = 0;
-          }
-          uint32_t m = __vmaxu2(u.x & 0x7FFF7FFFu, u.y & 0x7FFF7FFFu);
-          m = __vmaxu2(m, __vmaxu2(u.z & 0x7FFF7FFFu, u.w & 0x7FFF7FFFu));
-          cur = max(cur, max(m & 0xFFFFu, m >> 16));
-        }
-        if (cur_r >= 0) atomicMax(smax + cur_r, cur);
-      }
-      named_bar_sync(1, 128);
-      if (et < BNT) {
-        // scale and divisor of token row et, as the activation quantizer forms them
-        const uint32_t amax_bits = et < M ? smax[et] : 0u;
-        const float amax = __uint_as_float(amax_bits << 16);
-        const float sv = et < M ? __fdiv_rn(amax, kE4M3Max) : 0.0f;
-        if (et < M) {
-          if (amax_bits >= 0x7F80u) report(FP8_DEV_NONFINITE);
-          dv_s[et] = make_divisor(sv, amax);
-          if (blockIdx.x == 0 && have_x) fx.stok_out[et] = sv;
-        }
-        stok_s[et] = sv;
-      }
-      named_bar_sync(1, 128);
-      // Stage fill: one 16-byte chunk = 16 consecutive k of one token row; a
-      // thread owns chunks et and et + 128 of every stage. A stage's codes are
-      // formed before waiting for its slot to drain.
-      constexpr int kCPS = KBS * (kBK / 16);          // chunks per token row per stage
-      constexpr int kPer = (BNT * kCPS + 127) / 128;  // chunk slots per thread
-      const int nrc = M * kCPS;
-      int stage = 0;
-      uint32_t phase = 0;
-      for (int st = st0; have_x && st < st1; ++st) {
-        uint4 code[kPer];
-#pragma unroll
-        for (int p = 0; p < kPer; ++p) {
-          const int c = et + 128 * p;
-          code[p] = make_uint4(0, 0, 0, 0);
-          const int r = c / kCPS, rem = c % kCPS;
-          const int k0 = (st * KBS + rem / (kBK / 16)) * kBK + (rem % (kBK / 16)) * 16;
-          if (c < nrc && k0 < K) {
-            const float sv = stok_s[r];
-            if (sv != 0.0f) {
-              const RowDivisor dv = dv_s[r];
-              const uint4* src = reinterpret_cast<const uint4*>(xraw + (r * K + k0) * 2);
-              const uint4 a = src[0], b = src[1];
-              const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
-              float f[16];
-#pragma unroll
-              for (int i = 0; i < 8; ++i) {
-                f[2 * i] = div_rn(dv, __uint_as_float(w[i] << 16));
-                f[2 * i + 1] = div_rn(dv, __uint_as_float(w[i] & 0xFFFF0000u));
-              }
-              code[p] = make_uint4(pack4_e4m3(f[0], f[1], f[2], f[3]),
-                                   pack4_e4m3(f[4], f[5], f[6], f[7]),
-                                   pack4_e4m3(f[8], f[9], f[10], f[11]),
-                                   pack4_e4m3(f[12], f[13], f[14], f[15]));
-            }
-            if (blockIdx.x == 0)
-              *reinterpret_cast<uint4*>(fx.x8_out + static_cast<int64_t>(r) * K + k0) = code[p];
-          }
-        }
-        if (st - st0 >= STAGES && !mbar_wait(empty0 + 8 * stage, phase ^ 1)) break;
-#pragma unroll
-        for (int p = 0; p < kPer; ++p) {
-          const int c = et + 128 * p;
-          if (c < nrc) {
-            const int r = c / kCPS, rem = c % kCPS;
-            const int j = rem / (kBK / 16), q = rem % (kBK / 16);
-            uint8_t* tile = sX + (stage * KBS + j) * C::kXBytes;
-            *reinterpret_cast<uint4*>(tile + r * kBK + ((q ^ (r & 7)) * 16)) = code[p];
-          }
-        }
-        fence_proxy_async_shared();  // these generic stores -> visible to the tensor core
-        __syncwarp();
-        if (lane == 0) mbar_arrive(full0 + 8 * stage);
-        if (++stage == STAGES) { stage = 0; phase ^= 1; }
-      }
-    }
     // Stage both scale vectors while the main loop runs.
     {
       const int n = tile_n * kBM + et;
       sch_s[et] = n < N ? __ldg(s_ch + n) : 0.0f;
-      if (!FUSED) {
-        pdl_wait();  // per-token scales come from a preceding quantizer grid
-        if (et < BNT) stok_s[et] = et < M ? s_tok[et] : 0.0f;
-      }
+      pdl_wait();  // per-token scales come from a preceding quantizer grid
+      if (et < BNT) stok_s[et] = et < M ? s_tok[et] : 0.0f;
       named_bar_sync(1, 128);
     }
     if (have_acc && !mbar_wait(tfull, 0)) have_acc = false;

@@ -153,11 +153,9 @@ fp8_status fp8_rowwise_linear(const uint8_t* x8, const float* s_tok, const uint8
 /*
  * fp8_linear_bf16: the whole W8A8 linear from bf16 activations: per-token
  * quantization of x (exactly fp8_quant_act) followed by the row-wise GEMM
- * (exactly fp8_rowwise_linear), bit-identical to calling the two. For up to
- * 16 tokens (when the GEMM needs no K split) the quantization runs inside the
- * decode GEMM's prologue, one launch; otherwise the GEMM is launched as a
- * programmatic dependent of the quantizer, so its prologue and weight stream
- * start while the quantizer runs.
+ * (exactly fp8_rowwise_linear), bit-identical to calling the two. The GEMM
+ * is launched as a programmatic dependent of the quantizer, so its prologue
+ * and weight stream start while the quantizer runs.
  *   x [M, K] bf16 (pitch K); x8 [M, K] uint8 and s_tok [M] float32 are
  *   caller-provided scratch that also receive the quantized activations;
  *   w8, s_ch, y as in fp8_rowwise_linear.

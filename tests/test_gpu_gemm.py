@@ -184,11 +184,10 @@ def test_large_layer_sampled(lib, M):
 @pytest.mark.parametrize("M,N,K", [(1, 8192, 2048), (3, 8192, 2064), (8, 8192, 2048),
                                    (16, 6144, 1024), (1, 21504, 5376), (16, 8192, 2048),
                                    (4, 8192, 8176), (5, 8192, 8176)])
-def test_fused_quant_decode_is_bit_identical(lib, M, N, K):
-    """fp8_linear_bf16 quantizes a handful of short tokens (up to 64 KB of
-    bf16) inside the decode GEMM: its codes and scales equal the oracle's, and
-    y equals the two-kernel path (quantizer, then GEMM) bit for bit. The last
-    case is just over that size and takes the two-kernel path itself."""
+def test_linear_from_bf16_is_bit_identical_to_two_calls(lib, M, N, K):
+    """fp8_linear_bf16 on decode batches: its codes and scales equal the
+    oracle's, and y equals fp8_quant_act followed by fp8_rowwise_linear bit
+    for bit (shapes with a K tail, one-wave and two-wave tile counts)."""
     xb, a, w = _operands(M, N, K, seed=40 + M)
     wd, sd = to_dev(w.codes), to_dev(w.scales)
     x8 = torch.full((M, K), 0x7F, dtype=torch.uint8, device="cuda")
