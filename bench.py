@@ -9,10 +9,22 @@ spans the metric's M = 1..65536) a step is:
   3. the per-token activation quantization and the row-wise FP8 GEMM at
      M = 65536 (64 requests x 1,024 tokens), M = 1 and M = 64,
 
-with every input resident in HBM. The L2 is flushed (a 256 MiB write) before
-each decode-sized GEMM so its weights stream from HBM; the flushes are not
-counted in the step time. Other workloads (``--workload tiny|decode|prefill``)
-measure the other configurations.
+with every input resident in HBM. Decode GEMMs rotate over weight copies that
+together exceed L2 several times, and before each op that would otherwise hit
+in L2 the step flushes it (256 MiB written, then 256 MiB read); the flushes
+are timed separately and not counted in the step time. Other workloads:
+``decode`` (K=2048, N=8192, M = 1/8/64), ``prefill`` (K=4096, N=14336,
+M = 128/1024/8192 with the FNUZ load conversion), ``moe`` (8192 tokens,
+top-8 of 128 experts, hidden 2048, intermediate 704: routing, quantization,
+gather, grouped gate/up GEMM, GeGLU + quantization, grouped down GEMM,
+combine), ``tiny`` (K=256, N=128, M=4) and ``large8k`` (the large layer at
+M=8192, for profiling).
+
+Timing: the step is one CUDA graph replayed K times after W warm-up steps,
+with CUDA events on the launching stream; ops of at least 200 us are timed
+inside the step, shorter ones as the median of 5 replays of a graph of
+back-to-back launches of that op alone. SM clocks and throttle reasons are
+sampled with nvidia-smi during the timed region.
 
 Output: one JSON line (rank 0). ``value`` is GEMM TFLOP/s of the whole step
 (all ranks' FLOPs / max-over-ranks device time); ``kernels`` breaks the step
@@ -269,6 +281,25 @@ def setup_moe(torch, f, wl, seed, dev):
     return L, h, D, [out], cfg
 
 
+def max_over_ranks(vals, world, device):
+    """Element-wise maximum of per-rank float values over all ranks (a
+    float64 all-reduce on ``device``; the identity for one rank)."""
+    if world <= 1:
+        return [float(v) for v in vals]
+    import torch
+    import torch.distributed as dist
+
+    t = torch.tensor([float(v) for v in vals], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(v) for v in t.tolist()]
+
+
+def job_tflops(world, flops_per_rank_step, steps, ms):
+    """Whole-job throughput: every rank does ``flops_per_rank_step`` per step
+    (weak scaling), timed by the slowest rank's ``ms`` for ``steps`` steps."""
+    return world * flops_per_rank_step * steps / (ms * 1e-3) / 1e12
+
+
 def run_ours(args, rank, world, local_rank):
     import torch
     import torch.distributed as dist
@@ -304,28 +335,33 @@ def run_ours(args, rank, world, local_rank):
     assert f.device_status() == 0, "device status set during warm-up"
 
     # ---- each op alone: R back-to-back launches in one CUDA graph, one event
-    # pair around the replay (per-op event nodes would add several us to
-    # us-scale kernels).
-    def time_alone(fn, reps):
+    # pair around each replay (per-op event nodes would add several us to
+    # us-scale kernels); the median of 5 replays, and their spread.
+    def time_alone(fn, reps, trials=5):
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g):
             for r in range(reps):
                 fn(r)
         g.replay()
         torch.cuda.synchronize()
-        a = torch.cuda.Event(enable_timing=True)
-        b = torch.cuda.Event(enable_timing=True)
-        a.record(stream)
-        g.replay()
-        b.record(stream)
-        torch.cuda.synchronize()
+        per = []
+        for _ in range(trials):
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            g.replay()
+            b.record(stream)
+            torch.cuda.synchronize()
+            per.append(a.elapsed_time(b) / reps)
         del g
-        return a.elapsed_time(b) / reps
+        return statistics.median(per), (min(per), max(per))
 
-    alone_ms = []
+    alone_ms, alone_spread = [], []
     for name, fn, fl, by, bound, flushed, nl in step_ops:
         reps = 40 if flushed else 5
-        alone_ms.append(time_alone(fn, reps))
+        med, spread = time_alone(fn, reps)
+        alone_ms.append(med)
+        alone_spread.append(spread)
 
     # ---- the timed steps, replayed from one CUDA graph (the pages' GEMM
     # microbenchmark likewise ran inside a HIP graph; e2e below is eager).
@@ -394,12 +430,10 @@ def run_ours(args, rank, world, local_rank):
     step_ms = total_ms / args.steps
     graph_ms = t_all0.elapsed_time(t_all1)
     if world > 1:
-        t = torch.tensor([total_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+        total_ms = max_over_ranks([total_ms], world, dev)[0]
         step_ms = total_ms / args.steps
     flops_step = sum(o[2] for o in step_ops)
-    value = world * flops_step * args.steps / (total_ms * 1e-3) / 1e12
+    value = job_tflops(world, flops_step, args.steps, total_ms)
     op_ms = [in_step_ms.get(i, alone_ms[i]) for i in range(len(step_ops))]
 
     peaks = load_peaks()
@@ -408,7 +442,9 @@ def run_ours(args, rank, world, local_rank):
     for i, ((name, fn, fl, by, bound, pre, nl), ms) in enumerate(zip(step_ops, op_ms)):
         k = {"op": name, "us": round(ms * 1e3, 2), "gbs": round(by / (ms * 1e-3) / 1e9, 1),
              "tflops": round(fl / (ms * 1e-3) / 1e12, 1), "bound": bound,
-             "timed": "in step" if long_op[i] else "alone, back to back"}
+             "timed": "in step" if long_op[i] else "alone, back to back (median of 5)"}
+        if not long_op[i]:
+            k["us_range"] = [round(alone_spread[i][0] * 1e3, 2), round(alone_spread[i][1] * 1e3, 2)]
         if bound == "tensor":
             k["frac"] = round(k["tflops"] / fp8_sus, 3)
         elif bound == "hbm":
@@ -454,10 +490,8 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.synchronize()
     e2e_ms = ea.elapsed_time(eb)
     if world > 1:
-        t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
-    e2e_val = world * flops_step * e2e_steps / (e2e_ms * 1e-3) / 1e12
+        e2e_ms = max_over_ranks([e2e_ms], world, dev)[0]
+    e2e_val = job_tflops(world, flops_step, e2e_steps, e2e_ms)
     status |= f.device_status()
 
     out = None
