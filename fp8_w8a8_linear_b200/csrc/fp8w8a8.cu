@@ -603,13 +603,8 @@ fp8_status fp8_moe_route(const int32_t* topk_ids, int64_t tokens, int32_t top_k,
     return FP8_ERR_ALIGNMENT;
   DeviceInfo* dev;
   if (fp8_status st = device_info(&dev)) return st;
-  cudaStream_t s = as_stream(stream);
-  moe_count_kernel<<<num_experts, 256, 0, s>>>(topk_ids, n, offsets);
-  if (fp8_status st = last_launch()) return st;
-  if (fp8_status st = launch_pdl(moe_scatter_kernel, dim3(num_experts), dim3(256), s, topk_ids, n,
-                                 static_cast<const int32_t*>(offsets + 1), perm, inv))
-    return st;
-  return launch_pdl(moe_offsets_kernel, dim3(1), dim3(32), s, offsets, static_cast<int>(num_experts));
+  return launch_pdl(moe_route_kernel, dim3(num_experts), dim3(kRouteThreads), as_stream(stream),
+                    topk_ids, n, static_cast<int>(num_experts), perm, inv, offsets);
 }
 
 fp8_status fp8_moe_gather(const uint8_t* x8, const float* s_tok, const int32_t* perm,
@@ -671,7 +666,7 @@ fp8_status fp8_moe_geglu_quant(const uint16_t* gate_up, int64_t M, int64_t inter
 fp8_status fp8_moe_combine(const uint16_t* rows, const int32_t* inv, int64_t tokens,
                            int32_t top_k, int64_t H, const float* weights, uint16_t* out,
                            void* stream) {
-  if (tokens < 0 || top_k < 1 || H < 0) return FP8_ERR_INVALID_ARG;
+  if (tokens < 0 || top_k < 1 || top_k > kCombineMaxK || H < 0) return FP8_ERR_INVALID_ARG;
   if (H % 8 != 0) return FP8_ERR_SHAPE;
   if (tokens == 0 || H == 0) return FP8_OK;
   if (!rows || !inv || !out) return FP8_ERR_INVALID_ARG;

@@ -18,61 +18,114 @@
 namespace fp8k {
 
 // ------------------------------------------------------------------ routing
-// counts[e] (written to offsets[e + 1]) = number of flat entries equal to e.
-__global__ void __launch_bounds__(256) moe_count_kernel(const int32_t* __restrict__ ids,
-                                                         int64_t n, int32_t* __restrict__ offsets) {
-  pdl_launch_dependents();
-  __shared__ int red[8];
-  const int e = blockIdx.x;
-  int c = 0;
-  bool bad = false;
-  for (int64_t i = threadIdx.x; i < n; i += blockDim.x) {
-    const int32_t v = ids[i];
-    c += v == e;
-    bad |= e == 0 && (v < 0 || v >= static_cast<int>(gridDim.x));
-  }
-  if (bad) report(FP8_DEV_BAD_INDEX);
-  c = __reduce_add_sync(0xFFFFFFFFu, c);
-  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = c;
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    int t = 0;
-    for (int w = 0; w < 8; ++w) t += red[w];
-    offsets[e + 1] = t;
-  }
-}
+// One block per expert e over the n = tokens * top_k flat ids:
+//   pass 1: base = #{ids < e}, cnt = #{ids == e}; offsets[e + 1] = base + cnt;
+//   pass 2: the entries equal to e, in index order, go to perm[base ...] and
+//           their positions to inv[]: each thread takes kRouteIds consecutive
+//           ids of a chunk, and a block-wide exclusive scan of the per-thread
+//           match counts keeps the order. The next chunk's ids are loaded
+//           before the current one is scanned.
+// Positions are decided by counts alone (no atomics), so the result is unique.
+// Out-of-range ids are counted in no expert and set FP8_DEV_BAD_INDEX; every
+// position written is still < n.
+constexpr int kRouteThreads = 512;
+constexpr int kRouteIds = 32;                          // ids per thread per chunk
+constexpr int kRouteChunk = kRouteThreads * kRouteIds;
 
-// Block e writes the flat indices of its entries, in index order, to
-// perm[off_e ...] and their positions to inv[]; off_e = sum of counts < e.
-// Each thread takes 8 consecutive entries per 2048-entry chunk; a block-wide
-// exclusive scan of the per-thread match counts keeps the order.
-__global__ void __launch_bounds__(256) moe_scatter_kernel(const int32_t* __restrict__ ids,
-                                                           int64_t n,
-                                                           const int32_t* __restrict__ counts1,
-                                                           int32_t* __restrict__ perm,
-                                                           int32_t* __restrict__ inv) {
+__global__ void __launch_bounds__(kRouteThreads) moe_route_kernel(const int32_t* __restrict__ ids,
+                                                                   int64_t n, int E,
+                                                                   int32_t* __restrict__ perm,
+                                                                   int32_t* __restrict__ inv,
+                                                                   int32_t* __restrict__ offsets) {
   pdl_launch_dependents();
-  pdl_wait();  // counts come from the preceding count grid
-  __shared__ int wsum[8];
-  __shared__ int base_s;
+  pdl_wait();  // the ids may come from a preceding grid
+  constexpr int kWarps = kRouteThreads / 32;
+  __shared__ int wsum[kWarps];
+  __shared__ int wsum2[kWarps];
   const int e = blockIdx.x;
   const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
-  if (tid < 32) {
-    int s = 0;
-    for (int i = tid; i < e; i += 32) s += counts1[i];  // counts1[i] = count of expert i
-    s = __reduce_add_sync(0xFFFFFFFFu, s);
-    if (tid == 0) base_s = s;
+  // 16-byte loads when every int4 lies inside the ids.
+  const bool vec = (reinterpret_cast<uintptr_t>(ids) & 15) == 0 && n % 4 == 0;
+  const int4* ids4 = reinterpret_cast<const int4*>(ids);
+
+  // ---- pass 1
+  int lt = 0, eq = 0;
+  bool bad = false;
+  auto tally = [&](int v) {
+    lt += v < e;
+    eq += v == e;
+    bad |= static_cast<unsigned>(v) >= static_cast<unsigned>(E);
+  };
+  const int64_t nv = vec ? n / 4 : 0;
+  for (int64_t b0 = tid; b0 < nv; b0 += int64_t(kRouteThreads) * 8) {
+    int4 v[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int64_t j = b0 + int64_t(i) * kRouteThreads;
+      v[i] = j < nv ? __ldg(ids4 + j) : make_int4(0, 0, 0, 0);
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      if (b0 + int64_t(i) * kRouteThreads < nv) {
+        tally(v[i].x);
+        tally(v[i].y);
+        tally(v[i].z);
+        tally(v[i].w);
+      }
+    }
+  }
+  for (int64_t i = nv * 4 + tid; i < n; i += kRouteThreads) tally(__ldg(ids + i));
+  if (e == 0 && bad) report(FP8_DEV_BAD_INDEX);
+  lt = __reduce_add_sync(0xFFFFFFFFu, lt);
+  eq = __reduce_add_sync(0xFFFFFFFFu, eq);
+  if (lane == 0) {
+    wsum[w] = lt;
+    wsum2[w] = eq;
   }
   __syncthreads();
-  int base = base_s;
-  for (int64_t c0 = 0; c0 < n; c0 += 2048) {
-    const int64_t i0 = c0 + static_cast<int64_t>(tid) * 8;
+  int base = 0, cnt = 0;
+#pragma unroll
+  for (int k = 0; k < kWarps; ++k) {
+    base += wsum[k];
+    cnt += wsum2[k];
+  }
+  if (tid == 0) {
+    offsets[e + 1] = base + cnt;
+    if (e == 0) offsets[0] = 0;
+  }
+  __syncthreads();  // wsum is reused below
+  if (cnt == 0) return;
+
+  // ---- pass 2
+  int4 cur[kRouteIds / 4], nxt[kRouteIds / 4];
+  auto load = [&](int64_t c0, int4* v) {
+    const int64_t i0 = c0 + int64_t(tid) * kRouteIds;
+#pragma unroll
+    for (int q = 0; q < kRouteIds / 4; ++q) {
+      const int64_t i = i0 + 4 * q;
+      if (vec) {
+        v[q] = i < n ? __ldg(ids4 + i / 4) : make_int4(-1, -1, -1, -1);
+      } else {
+        v[q].x = i < n ? __ldg(ids + i) : -1;
+        v[q].y = i + 1 < n ? __ldg(ids + i + 1) : -1;
+        v[q].z = i + 2 < n ? __ldg(ids + i + 2) : -1;
+        v[q].w = i + 3 < n ? __ldg(ids + i + 3) : -1;
+      }
+    }
+  };
+  load(0, cur);
+  for (int64_t c0 = 0; c0 < n; c0 += kRouteChunk) {
+    if (c0 + kRouteChunk < n) load(c0 + kRouteChunk, nxt);
     uint32_t mask = 0;
 #pragma unroll
-    for (int j = 0; j < 8; ++j)
-      if (i0 + j < n && ids[i0 + j] == e) mask |= 1u << j;
-    const int cnt = __popc(mask);
-    int incl = cnt;
+    for (int q = 0; q < kRouteIds / 4; ++q) {
+      mask |= static_cast<uint32_t>(cur[q].x == e) << (4 * q);
+      mask |= static_cast<uint32_t>(cur[q].y == e) << (4 * q + 1);
+      mask |= static_cast<uint32_t>(cur[q].z == e) << (4 * q + 2);
+      mask |= static_cast<uint32_t>(cur[q].w == e) << (4 * q + 3);
+    }
+    const int c = __popc(mask);
+    int incl = c;
 #pragma unroll
     for (int d = 1; d < 32; d <<= 1) {
       const int v = __shfl_up_sync(0xFFFFFFFFu, incl, d);
@@ -82,12 +135,13 @@ __global__ void __launch_bounds__(256) moe_scatter_kernel(const int32_t* __restr
     __syncthreads();
     int wpre = 0, total = 0;
 #pragma unroll
-    for (int k = 0; k < 8; ++k) {
+    for (int k = 0; k < kWarps; ++k) {
       const int v = wsum[k];
       wpre += k < w ? v : 0;
       total += v;
     }
-    int pos = base + wpre + incl - cnt;
+    int pos = base + wpre + incl - c;
+    const int64_t i0 = c0 + int64_t(tid) * kRouteIds;
     while (mask) {
       const int j = __ffs(mask) - 1;
       mask &= mask - 1;
@@ -96,38 +150,10 @@ __global__ void __launch_bounds__(256) moe_scatter_kernel(const int32_t* __restr
       ++pos;
     }
     base += total;
-    __syncthreads();
-  }
-}
-
-// offsets[0] = 0, offsets[e + 1] = counts[0] + ... + counts[e], in place
-// (offsets[e + 1] holds counts[e] on entry). One warp.
-__global__ void moe_offsets_kernel(int32_t* __restrict__ offsets, int E) {
-  pdl_launch_dependents();
-  pdl_wait();  // counts come from the count grid, and the scatter grid reads them
-  const int lane = threadIdx.x;
-  const int per = (E + 31) / 32;
-  int sum = 0;
-  for (int i = 0; i < per; ++i) {
-    const int e = lane * per + i;
-    if (e < E) sum += offsets[e + 1];
-  }
-  int incl = sum;
+    __syncthreads();  // wsum is rewritten by the next chunk
 #pragma unroll
-  for (int d = 1; d < 32; d <<= 1) {
-    const int v = __shfl_up_sync(0xFFFFFFFFu, incl, d);
-    if (lane >= d) incl += v;
+    for (int q = 0; q < kRouteIds / 4; ++q) cur[q] = nxt[q];
   }
-  int run = incl - sum;
-  for (int i = 0; i < per; ++i) {
-    const int e = lane * per + i;
-    if (e < E) {
-      const int c = offsets[e + 1];
-      run += c;
-      offsets[e + 1] = run;
-    }
-  }
-  if (lane == 0) offsets[0] = 0;
 }
 
 // ------------------------------------------------------------------ gather
@@ -152,10 +178,15 @@ __global__ void __launch_bounds__(256) moe_gather_kernel(const uint8_t* __restri
 }
 
 // ------------------------------------------------------------------ GeGLU + quant
-// gelu_tanh(x) = 0.5 x (1 + tanh(sqrt(2/pi) (x + 0.044715 x^3))) in fp32.
+// gelu_tanh(x) = 0.5 x (1 + tanh(u)), u = sqrt(2/pi) (x + 0.044715 x^3), in
+// fp32 through the identity 0.5 (1 + tanh(u)) = 1 / (1 + exp(-2u)):
+// gelu_tanh(x) = x / (1 + exp(-2u)). For x -> -inf, exp(-2u) overflows to
+// +inf and the quotient is -0 (the limit); for x -> +inf it is x.
 __device__ __forceinline__ float gelu_tanh_f32(float x) {
-  const float inner = 0.7978845608028654f * __fmaf_rn(0.044715f * x, x * x, x);
-  return 0.5f * x * (1.0f + tanhf(inner));
+  constexpr float kA = -1.5957691216057308f;            // -2 sqrt(2/pi)
+  constexpr float kB = -1.5957691216057308f * 0.044715f;
+  const float m2u = x * __fmaf_rn(kB, x * x, kA);       // -2u
+  return __fdividef(x, 1.0f + __expf(m2u));
 }
 
 // Eight bf16 h values (packed) from eight gate and eight up values.
@@ -243,7 +274,11 @@ __global__ void __launch_bounds__(256) moe_geglu_quant_kernel(const uint16_t* __
 // ------------------------------------------------------------------ combine
 // out[t] = sum_{j < k} w[t, j] * rows[inv[t*k + j]] with fp32 products and
 // sums in slot order (w = 1/k when weights is null), rounded once to bf16.
-// One warp per token, 16-byte accesses (H % 8 == 0).
+// One warp per token, 16-byte accesses (H % 8 == 0). The token's k row
+// indices and weights are read once into lanes; for each 16-byte column
+// vector all k rows are loaded before the ordered sum (k <= kCombineMaxK).
+constexpr int kCombineMaxK = 16;
+
 __global__ void __launch_bounds__(256) moe_combine_kernel(const uint16_t* __restrict__ rows,
                                                            const int32_t* __restrict__ inv,
                                                            int64_t T, int top_k, int64_t H,
@@ -255,17 +290,30 @@ __global__ void __launch_bounds__(256) moe_combine_kernel(const uint16_t* __rest
   const int lane = threadIdx.x & 31;
   if (t >= T) return;
   const float wu = __fdiv_rn(1.0f, static_cast<float>(top_k));
-  for (int64_t j = lane; j < H / 8; j += 32) {
-    float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-    for (int s = 0; s < top_k; ++s) {
-      const int64_t r = inv[t * top_k + s];
-      const float w = weights ? weights[t * top_k + s] : wu;
-      const uint4 v = __ldg(reinterpret_cast<const uint4*>(rows + r * H) + j);
-      const uint32_t vw[4] = {v.x, v.y, v.z, v.w};
+  const int r_l = lane < top_k ? inv[t * top_k + lane] : 0;
+  const float w_l = lane < top_k ? (weights ? weights[t * top_k + lane] : wu) : 0.0f;
+  // Warp-uniform trip count: every lane takes part in the shuffles.
+  for (int64_t j0 = 0; j0 < H / 8; j0 += 32) {
+    const int64_t j = j0 + lane;
+    const bool live = j < H / 8;
+    uint4 v[kCombineMaxK];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        acc[2 * i] = __fadd_rn(acc[2 * i], __fmul_rn(w, __uint_as_float(vw[i] << 16)));
-        acc[2 * i + 1] = __fadd_rn(acc[2 * i + 1], __fmul_rn(w, __uint_as_float(vw[i] & 0xFFFF0000u)));
+    for (int s = 0; s < kCombineMaxK; ++s) {
+      const int64_t r = __shfl_sync(0xFFFFFFFFu, r_l, s);
+      if (s < top_k && live) v[s] = __ldg(reinterpret_cast<const uint4*>(rows + r * H) + j);
+    }
+    float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+#pragma unroll
+    for (int s = 0; s < kCombineMaxK; ++s) {
+      const float w = __shfl_sync(0xFFFFFFFFu, w_l, s);
+      if (s < top_k) {
+        const uint32_t vw[4] = {v[s].x, v[s].y, v[s].z, v[s].w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          acc[2 * i] = __fadd_rn(acc[2 * i], __fmul_rn(w, __uint_as_float(vw[i] << 16)));
+          acc[2 * i + 1] =
+              __fadd_rn(acc[2 * i + 1], __fmul_rn(w, __uint_as_float(vw[i] & 0xFFFF0000u)));
+        }
       }
     }
     uint32_t o[4];
@@ -275,7 +323,7 @@ __global__ void __launch_bounds__(256) moe_combine_kernel(const uint16_t* __rest
       asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(acc[2 * i + 1]), "f"(acc[2 * i]));
       o[i] = r;
     }
-    reinterpret_cast<uint4*>(out + t * H)[j] = make_uint4(o[0], o[1], o[2], o[3]);
+    if (live) reinterpret_cast<uint4*>(out + t * H)[j] = make_uint4(o[0], o[1], o[2], o[3]);
   }
 }
 

@@ -190,7 +190,8 @@ fp8_status fp8_cast_e4m3(const float* x, int64_t n, uint8_t* out, void* stream);
  *   offsets [num_experts + 1] int32 out: expert e owns rows offsets[e] ..
  *     offsets[e+1] - 1.
  * Deterministic (no atomics decide positions). 1 <= num_experts <= 1024.
- * Ids out of range set FP8_DEV_BAD_INDEX (their rows are missing).
+ * Ids out of range set FP8_DEV_BAD_INDEX; perm, inv and offsets are then
+ * unspecified (every write stays inside them).
  */
 fp8_status fp8_moe_route(const int32_t* topk_ids, int64_t tokens, int32_t top_k,
                          int32_t num_experts, int32_t* perm, int32_t* inv, int32_t* offsets,
@@ -234,7 +235,7 @@ fp8_status fp8_moe_geglu_quant(const uint16_t* gate_up, int64_t M, int64_t inter
  * fp8_moe_combine: out[t] = sum_{j<top_k} w[t,j] * rows[inv[t*top_k + j]]
  * (fp32 products and sums in slot order, one rounding to bf16); rows
  * [tokens*top_k, H] bf16 in expert order, weights [tokens, top_k] fp32 or
- * NULL for 1/top_k. Requires H % 8 == 0.
+ * NULL for 1/top_k. Requires H % 8 == 0 and 1 <= top_k <= 16.
  */
 fp8_status fp8_moe_combine(const uint16_t* rows, const int32_t* inv, int64_t tokens,
                            int32_t top_k, int64_t H, const float* weights, uint16_t* out,

@@ -55,6 +55,10 @@ def _sig(clib):
     clib.fp8_convert_fnuz.argtypes = [P, P, I, I, P, P, P]
     clib.fp8_cast_e4m3.argtypes = [P, I, P, P]
     clib.fp8_linear_bf16.argtypes = [P, P, P, I, I, I, P, P, P, P]
+    I32 = ctypes.c_int32
+    clib.fp8_moe_route.argtypes = [P, I, I32, I32, P, P, P, P]
+    clib.fp8_moe_combine.argtypes = [P, P, I, I32, I, P, P, P]
+    clib.fp8_moe_gather.argtypes = [P, P, P, I, I, I32, P, P, P]
 
 
 FAKE = 0x10000  # never dereferenced: every case below fails a host check first
@@ -87,3 +91,10 @@ def test_host_checks_return_before_any_launch(clib):
     assert clib.fp8_cast_e4m3(a, -5, a, None) == 1
     assert clib.fp8_cast_e4m3(a + 4, 5, a, None) == 2
     assert clib.fp8_cast_e4m3(a, 0, a, None) == 0
+    # MoE: expert count, top_k limits, alignment, K % 16
+    assert clib.fp8_moe_route(a, 16, 2, 0, a, a, a, None) == 1
+    assert clib.fp8_moe_route(a, 16, 2, 1025, a, a, a, None) == 1
+    assert clib.fp8_moe_route(a + 2, 16, 2, 8, a, a, a, None) == 2
+    assert clib.fp8_moe_combine(a, a, 16, 17, 64, None, a, None) == 1
+    assert clib.fp8_moe_combine(a, a, 16, 0, 64, None, a, None) == 1
+    assert clib.fp8_moe_gather(a, a, a, 32, 24, 2, a, a, None) == 3

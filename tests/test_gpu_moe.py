@@ -24,7 +24,8 @@ def _ids(T, E, k, seed):
 
 
 @pytest.mark.parametrize("T,E,k,seed", [(8192, 128, 8, 4), (1, 4, 2, 1), (100, 1, 1, 2),
-                                        (300, 64, 4, 3), (5000, 1024, 2, 5)])
+                                        (300, 64, 4, 3), (5000, 1024, 2, 5),
+                                        (20001, 96, 3, 8)])   # n % 4 != 0, several id chunks
 def test_route_matches_oracle(lib, T, E, k, seed):
     ids = _ids(T, E, k, seed)
     if T == 300:
@@ -130,8 +131,8 @@ def test_geglu_quant_against_oracle(lib):
     assert same_bits_f32(f32(s_h)[same], q.scales)
 
 
-def test_combine_within_bound(lib):
-    T, E, k, H = 2048, 128, 8, 2048
+@pytest.mark.parametrize("T,E,k,H", [(2048, 128, 8, 2048), (333, 16, 1, 512), (100, 64, 16, 264)])
+def test_combine_within_bound(lib, T, E, k, H):
     ids = _ids(T, E, k, 13)
     perm, inv, off = moe.route_sort(ids, E)
     rows = activations_bf16(T * k, H, seed=13)
