@@ -359,6 +359,10 @@ def run_ours(args, rank, world, local_rank):
     alone_ms, alone_spread = [], []
     for name, fn, fl, by, bound, flushed, nl in step_ops:
         reps = 40 if flushed else 5
+        # a pause first, so that the power state a long preceding op left
+        # behind (clocks lowered under the power cap) has recovered
+        torch.cuda.synchronize()
+        time.sleep(0.3)
         med, spread = time_alone(fn, reps)
         alone_ms.append(med)
         alone_spread.append(spread)

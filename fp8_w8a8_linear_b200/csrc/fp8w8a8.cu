@@ -27,6 +27,7 @@ bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0
 
 struct DeviceInfo {
   int sm_count = 0;
+  int smem_optin = 0;     // largest dynamic shared memory a block may opt into
   int pair_clusters = 0;  // co-resident 2-CTA clusters of the pair GEMM
   bool supported = false;
   bool attrs_set = false;
@@ -107,11 +108,14 @@ fp8_status set_prefill_attr() {
              : FP8_ERR_CUDA;
 }
 
+// Deep-ring variants whose split-K layout would not fit are set up (and
+// launched) without a K split only.
 template <int BNT, int STAGES, int KBS>
-fp8_status set_decode_attr() {
+fp8_status set_decode_attr(int smem_optin) {
+  using C = DecodeCfg<BNT, STAGES, KBS>;
+  const size_t smem = C::kSmemSplit <= static_cast<size_t>(smem_optin) ? C::kSmemSplit : C::kSmemSingle;
   return cudaFuncSetAttribute(gemm_decode_kernel<BNT, STAGES, KBS>,
-                              cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              static_cast<int>(DecodeCfg<BNT, STAGES, KBS>::kSmemSplit)) ==
+                              cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) ==
                  cudaSuccess
              ? FP8_OK
              : FP8_ERR_CUDA;
@@ -140,6 +144,7 @@ fp8_status device_info(DeviceInfo** out) {
     cudaDeviceProp prop;
     if (cudaGetDeviceProperties(&prop, dev) != cudaSuccess) return FP8_ERR_CUDA;
     d.sm_count = prop.multiProcessorCount;
+    d.smem_optin = static_cast<int>(prop.sharedMemPerBlockOptin);
     d.supported = prop.major == 10 && prop.minor == 0;
     if (!d.supported) return FP8_ERR_UNSUPPORTED;
     fp8_status st = FP8_OK;
@@ -165,13 +170,16 @@ fp8_status device_info(DeviceInfo** out) {
         st = FP8_ERR_CUDA;
       d.pair_clusters = n;
     }
-    st = st != FP8_OK ? st : set_decode_attr<16, 3, 2>();
-    st = st != FP8_OK ? st : set_decode_attr<32, 4, 1>();
-    st = st != FP8_OK ? st : set_decode_attr<32, 3, 2>();
-    st = st != FP8_OK ? st : set_decode_attr<64, 4, 1>();
-    st = st != FP8_OK ? st : set_decode_attr<64, 4, 2>();
-    st = st != FP8_OK ? st : set_decode_attr<128, 2, 1>();
-    st = st != FP8_OK ? st : set_decode_attr<128, 4, 1>();
+    const int so = d.smem_optin;
+    st = st != FP8_OK ? st : set_decode_attr<16, 3, 2>(so);
+    st = st != FP8_OK ? st : set_decode_attr<16, 6, 2>(so);
+    st = st != FP8_OK ? st : set_decode_attr<32, 4, 1>(so);
+    st = st != FP8_OK ? st : set_decode_attr<32, 3, 2>(so);
+    st = st != FP8_OK ? st : set_decode_attr<64, 4, 1>(so);
+    st = st != FP8_OK ? st : set_decode_attr<64, 4, 2>(so);
+    st = st != FP8_OK ? st : set_decode_attr<128, 3, 1>(so);
+    st = st != FP8_OK ? st : set_decode_attr<128, 4, 1>(so);
+    st = st != FP8_OK ? st : set_decode_attr<128, 6, 1>(so);
     if (st == FP8_OK &&
         cudaFuncSetAttribute(quant_act_staged_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              kStagedSmemBudget + 1024) != cudaSuccess)
@@ -322,6 +330,23 @@ fp8_status launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, cudaStrea
   return cudaLaunchKernelEx(&cfg, kernel, args...) == cudaSuccess ? FP8_OK : FP8_ERR_CUDA;
 }
 
+// As launch_pdl, with dynamic shared memory.
+template <typename... KArgs, typename... Args>
+fp8_status launch_pdl_smem(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                           cudaStream_t stream, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attrs[1];
+  int na = 0;
+  set_pdl(attrs, na, true);
+  cfg.attrs = attrs;
+  cfg.numAttrs = na;
+  return cudaLaunchKernelEx(&cfg, kernel, args...) == cudaSuccess ? FP8_OK : FP8_ERR_CUDA;
+}
+
 // Number of K splits the decode GEMM uses for N output channels.
 int decode_splits(const DeviceInfo& dev, int N, int K, int kbs) {
   const int tiles = (N + kBM - 1) / kBM;
@@ -348,6 +373,7 @@ fp8_status launch_decode_t(const DeviceInfo& dev, const uint8_t* x8, const float
   const int num_steps = (K + kBK * KBS - 1) / (kBK * KBS);
   int splits = decode_splits(dev, N, K, KBS);
   if (force_splits > 0) splits = force_splits;
+  if (splits > 1 && C::kSmemSplit > static_cast<size_t>(dev.smem_optin)) return FP8_ERR_UNSUPPORTED;
   const int steps_per_split = (num_steps + splits - 1) / splits;
   CUtensorMap tmY;
   std::memset(&tmY, 0, sizeof(tmY));
@@ -380,17 +406,27 @@ fp8_status launch_linear(const DeviceInfo& dev, const uint8_t* x8, const float* 
   // Decode-sized M: swap-AB kernel. Pipeline depth is chosen so that every
   // CTA is resident at once: with more 128-channel tiles than SMs, two CTAs
   // share an SM (<= ~110 KB of stages each), otherwise one CTA gets ~200 KB.
-  const bool one_per_sm = (N + kBM - 1) / kBM <= dev.sm_count;
-  if (M <= 16) return launch_decode_t<16, 3, 2>(dev, x8, s_tok, w8, s_ch, M, N, K, y, stream, pdl);
+  // The deepest rings (most of a CTA's weights requested before it waits for
+  // the preceding grid) are used when there is no K split.
+  const int tiles = (N + kBM - 1) / kBM;
+  const bool one_per_sm = tiles <= dev.sm_count;
+  const bool no_split = 4 * tiles >= dev.sm_count;  // decode_splits() gives 1
+  if (M <= 16)
+    return one_per_sm && no_split
+               ? launch_decode_t<16, 6, 2>(dev, x8, s_tok, w8, s_ch, M, N, K, y, stream, pdl)
+               : launch_decode_t<16, 3, 2>(dev, x8, s_tok, w8, s_ch, M, N, K, y, stream, pdl);
   if (M <= 32)
     return one_per_sm ? launch_decode_t<32, 3, 2>(dev, x8, s_tok, w8, s_ch, M, N, K, y, stream, pdl)
                       : launch_decode_t<32, 4, 1>(dev, x8, s_tok, w8, s_ch, M, N, K, y, stream, pdl);
   if (M <= 64)
     return one_per_sm ? launch_decode_t<64, 4, 2>(dev, x8, s_tok, w8, s_ch, M, N, K, y, stream, pdl)
                       : launch_decode_t<64, 4, 1>(dev, x8, s_tok, w8, s_ch, M, N, K, y, stream, pdl);
-  if (M <= 128)
-    return one_per_sm ? launch_decode_t<128, 4, 1>(dev, x8, s_tok, w8, s_ch, M, N, K, y, stream, pdl)
-                      : launch_decode_t<128, 2, 1>(dev, x8, s_tok, w8, s_ch, M, N, K, y, stream, pdl);
+  if (M <= 128) {
+    if (!one_per_sm)
+      return launch_decode_t<128, 3, 1>(dev, x8, s_tok, w8, s_ch, M, N, K, y, stream, pdl);
+    return no_split ? launch_decode_t<128, 6, 1>(dev, x8, s_tok, w8, s_ch, M, N, K, y, stream, pdl)
+                    : launch_decode_t<128, 4, 1>(dev, x8, s_tok, w8, s_ch, M, N, K, y, stream, pdl);
+  }
   // Prefill: 256 x 256 tiles on CTA pairs when there are at least two row
   // tiles of 256, single-SM 128 x 256 tiles below that.
   if (M >= 512 && dev.pair_clusters > 0)
@@ -399,6 +435,9 @@ fp8_status launch_linear(const DeviceInfo& dev, const uint8_t* x8, const float* 
 }
 
 // ----------------------------------------------------------------- quant plans
+// Every quantizer kernel waits for the preceding grid before it reads x and
+// writes nothing before that, so it is always launched as a programmatic
+// dependent: in a chain of linears it starts while the previous GEMM ends.
 fp8_status launch_quant_act(const DeviceInfo& dev, const uint16_t* x, int64_t M, int64_t K,
                             int64_t ldx, uint8_t* x8, float* s_tok, cudaStream_t stream) {
   const int64_t nvec = K / 8;
@@ -409,26 +448,22 @@ fp8_status launch_quant_act(const DeviceInfo& dev, const uint16_t* x, int64_t M,
     const int warps = static_cast<int>(staged_warps);
     const size_t smem = static_cast<size_t>(warps) * 2 * row_pad + 16 * warps;
     const int64_t blocks = std::min<int64_t>(dev.sm_count, (M + warps - 1) / warps);
-    quant_act_staged_kernel<<<static_cast<unsigned>(blocks), 32 * warps, smem, stream>>>(
-        x, M, K, ldx, x8, s_tok, row_pad);
-    return last_launch();
+    return launch_pdl_smem(quant_act_staged_kernel, dim3(static_cast<unsigned>(blocks)),
+                           dim3(32 * warps), smem, stream, x, M, K, ldx, x8, s_tok, row_pad);
   }
   if (M <= 1024) {
     // Few tokens: a whole block per token row, sized so that the row sits in
     // registers (one memory round trip for the amax, none for the quantize).
     const dim3 grid(static_cast<unsigned>(M));
     if (nvec <= 4 * 256)
-      quant_act_kernel<256, 4><<<grid, 256, 0, stream>>>(x, M, K, ldx, x8, s_tok);
-    else
-      quant_act_kernel<1024, 8, 1024><<<grid, 1024, 0, stream>>>(x, M, K, ldx, x8, s_tok);
-  } else {
-    const dim3 grid(static_cast<unsigned>((M + 7) / 8));
-    if (nvec <= 24 * 32)
-      quant_act_kernel<32, 24><<<grid, 256, 0, stream>>>(x, M, K, ldx, x8, s_tok);
-    else
-      quant_act_kernel<32, 0><<<grid, 256, 0, stream>>>(x, M, K, ldx, x8, s_tok);
+      return launch_pdl(quant_act_kernel<256, 4>, grid, dim3(256), stream, x, M, K, ldx, x8, s_tok);
+    return launch_pdl(quant_act_kernel<1024, 8, 1024>, grid, dim3(1024), stream, x, M, K, ldx, x8,
+                      s_tok);
   }
-  return last_launch();
+  const dim3 grid(static_cast<unsigned>((M + 7) / 8));
+  if (nvec <= 24 * 32)
+    return launch_pdl(quant_act_kernel<32, 24>, grid, dim3(256), stream, x, M, K, ldx, x8, s_tok);
+  return launch_pdl(quant_act_kernel<32, 0>, grid, dim3(256), stream, x, M, K, ldx, x8, s_tok);
 }
 
 bool dims_ok(int64_t v, int64_t lim) { return v >= 0 && v <= lim; }
@@ -552,7 +587,7 @@ fp8_status fp8_rowwise_linear(const uint8_t* x8, const float* s_tok, const uint8
     return FP8_OK;
   }
   return launch_linear(*dev, x8, s_tok, w8, s_ch, static_cast<int>(M), static_cast<int>(N),
-                       static_cast<int>(K), y, as_stream(stream), false);
+                       static_cast<int>(K), y, as_stream(stream), true);
 }
 
 fp8_status fp8_linear_bf16(const uint16_t* x, const uint8_t* w8, const float* s_ch, int64_t M,

@@ -618,6 +618,12 @@ __global__ void __launch_bounds__(192)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
+  // Let the next grid on the stream launch now: in a chain of decode linears
+  // its CTAs take the idle SMs and start their own weight streams while this
+  // one finishes. Signalled only once this CTA holds its TMEM, so a waiting
+  // dependent can never take the columns this CTA still has to allocate. The
+  // dependent touches nothing this grid writes before griddepcontrol.wait.
+  pdl_launch_dependents();
 
   if (warp == 0) {
     if (lane == 0 && have_acc) {

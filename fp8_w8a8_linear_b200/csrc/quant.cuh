@@ -94,6 +94,7 @@ __global__ void __launch_bounds__(BLOCK) quant_act_kernel(const uint16_t* __rest
                                                            uint8_t* __restrict__ x8,
                                                            float* __restrict__ s_tok) {
   pdl_launch_dependents();
+  pdl_wait();  // x may come from the preceding grid (a no-op without programmatic launch)
   __shared__ uint32_t red[BLOCK / 32];
   constexpr int RPB = BLOCK / TPR;  // rows per block
   const int64_t row = static_cast<int64_t>(blockIdx.x) * RPB + threadIdx.x / TPR;
@@ -174,6 +175,7 @@ __global__ void __launch_bounds__(256) quant_act_staged_kernel(const uint16_t* _
                                                                 float* __restrict__ s_tok,
                                                                 uint32_t row_bytes_padded) {
   pdl_launch_dependents();
+  pdl_wait();  // x may come from the preceding grid (a no-op without programmatic launch)
   extern __shared__ __align__(128) uint8_t qsm[];
   const int warps = blockDim.x >> 5;
   const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;

@@ -144,7 +144,18 @@ fp8_status fp8_quant_act(const uint16_t* x, int64_t M, int64_t K, int64_t ldx, u
  * is fixed per shape, so results are bit-reproducible run to run.
  * Requires K % 16 == 0 and K <= 65536; x8, w8, y 16-byte aligned.
  * Runs on tcgen05 tensor cores with TMA-staged tiles and a TMEM accumulator;
- * M <= 64 selects a swap-AB split-K variant bound by the weight stream.
+ * M <= 128 selects a swap-AB variant bound by the weight stream (K split over
+ * a thread-block cluster when there are few 128-channel tiles).
+ *
+ * Launch order (programmatic dependent launch): the GEMM is launched as a
+ * programmatic dependent of the preceding grid on the stream. Before it waits
+ * for that grid it reads only w8 and s_ch, so these must not be written by a
+ * preceding grid that lets dependents launch early
+ * (griddepcontrol.launch_dependents) before it has finished writing them; no
+ * kernel of this library that writes weights does. The decode variant and the
+ * quantizers let the next grid launch early; a grid launched after them with
+ * the programmatic attribute must wait (griddepcontrol.wait) before it reads
+ * y, x8 or s_tok. Grids launched without the attribute are ordered as usual.
  */
 fp8_status fp8_rowwise_linear(const uint8_t* x8, const float* s_tok, const uint8_t* w8,
                               const float* s_ch, int64_t M, int64_t N, int64_t K,
@@ -153,9 +164,10 @@ fp8_status fp8_rowwise_linear(const uint8_t* x8, const float* s_tok, const uint8
 /*
  * fp8_linear_bf16: the whole W8A8 linear from bf16 activations: per-token
  * quantization of x (exactly fp8_quant_act) followed by the row-wise GEMM
- * (exactly fp8_rowwise_linear), bit-identical to calling the two. The GEMM
- * is launched as a programmatic dependent of the quantizer, so its prologue
- * and weight stream start while the quantizer runs.
+ * (exactly fp8_rowwise_linear), bit-identical to calling the two. Both are
+ * launched as programmatic dependents (see fp8_rowwise_linear): the GEMM's
+ * prologue and weight stream start while the quantizer runs, and in a chain
+ * of decode linears the next quantizer and GEMM start while this GEMM ends.
  *   x [M, K] bf16 (pitch K); x8 [M, K] uint8 and s_tok [M] float32 are
  *   caller-provided scratch that also receive the quantized activations;
  *   w8, s_ch, y as in fp8_rowwise_linear.

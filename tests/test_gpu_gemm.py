@@ -55,6 +55,8 @@ GEMM_SHAPES = [
     (1000, 1000, 2000),
     (2048, 2304, 4096),
     (300, 4096, 5376),
+    (5, 6000, 1040),      # one CTA per SM, no split: the deep-ring decode variant
+    (120, 19000, 512),    # more 128-channel tiles than SMs at M = 128
 ]
 
 
