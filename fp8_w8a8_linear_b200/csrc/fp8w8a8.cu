@@ -124,7 +124,11 @@ fp8_status set_decode_attr(int smem_optin) {
 template <int STAGES>
 fp8_status set_pair_attr() {
   return cudaFuncSetAttribute(gemm_pair_kernel<STAGES>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              static_cast<int>(PairCfg<STAGES>::kSmem)) == cudaSuccess
+                              static_cast<int>(PairCfg<STAGES>::kSmem)) == cudaSuccess &&
+                 cudaFuncSetAttribute(gemm_pair_kernel<STAGES, true>,
+                                      cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      static_cast<int>(PairCfg<STAGES>::kSmem + 4 * (kMaxExperts + 1))) ==
+                     cudaSuccess
              ? FP8_OK
              : FP8_ERR_CUDA;
 }
@@ -308,6 +312,45 @@ fp8_status launch_grouped(const DeviceInfo& dev, const uint8_t* x8, const float*
   g.offsets = offsets;
   g.num_experts = E;
   if (cudaLaunchKernelEx(&cfg, gemm_prefill_kernel<BN, ST, true>, tmA, tmB, g) != cudaSuccess)
+    return FP8_ERR_CUDA;
+  return FP8_OK;
+}
+
+// Per-expert GEMM on CTA pairs (256-row pair tiles per expert): persistent
+// grid of the co-resident pairs, tiles decoded on the GPU from offsets.
+fp8_status launch_grouped_pair(const DeviceInfo& dev, const uint8_t* x8, const float* s_rows,
+                               const int32_t* offsets, int E, int M_total, const uint8_t* w8,
+                               const float* s_ch, int N, int K, uint16_t* y, cudaStream_t stream) {
+  CUtensorMap tmA, tmB;
+  if (!make_tmap_u8(&tmA, x8, M_total, K, 128) ||
+      !make_tmap_u8(&tmB, w8, static_cast<uint64_t>(E) * N, K, 128))
+    return FP8_ERR_CUDA;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * dev.pair_clusters);
+  cfg.blockDim = dim3(kPrefillThreads);
+  cfg.dynamicSmemBytes = PairCfg<kPairStages>::kSmem + 4 * (E + 1);
+  cfg.stream = stream;
+  cudaLaunchAttribute attrs[2];
+  int na = 0;
+  attrs[na].id = cudaLaunchAttributeClusterDimension;
+  attrs[na].val.clusterDim.x = 2;
+  attrs[na].val.clusterDim.y = 1;
+  attrs[na].val.clusterDim.z = 1;
+  ++na;
+  set_pdl(attrs, na, true);
+  cfg.attrs = attrs;
+  cfg.numAttrs = na;
+  GemmArgs g = {};
+  g.s_a = s_rows;
+  g.s_b = s_ch;
+  g.y = y;
+  g.M = M_total;
+  g.N = N;
+  g.K = K;
+  g.tiles_n = (N + 255) / 256;
+  g.offsets = offsets;
+  g.num_experts = E;
+  if (cudaLaunchKernelEx(&cfg, gemm_pair_kernel<kPairStages, true>, tmA, tmB, g) != cudaSuccess)
     return FP8_ERR_CUDA;
   return FP8_OK;
 }
@@ -678,6 +721,10 @@ fp8_status fp8_grouped_linear(const uint8_t* x8_rows, const float* s_rows, const
   // 256-column tiles even when N is not a multiple of 256: measured on B200,
   // the wider tile's halved operand traffic per MMA outweighs a partly empty
   // last tile (N = 1408: 245 us vs 265 us with 128-column tiles).
+  if (dev->pair_clusters > 0)
+    return launch_grouped_pair(*dev, x8_rows, s_rows, offsets, num_experts,
+                               static_cast<int>(M_total), w8, s_ch, static_cast<int>(N),
+                               static_cast<int>(K), y, as_stream(stream));
   return launch_grouped<256, kPrefillStages>(*dev, x8_rows, s_rows, offsets, num_experts,
                                              static_cast<int>(M_total), w8, s_ch,
                                              static_cast<int>(N), static_cast<int>(K), y,

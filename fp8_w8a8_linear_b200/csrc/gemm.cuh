@@ -65,6 +65,73 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return r;
 }
 
+// Epilogue store of one 32-row x 32-column bf16 chunk that a warp holds one
+// row per lane (pk = the lane's 64 bytes), through the warp's 2 KB staging
+// buffer: written row per lane, read back so that each global store
+// instruction covers 8 rows x 64 contiguous bytes (instead of 32 rows x 16
+// bytes). The 16-byte pieces of row r sit at piece index q ^ ((r >> 1) & 3),
+// which keeps both the writes and the reads free of bank conflicts. Rows at
+// or past row_end and columns at or past N (N % 8 == 0) are not written.
+constexpr int kStageChunkBytes = 32 * 64;
+// Epilogue staging of a 256-column tile kernel: one chunk per epilogue warp,
+// then the tile's column scales for each of the two accumulators.
+constexpr int kEpiStgBytes = 8 * kStageChunkBytes + 2 * 256 * 4;
+
+__device__ __forceinline__ void store_chunk_coalesced(uint8_t* stg, const uint4 (&pk)[4],
+                                                      uint16_t* __restrict__ y, int64_t row0,
+                                                      int64_t row_end, int N, int n0, int lane) {
+#pragma unroll
+  for (int q = 0; q < 4; ++q)
+    *reinterpret_cast<uint4*>(stg + lane * 64 + ((q ^ ((lane >> 1) & 3)) << 4)) = pk[q];
+  __syncwarp();
+  const int q = lane & 3;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int rr = i * 8 + (lane >> 2);
+    const uint4 v = *reinterpret_cast<const uint4*>(stg + rr * 64 + ((q ^ ((rr >> 1) & 3)) << 4));
+    const int64_t row = row0 + rr;
+    if (row < row_end && n0 + q * 8 < N)
+      *reinterpret_cast<uint4*>(y + row * static_cast<int64_t>(N) + n0 + q * 8) = v;
+  }
+  __syncwarp();  // the buffer is rewritten by the next chunk
+}
+
+// One 32-column chunk of the epilogue: a warp's 32 accumulator rows (r =
+// this lane's row `row`), scaled by s_a of the row and the chunk's 32 column
+// scales (sb_chunk, staged in shared memory), rounded to bf16 and stored -
+// through store_chunk_coalesced when rows are 16-byte storable (warp-uniform
+// vec_ok), else element by element with the scales from global memory.
+__device__ __forceinline__ void epi_chunk(const uint32_t (&r)[32], const float* sb_chunk,
+                                          const float* __restrict__ sb_glob, float sa, bool vec_ok,
+                                          uint8_t* stg, uint16_t* __restrict__ y, int row,
+                                          int64_t row_end, int N, int n0, int lane) {
+  if (n0 >= N) return;
+  if (vec_ok) {
+    uint4 pk[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const float4 b0 = reinterpret_cast<const float4*>(sb_chunk)[2 * q];
+      const float4 b1 = reinterpret_cast<const float4*>(sb_chunk)[2 * q + 1];
+      const float sb[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+      float v[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) v[i] = __fmul_rn(__fmul_rn(__uint_as_float(r[8 * q + i]), sa), sb[i]);
+      pk[q] = make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]),
+                         pack_bf16x2(v[4], v[5]), pack_bf16x2(v[6], v[7]));
+    }
+    store_chunk_coalesced(stg, pk, y, row - lane, row_end, N, n0, lane);
+  } else if (row < row_end) {
+    uint16_t* yrow = y + static_cast<int64_t>(row) * N;
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+      if (n0 + j < N) {
+        const float v = __fmul_rn(__fmul_rn(__uint_as_float(r[j]), sa), __ldg(sb_glob + n0 + j));
+        yrow[n0 + j] = f32_to_bf16_rn(v);
+      }
+    }
+  }
+}
+
 // Tile order: groups of `group_m` row tiles; inside a group, row tiles vary
 // fastest, then column tiles.
 __device__ __forceinline__ void tile_coords(int tile, int tiles_m, int tiles_n, int group_m,
@@ -86,7 +153,9 @@ struct PrefillCfg {
   static constexpr int kStageBytes = kABytes + kBBytes;
   static constexpr int kTmemCols = tmem_cols_for(2 * BN);
   static constexpr int kBarBytes = 8 * (2 * STAGES + 4) + 16;
-  static constexpr size_t kSmem = 1024 + static_cast<size_t>(STAGES) * kStageBytes + kBarBytes;
+  static constexpr int kStgBytes = kEpiStgBytes;  // epilogue staging (chunks, column scales)
+  static constexpr size_t kSmem =
+      1024 + static_cast<size_t>(STAGES) * kStageBytes + kStgBytes + kBarBytes;
   static_assert(BN % 32 == 0 && BN >= 32 && BN <= 256, "BN");
 };
 
@@ -116,9 +185,11 @@ struct Tile {
   int sb_off;   // offset of this tile's expert in s_b
 };
 
-// Tile t of the grouped problem: m-tiles are numbered expert by expert
-// (mt_off[e] = first m-tile of expert e), n-tiles vary fastest.
-__device__ __forceinline__ Tile grouped_tile(const GemmArgs& g, const int* mt_off, int t, int BN) {
+// Tile t of the grouped problem: m-tiles of tile_rows rows are numbered
+// expert by expert (mt_off[e] = first m-tile of expert e), n-tiles vary
+// fastest.
+__device__ __forceinline__ Tile grouped_tile(const GemmArgs& g, const int* mt_off, int t, int BN,
+                                             int tile_rows = kBM) {
   const int gmt = t / g.tiles_n, tn = t - (t / g.tiles_n) * g.tiles_n;
   int lo = 0, hi = g.num_experts;  // find e with mt_off[e] <= gmt < mt_off[e+1]
   while (hi - lo > 1) {
@@ -127,12 +198,42 @@ __device__ __forceinline__ Tile grouped_tile(const GemmArgs& g, const int* mt_of
   }
   const int e = lo;
   Tile T;
-  T.a_row = g.offsets[e] + (gmt - mt_off[e]) * kBM;
+  T.a_row = g.offsets[e] + (gmt - mt_off[e]) * tile_rows;
   T.row_end = g.offsets[e + 1];
   T.b_row = e * g.N + tn * BN;
   T.col0 = tn * BN;
   T.sb_off = e * g.N;
   return T;
+}
+
+// mt_off[e] = number of tile_rows-row m-tiles of experts 0..e-1 (mt_off[E]
+// = total), from the row offsets; one warp. The offsets may come from a
+// preceding routing grid, so the warp waits for it first.
+__device__ __forceinline__ void grouped_prefix(const GemmArgs& g, int* mt_off, int tile_rows,
+                                               int lane) {
+  pdl_wait();
+  const int E = g.num_experts;
+  const int per = (E + 31) / 32;
+  int sum = 0;
+  for (int i = 0; i < per; ++i) {
+    const int e = lane * per + i;
+    if (e < E) sum += (g.offsets[e + 1] - g.offsets[e] + tile_rows - 1) / tile_rows;
+  }
+  int incl = sum;
+#pragma unroll
+  for (int d = 1; d < 32; d <<= 1) {
+    const int v = __shfl_up_sync(0xFFFFFFFFu, incl, d);
+    if (lane >= d) incl += v;
+  }
+  int run = incl - sum;
+  for (int i = 0; i < per; ++i) {
+    const int e = lane * per + i;
+    if (e < E) {
+      mt_off[e] = run;
+      run += (g.offsets[e + 1] - g.offsets[e] + tile_rows - 1) / tile_rows;
+    }
+  }
+  if (lane == 31) mt_off[E] = incl;
 }
 
 __device__ __forceinline__ Tile dense_tile(const GemmArgs& g, int t, int BN) {
@@ -161,7 +262,8 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
   uint8_t* smem = align1024(smem_raw);
   uint8_t* sA = smem;
   uint8_t* sB = smem + STAGES * C::kABytes;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sB + STAGES * C::kBBytes);
+  uint8_t* stg_all = sB + STAGES * C::kBBytes;  // epilogue staging
+  uint64_t* bars = reinterpret_cast<uint64_t*>(stg_all + C::kStgBytes);
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 4);
   // grouped: E+1 ints after the barriers and the TMEM holder (the launch adds
   // 4 * (E + 1) bytes of dynamic shared memory for them)
@@ -192,33 +294,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     tmem_relinquish();
   }
   if constexpr (GROUPED) {
-    // m-tile prefix over experts: warp 2 scans ceil(rows_e / 128); the row
-    // offsets may come from a preceding routing grid.
-    if (warp == 2) {
-      pdl_wait();
-      const int E = g.num_experts;
-      const int per = (E + 31) / 32;
-      int sum = 0;
-      for (int i = 0; i < per; ++i) {
-        const int e = lane * per + i;
-        if (e < E) sum += (g.offsets[e + 1] - g.offsets[e] + kBM - 1) / kBM;
-      }
-      int incl = sum;
-#pragma unroll
-      for (int d = 1; d < 32; d <<= 1) {
-        const int v = __shfl_up_sync(0xFFFFFFFFu, incl, d);
-        if (lane >= d) incl += v;
-      }
-      int run = incl - sum;
-      for (int i = 0; i < per; ++i) {
-        const int e = lane * per + i;
-        if (e < E) {
-          mt_off[e] = run;
-          run += (g.offsets[e + 1] - g.offsets[e] + kBM - 1) / kBM;
-        }
-      }
-      if (lane == 31) mt_off[E] = incl;
-    }
+    if (warp == 2) grouped_prefix(g, mt_off, kBM, lane);  // m-tiles of 128 rows
   }
   tc_fence_before();
   __syncthreads();
@@ -279,53 +355,40 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     // and warps w and w+4 share a quadrant, splitting its column chunks.
     const int quad = warp & 3;
     const int half = (warp - 2) >> 2;
+    uint8_t* stg = stg_all + (warp - 2) * kStageChunkBytes;  // this warp's staging chunk
+    float* sb_tile = reinterpret_cast<float*>(stg_all + 8 * kStageChunkBytes);  // [2][256]
     const int N = g.N;
-    const bool vec_ok = (N % 8) == 0;
+    // 16-byte stores of y rows and 16-byte loads of the column scales
+    const bool vec_ok = (N % 8) == 0 && (reinterpret_cast<uintptr_t>(g.s_b) & 15) == 0;
     int acc = 0;
     uint32_t acc_phase = 0;
     bool waited = false;
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
       const Tile T = tile_of(tile);
-      if (!mbar_wait(tfull0 + 8 * acc, acc_phase)) break;
+      {
+        // The tile's column scales into this accumulator's buffer, one per
+        // epilogue thread (weight-side data, read before the tile is done;
+        // every warp left the buffer's previous tile before the last barrier).
+        const int col = T.col0 + (threadIdx.x - 64);
+        sb_tile[acc * 256 + (threadIdx.x - 64)] = col < N ? __ldg(g.s_b + T.sb_off + col) : 0.0f;
+      }
+      const bool got = mbar_wait(tfull0 + 8 * acc, acc_phase);
+      // all epilogue warps: scales visible; leave together if any wait failed
+      if (named_bar_or(2, 32 * kEpiWarps, !got)) break;
       tc_fence_after();
       if (!waited) { pdl_wait(); waited = true; }
       const int row = T.a_row + quad * 32 + lane;
-      const bool row_ok = row < T.row_end;
-      const float sa = row_ok ? __ldg(g.s_a + row) : 0.0f;
-      uint16_t* yrow = g.y + static_cast<int64_t>(row) * N;
+      const float sa = row < T.row_end ? __ldg(g.s_a + row) : 0.0f;
       const float* sb_base = g.s_b + T.sb_off;
       const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + acc * BN;
+      constexpr int kCh = BN / 64;  // 32-column chunks per warp
 #pragma unroll 1
-      for (int c = half * (BN / 64); c < (half + 1) * (BN / 64); ++c) {
+      for (int c = half * kCh; c < (half + 1) * kCh; ++c) {
         uint32_t r[32];
         tmem_ld32(t_row + c * 32, r);
         tmem_ld_wait();
-        const int n0 = T.col0 + c * 32;
-        if (row_ok && n0 < N) {
-          if (vec_ok && n0 + 32 <= N) {
-            const float4* sb4 = reinterpret_cast<const float4*>(sb_base + n0);
-            uint4* dst = reinterpret_cast<uint4*>(yrow + n0);
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              const float4 b0 = __ldg(sb4 + 2 * q), b1 = __ldg(sb4 + 2 * q + 1);
-              const float sb[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
-              float v[8];
-#pragma unroll
-              for (int i = 0; i < 8; ++i)
-                v[i] = __fmul_rn(__fmul_rn(__uint_as_float(r[8 * q + i]), sa), sb[i]);
-              dst[q] = make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]),
-                                  pack_bf16x2(v[4], v[5]), pack_bf16x2(v[6], v[7]));
-            }
-          } else {
-#pragma unroll
-            for (int j = 0; j < 32; ++j) {
-              if (n0 + j < N) {
-                const float v = __fmul_rn(__fmul_rn(__uint_as_float(r[j]), sa), __ldg(sb_base + n0 + j));
-                yrow[n0 + j] = f32_to_bf16_rn(v);
-              }
-            }
-          }
-        }
+        epi_chunk(r, sb_tile + acc * 256 + c * 32, sb_base, sa, vec_ok, stg, g.y, row, T.row_end, N,
+                  T.col0 + c * 32, lane);
       }
       tc_fence_before();
       __syncwarp();
@@ -362,10 +425,17 @@ struct PairCfg {
   static constexpr int kStageBytes = kABytes + kBBytes;
   static constexpr int kTmemCols = 512;              // two 256-column accumulators
   static constexpr int kBarBytes = 8 * (2 * STAGES + 4) + 16;
-  static constexpr size_t kSmem = 1024 + static_cast<size_t>(STAGES) * kStageBytes + kBarBytes;
+  static constexpr int kStgBytes = kEpiStgBytes;  // epilogue staging (chunks, column scales)
+  static constexpr size_t kSmem =
+      1024 + static_cast<size_t>(STAGES) * kStageBytes + kStgBytes + kBarBytes;
 };
 
-template <int STAGES>
+//
+// GROUPED: the per-expert GEMM on the same pairs. Expert e's rows are cut
+// into 256-row pair tiles (the last one masked at the expert's end); the
+// tiles are decoded on the GPU from the row offsets as in the single-SM
+// grouped kernel.
+template <int STAGES, bool GROUPED = false>
 __global__ void __launch_bounds__(kPrefillThreads, 1)
     gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                      const GemmArgs g) {
@@ -374,8 +444,11 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
   uint8_t* smem = align1024(smem_raw);
   uint8_t* sA = smem;
   uint8_t* sB = smem + STAGES * C::kABytes;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sB + STAGES * C::kBBytes);
+  uint8_t* stg_all = sB + STAGES * C::kBBytes;  // epilogue staging
+  uint64_t* bars = reinterpret_cast<uint64_t*>(stg_all + C::kStgBytes);
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 4);
+  // grouped: E+1 ints after the barriers (the launch adds 4 * (E + 1) bytes)
+  int* mt_off = reinterpret_cast<int*>(reinterpret_cast<uint8_t*>(bars) + C::kBarBytes);
   const uint32_t full0 = smem_u32(bars);
   const uint32_t empty0 = smem_u32(bars + STAGES);
   const uint32_t tfull0 = smem_u32(bars + 2 * STAGES);
@@ -385,7 +458,6 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
   const uint32_t rank = cluster_ctarank();        // 0 = leader (issues the MMAs)
   const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
   const int num_kb = (g.K + kBK - 1) / kBK;
-  const int num_tiles = g.tiles_m * g.tiles_n;    // tiles of 256 x 256
 
   if (warp == 0 && lane == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -404,10 +476,31 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     tmem_alloc_pair(smem_u32(tmem_holder), C::kTmemCols);
     tmem_relinquish_pair();
   }
+  if constexpr (GROUPED) {
+    if (warp == 2) grouped_prefix(g, mt_off, 256, lane);  // pair m-tiles of 256 rows
+  }
   tc_fence_before();
   cluster_sync();  // both CTAs' barriers exist before any cross-CTA arrive or load
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
+  // tiles of 256 x 256; the fields of a Tile here are the pair's (row 0 of
+  // the tile, column 0), each CTA adding rank * 128 to its A and B rows
+  const int num_tiles = GROUPED ? mt_off[g.num_experts] * g.tiles_n : g.tiles_m * g.tiles_n;
+  auto tile_of = [&](int t) {
+    if constexpr (GROUPED) {
+      return grouped_tile(g, mt_off, t, C::kBN, 256);
+    } else {
+      int tm, tn;
+      tile_coords(t, g.tiles_m, g.tiles_n, g.group_m, tm, tn);
+      Tile T;
+      T.a_row = tm * 256;
+      T.row_end = g.M;
+      T.b_row = tn * C::kBN;
+      T.col0 = tn * C::kBN;
+      T.sb_off = 0;
+      return T;
+    }
+  };
 
   if (warp == 0) {
     if (lane == 0) {
@@ -416,10 +509,9 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       uint32_t phase = 0;
       bool ok = true;
       for (int tile = pair; ok && tile < num_tiles; tile += npairs) {
-        int tm, tn;
-        tile_coords(tile, g.tiles_m, g.tiles_n, g.group_m, tm, tn);
-        const int a_row = tm * 256 + rank * C::kHalf;
-        const int b_row = tn * C::kBN + rank * C::kHalf;
+        const Tile T = tile_of(tile);
+        const int a_row = T.a_row + rank * C::kHalf;
+        const int b_row = T.b_row + rank * C::kHalf;
         for (int kb = 0; kb < num_kb; ++kb) {
           if (!mbar_wait(empty0 + 8 * stage, phase ^ 1)) { ok = false; break; }
           const uint32_t fb_local = full0 + 8 * stage;
@@ -465,54 +557,41 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     // Epilogue warps 2..9 of each CTA drain that CTA's 128 TMEM lanes.
     const int quad = warp & 3;
     const int half = (warp - 2) >> 2;
+    uint8_t* stg = stg_all + (warp - 2) * kStageChunkBytes;  // this warp's staging chunk
+    float* sb_tile = reinterpret_cast<float*>(stg_all + 8 * kStageChunkBytes);  // [2][256]
     const int N = g.N;
-    const bool vec_ok = (N % 8) == 0;
+    // 16-byte stores of y rows and 16-byte loads of the column scales
+    const bool vec_ok = (N % 8) == 0 && (reinterpret_cast<uintptr_t>(g.s_b) & 15) == 0;
     const uint32_t tempty_leader0 = mapa_shared(tempty0, 0);
     int acc = 0;
     uint32_t acc_phase = 0;
     bool waited = false;
     for (int tile = pair; tile < num_tiles; tile += npairs) {
-      int tm, tn;
-      tile_coords(tile, g.tiles_m, g.tiles_n, g.group_m, tm, tn);
-      if (!mbar_wait(tfull0 + 8 * acc, acc_phase)) break;
+      const Tile T = tile_of(tile);
+      {
+        // The tile's column scales into this accumulator's buffer, one per
+        // epilogue thread (weight-side data, read before the tile is done;
+        // every warp left the buffer's previous tile before the last barrier).
+        const int col = T.col0 + (threadIdx.x - 64);
+        sb_tile[acc * 256 + (threadIdx.x - 64)] = col < N ? __ldg(g.s_b + T.sb_off + col) : 0.0f;
+      }
+      const bool got = mbar_wait(tfull0 + 8 * acc, acc_phase);
+      // all epilogue warps: scales visible; leave together if any wait failed
+      if (named_bar_or(2, 32 * kEpiWarps, !got)) break;
       tc_fence_after();
       if (!waited) { pdl_wait(); waited = true; }
-      const int row = tm * 256 + rank * C::kHalf + quad * 32 + lane;
-      const bool row_ok = row < g.M;
-      const float sa = row_ok ? __ldg(g.s_a + row) : 0.0f;
-      uint16_t* yrow = g.y + static_cast<int64_t>(row) * N;
+      const int row = T.a_row + rank * C::kHalf + quad * 32 + lane;
+      const float sa = row < T.row_end ? __ldg(g.s_a + row) : 0.0f;
+      const float* sb_base = g.s_b + T.sb_off;
       const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + acc * C::kBN;
+      constexpr int kCh = 4;  // 32-column chunks per warp
 #pragma unroll 1
-      for (int c = half * 4; c < half * 4 + 4; ++c) {
+      for (int c = half * kCh; c < (half + 1) * kCh; ++c) {
         uint32_t r[32];
         tmem_ld32(t_row + c * 32, r);
         tmem_ld_wait();
-        const int n0 = tn * C::kBN + c * 32;
-        if (row_ok && n0 < N) {
-          if (vec_ok && n0 + 32 <= N) {
-            const float4* sb4 = reinterpret_cast<const float4*>(g.s_b + n0);
-            uint4* dst = reinterpret_cast<uint4*>(yrow + n0);
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              const float4 b0 = __ldg(sb4 + 2 * q), b1 = __ldg(sb4 + 2 * q + 1);
-              const float sb[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
-              float v[8];
-#pragma unroll
-              for (int i = 0; i < 8; ++i)
-                v[i] = __fmul_rn(__fmul_rn(__uint_as_float(r[8 * q + i]), sa), sb[i]);
-              dst[q] = make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]),
-                                  pack_bf16x2(v[4], v[5]), pack_bf16x2(v[6], v[7]));
-            }
-          } else {
-#pragma unroll
-            for (int j = 0; j < 32; ++j) {
-              if (n0 + j < N) {
-                const float v = __fmul_rn(__fmul_rn(__uint_as_float(r[j]), sa), __ldg(g.s_b + n0 + j));
-                yrow[n0 + j] = f32_to_bf16_rn(v);
-              }
-            }
-          }
-        }
+        epi_chunk(r, sb_tile + acc * 256 + c * 32, sb_base, sa, vec_ok, stg, g.y, row, T.row_end, N,
+                  T.col0 + c * 32, lane);
       }
       tc_fence_before();
       __syncwarp();
