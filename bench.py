@@ -531,9 +531,9 @@ def run_ours(args, rank, world, local_rank):
 # figure is the M=8192 capture of the same K and N scaled by 8 (x8, y and
 # the number of weight re-reads all grow in proportion to M).
 TRAFFIC = {
-    ("large8k", "gemm_prefill[M=8192]"): 855.08e6,
-    ("large", "gemm_prefill[M=65536]"): 8 * 855.08e6,
-    ("moe", "grouped_gate_up"): 663.91e6,
+    ("large8k", "gemm_prefill[M=8192]"): 847.42e6,
+    ("large", "gemm_prefill[M=65536]"): 8 * 847.42e6,
+    ("moe", "grouped_gate_up"): 669.47e6,
 }
 
 
