@@ -78,7 +78,8 @@ bool make_tmap_u8(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols
 // box_cols x box_rows, no swizzle; out-of-range parts of a stored box are
 // not written. Requires cols % 8 == 0 (16-byte pitch).
 bool make_tmap_bf16_store(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols,
-                          uint32_t box_cols, uint32_t box_rows) {
+                          uint32_t box_cols, uint32_t box_rows,
+                          CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_NONE) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
   cuuint64_t dims[2] = {cols, rows};
@@ -87,8 +88,18 @@ bool make_tmap_bf16_store(CUtensorMap* m, const void* base, uint64_t rows, uint6
   cuuint32_t estr[2] = {1, 1};
   std::memset(m, 0, sizeof(*m));
   return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
-            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
-            CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Store map of the prefill epilogues: y [rows, cols] bf16 in 32 x 32 boxes
+// whose 64-byte rows use the 64-byte swizzle of the staging buffers. Sets
+// g.use_tma_store when y can be stored that way (cols % 8 == 0).
+void make_epilogue_store_map(CUtensorMap* m, fp8k::GemmArgs& g, const uint16_t* y, uint64_t rows,
+                             uint64_t cols) {
+  std::memset(m, 0, sizeof(*m));
+  g.use_tma_store = (cols % 8 == 0) && (reinterpret_cast<uintptr_t>(y) & 15) == 0 &&
+                    make_tmap_bf16_store(m, y, rows, cols, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B);
 }
 
 fp8_status last_launch() {
@@ -237,7 +248,9 @@ fp8_status launch_prefill(const DeviceInfo& dev, const uint8_t* x8, const float*
   g.tiles_m = tiles_m;
   g.tiles_n = tiles_n;
   g.group_m = group_m;
-  if (cudaLaunchKernelEx(&cfg, gemm_prefill_kernel<BN, ST, false>, tmA, tmB, g) != cudaSuccess)
+  CUtensorMap tmY;
+  make_epilogue_store_map(&tmY, g, y, M, N);
+  if (cudaLaunchKernelEx(&cfg, gemm_prefill_kernel<BN, ST, false>, tmA, tmB, tmY, g) != cudaSuccess)
     return FP8_ERR_CUDA;
   return FP8_OK;
 }
@@ -277,7 +290,9 @@ fp8_status launch_pair(const DeviceInfo& dev, const uint8_t* x8, const float* s_
   g.tiles_m = tiles_m;
   g.tiles_n = tiles_n;
   g.group_m = std::min(tiles_m, 8);
-  if (cudaLaunchKernelEx(&cfg, gemm_pair_kernel<kPairStages>, tmA, tmB, g) != cudaSuccess)
+  CUtensorMap tmY;
+  make_epilogue_store_map(&tmY, g, y, M, N);
+  if (cudaLaunchKernelEx(&cfg, gemm_pair_kernel<kPairStages>, tmA, tmB, tmY, g) != cudaSuccess)
     return FP8_ERR_CUDA;
   return FP8_OK;
 }
@@ -311,7 +326,9 @@ fp8_status launch_grouped(const DeviceInfo& dev, const uint8_t* x8, const float*
   g.tiles_n = (N + BN - 1) / BN;
   g.offsets = offsets;
   g.num_experts = E;
-  if (cudaLaunchKernelEx(&cfg, gemm_prefill_kernel<BN, ST, true>, tmA, tmB, g) != cudaSuccess)
+  CUtensorMap tmY;
+  make_epilogue_store_map(&tmY, g, y, M_total, N);
+  if (cudaLaunchKernelEx(&cfg, gemm_prefill_kernel<BN, ST, true>, tmA, tmB, tmY, g) != cudaSuccess)
     return FP8_ERR_CUDA;
   return FP8_OK;
 }
@@ -350,7 +367,9 @@ fp8_status launch_grouped_pair(const DeviceInfo& dev, const uint8_t* x8, const f
   g.tiles_n = (N + 255) / 256;
   g.offsets = offsets;
   g.num_experts = E;
-  if (cudaLaunchKernelEx(&cfg, gemm_pair_kernel<kPairStages, true>, tmA, tmB, g) != cudaSuccess)
+  CUtensorMap tmY;
+  make_epilogue_store_map(&tmY, g, y, M_total, N);
+  if (cudaLaunchKernelEx(&cfg, gemm_pair_kernel<kPairStages, true>, tmA, tmB, tmY, g) != cudaSuccess)
     return FP8_ERR_CUDA;
   return FP8_OK;
 }

@@ -101,10 +101,17 @@ __device__ __forceinline__ void store_chunk_coalesced(uint8_t* stg, const uint4 
 // scales (sb_chunk, staged in shared memory), rounded to bf16 and stored -
 // through store_chunk_coalesced when rows are 16-byte storable (warp-uniform
 // vec_ok), else element by element with the scales from global memory.
+//
+// With tma_ok (warp-uniform: a store tensor map over y exists and all 32
+// rows of the chunk belong to the tile's row range) the staged chunk leaves
+// by one TMA store instead (the staging layout is the map's 64-byte swizzle;
+// the map clips columns at N); the buffer is reused only after the previous
+// store from it has read it.
 __device__ __forceinline__ void epi_chunk(const uint32_t (&r)[32], const float* sb_chunk,
                                           const float* __restrict__ sb_glob, float sa, bool vec_ok,
                                           uint8_t* stg, uint16_t* __restrict__ y, int row,
-                                          int64_t row_end, int N, int n0, int lane) {
+                                          int64_t row_end, int N, int n0, int lane,
+                                          const CUtensorMap* tmY, bool tma_ok) {
   if (n0 >= N) return;
   if (vec_ok) {
     uint4 pk[4];
@@ -119,7 +126,21 @@ __device__ __forceinline__ void epi_chunk(const uint32_t (&r)[32], const float* 
       pk[q] = make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]),
                          pack_bf16x2(v[4], v[5]), pack_bf16x2(v[6], v[7]));
     }
-    store_chunk_coalesced(stg, pk, y, row - lane, row_end, N, n0, lane);
+    if (lane == 0) bulk_wait_group_read_all();  // the previous store from stg has read it
+    __syncwarp();
+    if (tma_ok) {
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+        *reinterpret_cast<uint4*>(stg + lane * 64 + ((q ^ ((lane >> 1) & 3)) << 4)) = pk[q];
+      fence_proxy_async_shared();  // generic writes -> visible to the TMA store
+      __syncwarp();
+      if (lane == 0) {
+        tma_store_2d(tmY, smem_u32(stg), n0, row - lane);
+        bulk_commit_group();
+      }
+    } else {
+      store_chunk_coalesced(stg, pk, y, row - lane, row_end, N, n0, lane);
+    }
   } else if (row < row_end) {
     uint16_t* yrow = y + static_cast<int64_t>(row) * N;
 #pragma unroll
@@ -175,6 +196,7 @@ struct GemmArgs {
   int tiles_m, tiles_n, group_m;
   const int* offsets;  // grouped only
   int num_experts;     // grouped only
+  int use_tma_store;   // tmY is a 32 x 32 bf16 store map over y (64-byte swizzle)
 };
 
 struct Tile {
@@ -256,7 +278,8 @@ constexpr int kPrefillThreads = 64 + 32 * kEpiWarps;
 template <int BN, int STAGES, bool GROUPED>
 __global__ void __launch_bounds__(kPrefillThreads, 1)
     gemm_prefill_kernel(const __grid_constant__ CUtensorMap tmA,
-                        const __grid_constant__ CUtensorMap tmB, const GemmArgs g) {
+                        const __grid_constant__ CUtensorMap tmB,
+                        const __grid_constant__ CUtensorMap tmY, const GemmArgs g) {
   using C = PrefillCfg<BN, STAGES>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
@@ -380,6 +403,8 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       const int row = T.a_row + quad * 32 + lane;
       const float sa = row < T.row_end ? __ldg(g.s_a + row) : 0.0f;
       const float* sb_base = g.s_b + T.sb_off;
+      // whole 32-row chunk inside the tile's rows: one TMA store per chunk
+      const bool tma_rows = g.use_tma_store && (row - lane) + 32 <= T.row_end;
       const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + acc * BN;
       constexpr int kCh = BN / 64;  // 32-column chunks per warp
 #pragma unroll 1
@@ -388,13 +413,14 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         tmem_ld32(t_row + c * 32, r);
         tmem_ld_wait();
         epi_chunk(r, sb_tile + acc * 256 + c * 32, sb_base, sa, vec_ok, stg, g.y, row, T.row_end, N,
-                  T.col0 + c * 32, lane);
+                  T.col0 + c * 32, lane, &tmY, tma_rows);
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(tempty0 + 8 * acc);
       if (++acc == 2) { acc = 0; acc_phase ^= 1; }
     }
+    if (lane == 0) bulk_wait_group_all();  // this warp's TMA stores of y are complete
   }
   tc_fence_before();
   __syncthreads();
@@ -438,7 +464,7 @@ struct PairCfg {
 template <int STAGES, bool GROUPED = false>
 __global__ void __launch_bounds__(kPrefillThreads, 1)
     gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                     const GemmArgs g) {
+                     const __grid_constant__ CUtensorMap tmY, const GemmArgs g) {
   using C = PairCfg<STAGES>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
@@ -583,6 +609,8 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       const int row = T.a_row + rank * C::kHalf + quad * 32 + lane;
       const float sa = row < T.row_end ? __ldg(g.s_a + row) : 0.0f;
       const float* sb_base = g.s_b + T.sb_off;
+      // whole 32-row chunk inside the tile's rows: one TMA store per chunk
+      const bool tma_rows = g.use_tma_store && (row - lane) + 32 <= T.row_end;
       const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + acc * C::kBN;
       constexpr int kCh = 4;  // 32-column chunks per warp
 #pragma unroll 1
@@ -591,13 +619,14 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         tmem_ld32(t_row + c * 32, r);
         tmem_ld_wait();
         epi_chunk(r, sb_tile + acc * 256 + c * 32, sb_base, sa, vec_ok, stg, g.y, row, T.row_end, N,
-                  T.col0 + c * 32, lane);
+                  T.col0 + c * 32, lane, &tmY, tma_rows);
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(tempty_leader0 + 8 * acc);
       if (++acc == 2) { acc = 0; acc_phase ^= 1; }
     }
+    if (lane == 0) bulk_wait_group_all();  // this warp's TMA stores of y are complete
   }
   tc_fence_before();
   __syncthreads();

@@ -57,6 +57,9 @@ GEMM_SHAPES = [
     (300, 4096, 5376),
     (5, 6000, 1040),      # one CTA per SM, no split: the deep-ring decode variant
     (120, 19000, 512),    # more 128-channel tiles than SMs at M = 128
+    (200, 1001, 256),     # single-SM prefill, N % 8 != 0: element stores
+    (600, 1003, 512),     # CTA pairs, N % 8 != 0
+    (700, 2056, 384),     # CTA pairs, ragged M and N: TMA-stored and fallback chunks
 ]
 
 
