@@ -54,6 +54,9 @@ _SIGS = {
     "fp8_grouped_linear": ([_P, _P, _P, ctypes.c_int32, _I64, _P, _P, _I64, _I64, _P, _P],
                            ctypes.c_int),
     "fp8_moe_geglu_quant": ([_P, _I64, _I64, _P, _P, _P, _P], ctypes.c_int),
+    "fp8_moe_interleave_gate_up": ([_P, _P, ctypes.c_int32, _I64, _I64, _P, _P, _P], ctypes.c_int),
+    "fp8_grouped_linear_geglu": ([_P, _P, _P, ctypes.c_int32, _I64, _P, _P, _I64, _I64, _P, _P],
+                                 ctypes.c_int),
     "fp8_moe_combine": ([_P, _P, _I64, ctypes.c_int32, _I64, _P, _P, _P], ctypes.c_int),
 }
 for _name, (_args, _ret) in _SIGS.items():
@@ -229,6 +232,40 @@ def grouped_linear(x8_rows: torch.Tensor, s_rows: torch.Tensor, offsets: torch.T
     return y
 
 
+def moe_interleave_gate_up(w8: torch.Tensor, s_ch: torch.Tensor, num_experts: int, inter: int,
+                           w8_il: torch.Tensor | None = None, s_il: torch.Tensor | None = None):
+    """Gate/up weights [E, 2*inter, K] -> the interleaved layout of
+    grouped_linear_geglu: [E, 256*ceil(inter/128), K] and its scales."""
+    E = num_experts
+    K = w8.numel() // (E * 2 * inter)
+    rows = 256 * ((inter + 127) // 128)
+    dev = w8.device
+    w8_il = torch.empty((E * rows, K), dtype=torch.uint8, device=dev) if w8_il is None else w8_il
+    s_il = torch.empty((E * rows,), dtype=torch.float32, device=dev) if s_il is None else s_il
+    _check(_lib.fp8_moe_interleave_gate_up(_dev(w8, torch.uint8, "w8"), _dev(s_ch, torch.float32, "s_ch"),
+                                           E, inter, K, _dev(w8_il, torch.uint8, "w8_il"),
+                                           _dev(s_il, torch.float32, "s_il"), _stream()),
+           "fp8_moe_interleave_gate_up")
+    return w8_il, s_il
+
+
+def grouped_linear_geglu(x8_rows: torch.Tensor, s_rows: torch.Tensor, offsets: torch.Tensor,
+                         w8_il: torch.Tensor, s_il: torch.Tensor, inter: int,
+                         h: torch.Tensor | None = None):
+    """Expert gate/up GEMM with the GeGLU unit in its epilogue: h [M, inter] bf16."""
+    M, K = x8_rows.shape
+    E = offsets.numel() - 1
+    h = torch.empty((M, inter), dtype=torch.bfloat16, device=x8_rows.device) if h is None else h
+    _check(_lib.fp8_grouped_linear_geglu(_dev(x8_rows, torch.uint8, "x8_rows"),
+                                         _dev(s_rows, torch.float32, "s_rows", (M,)),
+                                         _dev(offsets, torch.int32, "offsets"), E, M,
+                                         _dev(w8_il, torch.uint8, "w8_il"),
+                                         _dev(s_il, torch.float32, "s_il"), inter, K,
+                                         _dev(h, torch.bfloat16, "h", (M, inter)), _stream()),
+           "fp8_grouped_linear_geglu")
+    return h
+
+
 def moe_geglu_quant(gate_up: torch.Tensor, inter: int, h8=None, s_h=None, h_out=None):
     M = gate_up.shape[0]
     dev = gate_up.device
@@ -286,5 +323,6 @@ __all__ = [
     "Fp8Error", "raw", "version", "device_supported", "device_status", "repack_qat",
     "convert_fnuz", "quant_act", "rowwise_linear", "linear", "linear_noalloc", "cast_e4m3",
     "moe_route", "moe_gather", "grouped_linear", "moe_geglu_quant", "moe_combine",
+    "moe_interleave_gate_up", "grouped_linear_geglu",
     "DEV_NONFINITE", "DEV_NAN_CODE", "DEV_INEXACT", "DEV_TIMEOUT", "LIB_PATH",
 ]

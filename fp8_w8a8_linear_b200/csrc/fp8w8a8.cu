@@ -139,6 +139,10 @@ fp8_status set_pair_attr() {
                  cudaFuncSetAttribute(gemm_pair_kernel<STAGES, true>,
                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
                                       static_cast<int>(PairCfg<STAGES>::kSmem + 4 * (kMaxExperts + 1))) ==
+                     cudaSuccess &&
+                 cudaFuncSetAttribute(gemm_pair_kernel<STAGES, true, true>,
+                                      cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      static_cast<int>(PairCfg<STAGES>::kSmem + 4 * (kMaxExperts + 1))) ==
                      cudaSuccess
              ? FP8_OK
              : FP8_ERR_CUDA;
@@ -335,9 +339,12 @@ fp8_status launch_grouped(const DeviceInfo& dev, const uint8_t* x8, const float*
 
 // Per-expert GEMM on CTA pairs (256-row pair tiles per expert): persistent
 // grid of the co-resident pairs, tiles decoded on the GPU from offsets.
+// With n_out > 0 the GeGLU epilogue writes h [M_total, n_out] (w8 / s_ch in
+// the interleaved gate/up layout, N = 256 * ceil(n_out / 128) rows per expert).
 fp8_status launch_grouped_pair(const DeviceInfo& dev, const uint8_t* x8, const float* s_rows,
                                const int32_t* offsets, int E, int M_total, const uint8_t* w8,
-                               const float* s_ch, int N, int K, uint16_t* y, cudaStream_t stream) {
+                               const float* s_ch, int N, int K, uint16_t* y, cudaStream_t stream,
+                               int n_out = 0) {
   CUtensorMap tmA, tmB;
   if (!make_tmap_u8(&tmA, x8, M_total, K, 128) ||
       !make_tmap_u8(&tmB, w8, static_cast<uint64_t>(E) * N, K, 128))
@@ -367,10 +374,12 @@ fp8_status launch_grouped_pair(const DeviceInfo& dev, const uint8_t* x8, const f
   g.tiles_n = (N + 255) / 256;
   g.offsets = offsets;
   g.num_experts = E;
+  g.n_out = n_out;
   CUtensorMap tmY;
-  make_epilogue_store_map(&tmY, g, y, M_total, N);
-  if (cudaLaunchKernelEx(&cfg, gemm_pair_kernel<kPairStages, true>, tmA, tmB, tmY, g) != cudaSuccess)
-    return FP8_ERR_CUDA;
+  make_epilogue_store_map(&tmY, g, y, M_total, n_out > 0 ? n_out : N);
+  const auto kernel = n_out > 0 ? gemm_pair_kernel<kPairStages, true, true>
+                                : gemm_pair_kernel<kPairStages, true, false>;
+  if (cudaLaunchKernelEx(&cfg, kernel, tmA, tmB, tmY, g) != cudaSuccess) return FP8_ERR_CUDA;
   return FP8_OK;
 }
 
@@ -506,10 +515,14 @@ fp8_status launch_quant_act(const DeviceInfo& dev, const uint16_t* x, int64_t M,
   const uint32_t row_pad = static_cast<uint32_t>((2 * K + 127) / 128 * 128);
   const int64_t staged_warps = std::min<int64_t>(8, kStagedSmemBudget / (2 * int64_t(row_pad) + 16));
   if (M > 1024 && staged_warps >= 2) {
-    // Large M: warp-per-row pipeline through shared memory, one block per SM.
+    // Large M: warp-per-row pipeline through shared memory; as many blocks per
+    // SM (up to 4) as their row buffers allow, so that short rows still keep
+    // enough rows in flight.
     const int warps = static_cast<int>(staged_warps);
     const size_t smem = static_cast<size_t>(warps) * 2 * row_pad + 16 * warps;
-    const int64_t blocks = std::min<int64_t>(dev.sm_count, (M + warps - 1) / warps);
+    const int64_t per_sm =
+        std::max<int64_t>(1, std::min<int64_t>(4, int64_t(dev.smem_optin) / int64_t(smem + 1024)));
+    const int64_t blocks = std::min<int64_t>(per_sm * dev.sm_count, (M + warps - 1) / warps);
     return launch_pdl_smem(quant_act_staged_kernel, dim3(static_cast<unsigned>(blocks)),
                            dim3(32 * warps), smem, stream, x, M, K, ldx, x8, s_tok, row_pad);
   }
@@ -748,6 +761,53 @@ fp8_status fp8_grouped_linear(const uint8_t* x8_rows, const float* s_rows, const
                                              static_cast<int>(M_total), w8, s_ch,
                                              static_cast<int>(N), static_cast<int>(K), y,
                                              as_stream(stream));
+}
+
+fp8_status fp8_moe_interleave_gate_up(const uint8_t* w8, const float* s_ch, int32_t num_experts,
+                                      int64_t inter, int64_t K, uint8_t* w8_il, float* s_il,
+                                      void* stream) {
+  if (num_experts < 1 || num_experts > kMaxExperts || inter < 1 || !dims_ok(K, 65536))
+    return FP8_ERR_INVALID_ARG;
+  if (K % 16 != 0 || inter % 16 != 0) return FP8_ERR_SHAPE;
+  const int64_t tiles = (inter + 127) / 128;
+  const int64_t rows_out = static_cast<int64_t>(num_experts) * 256 * tiles;
+  if (rows_out >= (int64_t(1) << 31) || static_cast<int64_t>(num_experts) * 2 * inter >= (int64_t(1) << 31))
+    return FP8_ERR_SHAPE;
+  if (!w8 || !s_ch || !w8_il || !s_il) return FP8_ERR_INVALID_ARG;
+  if (!aligned16(w8) || !aligned16(w8_il) || !aligned4(s_ch) || !aligned4(s_il))
+    return FP8_ERR_ALIGNMENT;
+  DeviceInfo* dev;
+  if (fp8_status st = device_info(&dev)) return st;
+  moe_interleave_gate_up_kernel<<<static_cast<unsigned>((rows_out + 7) / 8), 256, 0,
+                                  as_stream(stream)>>>(w8, s_ch, num_experts, inter, K, tiles, w8_il,
+                                                       s_il);
+  return last_launch();
+}
+
+fp8_status fp8_grouped_linear_geglu(const uint8_t* x8_rows, const float* s_rows,
+                                    const int32_t* offsets, int32_t num_experts, int64_t M_total,
+                                    const uint8_t* w8_il, const float* s_il, int64_t inter,
+                                    int64_t K, uint16_t* h, void* stream) {
+  if (num_experts < 1 || num_experts > kMaxExperts || inter < 1) return FP8_ERR_INVALID_ARG;
+  if (inter % 16 != 0) return FP8_ERR_SHAPE;
+  const int64_t n_il = 256 * ((inter + 127) / 128);  // interleaved rows per expert
+  if (fp8_status st = check_linear(x8_rows, s_rows, w8_il, s_il, M_total, n_il, K, h)) return st;
+  if (M_total == 0) return FP8_OK;
+  if (!offsets) return FP8_ERR_INVALID_ARG;
+  if (!aligned4(offsets) || !aligned16(s_il)) return FP8_ERR_ALIGNMENT;
+  if (static_cast<int64_t>(num_experts) * n_il >= (int64_t(1) << 31)) return FP8_ERR_SHAPE;
+  DeviceInfo* dev;
+  if (fp8_status st = device_info(&dev)) return st;
+  if (dev->pair_clusters <= 0) return FP8_ERR_UNSUPPORTED;
+  if (K == 0) {  // gate = up = 0, so h = 0
+    if (cudaMemsetAsync(h, 0, static_cast<size_t>(M_total) * inter * 2, as_stream(stream)) !=
+        cudaSuccess)
+      return FP8_ERR_CUDA;
+    return FP8_OK;
+  }
+  return launch_grouped_pair(*dev, x8_rows, s_rows, offsets, num_experts, static_cast<int>(M_total),
+                             w8_il, s_il, static_cast<int>(n_il), static_cast<int>(K), h,
+                             as_stream(stream), static_cast<int>(inter));
 }
 
 fp8_status fp8_moe_geglu_quant(const uint16_t* gate_up, int64_t M, int64_t inter, uint8_t* h8,

@@ -39,6 +39,7 @@
 
 #include <cstdint>
 
+#include "act.cuh"
 #include "ptx.cuh"
 
 namespace fp8k {
@@ -96,6 +97,33 @@ __device__ __forceinline__ void store_chunk_coalesced(uint8_t* stg, const uint4 
   __syncwarp();  // the buffer is rewritten by the next chunk
 }
 
+// Store of one 32 x 32 bf16 chunk a warp holds one row per lane (pk = the
+// lane's 64 bytes; `row` = this lane's row): one TMA store of the swizzled
+// staging buffer when tma_ok (warp-uniform: the map covers y and all 32 rows
+// belong to the tile's rows; the map clips columns at N), else through
+// store_chunk_coalesced. The buffer is rewritten only after the previous
+// store from it has read it.
+__device__ __forceinline__ void epi_store_chunk(const uint4 (&pk)[4], uint8_t* stg,
+                                                uint16_t* __restrict__ y, int row, int64_t row_end,
+                                                int N, int n0, int lane, const CUtensorMap* tmY,
+                                                bool tma_ok) {
+  if (lane == 0) bulk_wait_group_read_all();  // the previous store from stg has read it
+  __syncwarp();
+  if (tma_ok) {
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+      *reinterpret_cast<uint4*>(stg + lane * 64 + ((q ^ ((lane >> 1) & 3)) << 4)) = pk[q];
+    fence_proxy_async_shared();  // generic writes -> visible to the TMA store
+    __syncwarp();
+    if (lane == 0) {
+      tma_store_2d(tmY, smem_u32(stg), n0, row - lane);
+      bulk_commit_group();
+    }
+  } else {
+    store_chunk_coalesced(stg, pk, y, row - lane, row_end, N, n0, lane);
+  }
+}
+
 // One 32-column chunk of the epilogue: a warp's 32 accumulator rows (r =
 // this lane's row `row`), scaled by s_a of the row and the chunk's 32 column
 // scales (sb_chunk, staged in shared memory), rounded to bf16 and stored -
@@ -126,21 +154,7 @@ __device__ __forceinline__ void epi_chunk(const uint32_t (&r)[32], const float* 
       pk[q] = make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]),
                          pack_bf16x2(v[4], v[5]), pack_bf16x2(v[6], v[7]));
     }
-    if (lane == 0) bulk_wait_group_read_all();  // the previous store from stg has read it
-    __syncwarp();
-    if (tma_ok) {
-#pragma unroll
-      for (int q = 0; q < 4; ++q)
-        *reinterpret_cast<uint4*>(stg + lane * 64 + ((q ^ ((lane >> 1) & 3)) << 4)) = pk[q];
-      fence_proxy_async_shared();  // generic writes -> visible to the TMA store
-      __syncwarp();
-      if (lane == 0) {
-        tma_store_2d(tmY, smem_u32(stg), n0, row - lane);
-        bulk_commit_group();
-      }
-    } else {
-      store_chunk_coalesced(stg, pk, y, row - lane, row_end, N, n0, lane);
-    }
+    epi_store_chunk(pk, stg, y, row, row_end, N, n0, lane, tmY, tma_ok);
   } else if (row < row_end) {
     uint16_t* yrow = y + static_cast<int64_t>(row) * N;
 #pragma unroll
@@ -197,6 +211,7 @@ struct GemmArgs {
   const int* offsets;  // grouped only
   int num_experts;     // grouped only
   int use_tma_store;   // tmY is a 32 x 32 bf16 store map over y (64-byte swizzle)
+  int n_out;           // GeGLU epilogue only: columns of h (the features)
 };
 
 struct Tile {
@@ -461,11 +476,19 @@ struct PairCfg {
 // into 256-row pair tiles (the last one masked at the expert's end); the
 // tiles are decoded on the GPU from the row offsets as in the single-SM
 // grouped kernel.
-template <int STAGES, bool GROUPED = false>
+//
+// GEGLU (grouped only): B holds each expert's gate and up rows interleaved
+// in blocks of 128 (tile tn = gate rows of features 128 tn .. 128 tn + 127,
+// then up rows of the same features), so a tile's accumulator has gate and
+// up of 128 features side by side; the epilogue rounds both to bf16 as the
+// plain GEMM would store them and writes h = bf16(gelu_tanh(gate) * up)
+// [M_total, n_out] instead.
+template <int STAGES, bool GROUPED = false, bool GEGLU = false>
 __global__ void __launch_bounds__(kPrefillThreads, 1)
     gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                      const __grid_constant__ CUtensorMap tmY, const GemmArgs g) {
   using C = PairCfg<STAGES>;
+  static_assert(GROUPED || !GEGLU, "the GeGLU epilogue is for the grouped GEMM");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
   uint8_t* sA = smem;
@@ -612,14 +635,51 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       // whole 32-row chunk inside the tile's rows: one TMA store per chunk
       const bool tma_rows = g.use_tma_store && (row - lane) + 32 <= T.row_end;
       const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + acc * C::kBN;
-      constexpr int kCh = 4;  // 32-column chunks per warp
+      if constexpr (GEGLU) {
+        // accumulator columns 0..127: gate of the tile's 128 features,
+        // 128..255: their up; this warp takes 64 features in two chunks
+        const int f_base = T.col0 >> 1;
 #pragma unroll 1
-      for (int c = half * kCh; c < (half + 1) * kCh; ++c) {
-        uint32_t r[32];
-        tmem_ld32(t_row + c * 32, r);
-        tmem_ld_wait();
-        epi_chunk(r, sb_tile + acc * 256 + c * 32, sb_base, sa, vec_ok, stg, g.y, row, T.row_end, N,
-                  T.col0 + c * 32, lane, &tmY, tma_rows);
+        for (int fc = half * 2; fc < half * 2 + 2; ++fc) {
+          const int f0 = f_base + fc * 32;
+          if (f0 >= g.n_out) continue;  // warp-uniform
+          uint32_t rg[32], ru[32];
+          tmem_ld32(t_row + fc * 32, rg);
+          tmem_ld32(t_row + 128 + fc * 32, ru);
+          tmem_ld_wait();
+          const float* sbg = sb_tile + acc * 256 + fc * 32;
+          const float* sbu = sbg + 128;
+          uint4 pk[4];
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            float hv[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              const int j = 8 * q + i;
+              // gate and up exactly as the plain GEMM stores them in bf16
+              const float gv = __uint_as_float(static_cast<uint32_t>(f32_to_bf16_rn(
+                                   __fmul_rn(__fmul_rn(__uint_as_float(rg[j]), sa), sbg[j])))
+                               << 16);
+              const float uv = __uint_as_float(static_cast<uint32_t>(f32_to_bf16_rn(
+                                   __fmul_rn(__fmul_rn(__uint_as_float(ru[j]), sa), sbu[j])))
+                               << 16);
+              hv[i] = geglu_f32(gv, uv);
+            }
+            pk[q] = make_uint4(pack_bf16x2(hv[0], hv[1]), pack_bf16x2(hv[2], hv[3]),
+                               pack_bf16x2(hv[4], hv[5]), pack_bf16x2(hv[6], hv[7]));
+          }
+          epi_store_chunk(pk, stg, g.y, row, T.row_end, g.n_out, f0, lane, &tmY, tma_rows);
+        }
+      } else {
+        constexpr int kCh = 4;  // 32-column chunks per warp
+#pragma unroll 1
+        for (int c = half * kCh; c < (half + 1) * kCh; ++c) {
+          uint32_t r[32];
+          tmem_ld32(t_row + c * 32, r);
+          tmem_ld_wait();
+          epi_chunk(r, sb_tile + acc * 256 + c * 32, sb_base, sa, vec_ok, stg, g.y, row, T.row_end,
+                    N, T.col0 + c * 32, lane, &tmY, tma_rows);
+        }
       }
       tc_fence_before();
       __syncwarp();

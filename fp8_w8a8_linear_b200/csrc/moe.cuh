@@ -12,6 +12,7 @@
 
 #include <cstdint>
 
+#include "act.cuh"
 #include "ptx.cuh"
 #include "quant.cuh"
 
@@ -156,6 +157,29 @@ __global__ void __launch_bounds__(kRouteThreads) moe_route_kernel(const int32_t*
   }
 }
 
+// ------------------------------------------------------------------ weight layout
+// Gate/up weights of the GeGLU-fused grouped GEMM: per expert, row
+// t*256 + s*128 + j of the output is row s*I + t*128 + j of the input
+// (s = 0 gate, 1 up; features t*128 + j >= I give zero rows with scale 0).
+// One warp per output row, 16-byte copies (K % 16 == 0).
+__global__ void __launch_bounds__(256) moe_interleave_gate_up_kernel(
+    const uint8_t* __restrict__ w8, const float* __restrict__ s_ch, int64_t E, int64_t I, int64_t K,
+    int64_t tiles, uint8_t* __restrict__ w_il, float* __restrict__ s_il) {
+  const int64_t orow = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  const int64_t per = 256 * tiles;
+  if (orow >= E * per) return;
+  const int64_t e = orow / per, r = orow % per;
+  const int64_t t = r / 256, sg = (r % 256) / 128, j = r % 128;
+  const int64_t feat = t * 128 + j;
+  const bool live = feat < I;
+  const int64_t irow = e * 2 * I + sg * I + feat;
+  const uint4* src = reinterpret_cast<const uint4*>(w8 + irow * K);
+  uint4* dst = reinterpret_cast<uint4*>(w_il + orow * K);
+  for (int64_t v = lane; v < K / 16; v += 32) dst[v] = live ? __ldg(src + v) : make_uint4(0, 0, 0, 0);
+  if (lane == 0) s_il[orow] = live ? s_ch[irow] : 0.0f;
+}
+
 // ------------------------------------------------------------------ gather
 // rows_out[i] = x8[perm[i] / top_k], s_out[i] = s_tok[perm[i] / top_k].
 // One warp per row, 16-byte copies (K % 16 == 0).
@@ -178,17 +202,6 @@ __global__ void __launch_bounds__(256) moe_gather_kernel(const uint8_t* __restri
 }
 
 // ------------------------------------------------------------------ GeGLU + quant
-// gelu_tanh(x) = 0.5 x (1 + tanh(u)), u = sqrt(2/pi) (x + 0.044715 x^3), in
-// fp32 through the identity 0.5 (1 + tanh(u)) = 1 / (1 + exp(-2u)):
-// gelu_tanh(x) = x / (1 + exp(-2u)). For x -> -inf, exp(-2u) overflows to
-// +inf and the quotient is -0 (the limit); for x -> +inf it is x.
-__device__ __forceinline__ float gelu_tanh_f32(float x) {
-  constexpr float kA = -1.5957691216057308f;            // -2 sqrt(2/pi)
-  constexpr float kB = -1.5957691216057308f * 0.044715f;
-  const float m2u = x * __fmaf_rn(kB, x * x, kA);       // -2u
-  return __fdividef(x, 1.0f + __expf(m2u));
-}
-
 // Eight bf16 h values (packed) from eight gate and eight up values.
 __device__ __forceinline__ uint4 geglu8(const uint4& g, const uint4& u) {
   const uint32_t gw[4] = {g.x, g.y, g.z, g.w}, uw[4] = {u.x, u.y, u.z, u.w};
@@ -197,7 +210,7 @@ __device__ __forceinline__ uint4 geglu8(const uint4& g, const uint4& u) {
   for (int i = 0; i < 4; ++i) {
     const float g0 = __uint_as_float(gw[i] << 16), g1 = __uint_as_float(gw[i] & 0xFFFF0000u);
     const float u0 = __uint_as_float(uw[i] << 16), u1 = __uint_as_float(uw[i] & 0xFFFF0000u);
-    const float h0 = gelu_tanh_f32(g0) * u0, h1 = gelu_tanh_f32(g1) * u1;
+    const float h0 = geglu_f32(g0, u0), h1 = geglu_f32(g1, u1);
     uint32_t r;
     asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(h1), "f"(h0));
     o[i] = r;

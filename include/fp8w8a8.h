@@ -234,6 +234,40 @@ fp8_status fp8_grouped_linear(const uint8_t* x8_rows, const float* s_rows, const
                               const float* s_ch, int64_t N, int64_t K, uint16_t* y, void* stream);
 
 /*
+ * fp8_moe_interleave_gate_up: the gate/up weights of fp8_grouped_linear_geglu,
+ * a load-time reordering. w8 [num_experts, 2*inter, K] uint8 E4M3 (per
+ * expert the gate rows 0..inter-1, then the up rows) and s_ch
+ * [num_experts, 2*inter] fp32 become w8_il [num_experts, 256*T, K] and s_il
+ * [num_experts, 256*T], T = ceil(inter / 128): row t*256 + s*128 + j of an
+ * expert is its gate (s = 0) or up (s = 1) row of feature t*128 + j; features
+ * >= inter give zero rows with scale 0. Requires K % 16 == 0, inter % 16 ==
+ * 0; 16-byte aligned w8 and w8_il. No counterpart on the pages: a layout for
+ * the fused GeGLU below.
+ */
+fp8_status fp8_moe_interleave_gate_up(const uint8_t* w8, const float* s_ch, int32_t num_experts,
+                                      int64_t inter, int64_t K, uint8_t* w8_il, float* s_il,
+                                      void* stream);
+
+/*
+ * fp8_grouped_linear_geglu: the expert gate/up GEMM with the GeGLU unit in
+ * its epilogue. For each expert e and each of its rows i (offsets as in
+ * fp8_grouped_linear): gate and up are the row-wise scaled FP8 products of
+ * x8_rows[i] with the expert's gate and up rows, each rounded to bf16 exactly
+ * as fp8_grouped_linear stores them, and h [M_total, inter] bf16 receives
+ * bf16(gelu_tanh(gate) * up) - bit for bit what fp8_moe_geglu_quant writes
+ * to h_out from fp8_grouped_linear's output. Quantize h with fp8_quant_act
+ * (the same per-row quantization as fp8_moe_geglu_quant). w8_il / s_il in
+ * the layout of fp8_moe_interleave_gate_up (s_il 16-byte aligned). Requires
+ * inter % 16 == 0, K % 16 == 0; runs on CTA pairs (FP8_ERR_UNSUPPORTED if
+ * the device cannot co-schedule them). No counterpart on the pages beyond
+ * the expert MLP itself (readings as for fp8_moe_geglu_quant).
+ */
+fp8_status fp8_grouped_linear_geglu(const uint8_t* x8_rows, const float* s_rows,
+                                    const int32_t* offsets, int32_t num_experts, int64_t M_total,
+                                    const uint8_t* w8_il, const float* s_il, int64_t inter,
+                                    int64_t K, uint16_t* h, void* stream);
+
+/*
  * fp8_moe_geglu_quant: h = bf16(gelu_tanh(gate) * up) per element of
  * gate_up [M, 2*inter] bf16 (gate in columns 0..inter-1, up after it; fp32
  * arithmetic, one rounding to bf16), then per-row E4M3 quantization of h with

@@ -180,3 +180,50 @@ def test_small_moe_layer_end_to_end(lib):
     rel = np.linalg.norm(out - ref) / np.linalg.norm(ref)
     assert rel < 0.03, rel
     assert lib.device_status() == 0
+
+
+def test_interleave_gate_up_layout(lib):
+    """Row t*256 + s*128 + j of an expert is its gate (s=0) / up (s=1) row of
+    feature t*128 + j; features past inter are zero rows with scale 0."""
+    E, I, K = 3, 176, 96          # 2 feature tiles, the second one partial
+    rng = np.random.default_rng(20)
+    w = rng.integers(0, 0x7F, (E * 2 * I, K), dtype=np.uint8)
+    s = rng.uniform(0.5, 2.0, E * 2 * I).astype(np.float32)
+    w_il, s_il = lib.moe_interleave_gate_up(to_dev(w), to_dev(s), E, I)
+    T = (I + 127) // 128
+    ref_w = np.zeros((E * 256 * T, K), np.uint8)
+    ref_s = np.zeros(E * 256 * T, np.float32)
+    for e in range(E):
+        for t in range(T):
+            for sg in range(2):
+                for j in range(128):
+                    f = t * 128 + j
+                    if f < I:
+                        ref_w[e * 256 * T + t * 256 + sg * 128 + j] = w[e * 2 * I + sg * I + f]
+                        ref_s[e * 256 * T + t * 256 + sg * 128 + j] = s[e * 2 * I + sg * I + f]
+    assert np.array_equal(u8(w_il), ref_w) and same_bits_f32(f32(s_il), ref_s)
+
+
+@pytest.mark.parametrize("T,E,k,I,K", [(8192, 128, 8, 704, 2048), (300, 8, 2, 176, 512),
+                                       (64, 128, 8, 256, 704), (1000, 16, 4, 1408, 256)])
+def test_geglu_epilogue_bit_identical(lib, T, E, k, I, K):
+    """fp8_grouped_linear_geglu gives bit for bit the h that the plain grouped
+    GEMM followed by fp8_moe_geglu_quant gives, and fp8_quant_act of it the
+    same codes and scales."""
+    ids = _ids(T, E, k, 21)
+    perm, inv, off = moe.route_sort(ids, E)
+    xb = activations_bf16(T, K, seed=21, outlier_frac=0.01)
+    a = oracle.quant_act(xb)
+    xs, ss = moe.gather_rows(a.codes, a.scales, perm, k)
+    q4, d = q4_weights(E * 2 * I, K, seed=22)
+    wd, sd = lib.repack_qat(to_dev(q4), to_dev(d))
+    xd, sxd, offd = to_dev(xs), to_dev(ss), to_dev(off)
+    gu = lib.grouped_linear(xd, sxd, offd, wd, sd)
+    h_ref = torch.empty((T * k, I), dtype=torch.bfloat16, device="cuda")
+    h8_ref, sh_ref = lib.moe_geglu_quant(gu, I, h_out=h_ref)
+    w_il, s_il = lib.moe_interleave_gate_up(wd, sd, E, I)
+    h = lib.grouped_linear_geglu(xd, sxd, offd, w_il, s_il, I)
+    assert np.array_equal(bf16_to_np_bits(h), bf16_to_np_bits(h_ref))
+    h8, sh = lib.quant_act(h)
+    assert np.array_equal(u8(h8), u8(h8_ref)) and same_bits_f32(f32(sh), f32(sh_ref))
+    assert lib.device_status() == 0
