@@ -188,11 +188,13 @@ def test_large_layer_sampled(lib, M):
 
 @pytest.mark.parametrize("M,N,K", [(1, 8192, 2048), (3, 8192, 2064), (8, 8192, 2048),
                                    (16, 6144, 1024), (1, 21504, 5376), (16, 8192, 2048),
-                                   (4, 8192, 8176), (5, 8192, 8176)])
+                                   (4, 8192, 8176), (5, 8192, 8176), (4, 8192, 2048),
+                                   (2, 6144, 4096), (1, 1024, 4096)])
 def test_linear_from_bf16_is_bit_identical_to_two_calls(lib, M, N, K):
     """fp8_linear_bf16 on decode batches: its codes and scales equal the
     oracle's, and y equals fp8_quant_act followed by fp8_rowwise_linear bit
-    for bit (shapes with a K tail, one-wave and two-wave tile counts)."""
+    for bit (one- and two-wave tile counts, a K tail, a narrow layer whose K
+    is split)."""
     xb, a, w = _operands(M, N, K, seed=40 + M)
     wd, sd = to_dev(w.codes), to_dev(w.scales)
     x8 = torch.full((M, K), 0x7F, dtype=torch.uint8, device="cuda")
