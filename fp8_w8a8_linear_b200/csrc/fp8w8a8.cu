@@ -204,6 +204,10 @@ fp8_status device_info(DeviceInfo** out) {
                              kStagedSmemBudget + 1024) != cudaSuccess)
       st = FP8_ERR_CUDA;
     if (st == FP8_OK &&
+        cudaFuncSetAttribute(convert_fnuz_staged_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             kStagedSmemBudget + 1024) != cudaSuccess)
+      st = FP8_ERR_CUDA;
+    if (st == FP8_OK &&
         cudaFuncSetAttribute(repack_qat_staged_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              110 * 1024) != cudaSuccess)
       st = FP8_ERR_CUDA;
@@ -619,6 +623,18 @@ fp8_status fp8_convert_fnuz(const uint8_t* w8_fnuz, const float* s_fnuz, int64_t
     return FP8_ERR_ALIGNMENT;
   DeviceInfo* dev;
   if (fp8_status st = device_info(&dev)) return st;
+  const uint32_t row_pad = static_cast<uint32_t>((K + 127) / 128 * 128);
+  const int64_t warps = std::min<int64_t>(8, kStagedSmemBudget / (2 * int64_t(row_pad) + 16));
+  if (N >= 4 * dev->sm_count && K >= 128 && warps >= 2) {
+    // Rows staged through shared memory, as many 8-warp blocks per SM as fit.
+    const size_t smem = static_cast<size_t>(warps) * 2 * row_pad + 16 * warps;
+    const int64_t per_sm =
+        std::max<int64_t>(1, std::min<int64_t>(4, int64_t(dev->smem_optin) / int64_t(smem + 1024)));
+    const int64_t blocks = std::min<int64_t>(per_sm * dev->sm_count, (N + warps - 1) / warps);
+    convert_fnuz_staged_kernel<<<static_cast<unsigned>(blocks), static_cast<unsigned>(32 * warps),
+                                 smem, as_stream(stream)>>>(w8_fnuz, s_fnuz, N, K, w8, s_ch, row_pad);
+    return last_launch();
+  }
   const dim3 grid(static_cast<unsigned>((N + 7) / 8));
   convert_fnuz_kernel<32><<<grid, 256, 0, as_stream(stream)>>>(w8_fnuz, s_fnuz, N, K, w8, s_ch);
   return last_launch();

@@ -604,6 +604,102 @@ __global__ void __launch_bounds__(256) convert_fnuz_kernel(const uint8_t* src,
   if (t == 0) s_dst[row] = keep ? half : s_in;
 }
 
+// The same conversion with one warp per row and the rows staged in shared
+// memory by 1-D bulk copies, two buffers per warp (as the staged activation
+// quantizer): the flag pass and the copy or re-encode pass both read shared
+// memory, so each row crosses HBM once each way; the next row is in flight
+// while this one is converted. In-place use (dst == src) is safe: a row is
+// wholly in shared memory before any of it is written back.
+__global__ void __launch_bounds__(256) convert_fnuz_staged_kernel(const uint8_t* src,
+                                                                   const float* s_src, int64_t N,
+                                                                   int64_t K, uint8_t* dst,
+                                                                   float* s_dst,
+                                                                   uint32_t row_bytes_padded) {
+  extern __shared__ __align__(128) uint8_t qsm[];
+  const int warps = blockDim.x >> 5;
+  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  uint8_t* buf0 = qsm + static_cast<size_t>(w) * 2 * row_bytes_padded;
+  uint64_t* bars =
+      reinterpret_cast<uint64_t*>(qsm + static_cast<size_t>(warps) * 2 * row_bytes_padded);
+  const uint32_t bar0 = smem_u32(bars + 2 * w);
+  const uint32_t row_bytes = static_cast<uint32_t>(K);
+  const int64_t nvec = K / 16;
+  const int64_t gw = static_cast<int64_t>(blockIdx.x) * warps + w;
+  const int64_t nw = static_cast<int64_t>(gridDim.x) * warps;
+  if (lane == 0) {
+    mbar_init(bar0, 1);
+    mbar_init(bar0 + 8, 1);
+    fence_barrier_init();
+  }
+  __syncwarp();
+  auto issue = [&](int64_t row, int b) {
+    if (lane == 0) {
+      fence_proxy_async_shared();
+      mbar_arrive_expect_tx(bar0 + 8 * b, row_bytes);
+      bulk_load(smem_u32(buf0 + b * row_bytes_padded), src + row * K, row_bytes, bar0 + 8 * b);
+    }
+  };
+  if (gw < N) issue(gw, 0);
+  if (gw + nw < N) issue(gw + nw, 1);
+  uint32_t phases = 0u;  // bit b: parity to wait for on buffer b
+  int b = 0;
+  for (int64_t row = gw; row < N; row += nw, b ^= 1) {
+    if (!mbar_wait(bar0 + 8 * b, (phases >> b) & 1u)) return;
+    phases ^= 1u << b;
+    const uint4* in = reinterpret_cast<const uint4*>(buf0 + b * row_bytes_padded);
+    const float s_in = s_src[row];
+    uint32_t flags = 0;  // bit 0: a 0x80 code, bit 1: a +-240 code
+#pragma unroll 4
+    for (int64_t j = lane; j < nvec; j += 32) {
+      const uint4 u = in[j];
+      const uint32_t wv[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        if (has_zero_byte(wv[i] ^ 0x80808080u)) flags |= 1u;
+        if (has_zero_byte((wv[i] & 0x7F7F7F7Fu) ^ 0x7F7F7F7Fu)) flags |= 2u;
+      }
+    }
+    flags = __reduce_or_sync(0xFFFFFFFFu, flags);
+    const float half = __fmul_rn(s_in, 0.5f);
+    const bool finite = isfinite(s_in);
+    const bool keep = !(flags & 2u) && finite && __fmul_rn(half, 2.0f) == s_in;
+    if (lane == 0) {
+      if (flags & 1u) report(FP8_DEV_NAN_CODE);
+      if (!finite) report(FP8_DEV_NONFINITE);
+    }
+    uint4* out = reinterpret_cast<uint4*>(dst + row * K);
+    bool inexact = false;
+    if (keep) {
+#pragma unroll 4
+      for (int64_t j = lane; j < nvec; j += 32) out[j] = in[j];
+    } else {
+      for (int64_t j = lane; j < nvec; j += 32) {
+        const uint4 u = in[j];
+        uint32_t wv[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          float f[4];
+#pragma unroll
+          for (int q = 0; q < 4; ++q) f[q] = dec_fnuz((wv[i] >> (8 * q)) & 0xFFu);
+          const uint32_t c = pack4_e4m3(f[0], f[1], f[2], f[3]);
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const uint32_t cb = (c >> (8 * q)) & 0xFFu;
+            const uint32_t ib = (wv[i] >> (8 * q)) & 0xFFu;
+            if (ib != 0x80u && dec_e4m3(cb) != f[q]) inexact = true;
+          }
+          wv[i] = c;
+        }
+        out[j] = make_uint4(wv[0], wv[1], wv[2], wv[3]);
+      }
+    }
+    if (__any_sync(0xFFFFFFFFu, inexact) && lane == 0) report(FP8_DEV_INEXACT);
+    if (lane == 0) s_dst[row] = keep ? half : s_in;
+    __syncwarp();  // every lane is done reading this buffer before it is refilled
+    if (row + 2 * nw < N) issue(row + 2 * nw, b);
+  }
+}
+
 // ----------------------------------------------------------- cast
 __global__ void __launch_bounds__(256) cast_e4m3_kernel(const float* __restrict__ x, int64_t n,
                                                          uint8_t* __restrict__ out) {

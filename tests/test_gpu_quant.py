@@ -217,6 +217,34 @@ def test_native_fnuz_conversion_matches_oracle(lib):
     assert not st & lib.DEV_NAN_CODE
 
 
+def test_fnuz_staged_rows_in_place_and_special_rows(lib):
+    """The row-staged conversion (N >= 4 x SMs): in place, K not a multiple of
+    128, +-240 rows re-encoded, odd-subnormal and zero scales, 0x80 flagged."""
+    N, K = 1200, 1040
+    rng = np.random.default_rng(31)
+    codes = rng.integers(0, 0x7F, size=(N, K)).astype(np.uint8)
+    codes[rng.random((N, K)) < 0.5] |= 0x80                        # negative codes
+    codes[codes == 0x80] = 0x00                                     # no NaN code yet
+    codes[3, 17] = 0x7F                                             # +240
+    codes[700, 1039] = 0x7F
+    codes[11, 0] = 0xFF                                             # -240
+    s = rng.uniform(0.01, 2.0, N).astype(np.float32)
+    s[5] = np.float32(2.0 ** -149 * 5)                              # odd subnormal: not halved
+    s[6] = 0.0
+    ref = oracle.convert_fnuz_to_e4m3(codes, s)
+    cd, sd = to_dev(codes), to_dev(s)
+    lib.device_status()
+    lib.convert_fnuz(cd, sd, w8=cd, s_ch=sd)
+    assert np.array_equal(u8(cd), ref.codes)
+    assert same_bits_f32(f32(sd), ref.scales)
+    st = lib.device_status()
+    assert bool(st & lib.DEV_INEXACT) == bool(ref.inexact_rows.any())
+    assert not st & lib.DEV_NAN_CODE
+    codes[900, 33] = 0x80
+    lib.convert_fnuz(to_dev(codes), to_dev(s))
+    assert lib.device_status() & lib.DEV_NAN_CODE
+
+
 def test_fnuz_in_place_and_special_cases(lib):
     N, K = 5, 64
     rng = np.random.default_rng(3)
