@@ -851,8 +851,12 @@ fp8_status fp8_moe_combine(const uint16_t* rows, const int32_t* inv, int64_t tok
     return FP8_ERR_ALIGNMENT;
   DeviceInfo* dev;
   if (fp8_status st = device_info(&dev)) return st;
-  return launch_pdl(moe_combine_kernel, dim3(static_cast<unsigned>((tokens + 7) / 8)), dim3(256),
-                    as_stream(stream), rows, inv, tokens, static_cast<int>(top_k), H, weights, out);
+  const dim3 grid(static_cast<unsigned>((tokens + 7) / 8));
+  if (top_k <= 8)
+    return launch_pdl(moe_combine_kernel<8>, grid, dim3(256), as_stream(stream), rows, inv, tokens,
+                      static_cast<int>(top_k), H, weights, out);
+  return launch_pdl(moe_combine_kernel<kCombineMaxK>, grid, dim3(256), as_stream(stream), rows, inv,
+                    tokens, static_cast<int>(top_k), H, weights, out);
 }
 
 }  // extern "C"

@@ -197,7 +197,16 @@ __global__ void __launch_bounds__(256) moe_gather_kernel(const uint8_t* __restri
   const int64_t src = perm[row] / top_k;
   const uint4* a = reinterpret_cast<const uint4*>(x8 + src * K);
   uint4* b = reinterpret_cast<uint4*>(x8_out + row * K);
-  for (int64_t j = lane; j < K / 16; j += 32) b[j] = __ldg(a + j);
+  // four 16-byte vectors per lane in flight before their stores
+  for (int64_t j0 = lane; j0 < K / 16; j0 += 128) {
+    uint4 v[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      if (j0 + 32 * i < K / 16) v[i] = __ldg(a + j0 + 32 * i);
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      if (j0 + 32 * i < K / 16) b[j0 + 32 * i] = v[i];
+  }
   if (lane == 0) s_out[row] = s_tok[src];
 }
 
@@ -292,6 +301,7 @@ __global__ void __launch_bounds__(256) moe_geglu_quant_kernel(const uint16_t* __
 // vector all k rows are loaded before the ordered sum (k <= kCombineMaxK).
 constexpr int kCombineMaxK = 16;
 
+template <int KMAX>  // slots held per column vector (top_k <= KMAX <= kCombineMaxK)
 __global__ void __launch_bounds__(256) moe_combine_kernel(const uint16_t* __restrict__ rows,
                                                            const int32_t* __restrict__ inv,
                                                            int64_t T, int top_k, int64_t H,
@@ -309,15 +319,15 @@ __global__ void __launch_bounds__(256) moe_combine_kernel(const uint16_t* __rest
   for (int64_t j0 = 0; j0 < H / 8; j0 += 32) {
     const int64_t j = j0 + lane;
     const bool live = j < H / 8;
-    uint4 v[kCombineMaxK];
+    uint4 v[KMAX];
 #pragma unroll
-    for (int s = 0; s < kCombineMaxK; ++s) {
+    for (int s = 0; s < KMAX; ++s) {
       const int64_t r = __shfl_sync(0xFFFFFFFFu, r_l, s);
       if (s < top_k && live) v[s] = __ldg(reinterpret_cast<const uint4*>(rows + r * H) + j);
     }
     float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
 #pragma unroll
-    for (int s = 0; s < kCombineMaxK; ++s) {
+    for (int s = 0; s < KMAX; ++s) {
       const float w = __shfl_sync(0xFFFFFFFFu, w_l, s);
       if (s < top_k) {
         const uint32_t vw[4] = {v[s].x, v[s].y, v[s].z, v[s].w};
