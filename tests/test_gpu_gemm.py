@@ -56,6 +56,7 @@ GEMM_SHAPES = [
     (2048, 2304, 4096),
     (300, 4096, 5376),
     (5, 6000, 1040),      # one CTA per SM, no split: the deep-ring decode variant
+    (3, 4000, 2096),      # few tokens, narrow layer: K split 4 ways, ragged N and K
     (120, 19000, 512),    # more 128-channel tiles than SMs at M = 128
     (200, 1001, 256),     # single-SM prefill, N % 8 != 0: element stores
     (600, 1003, 512),     # CTA pairs, N % 8 != 0
