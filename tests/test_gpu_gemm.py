@@ -207,3 +207,23 @@ def test_linear_from_bf16_is_bit_identical_to_two_calls(lib, M, N, K):
     assert np.array_equal(bf16_to_np_bits(y_fused), bf16_to_np_bits(y_two))
     _check(y_fused, a, w)
     assert lib.device_status() == 0
+
+
+def test_bf16_weights_quantized_per_channel_online(lib):
+    """bf16 weights quantized per output channel at load time (the vLLM
+    fp8_per_channel path for bf16 checkpoints): fp8_quant_act over the
+    weight rows gives one amax/448 scale per channel, bit-exact against the
+    oracle, and the GEMM with those weights stays within the bound."""
+    M, N, K = 37, 3000, 2048
+    wb = activations_bf16(N, K, seed=41)                  # bf16 weight rows [N, K]
+    xb = activations_bf16(M, K, seed=42, outlier_frac=0.01)
+    w_ref = oracle.quant_act(wb)
+    a = oracle.quant_act(xb)
+    w8, s_ch = lib.quant_act(to_dev(wb))
+    assert np.array_equal(u8(w8), w_ref.codes) and same_bits_f32(f32(s_ch), w_ref.scales)
+    y = lib.linear(to_dev(xb), w8, s_ch)
+    y_ref, abs_s = oracle.rowwise_linear_ref(a.codes, a.scales, w_ref.codes, w_ref.scales,
+                                             return_abs=True)
+    ok, worst = oracle.check_linear(bf16_values(y), y_ref, abs_s)
+    assert ok, worst
+    assert lib.device_status() == 0
