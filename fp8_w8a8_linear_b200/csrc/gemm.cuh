@@ -245,7 +245,18 @@ __device__ __forceinline__ Tile grouped_tile(const GemmArgs& g, const int* mt_of
 
 // mt_off[e] = number of tile_rows-row m-tiles of experts 0..e-1 (mt_off[E]
 // = total), from the row offsets; one warp. The offsets may come from a
-// preceding routing grid, so the warp waits for it first.
+// preceding routing grid, so the warp waits for it first. An expert whose
+// row range is not inside [0, M) (or runs backwards) gets no tiles and sets
+// FP8_DEV_BAD_INDEX, so no tile can read or write outside x, s_a or y.
+__device__ __forceinline__ int grouped_expert_rows(const GemmArgs& g, int e) {
+  const int lo = g.offsets[e], hi = g.offsets[e + 1];
+  if (lo < 0 || hi < lo || hi > g.M) {
+    report(FP8_DEV_BAD_INDEX);
+    return 0;
+  }
+  return hi - lo;
+}
+
 __device__ __forceinline__ void grouped_prefix(const GemmArgs& g, int* mt_off, int tile_rows,
                                                int lane) {
   pdl_wait();
@@ -254,7 +265,7 @@ __device__ __forceinline__ void grouped_prefix(const GemmArgs& g, int* mt_off, i
   int sum = 0;
   for (int i = 0; i < per; ++i) {
     const int e = lane * per + i;
-    if (e < E) sum += (g.offsets[e + 1] - g.offsets[e] + tile_rows - 1) / tile_rows;
+    if (e < E) sum += (grouped_expert_rows(g, e) + tile_rows - 1) / tile_rows;
   }
   int incl = sum;
 #pragma unroll
@@ -267,7 +278,7 @@ __device__ __forceinline__ void grouped_prefix(const GemmArgs& g, int* mt_off, i
     const int e = lane * per + i;
     if (e < E) {
       mt_off[e] = run;
-      run += (g.offsets[e + 1] - g.offsets[e] + tile_rows - 1) / tile_rows;
+      run += (grouped_expert_rows(g, e) + tile_rows - 1) / tile_rows;
     }
   }
   if (lane == 31) mt_off[E] = incl;

@@ -194,20 +194,24 @@ __global__ void __launch_bounds__(256) moe_gather_kernel(const uint8_t* __restri
   const int64_t row = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (row >= rows) return;
-  const int64_t src = perm[row] / top_k;
-  const uint4* a = reinterpret_cast<const uint4*>(x8 + src * K);
+  const int32_t p = perm[row];
+  // not a flat (token, slot) index: a zero row and scale, flagged
+  const bool ok = p >= 0 && p < rows;
+  if (!ok && lane == 0) report(FP8_DEV_BAD_INDEX);
+  const int64_t src = ok ? p / top_k : 0;
   uint4* b = reinterpret_cast<uint4*>(x8_out + row * K);
+  const uint4* a = reinterpret_cast<const uint4*>(x8 + src * K);
   // four 16-byte vectors per lane in flight before their stores
   for (int64_t j0 = lane; j0 < K / 16; j0 += 128) {
     uint4 v[4];
 #pragma unroll
     for (int i = 0; i < 4; ++i)
-      if (j0 + 32 * i < K / 16) v[i] = __ldg(a + j0 + 32 * i);
+      v[i] = ok && j0 + 32 * i < K / 16 ? __ldg(a + j0 + 32 * i) : make_uint4(0, 0, 0, 0);
 #pragma unroll
     for (int i = 0; i < 4; ++i)
       if (j0 + 32 * i < K / 16) b[j0 + 32 * i] = v[i];
   }
-  if (lane == 0) s_out[row] = s_tok[src];
+  if (lane == 0) s_out[row] = ok ? s_tok[src] : 0.0f;
 }
 
 // ------------------------------------------------------------------ GeGLU + quant
@@ -313,7 +317,11 @@ __global__ void __launch_bounds__(256) moe_combine_kernel(const uint16_t* __rest
   const int lane = threadIdx.x & 31;
   if (t >= T) return;
   const float wu = __fdiv_rn(1.0f, static_cast<float>(top_k));
-  const int r_l = lane < top_k ? inv[t * top_k + lane] : 0;
+  int r_l = lane < top_k ? inv[t * top_k + lane] : 0;
+  if (r_l < 0 || r_l >= T * top_k) {  // not a row of `rows`: contributes nothing, flagged
+    report(FP8_DEV_BAD_INDEX);
+    r_l = -1;
+  }
   const float w_l = lane < top_k ? (weights ? weights[t * top_k + lane] : wu) : 0.0f;
   // Warp-uniform trip count: every lane takes part in the shuffles.
   for (int64_t j0 = 0; j0 < H / 8; j0 += 32) {
@@ -323,7 +331,8 @@ __global__ void __launch_bounds__(256) moe_combine_kernel(const uint16_t* __rest
 #pragma unroll
     for (int s = 0; s < KMAX; ++s) {
       const int64_t r = __shfl_sync(0xFFFFFFFFu, r_l, s);
-      if (s < top_k && live) v[s] = __ldg(reinterpret_cast<const uint4*>(rows + r * H) + j);
+      v[s] = make_uint4(0, 0, 0, 0);
+      if (s < top_k && live && r >= 0) v[s] = __ldg(reinterpret_cast<const uint4*>(rows + r * H) + j);
     }
     float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
 #pragma unroll

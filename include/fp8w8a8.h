@@ -213,7 +213,9 @@ fp8_status fp8_moe_route(const int32_t* topk_ids, int64_t tokens, int32_t top_k,
  * fp8_moe_gather: rows of per-token quantized activations in expert order:
  *   x8_rows[i] = x8[perm[i] / top_k], s_rows[i] = s_tok[perm[i] / top_k].
  *   x8 [tokens, K] uint8, s_tok [tokens] fp32 (from fp8_quant_act); rows =
- *   tokens * top_k. Requires K % 16 == 0, 16-byte aligned x8 / x8_rows.
+ *   tokens * top_k. Requires K % 16 == 0, 16-byte aligned x8 / x8_rows. A
+ *   perm entry outside [0, rows) gives a zero row and scale and sets
+ *   FP8_DEV_BAD_INDEX.
  */
 fp8_status fp8_moe_gather(const uint8_t* x8, const float* s_tok, const int32_t* perm,
                           int64_t rows, int64_t K, int32_t top_k, uint8_t* x8_rows,
@@ -226,8 +228,9 @@ fp8_status fp8_moe_gather(const uint8_t* x8, const float* s_tok, const int32_t* 
  * s_ch [num_experts * N]) into y [M_total, N] bf16, with the same arithmetic
  * and bound as fp8_rowwise_linear. One persistent tcgen05 kernel walks
  * (expert, 128-row tile, column tile) work items derived on the GPU from
- * offsets. Requires K % 16 == 0, num_experts <= 1024, offsets[num_experts]
- * <= M_total.
+ * offsets. Requires K % 16 == 0, num_experts <= 1024; offsets must be
+ * non-decreasing within [0, M_total]: an expert whose row range is not (a
+ * device-side error) is skipped and sets FP8_DEV_BAD_INDEX.
  */
 fp8_status fp8_grouped_linear(const uint8_t* x8_rows, const float* s_rows, const int32_t* offsets,
                               int32_t num_experts, int64_t M_total, const uint8_t* w8,
@@ -281,7 +284,8 @@ fp8_status fp8_moe_geglu_quant(const uint16_t* gate_up, int64_t M, int64_t inter
  * fp8_moe_combine: out[t] = sum_{j<top_k} w[t,j] * rows[inv[t*top_k + j]]
  * (fp32 products and sums in slot order, one rounding to bf16); rows
  * [tokens*top_k, H] bf16 in expert order, weights [tokens, top_k] fp32 or
- * NULL for 1/top_k. Requires H % 8 == 0 and 1 <= top_k <= 16.
+ * NULL for 1/top_k. Requires H % 8 == 0 and 1 <= top_k <= 16. An inv entry
+ * outside [0, tokens*top_k) contributes nothing and sets FP8_DEV_BAD_INDEX.
  */
 fp8_status fp8_moe_combine(const uint16_t* rows, const int32_t* inv, int64_t tokens,
                            int32_t top_k, int64_t H, const float* weights, uint16_t* out,

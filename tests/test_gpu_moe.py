@@ -227,3 +227,48 @@ def test_geglu_epilogue_bit_identical(lib, T, E, k, I, K):
     h8, sh = lib.quant_act(h)
     assert np.array_equal(u8(h8), u8(h8_ref)) and same_bits_f32(f32(sh), f32(sh_ref))
     assert lib.device_status() == 0
+
+
+def test_bad_device_indices_are_flagged_not_followed(lib):
+    """Expert offsets outside [0, M] or running backwards, perm entries
+    outside [0, rows) and inv entries outside [0, tokens*top_k) are device
+    errors: flagged with FP8_DEV_BAD_INDEX and never used as addresses."""
+    E, N, K, R = 4, 256, 128, 64
+    rng = np.random.default_rng(50)
+    xr = rng.integers(0, 0x7F, (R, K), dtype=np.uint8)
+    sr = np.ones(R, np.float32)
+    w8, sc = _expert_weights(E, N, K, seed=51)
+    lib.device_status()
+    y = torch.full((R, N), 7.0, dtype=torch.bfloat16, device="cuda")
+    bad_off = np.array([0, 40, 20, 64, 64], np.int32)            # expert 1 runs backwards
+    lib.grouped_linear(to_dev(xr), to_dev(sr), to_dev(bad_off), to_dev(w8), to_dev(sc), y)
+    assert lib.device_status() & lib.DEV_BAD_INDEX
+    big_off = np.array([0, 16, 32, 48, 10 ** 6], np.int32)       # past M_total
+    lib.grouped_linear(to_dev(xr), to_dev(sr), to_dev(big_off), to_dev(w8), to_dev(sc), y)
+    assert lib.device_status() & lib.DEV_BAD_INDEX
+    # a valid expert next to the bad one is still computed
+    yv = bf16_values(y)
+    y_ref, abs_s = oracle.rowwise_linear_ref(xr[:16], sr[:16], w8[0], sc[0], return_abs=True)
+    ok, worst = oracle.check_linear(yv[:16], y_ref, abs_s)
+    assert ok, worst
+    # gather: perm entries -1 and rows give zero rows
+    T, k, Kx = 8, 2, 64
+    x8 = rng.integers(1, 0x7F, (T, Kx), dtype=np.uint8)
+    st = np.full(T, 2.0, np.float32)
+    perm = np.arange(T * k, dtype=np.int32)
+    perm[3], perm[5] = -1, T * k
+    g8, gs = lib.moe_gather(to_dev(x8), to_dev(st), to_dev(perm), k)
+    assert lib.device_status() & lib.DEV_BAD_INDEX
+    g8, gs = u8(g8), f32(gs)
+    assert not g8[3].any() and not g8[5].any() and gs[3] == 0 and gs[5] == 0
+    assert np.array_equal(g8[4], x8[2]) and gs[4] == 2.0
+    # combine: an inv entry past the rows contributes nothing
+    H = 64
+    rows = f32_to_bf16_bits(rng.standard_normal((T * k, H)).astype(np.float32))
+    inv = np.arange(T * k, dtype=np.int32)
+    inv[1] = 10 ** 6
+    out = bf16_values(lib.moe_combine(to_dev(rows), to_dev(inv), T, k))
+    assert lib.device_status() & lib.DEV_BAD_INDEX
+    vals = (rows.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    assert np.allclose(out[0], 0.5 * vals[0], rtol=2 ** -7, atol=1e-30)   # slot 1 dropped
+    assert np.allclose(out[1], 0.5 * (vals[2] + vals[3]), rtol=2 ** -7, atol=1e-6)
