@@ -516,10 +516,20 @@ fp8_status launch_linear(const DeviceInfo& dev, const uint8_t* x8, const float* 
     return no_split ? launch_decode_t<128, 6, 1>(dev, x8, s_tok, w8, s_ch, M, N, K, y, stream, pdl)
                     : launch_decode_t<128, 4, 1>(dev, x8, s_tok, w8, s_ch, M, N, K, y, stream, pdl);
   }
-  // Prefill: 256 x 256 tiles on CTA pairs when there are at least two row
-  // tiles of 256, single-SM 128 x 256 tiles below that.
-  if (M >= 512 && dev.pair_clusters > 0)
-    return launch_pair(dev, x8, s_tok, w8, s_ch, M, N, K, y, stream, pdl);
+  // Prefill: 256 x 256 tiles on CTA pairs or 128 x 256 tiles on single SMs
+  // (the same work per SM per tile). Pairs move a third less operand traffic
+  // per tile, so they win whenever they need no more waves of tiles than the
+  // single-SM grid - on equal waves only when K is long enough to amortize
+  // their heavier start (measured on B200 for M = 160..512: 14336 x 4096 and
+  // 21504 x 5376 favour pairs except where pairs need 3 waves against 2;
+  // 8192 x 2048 favours single SMs).
+  if (dev.pair_clusters > 0) {
+    const int64_t tiles_n = (N + 255) / 256;
+    const int64_t pair_waves = ((M + 255) / 256 * tiles_n + dev.pair_clusters - 1) / dev.pair_clusters;
+    const int64_t sm_waves = ((M + kBM - 1) / kBM * tiles_n + dev.sm_count - 1) / dev.sm_count;
+    if (pair_waves < sm_waves || (pair_waves == sm_waves && K >= 4096))
+      return launch_pair(dev, x8, s_tok, w8, s_ch, M, N, K, y, stream, pdl);
+  }
   return launch_prefill(dev, x8, s_tok, w8, s_ch, M, N, K, y, stream, pdl);
 }
 

@@ -52,15 +52,15 @@ GEMM_SHAPES = [
     (128, 520, 1040),
     (129, 520, 1040),
     (255, 256, 128),
-    (1000, 1000, 2000),
+    (1000, 1000, 2000),   # single-SM prefill at larger M (fewer waves than pairs would take)
     (2048, 2304, 4096),
     (300, 4096, 5376),
     (5, 6000, 1040),      # one CTA per SM, no split: the deep-ring decode variant
     (3, 4000, 2096),      # few tokens, narrow layer: K split 4 ways, ragged N and K
     (120, 19000, 512),    # more 128-channel tiles than SMs at M = 128
     (200, 1001, 256),     # single-SM prefill, N % 8 != 0: element stores
-    (600, 1003, 512),     # CTA pairs, N % 8 != 0
-    (700, 2056, 384),     # CTA pairs, ragged M and N: TMA-stored and fallback chunks
+    (600, 1003, 4096),    # CTA pairs, N % 8 != 0
+    (700, 2056, 4096),    # CTA pairs, ragged M and N: TMA-stored and fallback chunks
 ]
 
 
