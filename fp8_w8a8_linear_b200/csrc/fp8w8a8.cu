@@ -111,7 +111,7 @@ using namespace fp8k;
 
 template <int BN, int STAGES, bool GROUPED>
 fp8_status set_prefill_attr() {
-  const size_t smem = PrefillCfg<BN, STAGES>::kSmem + (GROUPED ? 4 * (kMaxExperts + 1) : 0);
+  const size_t smem = PrefillCfg<BN, STAGES>::kSmem + (GROUPED ? grouped_smem_bytes(kMaxExperts) : 0);
   return cudaFuncSetAttribute(gemm_prefill_kernel<BN, STAGES, GROUPED>,
                               cudaFuncAttributeMaxDynamicSharedMemorySize,
                               static_cast<int>(smem)) == cudaSuccess
@@ -138,11 +138,11 @@ fp8_status set_pair_attr() {
                               static_cast<int>(PairCfg<STAGES>::kSmem)) == cudaSuccess &&
                  cudaFuncSetAttribute(gemm_pair_kernel<STAGES, true>,
                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                      static_cast<int>(PairCfg<STAGES>::kSmem + 4 * (kMaxExperts + 1))) ==
+                                      static_cast<int>(PairCfg<STAGES>::kSmem + grouped_smem_bytes(kMaxExperts))) ==
                      cudaSuccess &&
                  cudaFuncSetAttribute(gemm_pair_kernel<STAGES, true, true>,
                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                      static_cast<int>(PairCfg<STAGES>::kSmem + 4 * (kMaxExperts + 1))) ==
+                                      static_cast<int>(PairCfg<STAGES>::kSmem + grouped_smem_bytes(kMaxExperts))) ==
                      cudaSuccess
              ? FP8_OK
              : FP8_ERR_CUDA;
@@ -322,7 +322,7 @@ fp8_status launch_grouped(const DeviceInfo& dev, const uint8_t* x8, const float*
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(dev.sm_count);
   cfg.blockDim = dim3(kPrefillThreads);
-  cfg.dynamicSmemBytes = PrefillCfg<BN, ST>::kSmem + 4 * (E + 1);
+  cfg.dynamicSmemBytes = PrefillCfg<BN, ST>::kSmem + grouped_smem_bytes(E);
   cfg.stream = stream;
   cudaLaunchAttribute attrs[1];
   int na = 0;
@@ -361,7 +361,7 @@ fp8_status launch_grouped_pair(const DeviceInfo& dev, const uint8_t* x8, const f
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2 * dev.pair_clusters);
   cfg.blockDim = dim3(kPrefillThreads);
-  cfg.dynamicSmemBytes = PairCfg<kPairStages>::kSmem + 4 * (E + 1);
+  cfg.dynamicSmemBytes = PairCfg<kPairStages>::kSmem + grouped_smem_bytes(E);
   cfg.stream = stream;
   cudaLaunchAttribute attrs[2];
   int na = 0;

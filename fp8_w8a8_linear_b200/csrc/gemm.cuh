@@ -59,6 +59,16 @@ __device__ __forceinline__ uint16_t f32_to_bf16_rn(float f) {
   return __bfloat16_as_ushort(__float2bfloat16_rn(f));
 }
 
+// Two IEEE fp32 products, each rounded to nearest even (one packed
+// instruction; per lane identical to __fmul_rn).
+__device__ __forceinline__ void fmul2_rn(float& d0, float& d1, float a0, float a1, float b0, float b1) {
+  asm("{\n\t.reg .b64 pa, pb, pd;\n\t"
+      "mov.b64 pa, {%2, %3};\n\tmov.b64 pb, {%4, %5};\n\t"
+      "mul.rn.f32x2 pd, pa, pb;\n\tmov.b64 {%0, %1}, pd;\n\t}"
+      : "=f"(d0), "=f"(d1)
+      : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+}
+
 // Two fp32 -> bf16 (round to nearest even), `lo` in bits [0,16).
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   uint32_t r;
@@ -150,7 +160,10 @@ __device__ __forceinline__ void epi_chunk(const uint32_t (&r)[32], const float* 
       const float sb[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
       float v[8];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) v[i] = __fmul_rn(__fmul_rn(__uint_as_float(r[8 * q + i]), sa), sb[i]);
+      for (int i = 0; i < 8; i += 2) {  // v = (acc * s_a) * s_b, two values per instruction
+        fmul2_rn(v[i], v[i + 1], __uint_as_float(r[8 * q + i]), __uint_as_float(r[8 * q + i + 1]), sa, sa);
+        fmul2_rn(v[i], v[i + 1], v[i], v[i + 1], sb[i], sb[i + 1]);
+      }
       pk[q] = make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]),
                          pack_bf16x2(v[4], v[5]), pack_bf16x2(v[6], v[7]));
     }
@@ -165,6 +178,34 @@ __device__ __forceinline__ void epi_chunk(const uint32_t (&r)[32], const float* 
       }
     }
   }
+}
+
+// K blocking of the prefill kernels: 128-byte k-blocks, each four 32-deep
+// MMA k-steps. When K is not a multiple of 128 but is one of 32 (and
+// K > 128), the last k-block is loaded at K - 128, wholly inside the operands,
+// and its first k-steps - the columns the previous block already covered -
+// are not issued. Every column enters the sum once, in the same order, and
+// the partly out-of-range TMA box (whose zero fill costs more than a full
+// box) is never requested.
+struct KBlocking {
+  int num_kb;
+  int last_x;   // K coordinate of the last k-block
+  int last_k0;  // first MMA k-step of the last k-block
+  __device__ __forceinline__ int x(int kb) const { return kb == num_kb - 1 ? last_x : kb * kBK; }
+};
+
+__device__ __forceinline__ KBlocking k_blocking(int K) {
+  KBlocking b;
+  b.num_kb = (K + kBK - 1) / kBK;
+  const int tail = K % kBK;
+  if (tail != 0 && tail % 32 == 0 && K > kBK) {
+    b.last_x = K - kBK;
+    b.last_k0 = (kBK - tail) / 32;
+  } else {
+    b.last_x = (b.num_kb - 1) * kBK;
+    b.last_k0 = 0;
+  }
+  return b;
 }
 
 // Tile order: groups of `group_m` row tiles; inside a group, row tiles vary
@@ -197,6 +238,9 @@ struct PrefillCfg {
 // Largest number of experts the grouped GEMM handles (its m-tile prefix
 // lives in shared memory).
 constexpr int kMaxExperts = 1024;
+// Dynamic shared memory a grouped launch adds for E experts: the m-tile
+// prefix and a copy of the row offsets, E + 1 ints each.
+constexpr size_t grouped_smem_bytes(int E) { return 8 * (static_cast<size_t>(E) + 1); }
 
 // Arguments shared by the dense and the grouped (per-expert) GEMM.
 //  dense:   A rows [0, M), B rows [0, N); tiles walked in groups of group_m.
@@ -224,9 +268,11 @@ struct Tile {
 
 // Tile t of the grouped problem: m-tiles of tile_rows rows are numbered
 // expert by expert (mt_off[e] = first m-tile of expert e), n-tiles vary
-// fastest.
+// fastest. The experts' row offsets are read from their shared-memory copy
+// (row_off = mt_off + E + 1), so decoding a tile touches no global memory.
 __device__ __forceinline__ Tile grouped_tile(const GemmArgs& g, const int* mt_off, int t, int BN,
                                              int tile_rows = kBM) {
+  const int* row_off = mt_off + g.num_experts + 1;
   const int gmt = t / g.tiles_n, tn = t - (t / g.tiles_n) * g.tiles_n;
   int lo = 0, hi = g.num_experts;  // find e with mt_off[e] <= gmt < mt_off[e+1]
   while (hi - lo > 1) {
@@ -235,8 +281,8 @@ __device__ __forceinline__ Tile grouped_tile(const GemmArgs& g, const int* mt_of
   }
   const int e = lo;
   Tile T;
-  T.a_row = g.offsets[e] + (gmt - mt_off[e]) * tile_rows;
-  T.row_end = g.offsets[e + 1];
+  T.a_row = row_off[e] + (gmt - mt_off[e]) * tile_rows;
+  T.row_end = row_off[e + 1];
   T.b_row = e * g.N + tn * BN;
   T.col0 = tn * BN;
   T.sb_off = e * g.N;
@@ -244,7 +290,8 @@ __device__ __forceinline__ Tile grouped_tile(const GemmArgs& g, const int* mt_of
 }
 
 // mt_off[e] = number of tile_rows-row m-tiles of experts 0..e-1 (mt_off[E]
-// = total), from the row offsets; one warp. The offsets may come from a
+// = total), from the row offsets, and mt_off[E + 1 + e] = offsets[e] (e = 0..E,
+// the copy grouped_tile reads); one warp. The offsets may come from a
 // preceding routing grid, so the warp waits for it first. An expert whose
 // row range is not inside [0, M) (or runs backwards) gets no tiles and sets
 // FP8_DEV_BAD_INDEX, so no tile can read or write outside x, s_a or y.
@@ -282,6 +329,7 @@ __device__ __forceinline__ void grouped_prefix(const GemmArgs& g, int* mt_off, i
     }
   }
   if (lane == 31) mt_off[E] = incl;
+  for (int e = lane; e <= E; e += 32) mt_off[E + 1 + e] = g.offsets[e];
 }
 
 __device__ __forceinline__ Tile dense_tile(const GemmArgs& g, int t, int BN) {
@@ -314,8 +362,8 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
   uint8_t* stg_all = sB + STAGES * C::kBBytes;  // epilogue staging
   uint64_t* bars = reinterpret_cast<uint64_t*>(stg_all + C::kStgBytes);
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 4);
-  // grouped: E+1 ints after the barriers and the TMEM holder (the launch adds
-  // 4 * (E + 1) bytes of dynamic shared memory for them)
+  // grouped: 2 * (E + 1) ints after the barriers and the TMEM holder (the
+  // launch adds grouped_smem_bytes(E) of dynamic shared memory for them)
   int* mt_off = reinterpret_cast<int*>(reinterpret_cast<uint8_t*>(bars) + C::kBarBytes);
   const uint32_t full0 = smem_u32(bars);
   const uint32_t empty0 = smem_u32(bars + STAGES);
@@ -323,7 +371,8 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
   const uint32_t tempty0 = smem_u32(bars + 2 * STAGES + 2);
 
   const int warp = warp_id(), lane = lane_id();
-  const int num_kb = (g.K + kBK - 1) / kBK;
+  const KBlocking kblk = k_blocking(g.K);
+  const int num_kb = kblk.num_kb;
 
   if (warp == 0 && lane == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -364,8 +413,8 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
           if (!mbar_wait(empty0 + 8 * stage, phase ^ 1)) { ok = false; break; }
           const uint32_t fb = full0 + 8 * stage;
           mbar_arrive_expect_tx(fb, C::kStageBytes);
-          tma_load_2d(smem_u32(sA + stage * C::kABytes), &tmA, fb, kb * kBK, T.a_row, 0ull);
-          tma_load_2d(smem_u32(sB + stage * C::kBBytes), &tmB, fb, kb * kBK, T.b_row, 0ull);
+          tma_load_2d(smem_u32(sA + stage * C::kABytes), &tmA, fb, kblk.x(kb), T.a_row, 0ull);
+          tma_load_2d(smem_u32(sB + stage * C::kBBytes), &tmB, fb, kblk.x(kb), T.b_row, 0ull);
           if (++stage == STAGES) { stage = 0; phase ^= 1; }
         }
       }
@@ -382,19 +431,25 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         if (!mbar_wait(tempty0 + 8 * acc, acc_phase ^ 1)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * BN;
-        for (int kb = 0; kb < num_kb; ++kb) {
-          if (!mbar_wait(full0 + 8 * stage, phase)) { ok = false; break; }
+        // one k-block's MMAs from k-step k0 on (k0 > 0 only for a shifted last block)
+        auto kblock = [&](int kb, int k0) {
+          if (!mbar_wait(full0 + 8 * stage, phase)) return false;
           tc_fence_after();
           const uint32_t a0 = smem_u32(sA + stage * C::kABytes);
           const uint32_t b0 = smem_u32(sB + stage * C::kBBytes);
 #pragma unroll
-          for (int k = 0; k < kBK / 32; ++k) {
+          for (int k = k0; k < kBK / 32; ++k) {
             umma_f8(d_tmem, sw128_kmajor_desc(a0 + 32 * k), sw128_kmajor_desc(b0 + 32 * k), idesc,
                     (kb | k) != 0);
           }
           umma_commit(empty0 + 8 * stage);
           if (++stage == STAGES) { stage = 0; phase ^= 1; }
-        }
+          return true;
+        };
+        // the hot loop keeps constant k-steps; a shifted last block is peeled off
+        const int kb_full = kblk.last_k0 != 0 ? num_kb - 1 : num_kb;
+        for (int kb = 0; ok && kb < kb_full; ++kb) ok = kblock(kb, 0);
+        if (ok && kb_full < num_kb) ok = kblock(num_kb - 1, kblk.last_k0);
         umma_commit(tfull0 + 8 * acc);
         if (++acc == 2) { acc = 0; acc_phase ^= 1; }
       }
@@ -507,7 +562,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
   uint8_t* stg_all = sB + STAGES * C::kBBytes;  // epilogue staging
   uint64_t* bars = reinterpret_cast<uint64_t*>(stg_all + C::kStgBytes);
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 4);
-  // grouped: E+1 ints after the barriers (the launch adds 4 * (E + 1) bytes)
+  // grouped: 2 * (E + 1) ints after the barriers (the launch adds grouped_smem_bytes(E))
   int* mt_off = reinterpret_cast<int*>(reinterpret_cast<uint8_t*>(bars) + C::kBarBytes);
   const uint32_t full0 = smem_u32(bars);
   const uint32_t empty0 = smem_u32(bars + STAGES);
@@ -517,7 +572,8 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
   const int warp = warp_id(), lane = lane_id();
   const uint32_t rank = cluster_ctarank();        // 0 = leader (issues the MMAs)
   const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
-  const int num_kb = (g.K + kBK - 1) / kBK;
+  const KBlocking kblk = k_blocking(g.K);
+  const int num_kb = kblk.num_kb;
 
   if (warp == 0 && lane == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -578,8 +634,8 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
           const uint32_t fb_leader = mapa_shared(fb_local, 0);
           // Both CTAs' bytes complete on the leader's full barrier.
           if (rank == 0) mbar_arrive_expect_tx(fb_local, 2 * C::kStageBytes);
-          tma_load_2d_pair(smem_u32(sA + stage * C::kABytes), &tmA, fb_leader, kb * kBK, a_row);
-          tma_load_2d_pair(smem_u32(sB + stage * C::kBBytes), &tmB, fb_leader, kb * kBK, b_row);
+          tma_load_2d_pair(smem_u32(sA + stage * C::kABytes), &tmA, fb_leader, kblk.x(kb), a_row);
+          tma_load_2d_pair(smem_u32(sB + stage * C::kBBytes), &tmB, fb_leader, kblk.x(kb), b_row);
           if (++stage == STAGES) { stage = 0; phase ^= 1; }
         }
       }
@@ -596,19 +652,25 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         if (!mbar_wait(tempty0 + 8 * acc, acc_phase ^ 1)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * C::kBN;
-        for (int kb = 0; kb < num_kb; ++kb) {
-          if (!mbar_wait(full0 + 8 * stage, phase)) { ok = false; break; }
+        // one k-block's MMAs from k-step k0 on (k0 > 0 only for a shifted last block)
+        auto kblock = [&](int kb, int k0) {
+          if (!mbar_wait(full0 + 8 * stage, phase)) return false;
           tc_fence_after();
           const uint32_t a0 = smem_u32(sA + stage * C::kABytes);
           const uint32_t b0 = smem_u32(sB + stage * C::kBBytes);
 #pragma unroll
-          for (int k = 0; k < kBK / 32; ++k) {
+          for (int k = k0; k < kBK / 32; ++k) {
             umma_f8_pair(d_tmem, sw128_kmajor_desc(a0 + 32 * k), sw128_kmajor_desc(b0 + 32 * k), idesc,
                          (kb | k) != 0);
           }
           umma_commit_pair(empty0 + 8 * stage, 0x3);
           if (++stage == STAGES) { stage = 0; phase ^= 1; }
-        }
+          return true;
+        };
+        // the hot loop keeps constant k-steps; a shifted last block is peeled off
+        const int kb_full = kblk.last_k0 != 0 ? num_kb - 1 : num_kb;
+        for (int kb = 0; ok && kb < kb_full; ++kb) ok = kblock(kb, 0);
+        if (ok && kb_full < num_kb) ok = kblock(num_kb - 1, kblk.last_k0);
         umma_commit_pair(tfull0 + 8 * acc, 0x3);
         if (++acc == 2) { acc = 0; acc_phase ^= 1; }
       }
@@ -623,25 +685,41 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     // 16-byte stores of y rows and 16-byte loads of the column scales
     const bool vec_ok = (N % 8) == 0 && (reinterpret_cast<uintptr_t>(g.s_b) & 15) == 0;
     const uint32_t tempty_leader0 = mapa_shared(tempty0, 0);
+    const int et = threadIdx.x - 64;  // epilogue thread 0..255: one column of the tile
     int acc = 0;
     uint32_t acc_phase = 0;
-    bool waited = false;
+    // Tiles are drained in the order the MMAs produce them, with their
+    // coordinates and scales fetched ahead: the tile after next is decoded
+    // and the next tile's s_a and s_b are loaded while the current tile
+    // drains, so no global-load latency sits between tiles (with short K the
+    // epilogue paces the kernel).
+    pdl_wait();  // s_a and the expert offsets may come from the preceding grid
+    auto fetch_scales = [&](const Tile& Tt, float& sbv, float& sav) {
+      const int col = Tt.col0 + et;
+      sbv = col < N ? __ldg(g.s_b + Tt.sb_off + col) : 0.0f;
+      const int rr = Tt.a_row + rank * C::kHalf + quad * 32 + lane;
+      sav = rr < Tt.row_end ? __ldg(g.s_a + rr) : 0.0f;
+    };
+    Tile T = {}, T1 = {};
+    float sb_v = 0.0f, sa = 0.0f;
+    if (pair < num_tiles) {
+      T = tile_of(pair);
+      fetch_scales(T, sb_v, sa);
+    }
+    if (pair + npairs < num_tiles) T1 = tile_of(pair + npairs);
     for (int tile = pair; tile < num_tiles; tile += npairs) {
-      const Tile T = tile_of(tile);
-      {
-        // The tile's column scales into this accumulator's buffer, one per
-        // epilogue thread (weight-side data, read before the tile is done;
-        // every warp left the buffer's previous tile before the last barrier).
-        const int col = T.col0 + (threadIdx.x - 64);
-        sb_tile[acc * 256 + (threadIdx.x - 64)] = col < N ? __ldg(g.s_b + T.sb_off + col) : 0.0f;
-      }
+      const int tile1 = tile + npairs, tile2 = tile + 2 * npairs;
+      float sb_v1 = 0.0f, sa1 = 0.0f;
+      if (tile1 < num_tiles) fetch_scales(T1, sb_v1, sa1);
+      const Tile T2 = tile2 < num_tiles ? tile_of(tile2) : T1;
+      // This tile's column scales into this accumulator's buffer (every warp
+      // left the buffer's previous tile before the last barrier).
+      sb_tile[acc * 256 + et] = sb_v;
       const bool got = mbar_wait(tfull0 + 8 * acc, acc_phase);
       // all epilogue warps: scales visible; leave together if any wait failed
       if (named_bar_or(2, 32 * kEpiWarps, !got)) break;
       tc_fence_after();
-      if (!waited) { pdl_wait(); waited = true; }
       const int row = T.a_row + rank * C::kHalf + quad * 32 + lane;
-      const float sa = row < T.row_end ? __ldg(g.s_a + row) : 0.0f;
       const float* sb_base = g.s_b + T.sb_off;
       // whole 32-row chunk inside the tile's rows: one TMA store per chunk
       const bool tma_rows = g.use_tma_store && (row - lane) + 32 <= T.row_end;
@@ -696,6 +774,10 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(tempty_leader0 + 8 * acc);
       if (++acc == 2) { acc = 0; acc_phase ^= 1; }
+      T = T1;
+      sb_v = sb_v1;
+      sa = sa1;
+      T1 = T2;
     }
     if (lane == 0) bulk_wait_group_all();  // this warp's TMA stores of y are complete
   }

@@ -304,10 +304,14 @@ __device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap
       "l"(reinterpret_cast<uint64_t>(map)), "r"(bar_cluster), "r"(x), "r"(y)
       : "memory");
 }
-// Arrive on an mbarrier of another CTA of the cluster (release, cluster scope).
+// Arrive on an mbarrier of a CTA of the cluster (`bar_cluster` from mapa),
+// with the default semantics (release at CTA scope). The pair epilogue uses it
+// to hand a drained accumulator back to the MMA thread: the ordering that
+// matters there is tcgen05's (wait::ld, then fence::before_thread_sync), and a
+// cluster-scope release would make the arriving thread wait for all of its
+// outstanding memory operations (measured at about 1.8k cycles per tile).
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t bar_cluster) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(bar_cluster)
-               : "memory");
+  asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(bar_cluster) : "memory");
 }
 
 // ---------------------------------------------------------------- clusters

@@ -61,6 +61,13 @@ GEMM_SHAPES = [
     (200, 1001, 256),     # single-SM prefill, N % 8 != 0: element stores
     (600, 1003, 4096),    # CTA pairs, N % 8 != 0
     (700, 2056, 4096),    # CTA pairs, ragged M and N: TMA-stored and fallback chunks
+    # K % 128 in {32, 64, 96}: the last k-block is loaded at K - 128 and its
+    # first 1-3 MMA k-steps are skipped (single-SM kernel, then CTA pairs)
+    (300, 520, 704),
+    (1000, 1024, 416),
+    (600, 768, 224),
+    (129, 256, 160),
+    (1024, 2048, 4160),
 ]
 
 

@@ -65,7 +65,11 @@ def _expert_weights(E, N, K, seed):
 
 
 @pytest.mark.parametrize("T,E,k,N,K", [(300, 8, 2, 384, 512), (300, 8, 2, 512, 512),
-                                       (1000, 16, 4, 1408, 256), (64, 128, 8, 256, 704)])
+                                       (1000, 16, 4, 1408, 256), (64, 128, 8, 256, 704),
+                                       # K <= 768 keeps A resident over several column
+                                       # tiles (5 here: units of unequal length); 800 does not
+                                       (2000, 4, 2, 1280, 768), (2000, 4, 2, 1280, 800),
+                                       (500, 3, 1, 520, 32)])
 def test_grouped_gemm_within_bound(lib, T, E, k, N, K):
     ids = _ids(T, E, k, 7)
     xb = activations_bf16(T, K, seed=7, outlier_frac=0.01)
