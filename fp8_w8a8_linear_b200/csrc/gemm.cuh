@@ -270,16 +270,15 @@ struct Tile {
 // expert by expert (mt_off[e] = first m-tile of expert e), n-tiles vary
 // fastest. The experts' row offsets are read from their shared-memory copy
 // (row_off = mt_off + E + 1), so decoding a tile touches no global memory.
+// Each thread decodes its tiles in increasing order, so the expert index only
+// moves forward: `e` carries it from one call to the next (start at 0) and is
+// advanced to the expert with mt_off[e] <= m-tile < mt_off[e + 1] - usually a
+// step or two, at most E steps over all of a thread's tiles.
 __device__ __forceinline__ Tile grouped_tile(const GemmArgs& g, const int* mt_off, int t, int BN,
-                                             int tile_rows = kBM) {
+                                             int tile_rows, int& e) {
   const int* row_off = mt_off + g.num_experts + 1;
   const int gmt = t / g.tiles_n, tn = t - (t / g.tiles_n) * g.tiles_n;
-  int lo = 0, hi = g.num_experts;  // find e with mt_off[e] <= gmt < mt_off[e+1]
-  while (hi - lo > 1) {
-    const int mid = (lo + hi) >> 1;
-    if (mt_off[mid] <= gmt) lo = mid; else hi = mid;
-  }
-  const int e = lo;
+  while (mt_off[e + 1] <= gmt) ++e;  // t < mt_off[E] * tiles_n, so this stops at e < E
   Tile T;
   T.a_row = row_off[e] + (gmt - mt_off[e]) * tile_rows;
   T.row_end = row_off[e + 1];
@@ -399,7 +398,10 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
   const int num_tiles = GROUPED ? mt_off[g.num_experts] * g.tiles_n : g.tiles_m * g.tiles_n;
-  auto tile_of = [&](int t) { return GROUPED ? grouped_tile(g, mt_off, t, BN) : dense_tile(g, t, BN); };
+  int e_seen = 0;  // this thread's expert cursor (tiles are decoded in increasing order)
+  auto tile_of = [&](int t) {
+    return GROUPED ? grouped_tile(g, mt_off, t, BN, kBM, e_seen) : dense_tile(g, t, BN);
+  };
 
   if (warp == 0) {
     if (lane == 0) {
@@ -602,9 +604,10 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
   // tiles of 256 x 256; the fields of a Tile here are the pair's (row 0 of
   // the tile, column 0), each CTA adding rank * 128 to its A and B rows
   const int num_tiles = GROUPED ? mt_off[g.num_experts] * g.tiles_n : g.tiles_m * g.tiles_n;
+  int e_seen = 0;  // this thread's expert cursor (tiles are decoded in increasing order)
   auto tile_of = [&](int t) {
     if constexpr (GROUPED) {
-      return grouped_tile(g, mt_off, t, C::kBN, 256);
+      return grouped_tile(g, mt_off, t, C::kBN, 256, e_seen);
     } else {
       int tm, tn;
       tile_coords(t, g.tiles_m, g.tiles_n, g.group_m, tm, tn);
