@@ -534,7 +534,8 @@ struct PairCfg {
   static constexpr int kStageBytes = kABytes + kBBytes;
   static constexpr int kTmemCols = 512;              // two 256-column accumulators
   static constexpr int kBarBytes = 8 * (2 * STAGES + 4) + 16;
-  static constexpr int kStgBytes = kEpiStgBytes;  // epilogue staging (chunks, column scales)
+  // epilogue staging: one 2 KB chunk and 128 column scales per epilogue warp
+  static constexpr int kStgBytes = kEpiWarps * (kStageChunkBytes + 128 * 4);
   static constexpr size_t kSmem =
       1024 + static_cast<size_t>(STAGES) * kStageBytes + kStgBytes + kBarBytes;
 };
@@ -679,16 +680,22 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       }
     }
   } else {
-    // Epilogue warps 2..9 of each CTA drain that CTA's 128 TMEM lanes.
+    // Epilogue warps 2..9 of each CTA drain that CTA's 128 TMEM lanes: warp
+    // (quad, half) takes TMEM lane quadrant quad (32 rows) and half of the
+    // tile's columns. Each warp stages its own 128 column scales (GeGLU: its
+    // 64 gate and 64 up columns), so the warps of a tile never wait for one
+    // another: a tile is a TMEM-full wait, the warp's chunks and an arrive.
     const int quad = warp & 3;
     const int half = (warp - 2) >> 2;
     uint8_t* stg = stg_all + (warp - 2) * kStageChunkBytes;  // this warp's staging chunk
-    float* sb_tile = reinterpret_cast<float*>(stg_all + 8 * kStageChunkBytes);  // [2][256]
+    float* sbw = reinterpret_cast<float*>(stg_all + kEpiWarps * kStageChunkBytes) + (warp - 2) * 128;
     const int N = g.N;
     // 16-byte stores of y rows and 16-byte loads of the column scales
     const bool vec_ok = (N % 8) == 0 && (reinterpret_cast<uintptr_t>(g.s_b) & 15) == 0;
     const uint32_t tempty_leader0 = mapa_shared(tempty0, 0);
-    const int et = threadIdx.x - 64;  // epilogue thread 0..255: one column of the tile
+    // this lane's 4 of the warp's 128 column scales (tile-relative column)
+    const int scol = GEGLU ? (lane < 16 ? half * 64 + 4 * lane : 128 + half * 64 + 4 * (lane - 16))
+                           : half * 128 + 4 * lane;
     int acc = 0;
     uint32_t acc_phase = 0;
     // Tiles are drained in the order the MMAs produce them, with their
@@ -697,14 +704,23 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     // drains, so no global-load latency sits between tiles (with short K the
     // epilogue paces the kernel).
     pdl_wait();  // s_a and the expert offsets may come from the preceding grid
-    auto fetch_scales = [&](const Tile& Tt, float& sbv, float& sav) {
-      const int col = Tt.col0 + et;
-      sbv = col < N ? __ldg(g.s_b + Tt.sb_off + col) : 0.0f;
+    auto fetch_scales = [&](const Tile& Tt, float4& sbv, float& sav) {
+      const int col = Tt.col0 + scol;
+      const float* src = g.s_b + Tt.sb_off + col;
+      if (vec_ok) {  // N % 8 == 0: the lane's 4 columns are all inside N or all past it
+        sbv = col < N ? __ldg(reinterpret_cast<const float4*>(src)) : make_float4(0.f, 0.f, 0.f, 0.f);
+      } else {
+        sbv.x = col < N ? __ldg(src) : 0.0f;
+        sbv.y = col + 1 < N ? __ldg(src + 1) : 0.0f;
+        sbv.z = col + 2 < N ? __ldg(src + 2) : 0.0f;
+        sbv.w = col + 3 < N ? __ldg(src + 3) : 0.0f;
+      }
       const int rr = Tt.a_row + rank * C::kHalf + quad * 32 + lane;
       sav = rr < Tt.row_end ? __ldg(g.s_a + rr) : 0.0f;
     };
     Tile T = {}, T1 = {};
-    float sb_v = 0.0f, sa = 0.0f;
+    float4 sb_v = make_float4(0.f, 0.f, 0.f, 0.f);
+    float sa = 0.0f;
     if (pair < num_tiles) {
       T = tile_of(pair);
       fetch_scales(T, sb_v, sa);
@@ -712,15 +728,16 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     if (pair + npairs < num_tiles) T1 = tile_of(pair + npairs);
     for (int tile = pair; tile < num_tiles; tile += npairs) {
       const int tile1 = tile + npairs, tile2 = tile + 2 * npairs;
-      float sb_v1 = 0.0f, sa1 = 0.0f;
+      float4 sb_v1 = make_float4(0.f, 0.f, 0.f, 0.f);
+      float sa1 = 0.0f;
       if (tile1 < num_tiles) fetch_scales(T1, sb_v1, sa1);
       const Tile T2 = tile2 < num_tiles ? tile_of(tile2) : T1;
-      // This tile's column scales into this accumulator's buffer (every warp
-      // left the buffer's previous tile before the last barrier).
-      sb_tile[acc * 256 + et] = sb_v;
+      // this tile's column scales into the warp's buffer (its lanes finished
+      // reading the previous tile's before the last __syncwarp)
+      *reinterpret_cast<float4*>(sbw + 4 * lane) = sb_v;
       const bool got = mbar_wait(tfull0 + 8 * acc, acc_phase);
-      // all epilogue warps: scales visible; leave together if any wait failed
-      if (named_bar_or(2, 32 * kEpiWarps, !got)) break;
+      __syncwarp();  // the scales are visible to the whole warp
+      if (!__all_sync(0xFFFFFFFFu, got)) break;
       tc_fence_after();
       const int row = T.a_row + rank * C::kHalf + quad * 32 + lane;
       const float* sb_base = g.s_b + T.sb_off;
@@ -739,23 +756,26 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
           tmem_ld32(t_row + fc * 32, rg);
           tmem_ld32(t_row + 128 + fc * 32, ru);
           tmem_ld_wait();
-          const float* sbg = sb_tile + acc * 256 + fc * 32;
-          const float* sbu = sbg + 128;
+          const float* sbg = sbw + (fc - half * 2) * 32;
+          const float* sbu = sbg + 64;
           uint4 pk[4];
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
-            float hv[8];
+            float gv[8], uv[8], hv[8];
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
+            for (int i = 0; i < 8; i += 2) {
               const int j = 8 * q + i;
               // gate and up exactly as the plain GEMM stores them in bf16
-              const float gv = __uint_as_float(static_cast<uint32_t>(f32_to_bf16_rn(
-                                   __fmul_rn(__fmul_rn(__uint_as_float(rg[j]), sa), sbg[j])))
-                               << 16);
-              const float uv = __uint_as_float(static_cast<uint32_t>(f32_to_bf16_rn(
-                                   __fmul_rn(__fmul_rn(__uint_as_float(ru[j]), sa), sbu[j])))
-                               << 16);
-              hv[i] = geglu_f32(gv, uv);
+              fmul2_rn(gv[i], gv[i + 1], __uint_as_float(rg[j]), __uint_as_float(rg[j + 1]), sa, sa);
+              fmul2_rn(gv[i], gv[i + 1], gv[i], gv[i + 1], sbg[j], sbg[j + 1]);
+              fmul2_rn(uv[i], uv[i + 1], __uint_as_float(ru[j]), __uint_as_float(ru[j + 1]), sa, sa);
+              fmul2_rn(uv[i], uv[i + 1], uv[i], uv[i + 1], sbu[j], sbu[j + 1]);
+            }
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              const float gb = __uint_as_float(static_cast<uint32_t>(f32_to_bf16_rn(gv[i])) << 16);
+              const float ub = __uint_as_float(static_cast<uint32_t>(f32_to_bf16_rn(uv[i])) << 16);
+              hv[i] = geglu_f32(gb, ub);
             }
             pk[q] = make_uint4(pack_bf16x2(hv[0], hv[1]), pack_bf16x2(hv[2], hv[3]),
                                pack_bf16x2(hv[4], hv[5]), pack_bf16x2(hv[6], hv[7]));
@@ -769,7 +789,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
           uint32_t r[32];
           tmem_ld32(t_row + c * 32, r);
           tmem_ld_wait();
-          epi_chunk(r, sb_tile + acc * 256 + c * 32, sb_base, sa, vec_ok, stg, g.y, row, T.row_end,
+          epi_chunk(r, sbw + (c - half * kCh) * 32, sb_base, sa, vec_ok, stg, g.y, row, T.row_end,
                     N, T.col0 + c * 32, lane, &tmY, tma_rows);
         }
       }
