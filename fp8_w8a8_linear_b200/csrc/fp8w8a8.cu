@@ -305,7 +305,7 @@ fp8_status launch_pair(const DeviceInfo& dev, const uint8_t* x8, const float* s_
   g.group_m = std::min(tiles_m, 16);
   CUtensorMap tmY;
   make_epilogue_store_map(&tmY, g, y, M, N);
-  if (cudaLaunchKernelEx(&cfg, gemm_pair_kernel<kPairStages>, tmA, tmB, tmY, g) != cudaSuccess)
+  if (cudaLaunchKernelEx(&cfg, gemm_pair_kernel<kPairStages>, tmA, tmB, tmB, tmY, g) != cudaSuccess)
     return FP8_ERR_CUDA;
   return FP8_OK;
 }
@@ -386,9 +386,12 @@ fp8_status launch_grouped_pair(const DeviceInfo& dev, const uint8_t* x8, const f
   g.n_out = n_out;
   CUtensorMap tmY;
   make_epilogue_store_map(&tmY, g, y, M_total, n_out > 0 ? n_out : N);
+  // GeGLU: half-width last feature tiles load 64 B rows per CTA through tmBh
+  CUtensorMap tmBh = tmB;
+  if (n_out > 0 && !make_tmap_u8(&tmBh, w8, static_cast<uint64_t>(E) * N, K, 64)) return FP8_ERR_CUDA;
   const auto kernel = n_out > 0 ? gemm_pair_kernel<kPairStages, true, true>
                                 : gemm_pair_kernel<kPairStages, true, false>;
-  if (cudaLaunchKernelEx(&cfg, kernel, tmA, tmB, tmY, g) != cudaSuccess) return FP8_ERR_CUDA;
+  if (cudaLaunchKernelEx(&cfg, kernel, tmA, tmB, tmBh, tmY, g) != cudaSuccess) return FP8_ERR_CUDA;
   return FP8_OK;
 }
 

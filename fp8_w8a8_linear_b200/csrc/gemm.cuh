@@ -551,11 +551,15 @@ struct PairCfg {
 // then up rows of the same features), so a tile's accumulator has gate and
 // up of 128 features side by side; the epilogue rounds both to bf16 as the
 // plain GEMM would store them and writes h = bf16(gelu_tanh(gate) * up)
-// [M_total, n_out] instead.
+// [M_total, n_out] instead. A last feature tile with at most 64 features
+// is half width: each CTA loads 64 B rows (through tmBh, a map with 64-row
+// boxes) and the MMAs run with N = 128, so the leader's gate rows fill
+// accumulator columns 0..63 and the peer's up rows columns 64..127.
 template <int STAGES, bool GROUPED = false, bool GEGLU = false>
 __global__ void __launch_bounds__(kPrefillThreads, 1)
     gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                     const __grid_constant__ CUtensorMap tmY, const GemmArgs g) {
+                     const __grid_constant__ CUtensorMap tmBh, const __grid_constant__ CUtensorMap tmY,
+                     const GemmArgs g) {
   using C = PairCfg<STAGES>;
   static_assert(GROUPED || !GEGLU, "the GeGLU epilogue is for the grouped GEMM");
   extern __shared__ uint8_t smem_raw[];
@@ -590,6 +594,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     fence_barrier_init();
     tma_prefetch_desc(&tmA);
     tma_prefetch_desc(&tmB);
+    if (GEGLU) tma_prefetch_desc(&tmBh);
   }
   if (warp == 1) {
     tmem_alloc_pair(smem_u32(tmem_holder), C::kTmemCols);
@@ -605,6 +610,9 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
   // tiles of 256 x 256; the fields of a Tile here are the pair's (row 0 of
   // the tile, column 0), each CTA adding rank * 128 to its A and B rows
   const int num_tiles = GROUPED ? mt_off[g.num_experts] * g.tiles_n : g.tiles_m * g.tiles_n;
+  // GeGLU: the last feature tile holds at most 64 features (tiles are
+  // numbered m-tile major, so tile % tiles_n is the feature tile)
+  auto half_width = [&](int t) { return GEGLU && g.n_out - 128 * (t % g.tiles_n) <= 64; };
   int e_seen = 0;  // this thread's expert cursor (tiles are decoded in increasing order)
   auto tile_of = [&](int t) {
     if constexpr (GROUPED) {
@@ -632,21 +640,25 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         const Tile T = tile_of(tile);
         const int a_row = T.a_row + rank * C::kHalf;
         const int b_row = T.b_row + rank * C::kHalf;
+        const bool half = half_width(tile);  // 64 B rows per CTA
+        const CUtensorMap* mapB = half ? &tmBh : &tmB;
+        const uint32_t stage_tx = 2 * (C::kABytes + (half ? C::kBBytes / 2 : C::kBBytes));
         for (int kb = 0; kb < num_kb; ++kb) {
           if (!mbar_wait(empty0 + 8 * stage, phase ^ 1)) { ok = false; break; }
           const uint32_t fb_local = full0 + 8 * stage;
           const uint32_t fb_leader = mapa_shared(fb_local, 0);
           // Both CTAs' bytes complete on the leader's full barrier.
-          if (rank == 0) mbar_arrive_expect_tx(fb_local, 2 * C::kStageBytes);
+          if (rank == 0) mbar_arrive_expect_tx(fb_local, stage_tx);
           tma_load_2d_pair(smem_u32(sA + stage * C::kABytes), &tmA, fb_leader, kblk.x(kb), a_row);
-          tma_load_2d_pair(smem_u32(sB + stage * C::kBBytes), &tmB, fb_leader, kblk.x(kb), b_row);
+          tma_load_2d_pair(smem_u32(sB + stage * C::kBBytes), mapB, fb_leader, kblk.x(kb), b_row);
           if (++stage == STAGES) { stage = 0; phase ^= 1; }
         }
       }
     }
   } else if (warp == 1) {
     if (lane == 0 && rank == 0) {
-      constexpr uint32_t idesc = idesc_e4m3_f32(256, C::kBN);
+      constexpr uint32_t kIdescFull = idesc_e4m3_f32(256, C::kBN);
+      constexpr uint32_t kIdescHalf = idesc_e4m3_f32(256, C::kBN / 2);
       int stage = 0;
       uint32_t phase = 0;
       int acc = 0;
@@ -656,6 +668,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         if (!mbar_wait(tempty0 + 8 * acc, acc_phase ^ 1)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * C::kBN;
+        const uint32_t idesc = half_width(tile) ? kIdescHalf : kIdescFull;
         // one k-block's MMAs from k-step k0 on (k0 > 0 only for a shifted last block)
         auto kblock = [&](int kb, int k0) {
           if (!mbar_wait(full0 + 8 * stage, phase)) return false;
@@ -746,15 +759,17 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + acc * C::kBN;
       if constexpr (GEGLU) {
         // accumulator columns 0..127: gate of the tile's 128 features,
-        // 128..255: their up; this warp takes 64 features in two chunks
+        // 128..255: their up (a half-width tile: 0..63 and 64..127); this
+        // warp takes 64 features in two chunks
         const int f_base = T.col0 >> 1;
+        const int up_col = half_width(tile) ? 64 : 128;
 #pragma unroll 1
         for (int fc = half * 2; fc < half * 2 + 2; ++fc) {
           const int f0 = f_base + fc * 32;
           if (f0 >= g.n_out) continue;  // warp-uniform
           uint32_t rg[32], ru[32];
           tmem_ld32(t_row + fc * 32, rg);
-          tmem_ld32(t_row + 128 + fc * 32, ru);
+          tmem_ld32(t_row + up_col + fc * 32, ru);
           tmem_ld_wait();
           const float* sbg = sbw + (fc - half * 2) * 32;
           const float* sbu = sbg + 64;

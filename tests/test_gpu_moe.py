@@ -209,7 +209,10 @@ def test_interleave_gate_up_layout(lib):
 
 
 @pytest.mark.parametrize("T,E,k,I,K", [(8192, 128, 8, 704, 2048), (300, 8, 2, 176, 512),
-                                       (64, 128, 8, 256, 704), (1000, 16, 4, 1408, 256)])
+                                       (64, 128, 8, 256, 704), (1000, 16, 4, 1408, 256),
+                                       # last feature tile of 80 features (full width) and a
+                                       # single tile of 64 (half width: N = 128 MMAs)
+                                       (300, 8, 2, 720, 256), (200, 4, 2, 64, 256)])
 def test_geglu_epilogue_bit_identical(lib, T, E, k, I, K):
     """fp8_grouped_linear_geglu gives bit for bit the h that the plain grouped
     GEMM followed by fp8_moe_geglu_quant gives, and fp8_quant_act of it the
