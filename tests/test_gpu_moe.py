@@ -25,7 +25,10 @@ def _ids(T, E, k, seed):
 
 @pytest.mark.parametrize("T,E,k,seed", [(8192, 128, 8, 4), (1, 4, 2, 1), (100, 1, 1, 2),
                                         (300, 64, 4, 3), (5000, 1024, 2, 5),
-                                        (20001, 96, 3, 8)])   # n % 4 != 0, several id chunks
+                                        (20001, 96, 3, 8),    # n % 4 != 0, ragged last chunk
+                                        # many experts at larger n, and a handful
+                                        (4096, 512, 2, 9), (8192, 1024, 8, 11),
+                                        (5000, 7, 1, 10)])
 def test_route_matches_oracle(lib, T, E, k, seed):
     ids = _ids(T, E, k, seed)
     if T == 300:
@@ -39,9 +42,11 @@ def test_route_matches_oracle(lib, T, E, k, seed):
     assert lib.device_status() == 0
 
 
-def test_route_flags_out_of_range_ids(lib):
-    ids = np.zeros((16, 2), np.int32)
+@pytest.mark.parametrize("T", [16, 4096])
+def test_route_flags_out_of_range_ids(lib, T):
+    ids = np.zeros((T, 2), np.int32)
     ids[3, 1] = 9
+    ids[T - 1, 0] = -1
     lib.moe_route(to_dev(ids), 4)
     assert lib.device_status() & lib.DEV_BAD_INDEX
 
