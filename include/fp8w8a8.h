@@ -227,10 +227,11 @@ fp8_status fp8_moe_gather(const uint8_t* x8, const float* s_tok, const int32_t* 
  * are multiplied by w8[e] (stacked [num_experts * N, K], K-major, scales
  * s_ch [num_experts * N]) into y [M_total, N] bf16, with the same arithmetic
  * and bound as fp8_rowwise_linear. One persistent tcgen05 kernel walks
- * (expert, 128-row tile, column tile) work items derived on the GPU from
- * offsets. Requires K % 16 == 0, num_experts <= 1024; offsets must be
- * non-decreasing within [0, M_total]: an expert whose row range is not (a
- * device-side error) is skipped and sets FP8_DEV_BAD_INDEX.
+ * (expert, row tile, column tile) work items derived on the GPU from
+ * offsets: 256-row tiles on pairs of SMs (128-row tiles on single SMs where
+ * no pair can be scheduled). Requires K % 16 == 0, num_experts <= 1024;
+ * offsets must be non-decreasing within [0, M_total]: an expert whose row
+ * range is not (a device-side error) is skipped and sets FP8_DEV_BAD_INDEX.
  */
 fp8_status fp8_grouped_linear(const uint8_t* x8_rows, const float* s_rows, const int32_t* offsets,
                               int32_t num_experts, int64_t M_total, const uint8_t* w8,
