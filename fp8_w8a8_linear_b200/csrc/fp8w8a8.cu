@@ -201,8 +201,12 @@ fp8_status device_info(DeviceInfo** out) {
     st = st != FP8_OK ? st : set_decode_attr<128, 4, 1>(so);
     st = st != FP8_OK ? st : set_decode_attr<128, 6, 1>(so);
     if (st == FP8_OK &&
-        cudaFuncSetAttribute(quant_act_staged_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             kStagedSmemBudget + 1024) != cudaSuccess)
+        (cudaFuncSetAttribute(quant_act_staged_kernel<false>,
+                              cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              kStagedSmemBudget + 1024) != cudaSuccess ||
+         cudaFuncSetAttribute(quant_act_staged_kernel<true>,
+                              cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              kStagedSmemBudget + 1024) != cudaSuccess))
       st = FP8_ERR_CUDA;
     if (st == FP8_OK &&
         cudaFuncSetAttribute(convert_fnuz_staged_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -562,10 +566,13 @@ fp8_status launch_quant_act(const DeviceInfo& dev, const uint16_t* x, int64_t M,
     // enough rows in flight.
     const int warps = static_cast<int>(staged_warps);
     const size_t smem = static_cast<size_t>(warps) * 2 * row_pad + 16 * warps;
-    const int64_t per_sm = staged_blocks_per_sm(quant_act_staged_kernel, 32 * warps, smem);
+    const int64_t per_sm = staged_blocks_per_sm(quant_act_staged_kernel<false>, 32 * warps, smem);
     const int64_t blocks = std::min<int64_t>(per_sm * dev.sm_count, (M + warps - 1) / warps);
-    return launch_pdl_smem(quant_act_staged_kernel, dim3(static_cast<unsigned>(blocks)),
-                           dim3(32 * warps), smem, stream, x, M, K, ldx, x8, s_tok, row_pad);
+    // Short rows (16 or more warps per SM) are issue-bound: packed divisions.
+    const auto kernel = per_sm * warps >= 16 ? quant_act_staged_kernel<true>
+                                             : quant_act_staged_kernel<false>;
+    return launch_pdl_smem(kernel, dim3(static_cast<unsigned>(blocks)), dim3(32 * warps), smem,
+                           stream, x, M, K, ldx, x8, s_tok, row_pad);
   }
   if (M <= 1024) {
     // Few tokens: a whole block per token row, sized so that the row sits in

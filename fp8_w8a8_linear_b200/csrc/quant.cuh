@@ -62,6 +62,35 @@ __device__ __forceinline__ float div_rn(const RowDivisor& d, float v) {
   return __fmaf_rn(e, d.r, q);
 }
 
+// div_rn's fast path for two values at once: the same multiply and four
+// FMAs per lane, issued as packed fp32x2 instructions (each lane rounded as
+// the scalar instruction rounds it, so the quotients are identical). The
+// correction steps use fma(q, -s, v), which equals fma(-q, s, v) exactly.
+struct RowDivisor2 {
+  uint64_t r2, ns2;  // {r, r} and {-s, -s}
+};
+
+__device__ __forceinline__ RowDivisor2 make_divisor2(const RowDivisor& d) {
+  RowDivisor2 d2;
+  asm("mov.b64 %0, {%1, %1};" : "=l"(d2.r2) : "f"(d.r));
+  asm("mov.b64 %0, {%1, %1};" : "=l"(d2.ns2) : "f"(-d.s));
+  return d2;
+}
+
+__device__ __forceinline__ void div2_rn(const RowDivisor2& d2, float v0, float v1, float& q0,
+                                        float& q1) {
+  asm("{\n\t.reg .b64 v, q, e;\n\t"
+      "mov.b64 v, {%2, %3};\n\t"
+      "mul.rn.f32x2 q, v, %4;\n\t"
+      "fma.rn.f32x2 e, q, %5, v;\n\t"
+      "fma.rn.f32x2 q, e, %4, q;\n\t"
+      "fma.rn.f32x2 e, q, %5, v;\n\t"
+      "fma.rn.f32x2 q, e, %4, q;\n\t"
+      "mov.b64 {%0, %1}, q;\n\t}"
+      : "=f"(q0), "=f"(q1)
+      : "f"(v0), "f"(v1), "l"(d2.r2), "l"(d2.ns2));
+}
+
 // Reduction of a 32-bit unsigned max across the TPR threads of one row.
 // TPR is 32 (one warp per row) or a multiple of 32 up to the block size (a
 // whole block per row); `red` holds one word per warp of the block.
@@ -139,15 +168,23 @@ __global__ void __launch_bounds__(BLOCK) quant_act_kernel(const uint16_t* __rest
   if (t == 0) s_tok[row] = s;
   uint2* dst = reinterpret_cast<uint2*>(x8 + row * K);
   const RowDivisor dv = make_divisor(s, amax);
+  const RowDivisor2 dv2 = make_divisor2(dv);
 
   auto quant8 = [&](const uint4& u) -> uint2 {
     if (s == 0.0f) return make_uint2(0, 0);
     const uint32_t w[4] = {u.x, u.y, u.z, u.w};
     float f[8];
+    if (dv.fast) {
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      f[2 * i] = div_rn(dv, __uint_as_float(w[i] << 16));
-      f[2 * i + 1] = div_rn(dv, __uint_as_float(w[i] & 0xFFFF0000u));
+      for (int i = 0; i < 4; ++i)
+        div2_rn(dv2, __uint_as_float(w[i] << 16), __uint_as_float(w[i] & 0xFFFF0000u), f[2 * i],
+                f[2 * i + 1]);
+    } else {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        f[2 * i] = div_rn(dv, __uint_as_float(w[i] << 16));
+        f[2 * i + 1] = div_rn(dv, __uint_as_float(w[i] & 0xFFFF0000u));
+      }
     }
     return make_uint2(pack4_e4m3(f[0], f[1], f[2], f[3]), pack4_e4m3(f[4], f[5], f[6], f[7]));
   };
@@ -169,6 +206,11 @@ __global__ void __launch_bounds__(BLOCK) quant_act_kernel(const uint16_t* __rest
 // in flight. Few registers, so many warps per SM; the row is read from HBM
 // exactly once and from shared memory twice (amax pass, quantize pass).
 // Dynamic shared memory: warps * 2 * row_bytes_padded, then 2 barriers per warp.
+// PACKED: the divisions as packed fp32x2 instructions (div2_rn), for launches
+// with many warps per SM, where issue slots are what limits short rows; with
+// few warps per SM (long rows) the scalar form's independent chains hide
+// latency better.
+template <bool PACKED>
 __global__ void __launch_bounds__(256) quant_act_staged_kernel(const uint16_t* __restrict__ x,
                                                                 int64_t M, int64_t K, int64_t ldx,
                                                                 uint8_t* __restrict__ x8,
@@ -228,6 +270,7 @@ __global__ void __launch_bounds__(256) quant_act_staged_kernel(const uint16_t* _
     if (s == 0.0f) {
       for (int64_t j = lane; j < nvec; j += 32) dst[j] = make_uint2(0, 0);
     } else if (dv.fast) {
+      const RowDivisor2 dv2 = make_divisor2(dv);
 #pragma unroll 2
       for (int64_t j = lane; j < nvec; j += 32) {
         const uint4 u = src[j];
@@ -235,8 +278,13 @@ __global__ void __launch_bounds__(256) quant_act_staged_kernel(const uint16_t* _
         float f[8];
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-          f[2 * i] = div_rn(dv, __uint_as_float(wv[i] << 16));
-          f[2 * i + 1] = div_rn(dv, __uint_as_float(wv[i] & 0xFFFF0000u));
+          if constexpr (PACKED) {
+            div2_rn(dv2, __uint_as_float(wv[i] << 16), __uint_as_float(wv[i] & 0xFFFF0000u),
+                    f[2 * i], f[2 * i + 1]);
+          } else {
+            f[2 * i] = div_rn(dv, __uint_as_float(wv[i] << 16));
+            f[2 * i + 1] = div_rn(dv, __uint_as_float(wv[i] & 0xFFFF0000u));
+          }
         }
         dst[j] = make_uint2(canon_zero4(cvt_e4m3x2(f[1], f[0]) | (cvt_e4m3x2(f[3], f[2]) << 16)),
                             canon_zero4(cvt_e4m3x2(f[5], f[4]) | (cvt_e4m3x2(f[7], f[6]) << 16)));
@@ -300,12 +348,10 @@ __device__ __forceinline__ GroupLUT group_lut_from(const float (&f)[8]) {
 // by 2 is exact, so fp32(d*2q) = 2 fp32(d*q) and fp32(2w/s) = 2 fp32(w/s);
 // the even q's quotients are therefore doublings, bit for bit. (Quotients
 // too small to be normal encode to 0 either way.)
-__device__ __forceinline__ GroupLUT group_lut_fast(float d, const RowDivisor& dv) {
+__device__ __forceinline__ GroupLUT group_lut_fast(float d, const RowDivisor2& dv2) {
   float f[8];
-  f[0] = div_rn(dv, d);
-  f[2] = div_rn(dv, __fmul_rn(d, 3.0f));
-  f[4] = div_rn(dv, __fmul_rn(d, 5.0f));
-  f[6] = div_rn(dv, __fmul_rn(d, 7.0f));
+  div2_rn(dv2, d, __fmul_rn(d, 3.0f), f[0], f[2]);
+  div2_rn(dv2, __fmul_rn(d, 5.0f), __fmul_rn(d, 7.0f), f[4], f[6]);
   f[1] = __fmul_rn(f[0], 2.0f);
   f[3] = __fmul_rn(f[1], 2.0f);
   f[5] = __fmul_rn(f[2], 2.0f);
@@ -403,6 +449,7 @@ __global__ void __launch_bounds__(256) repack_qat_kernel(const uint8_t* __restri
   if (t == 0) s_ch[row] = s;
   uint4* dst = reinterpret_cast<uint4*>(w8 + row * K);
   const RowDivisor dv = make_divisor(s, amax);
+  const RowDivisor2 dv2 = make_divisor2(dv);
 
   auto emit = [&](int64_t g, const uint4& u, float dg) {
     uint4 o0, o1;
@@ -410,7 +457,7 @@ __global__ void __launch_bounds__(256) repack_qat_kernel(const uint8_t* __restri
       o0 = make_uint4(0, 0, 0, 0);
       o1 = o0;
     } else {
-      const GroupLUT L = dv.fast ? group_lut_fast(dg, dv) : group_lut_slow(dg, s);
+      const GroupLUT L = dv.fast ? group_lut_fast(dg, dv2) : group_lut_slow(dg, s);
       o0.x = lut4(L, u.x);
       o0.y = lut4(L, u.x >> 16);
       o0.z = lut4(L, u.y);
@@ -512,8 +559,9 @@ __global__ void __launch_bounds__(256) repack_qat_staged_kernel(const uint8_t* _
         dst[2 * g + 1] = make_uint4(0, 0, 0, 0);
       }
     } else if (dv.fast) {
+      const RowDivisor2 dv2 = make_divisor2(dv);
 #pragma unroll 2
-      for (int64_t g = lane; g < ng; g += 32) emit_group(dst + 2 * g, qs[g], group_lut_fast(ds[g], dv));
+      for (int64_t g = lane; g < ng; g += 32) emit_group(dst + 2 * g, qs[g], group_lut_fast(ds[g], dv2));
     } else {
       for (int64_t g = lane; g < ng; g += 32) emit_group(dst + 2 * g, qs[g], group_lut_slow(ds[g], s));
     }
