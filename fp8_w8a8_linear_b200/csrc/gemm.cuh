@@ -84,8 +84,9 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 // which keeps both the writes and the reads free of bank conflicts. Rows at
 // or past row_end and columns at or past N (N % 8 == 0) are not written.
 constexpr int kStageChunkBytes = 32 * 64;
-// Epilogue staging of a 256-column tile kernel: one chunk per epilogue warp,
-// then the tile's column scales for each of the two accumulators.
+// Epilogue staging of the single-SM tile kernel: one chunk per epilogue warp,
+// then the tile's column scales for each of the two accumulators (the pair
+// kernel stages 128 column scales per warp instead).
 constexpr int kEpiStgBytes = 8 * kStageChunkBytes + 2 * 256 * 4;
 
 __device__ __forceinline__ void store_chunk_coalesced(uint8_t* stg, const uint4 (&pk)[4],
