@@ -562,8 +562,8 @@ fp8_status launch_quant_act(const DeviceInfo& dev, const uint16_t* x, int64_t M,
   const int64_t staged_warps = std::min<int64_t>(8, kStagedSmemBudget / (2 * int64_t(row_pad) + 16));
   if (M > 1024 && staged_warps >= 2) {
     // Large M: warp-per-row pipeline through shared memory; as many blocks per
-    // SM (up to 4) as their row buffers allow, so that short rows still keep
-    // enough rows in flight.
+    // SM as registers and row buffers allow (the occupancy query), so that
+    // short rows still keep enough rows in flight.
     const int warps = static_cast<int>(staged_warps);
     const size_t smem = static_cast<size_t>(warps) * 2 * row_pad + 16 * warps;
     const int64_t per_sm = staged_blocks_per_sm(quant_act_staged_kernel<false>, 32 * warps, smem);
