@@ -1,5 +1,6 @@
 """Pins of the oracle's mixture-of-experts pieces (CPU only)."""
 
+from decimal import Decimal, localcontext
 from fractions import Fraction
 
 import numpy as np
@@ -45,6 +46,48 @@ def test_gelu_tanh_against_torch_and_limits():
     assert moe.gelu_tanh(np.array([0.0]))[0] == 0.0
     assert abs(moe.gelu_tanh(np.array([30.0]))[0] - 30.0) < 1e-12
     assert abs(moe.gelu_tanh(np.array([-30.0]))[0]) < 1e-12
+
+
+def _gelu_tanh_decimal(x: float) -> Decimal:
+    """0.5 x (1 + tanh(v)), v = sqrt(2/pi) (x + 0.044715 x^3), in 300-digit
+    decimal arithmetic, with tanh(v) = (e^v - e^-v) / (e^v + e^-v) from its
+    exponential definition: at this precision 1 + tanh(v) keeps well over 100
+    correct digits even where it is near 1e-138 (x = -16)."""
+    with localcontext() as ctx:
+        ctx.prec = 300
+        pi = Decimal(0)
+        # pi from Machin's formula, 4 (4 atan(1/5) - atan(1/239))
+        def atan_inv(n):
+            n = Decimal(n)
+            term, total, k = 1 / n, 1 / n, 1
+            while True:
+                term = -term / (n * n)
+                t = term / (2 * k + 1)
+                if abs(t) < Decimal(10) ** -310:
+                    return total
+                total += t
+                k += 1
+        pi = 4 * (4 * atan_inv(5) - atan_inv(239))
+        X = Decimal(x)
+        v = (2 / pi).sqrt() * (X + Decimal("0.044715") * X ** 3)
+        ep, em = v.exp(), (-v).exp()
+        return Decimal("0.5") * X * (1 + (ep - em) / (ep + em))
+
+
+def test_gelu_tanh_relative_accuracy_against_high_precision():
+    """Relative error of the fp64 oracle below 1e-13 everywhere, the far
+    negative tail (values down to 1e-138) included; a plain fp64 evaluation of
+    0.5 x (1 + tanh v) has no correct digit below x = -7."""
+    xs = np.concatenate([np.linspace(-16, 16, 321), [-7.0, -9.3, -10.0, -10.3, -12.5, -15.9921875,
+                                                     1e-30, -1e-30, 2.0 ** -130, -2.0 ** -130]])
+    got = moe.gelu_tanh(xs)
+    for x, g in zip(xs, got):
+        ref = _gelu_tanh_decimal(float(x))
+        if x == 0:
+            assert g == 0 and ref == 0
+            continue
+        rel = abs((Decimal(float(g)) - ref) / ref)
+        assert rel < Decimal("1e-13"), (x, float(g), ref)
 
 
 def test_geglu_rounds_once_to_bf16():
@@ -117,3 +160,41 @@ def test_combine_is_the_weighted_sum_of_a_tokens_rows():
         for j in range(k):
             same[inv[t * k + j]] = v[t]
     assert np.allclose(moe.combine(same, inv, T, k), v, rtol=0, atol=1e-15)
+
+
+def test_combine_weighted_exact_rational():
+    """With explicit weights the fp64 combine equals the exact-rational
+    weighted sum of the token's rows, up to fp64 rounding of the k-term sum."""
+    rng = np.random.default_rng(4)
+    T, k, E, H = 6, 4, 9, 5
+    ids = np.stack([rng.choice(E, k, replace=False) for _ in range(T)]).astype(np.int32)
+    perm, inv, off = moe.route_sort(ids, E)
+    y = rng.standard_normal((T * k, H)).astype(np.float32).astype(np.float64)
+    w = rng.uniform(0, 1, (T, k)).astype(np.float32)
+    out = moe.combine(y, inv, T, k, weights=w)
+    for t in range(T):
+        for h in range(H):
+            exact = sum(Fraction(float(w[t, j])) * Fraction(float(y[inv[t * k + j], h]))
+                        for j in range(k))
+            mag = sum(abs(Fraction(float(w[t, j])) * Fraction(float(y[inv[t * k + j], h])))
+                      for j in range(k))
+            assert abs(Fraction(float(out[t, h])) - exact) <= mag * Fraction(2 * k, 2 ** 53)
+
+
+def test_combine_weighted_hand_worked():
+    """Two tokens, top-2 over 3 experts, by hand:
+    token 0 -> experts (2, 0) with weights (0.75, 0.25); token 1 -> (1, 2)
+    with weights (0.5, 0.5). The expert-sorted rows are
+    [t0s1 (e0), t1s0 (e1), t0s0 (e2), t1s1 (e2)]."""
+    ids = np.array([[2, 0], [1, 2]], dtype=np.int32)
+    perm, inv, off = moe.route_sort(ids, 3)
+    assert perm.tolist() == [1, 2, 0, 3] and inv.tolist() == [2, 0, 1, 3]
+    rows = np.array([[4.0, -8.0],     # t0 slot 1 (expert 0)
+                     [2.0, 6.0],      # t1 slot 0 (expert 1)
+                     [1.0, 2.0],      # t0 slot 0 (expert 2)
+                     [-2.0, 10.0]])   # t1 slot 1 (expert 2)
+    w = np.array([[0.75, 0.25], [0.5, 0.5]], dtype=np.float32)
+    out = moe.combine(rows, inv, 2, 2, weights=w)
+    # token 0: 0.75 * [1, 2] + 0.25 * [4, -8] = [1.75, -0.5]
+    # token 1: 0.5 * [2, 6] + 0.5 * [-2, 10] = [0, 8]
+    assert out.tolist() == [[1.75, -0.5], [0.0, 8.0]]
