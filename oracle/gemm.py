@@ -6,20 +6,23 @@ RowWiseTorchFP8ScaledMMLinearKernel for the CompressedTensorsW8A8Fp8 scheme;
 paragraph — per-output-channel fp32 weight scales, per-token activation
 scales, bf16 other tensors. The output is bf16.
 
-Exactness: every E4M3 value has at most 4 significant bits, so every product
-has at most 8, between 2^-18 and 448^2 < 2^18; a sum of K <= 2^13 such terms
-spans fewer than 2^13 * 2^18 / 2^-18 = 2^49 units of the smallest product, so
-fp64 (53-bit significand) holds every partial sum exactly, in any order.
-Hence the fp64 matrix product below (a library primitive) is the exact
-integer-scaled dot product, whatever blocking the library uses, for any
-K < 2^13; larger K is refused.
+Exactness: every E4M3 value is an integer multiple of 2^-9 (the smallest
+subnormal) below 448, so every product is an integer multiple of 2^-18 of
+magnitude at most 448^2 < 2^18, i.e. fewer than 2^36 units of 2^-18. Every
+partial sum of K such terms is again an integer number of units, fewer than
+K * 2^36; for K < 2^17 that is below 2^53, so fp64 (53-bit significand) holds
+every partial sum exactly, in any order. Hence the fp64 matrix product below
+(a library primitive) is the exact integer-scaled dot product, whatever
+blocking the library uses, for any K < 2^17; larger K is refused.
 
 Acceptance bound (the contract for the GPU result, which accumulates in fp32
 in an order this oracle does not fix):
 ``|y - y_ref| <= 4e-3 * s_tok * s_ch * sum_k |x8 * w8| + 1 ulp_bf16(y_ref)``.
 
 Pinned by tests/test_oracle_gemm.py against an exact-rational triple loop on
-small shapes, one-hot rows, negation and scale-doubling identities.
+small shapes, exact integer sums at K = 65536 with the largest products and
+the smallest units mixed, one-hot rows, negation and scale-doubling
+identities.
 """
 
 from __future__ import annotations
@@ -29,7 +32,7 @@ import numpy as np
 from .formats import dec_e4m3
 
 GEMM_REL_TOL = 4e-3
-_MAX_EXACT_K = 1 << 13
+_MAX_EXACT_K = 1 << 17
 
 
 def _dec(codes) -> np.ndarray:

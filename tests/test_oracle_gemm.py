@@ -1,7 +1,8 @@
 """Pins of the oracle's row-wise scaled GEMM (CPU only): an exact-rational
 triple loop on small shapes (including the whole tiny W8A8 linear, M=4 K=256
-N=128, from its q4_0-grid weights and bf16 activations), one-hot rows, and
-the negation / scale-doubling identities."""
+N=128, from its q4_0-grid weights and bf16 activations), exact integer sums
+at the largest K the library accepts, one-hot rows, and the negation /
+scale-doubling identities."""
 
 from fractions import Fraction
 
@@ -95,3 +96,29 @@ def test_tolerance_and_bf16_ulp():
     assert ok and r == 1.0
     ok, _ = oracle.check_linear(np.array([[1.0 + 2.0 ** -6]]), y, np.array([[0.0]]))
     assert not ok
+
+
+def test_exact_at_the_largest_k():
+    """K = 65536 (the library's limit): the fp64 product equals the exact sum,
+    computed with Python integers in units of 2^-18 (E4M3 values are integer
+    multiples of 2^-9), on rows that mix the largest products (+-448 * 448),
+    the smallest (2^-9 * 2^-9) and random codes, so that a partial sum needs
+    every one of fp64's 53 bits."""
+    K = 65536
+    rng = np.random.default_rng(7)
+    units = [None if np.isnan(v) else int(round(float(v) * 512)) for v in F.DEC_E4M3]
+    x8 = _finite_codes(rng, (3, K))
+    w8 = _finite_codes(rng, (4, K))
+    x8[0, :] = 0x7E                     # +448
+    w8[0, : K // 2] = 0x7E              # +448 * 448 on half the terms ...
+    w8[0, K // 2:] = 0x01               # ... then 2^-9 * 448 units
+    x8[1, 1::2] = 0x01                  # 2^-9 on every other term
+    w8[1, 0::2] = 0xFE                  # -448
+    w8[1, 1::2] = 0x01                  # 2^-9: adds 2^-18 per odd term
+    ones = np.ones(3, np.float32)
+    got = oracle.rowwise_linear_ref(x8, ones, w8, np.ones(4, np.float32))
+    for m in range(3):
+        xu = [units[int(c)] for c in x8[m]]
+        for n in range(4):
+            exact = sum(a * units[int(b)] for a, b in zip(xu, w8[n]))     # units of 2^-18
+            assert Fraction(float(got[m, n])) == Fraction(exact, 2 ** 18), (m, n)
