@@ -10,20 +10,33 @@
 
 namespace fp8k {
 
-// gelu_tanh(x) = 0.5 x (1 + tanh(u)), u = sqrt(2/pi) (x + 0.044715 x^3), in
-// fp32 through the identity 0.5 (1 + tanh(u)) = 1 / (1 + exp(-2u)):
-// gelu_tanh(x) = x / (1 + exp(-2u)). For x -> -inf, exp(-2u) overflows to
-// +inf and the quotient is -0 (the limit); for x -> +inf it is x.
-__device__ __forceinline__ float gelu_tanh_f32(float x) {
+// h = gelu_tanh(g) * up for g, up that are bf16 values held in fp32, in fp32,
+// within one bf16 ulp of the exact product for every bf16 g and every
+// |up| <= 2^40 (the caller rounds h to bf16 once).
+//
+// gelu_tanh(g) = 0.5 g (1 + tanh(v)), v = sqrt(2/pi) (g + 0.044715 g^3),
+// evaluated through 0.5 (1 + tanh(v)) = sigmoid(2v) = 1 / (1 + exp(-2v)).
+// With a = -2|v| <= 0 and e = exp(a) in (0, 1] (no overflow for any g):
+//   g >= 0:  sigmoid(2v) = 1 / (1 + e),   gelu = g / (1 + e);
+//   g <  0:  sigmoid(2v) = e / (1 + e),   gelu = g e / (1 + e).
+// e is computed with the accurate expf (subnormal results kept) and the
+// quotient with IEEE division, so no step loses a representable result.
+// When g < 0 and -2v > 86 (g < -9.3), e is near or below the smallest normal
+// fp32 value and 1 + e == 1; the product g e up is then taken in the log
+// domain, exp(2v + ln|g| + ln|up|), so that it neither flushes through a
+// subnormal intermediate nor depends on how small e is (its relative error
+// stays below 1e-5, far inside one bf16 ulp).
+__device__ __forceinline__ float geglu_f32(float g, float up) {
   constexpr float kA = -1.5957691216057308f;            // -2 sqrt(2/pi)
   constexpr float kB = -1.5957691216057308f * 0.044715f;
-  const float m2u = x * __fmaf_rn(kB, x * x, kA);       // -2u
-  return __fdividef(x, 1.0f + __expf(m2u));
-}
-
-// h = bf16(gelu_tanh(g) * u) for g, u that are bf16 values held in fp32.
-__device__ __forceinline__ float geglu_f32(float g, float u) {
-  return __fmul_rn(gelu_tanh_f32(g), u);
+  const float m2v = __fmul_rn(g, __fmaf_rn(kB, __fmul_rn(g, g), kA));  // -2v, sign opposite to g
+  if (g < 0.0f && m2v > 86.0f) {
+    const float L = __fadd_rn(__fadd_rn(-m2v, logf(-g)), logf(fabsf(up)));
+    return copysignf(expf(L), -up);  // sign of g * up with g < 0
+  }
+  const float e = expf(-fabsf(m2v));
+  const float num = g < 0.0f ? __fmul_rn(g, e) : g;
+  return __fmul_rn(__fdiv_rn(num, __fadd_rn(1.0f, e)), up);
 }
 
 }  // namespace fp8k

@@ -32,6 +32,15 @@
  *     unspecified.
  *   - Shapes are int64_t; all must be >= 0. A zero-sized problem enqueues
  *     nothing and returns FP8_OK.
+ *   - When the status word reports FP8_DEV_TIMEOUT, the outputs of every call
+ *     enqueued since the word was last read are undefined (a kernel whose
+ *     wait gave up still stores its output tile, from whatever its buffers
+ *     held).
+ *   - Per-device state (kernel attributes, occupancy figures, the address of
+ *     the no-allocation scratch array) is set up on the first call on each
+ *     device and cached for the life of the process: the library assumes the
+ *     device's primary context lives until the process exits. After a
+ *     cudaDeviceReset the library must not be called again in that process.
  *
  * Quantization arithmetic (bit-exact contract, the same in every kernel):
  *   per row r of fp32 values v:  amax = max_k |v[k]|,
@@ -319,8 +328,9 @@ fp8_status fp8_moe_combine(const uint16_t* rows, const int32_t* inv, int64_t tok
  * serialized by the caller.
  *
  * The first call on each device looks up that device's address of the array
- * (cudaGetSymbolAddress, with that device current) and caches it; make that
- * first call before any stream capture begins.
+ * (cudaGetSymbolAddress, with that device current) and caches it for the
+ * life of the process (see the conventions above: no cudaDeviceReset); make
+ * that first call before any stream capture begins.
  */
 #define FP8_NOALLOC_SCRATCH_BYTES (4u << 20)
 fp8_status fp8_linear_bf16_noalloc(const uint16_t* x, const uint8_t* w8, const float* s_ch,

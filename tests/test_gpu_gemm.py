@@ -79,6 +79,38 @@ def test_gemm_within_bound(lib, M, N, K):
     assert lib.device_status() == 0
 
 
+# The long reductions the C ABI accepts (K up to 65536): decode (swap-AB, K
+# split over a cluster) and prefill (single SMs and CTA pairs), including a
+# K that is not a multiple of 128 bytes.
+LONG_K_SHAPES = [
+    (1, 256, 8192),
+    (16, 384, 16384),
+    (1, 200, 65536),
+    (16, 256, 65536),
+    (300, 512, 8192),
+    (1000, 256, 16384),
+    (300, 256, 65536),
+    (640, 264, 65536),
+    (130, 256, 65520),
+]
+
+
+@pytest.mark.parametrize("M,N,K", LONG_K_SHAPES)
+def test_long_k_within_bound(lib, M, N, K):
+    xb, a, w = _operands(M, N, K, seed=M + N + K)
+    y = lib.rowwise_linear(to_dev(a.codes), to_dev(a.scales), to_dev(w.codes), to_dev(w.scales))
+    _check(y, a, w)
+    assert lib.device_status() == 0
+
+
+def test_k_beyond_the_limit_is_refused(lib):
+    x8 = torch.zeros((1, 65552), dtype=torch.uint8, device="cuda")
+    w8 = torch.zeros((128, 65552), dtype=torch.uint8, device="cuda")
+    s = torch.ones(128, dtype=torch.float32, device="cuda")
+    with pytest.raises(lib.Fp8Error):
+        lib.rowwise_linear(x8, s[:1], w8, s)
+
+
 @pytest.mark.parametrize("M", [1, 8, 64])
 def test_decode_sweep_shapes(lib, M):
     """Decode GEMM sweep: K=2048, N=8192, activations with 1% outlier channels."""

@@ -2,9 +2,12 @@
 
 Routing, gather and the per-row quantization of h are bit-exact; the grouped
 GEMM is within the row-wise GEMM bound; GeGLU may differ from the fp64 oracle
-by one bf16 rounding (fp32 arithmetic with tanhf), so h is compared within one
-bf16 ulp and h8 bit-exactly on the rows whose h matches; the combine is within
-its fp32-summation bound. Every stage is fed the oracle's own inputs.
+by one bf16 rounding (fp32 arithmetic), so h is compared within one bf16 ulp -
+for every bf16 gate value in [-16, 16] - and h8 bit-exactly against the
+oracle's quantization of the GPU's own h; the combine is within its
+fp32-summation bound. The layer tests run the whole GPU chain and check each
+stage element by element against the oracle applied to that stage's GPU
+inputs, so every comparison is with the oracle and none compounds.
 """
 
 import numpy as np
@@ -130,14 +133,89 @@ def test_geglu_quant_against_oracle(lib):
     h_out = torch.empty((M, I), dtype=torch.bfloat16, device="cuda")
     h8, s_h = lib.moe_geglu_quant(to_dev(gu), I, h_out=h_out)
     h_gpu = bf16_to_np_bits(h_out)
-    ref_v = (h_ref.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
-    gpu_v = (h_gpu.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
-    assert np.all(np.abs(gpu_v - ref_v) <= oracle.bf16_ulp(ref_v))
-    same = np.all(h_gpu == h_ref, axis=1)
-    assert same.mean() > 0.5
-    q = oracle.quant_act(h_ref[same])
-    assert np.array_equal(u8(h8)[same], q.codes)
-    assert same_bits_f32(f32(s_h)[same], q.scales)
+    _assert_h_within_one_ulp(h_gpu, h_ref)
+    # the quantization of h: the oracle's, of the GPU's own h, bit for bit
+    q = oracle.quant_act(h_gpu)
+    assert np.array_equal(u8(h8), q.codes) and same_bits_f32(f32(s_h), q.scales)
+
+
+def _bf16_vals(bits):
+    return (np.asarray(bits, np.uint16).astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
+def _assert_h_within_one_ulp(h_gpu_bits, h_ref_bits):
+    ref_v, gpu_v = _bf16_vals(h_ref_bits), _bf16_vals(h_gpu_bits)
+    bad = ~(np.abs(gpu_v - ref_v) <= oracle.bf16_ulp(ref_v))
+    assert not bad.any(), (int(bad.sum()), gpu_v[bad][:4], ref_v[bad][:4])
+
+
+# Every finite bf16 gate value in [-16, 16] (33,538 of them), each paired with
+# these up values (bf16 numbers; |up| <= 2^40 is the range the GeGLU unit
+# holds to one bf16 ulp for every gate).
+_UPS = [1.0, -1.0, 0.71875, 448.0, -0.0029296875, 2.0 ** 20, -(2.0 ** 40), 2.0 ** -60]
+
+
+def _gate_up_sweep():
+    b = np.arange(1 << 16, dtype=np.uint32).astype(np.uint16)
+    v = _bf16_vals(b)
+    gates = b[np.isfinite(v) & (np.abs(v) <= 16)]
+    ups = f32_to_bf16_bits(np.array(_UPS, np.float32))
+    assert np.array_equal(_bf16_vals(ups), np.array(_UPS))
+    g = np.tile(gates, len(ups))
+    u = np.repeat(ups, len(gates))
+    return g, u
+
+
+def test_geglu_every_bf16_gate_through_geglu_quant(lib):
+    """fp8_moe_geglu_quant on every bf16 gate in [-16, 16] (down to the
+    subnormals and the far negative tail, where the exact GELU is 1e-37 ...
+    1e-138) against the oracle's fp64 GeGLU, within one bf16 ulp."""
+    g, u = _gate_up_sweep()
+    I = 704
+    M = -(-g.size // I)
+    pad = M * I - g.size
+    gate = np.concatenate([g, np.zeros(pad, np.uint16)]).reshape(M, I)
+    up = np.concatenate([u, np.zeros(pad, np.uint16)]).reshape(M, I)
+    gu = np.concatenate([gate, up], axis=1)
+    h_out = torch.empty((M, I), dtype=torch.bfloat16, device="cuda")
+    h8, s_h = lib.moe_geglu_quant(to_dev(gu), I, h_out=h_out)
+    h_gpu = bf16_to_np_bits(h_out)
+    _assert_h_within_one_ulp(h_gpu, moe.geglu_bf16(gu, I))
+    q = oracle.quant_act(h_gpu)
+    assert np.array_equal(u8(h8), q.codes) and same_bits_f32(f32(s_h), q.scales)
+    assert lib.device_status() == 0
+
+
+def test_geglu_every_bf16_gate_through_the_fused_epilogue(lib):
+    """fp8_grouped_linear_geglu on the same sweep. Each expert's gate and up
+    rows hold E4M3 1.0 in column 0 and the rows of x8 hold 1.0 there too, so
+    every accumulator is exactly 1 and gate = bf16(1 * 1 * s_gate) = s_gate,
+    up = s_up: the channel scales carry the swept (gate, up) values into the
+    epilogue, whose h is checked against the oracle's fp64 GeGLU."""
+    g, u = _gate_up_sweep()
+    I, K, rows_per_expert = 704, 32, 3
+    E = -(-g.size // I)
+    assert E <= 1024
+    pad = E * I - g.size
+    gate = _bf16_vals(np.concatenate([g, np.zeros(pad, np.uint16)])).astype(np.float32).reshape(E, I)
+    up = _bf16_vals(np.concatenate([u, np.zeros(pad, np.uint16)])).astype(np.float32).reshape(E, I)
+    w = np.zeros((E, 2 * I, K), np.uint8)
+    w[:, :, 0] = 0x38                       # E4M3 1.0
+    s = np.concatenate([gate, up], axis=1)  # [E, 2I]: gate rows, then up rows
+    R = E * rows_per_expert
+    x8 = np.zeros((R, K), np.uint8)
+    x8[:, 0] = 0x38
+    s_rows = np.ones(R, np.float32)
+    off = (np.arange(E + 1) * rows_per_expert).astype(np.int32)
+    w_il, s_il = lib.moe_interleave_gate_up(to_dev(w), to_dev(s), E, I)
+    h = bf16_to_np_bits(lib.grouped_linear_geglu(to_dev(x8), to_dev(s_rows), to_dev(off),
+                                                 w_il, s_il, I))
+    gate_b = f32_to_bf16_bits(gate)
+    up_b = f32_to_bf16_bits(up)
+    gu = np.concatenate([np.repeat(gate_b, rows_per_expert, axis=0),
+                         np.repeat(up_b, rows_per_expert, axis=0)], axis=1)
+    _assert_h_within_one_ulp(h, moe.geglu_bf16(gu, I))
+    assert lib.device_status() == 0
 
 
 @pytest.mark.parametrize("T,E,k,H", [(2048, 128, 8, 2048), (333, 16, 1, 512), (100, 64, 16, 264)])
@@ -158,37 +236,98 @@ def test_combine_within_bound(lib, T, E, k, H):
     assert np.all(np.abs(bf16_values(out_w) - ref_w) <= 2 * k * 2.0 ** -24 * abs_w + oracle.bf16_ulp(ref_w))
 
 
-def test_small_moe_layer_end_to_end(lib):
-    """The whole layer on the GPU (route, quantize, gather, gate/up GEMM, GeGLU
-    + quant, down GEMM, combine) against the oracle's fp64 chain: final
-    output within 3% relative (Frobenius) - the stages' own bounds are checked
-    above; here the chain is checked as a whole."""
-    T, E, k, Hd, I = 512, 16, 4, 512, 256
-    ids = _ids(T, E, k, 14)
-    xb = activations_bf16(T, Hd, seed=14, outlier_frac=0.01)
-    wgu, sgu = _expert_weights(E, 2 * I, Hd, seed=15)
-    wdn, sdn = _expert_weights(E, Hd, I, seed=16)
-    # oracle chain
-    perm, inv, off = moe.route_sort(ids, E)
-    a = oracle.quant_act(xb)
-    xs, ss = moe.gather_rows(a.codes, a.scales, perm, k)
-    gu = moe.grouped_linear_ref(xs, ss, off, wgu, sgu)
-    gu_b = f32_to_bf16_bits(gu.astype(np.float32))
-    h = moe.geglu_bf16(gu_b, I)
-    hq = oracle.quant_act(h)
-    dn = moe.grouped_linear_ref(hq.codes, hq.scales, off, wdn, sdn)
-    ref = moe.combine(dn, inv, T, k)
+def _check_moe_layer_stagewise(lib, T, E, k, Hd, I, seed, row_sample=None, expert_sample=None):
+    """The whole layer on the GPU - route, quantize x, gather, gate/up GEMM
+    (plain, and with the fused GeGLU epilogue), GeGLU + quantization of h,
+    down GEMM, weighted combine - with every stage checked element by element
+    against the oracle applied to that stage's GPU inputs: routing, x8,
+    gather and h8 bit-exact; gate/up and down within the row-wise GEMM bound;
+    h within one bf16 ulp of the fp64 GeGLU of the GPU's gate/up; the fused
+    epilogue's h bit-identical to the unfused h; the combine within its fp32
+    bound. row_sample(e, r0, r1) picks the rows of expert e the GEMM stages
+    check (all rows when None); expert_sample the experts whose repacked
+    weights are compared with the oracle's repack (all when None)."""
+    ids = _ids(T, E, k, seed)
+    xb = activations_bf16(T, Hd, seed=seed, outlier_frac=0.01)
+    q4g, dg = q4_weights(E * 2 * I, Hd, seed=seed + 1)
+    q4d, dd = q4_weights(E * Hd, I, seed=seed + 2)
+    wts = np.random.default_rng(seed + 3).dirichlet(np.ones(k), T).astype(np.float32)
     # GPU chain
+    wgu, sgu = lib.repack_qat(to_dev(q4g), to_dev(dg))
+    wdn, sdn = lib.repack_qat(to_dev(q4d), to_dev(dd))
     p, iv, of = lib.moe_route(to_dev(ids), E)
     x8, st = lib.quant_act(to_dev(xb))
     g8, gs = lib.moe_gather(x8, st, p, k)
-    y1 = lib.grouped_linear(g8, gs, of, to_dev(wgu), to_dev(sgu))
-    h8, sh = lib.moe_geglu_quant(y1, I)
-    y2 = lib.grouped_linear(h8, sh, of, to_dev(wdn), to_dev(sdn))
-    out = bf16_values(lib.moe_combine(y2, iv, T, k))
-    rel = np.linalg.norm(out - ref) / np.linalg.norm(ref)
-    assert rel < 0.03, rel
+    y1 = lib.grouped_linear(g8, gs, of, wgu, sgu)
+    h_gpu = torch.empty((T * k, I), dtype=torch.bfloat16, device="cuda")
+    h8, sh = lib.moe_geglu_quant(y1, I, h_out=h_gpu)
+    w_il, s_il = lib.moe_interleave_gate_up(wgu, sgu, E, I)
+    h_fused = lib.grouped_linear_geglu(g8, gs, of, w_il, s_il, I)
+    y2 = lib.grouped_linear(h8, sh, of, wdn, sdn)
+    out = lib.moe_combine(y2, iv, T, k, weights=to_dev(wts))
     assert lib.device_status() == 0
+    # routing, quantization, gather: exact
+    rp, ri, ro = moe.route_sort(ids, E)
+    assert np.array_equal(p.cpu().numpy(), rp) and np.array_equal(iv.cpu().numpy(), ri)
+    assert np.array_equal(of.cpu().numpy(), ro)
+    a = oracle.quant_act(xb)
+    assert np.array_equal(u8(x8), a.codes) and same_bits_f32(f32(st), a.scales)
+    xs, ss = moe.gather_rows(a.codes, a.scales, rp, k)
+    assert np.array_equal(u8(g8), xs) and same_bits_f32(f32(gs), ss)
+    # weights: the oracle's repack, bit for bit, on the sampled experts (the
+    # GEMM stages below take the GPU's repacked weights as their inputs)
+    wg8, wgs = u8(wgu).reshape(E, 2 * I, Hd), f32(sgu).reshape(E, 2 * I)
+    wd8, wds = u8(wdn).reshape(E, Hd, I), f32(sdn).reshape(E, Hd)
+    for e in (range(E) if expert_sample is None else expert_sample):
+        wg = oracle.repack_qat(q4g[e * 2 * I:(e + 1) * 2 * I], dg[e * 2 * I:(e + 1) * 2 * I])
+        wd = oracle.repack_qat(q4d[e * Hd:(e + 1) * Hd], dd[e * Hd:(e + 1) * Hd])
+        assert np.array_equal(wg8[e], wg.codes) and same_bits_f32(wgs[e], wg.scales)
+        assert np.array_equal(wd8[e], wd.codes) and same_bits_f32(wds[e], wd.scales)
+    y1v, y2v = bf16_values(y1), bf16_values(y2)
+    h8n, shn = u8(h8), f32(sh)
+    for e in range(E):
+        r0, r1 = int(ro[e]), int(ro[e + 1])
+        if r1 == r0:
+            continue
+        rows = np.arange(r0, r1) if row_sample is None else row_sample(e, r0, r1)
+        ref, abs_s = oracle.rowwise_linear_ref(xs[rows], ss[rows], wg8[e], wgs[e], return_abs=True)
+        ok, worst = oracle.check_linear(y1v[rows], ref, abs_s)
+        assert ok, ("gate/up", e, worst)
+        ref, abs_s = oracle.rowwise_linear_ref(h8n[rows], shn[rows], wd8[e], wds[e], return_abs=True)
+        ok, worst = oracle.check_linear(y2v[rows], ref, abs_s)
+        assert ok, ("down", e, worst)
+    # GeGLU of the GPU's own gate/up, and the quantization of the GPU's own h
+    hb = bf16_to_np_bits(h_gpu)
+    _assert_h_within_one_ulp(hb, moe.geglu_bf16(bf16_to_np_bits(y1), I))
+    assert np.array_equal(bf16_to_np_bits(h_fused), hb)
+    q = oracle.quant_act(hb)
+    assert np.array_equal(h8n, q.codes) and same_bits_f32(shn, q.scales)
+    # combine of the GPU's own down rows with the router weights
+    ref = moe.combine(y2v, ri, T, k, weights=wts)
+    absum = moe.combine(np.abs(y2v), ri, T, k, weights=wts)
+    tol = 2 * k * 2.0 ** -24 * absum + oracle.bf16_ulp(ref)
+    assert np.all(np.abs(bf16_values(out) - ref) <= tol)
+
+
+def test_small_moe_layer_stage_by_stage(lib):
+    _check_moe_layer_stagewise(lib, T=512, E=16, k=4, Hd=512, I=256, seed=14)
+
+
+def test_moe_config_layer_stage_by_stage(lib):
+    """The MoE workload itself (8192 tokens, top-8 of 128 experts, hidden 2048,
+    intermediate 704), every expert's GEMMs checked on 12 of its rows: the
+    first 4, the last 4 (a partial pair tile) and 4 drawn at random; the
+    repack on 6 experts; every other stage on every row."""
+    rng = np.random.default_rng(30)
+
+    def sample(e, r0, r1):
+        n = r1 - r0
+        pick = set(range(min(4, n))) | set(range(max(0, n - 4), n))
+        pick |= set(rng.choice(n, min(4, n), replace=False).tolist())
+        return r0 + np.array(sorted(pick))
+
+    _check_moe_layer_stagewise(lib, T=8192, E=128, k=8, Hd=2048, I=704, seed=4, row_sample=sample,
+                               expert_sample=[0, 1, 57, 64, 126, 127])
 
 
 def test_interleave_gate_up_layout(lib):

@@ -6,9 +6,12 @@ framework owns all of device memory, or a latency-critical serving loop that
 cannot take cudaMalloc's implicit device synchronization. For them the library
 keeps the quantized activations in its own fixed device scratch array. These
 tests call that entry point through the C ABI and check, on two calls in a row
-with different inputs, that its output matches the regular fp8_linear_bf16
-entry point's within the GEMM tolerance every test here uses (and, as the
-kernels are the same, bit for bit); and that a problem too large for the
+with different inputs, that its output is within the GEMM tolerance every test
+here uses of the oracle's exact result and bit for bit the regular
+fp8_linear_bf16 entry point's (the kernels are the same); that two calls
+enqueued back to back on one stream with no host synchronization - the second
+with fewer tokens, so its scales sit at another offset of the shared array -
+each give their own correct result; and that a problem too large for the
 scratch array is refused before anything runs.
 """
 
@@ -45,11 +48,37 @@ def test_noalloc_matches_regular_entry_point_on_two_calls(lib, M, N, K):
         assert _noalloc(lib, x, w8, s_ch, y) == 0
         torch.cuda.synchronize()
         a = oracle.quant_act(xb)
-        _, abs_scaled = oracle.rowwise_linear_ref(a.codes, a.scales, w.codes, w.scales,
-                                                  return_abs=True)
-        ok, worst = oracle.check_linear(bf16_values(y), bf16_values(y_regular), abs_scaled)
+        y_ref, abs_scaled = oracle.rowwise_linear_ref(a.codes, a.scales, w.codes, w.scales,
+                                                      return_abs=True)
+        ok, worst = oracle.check_linear(bf16_values(y), y_ref, abs_scaled)
         assert ok, f"worst error / tolerance = {worst}"
         assert np.array_equal(bf16_to_np_bits(y), bf16_to_np_bits(y_regular))
+    assert lib.device_status() == 0
+
+
+@pytest.mark.parametrize("N,K,Ms", [(8192, 2048, (64, 8)), (1024, 2048, (1000, 300))])
+def test_noalloc_back_to_back_on_one_stream(lib, N, K, Ms):
+    """Two calls with different inputs enqueued on one stream with no host
+    synchronization in between: the second call's quantizer may only rewrite
+    the shared scratch once the first call's GEMM has read it. The second call
+    has fewer tokens, so its per-token scales start at another offset of the
+    array than the first call's; it goes through the Python wrapper."""
+    q4, d = q4_weights(N, K, seed=33)
+    w = oracle.repack_qat(q4, d)
+    w8, s_ch = to_dev(w.codes), to_dev(w.scales)
+    xbs = [activations_bf16(M, K, seed=60 + i, outlier_frac=0.01) for i, M in enumerate(Ms)]
+    xs = [to_dev(xb) for xb in xbs]
+    ys = [torch.full((M, N), float("nan"), dtype=torch.bfloat16, device="cuda") for M in Ms]
+    torch.cuda.synchronize()
+    assert _noalloc(lib, xs[0], w8, s_ch, ys[0]) == 0
+    lib.linear_noalloc(xs[1], w8, s_ch, y=ys[1])
+    torch.cuda.synchronize()
+    for xb, y in zip(xbs, ys):
+        a = oracle.quant_act(xb)
+        y_ref, abs_scaled = oracle.rowwise_linear_ref(a.codes, a.scales, w.codes, w.scales,
+                                                      return_abs=True)
+        ok, worst = oracle.check_linear(bf16_values(y), y_ref, abs_scaled)
+        assert ok, f"worst error / tolerance = {worst}"
     assert lib.device_status() == 0
 
 
