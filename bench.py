@@ -29,9 +29,16 @@ sampled with nvidia-smi during the timed region.
 Output: one JSON line (rank 0). ``value`` is GEMM TFLOP/s of the whole step
 (all ranks' FLOPs / max-over-ranks device time); ``kernels`` breaks the step
 into ops with their own time, TFLOP/s, GB/s of algorithmic bytes and roofline
-fraction; ``roofline`` is the dominant kernel's; ``e2e`` repeats the step
-through the public API from pinned host buffers with the copies in the timed
-region; ``cpu_baseline`` times the CPU oracle on a bounded sample.
+fractions - against the measured denominators (the HBM copy; FP8 dense = 2 x
+the bf16 cuBLAS figure, the burst one for timed regions under 2 s, else the
+sustained one) and against the spec (8 TB/s, 4.5 PF), and for tensor-bound ops
+against the FP8 ceiling torch._scaled_mm reaches on the box; ``roofline`` is
+the dominant kernel's; ``e2e`` repeats the step through the public API from
+pinned host buffers with the copies in the timed region; ``cpu_baseline`` times
+the CPU oracle on a bounded sample. A default single-GPU run of ``large`` also
+times the ops of ``decode``, ``prefill`` and ``moe`` (each in its own step
+graph) and appends them to ``kernels``, so one line covers every
+configuration; ``value`` and ``roofline`` stay those of ``large``.
 
 ``--impl reference`` times the CPU oracle itself (rank 0 only) on a bounded
 sample of the same workload and prints the same JSON line with
@@ -63,6 +70,8 @@ FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
 FALLBACK_BF16_TFLOPS_SUSTAINED = 1400.0
 FP8_PER_BF16 = 2.0  # nominal dense ratio, 4.5 PF fp8 / 2.25 PF bf16
+SPEC_FP8_TFLOPS = 4500.0  # B200 dense FP8, vendor spec
+SPEC_HBM_GBS = 8000.0     # B200 HBM3e, about 8 TB/s
 
 
 def load_peaks():
@@ -302,43 +311,20 @@ def job_tflops(world, flops_per_rank_step, steps, ms):
     return world * flops_per_rank_step * steps / (ms * 1e-3) / 1e12
 
 
-def run_ours(args, rank, world, local_rank):
-    import torch
-    import torch.distributed as dist
-
-    import fp8_w8a8_linear_b200 as f
-
-    torch.cuda.set_device(local_rank)
-    dev = torch.device("cuda", local_rank)
-    wl = WORKLOADS[args.workload]
-    seed = wl["seed"] + 1000 * rank  # each rank has its own batch (weak scaling)
-    stream = torch.cuda.current_stream()
-
-    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
-    flush_rd = torch.ones(64 << 20, dtype=torch.float32, device=dev)   # 256 MiB
-    flush_sum = torch.empty((), dtype=torch.float32, device=dev)
-
-    def flush_l2():
-        # Write 256 MiB (evicts the cache), then read another 256 MiB so the
-        # write-back of those dirty lines happens here, not inside the next op.
-        flush.zero_()
-        torch.sum(flush_rd, dim=0, out=flush_sum)
-
-    if wl.get("moe"):
-        step_ops, h, D, outs, cfg = setup_moe(torch, f, wl, seed, dev)
-    else:
-        step_ops, h, D, outs, cfg = setup_dense(torch, f, wl, seed, dev, True)
-    n_launch_per_step = sum(o[6] for o in step_ops)
-
-    for _ in range(args.warmup):
+def time_ops(torch, step_ops, steps, warmup, flush_l2, stream, on_timed=None):
+    """Times one workload's ops. Each op alone: R back-to-back launches in one
+    CUDA graph, one event pair around each replay (per-op event nodes would
+    add several us to us-scale kernels), the median of 5 replays and their
+    spread. Then `steps` steps replayed from one CUDA graph with an event pair
+    per step, one per L2 flush (subtracted) and one around every op that runs
+    >= 200 us alone (too long for the pair to matter). `on_timed(replay)` is
+    called to run the timed replay (it may bracket it with barriers and the
+    clock sampler). Returns a dict of per-op and per-step times in ms."""
+    for _ in range(warmup):
         for name, fn, *_rest in step_ops:
             fn(0)
     torch.cuda.synchronize()
-    assert f.device_status() == 0, "device status set during warm-up"
 
-    # ---- each op alone: R back-to-back launches in one CUDA graph, one event
-    # pair around each replay (per-op event nodes would add several us to
-    # us-scale kernels); the median of 5 replays, and their spread.
     def time_alone(fn, reps, trials=5):
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g):
@@ -369,10 +355,6 @@ def run_ours(args, rank, world, local_rank):
         alone_ms.append(med)
         alone_spread.append(spread)
 
-    # ---- the timed steps, replayed from one CUDA graph (the pages' GEMM
-    # microbenchmark likewise ran inside a HIP graph; e2e below is eager).
-    # Event pairs: one per step, one per flush (subtracted), and one around
-    # every op that runs >= 200 us alone (too long for the pair to matter).
     long_op = [ms >= 0.2 for ms in alone_ms]
 
     def ev():
@@ -381,7 +363,7 @@ def run_ours(args, rank, world, local_rank):
     graph = torch.cuda.CUDAGraph()
     steps_ev, flush_ev, op_ev = [], [], []
     with torch.cuda.graph(graph):
-        for _ in range(args.steps):
+        for _ in range(steps):
             e0, e1 = ev(), ev()
             fl_pairs, op_pairs = [], {}
             e0.record()
@@ -406,66 +388,186 @@ def run_ours(args, rank, world, local_rank):
             op_ev.append(op_pairs)
     graph.replay()  # untimed graph warm-up
     torch.cuda.synchronize()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
 
-    gpu_uuid = str(torch.cuda.get_device_properties(dev).uuid)
-    sampler = ClockSampler(gpu_uuid if gpu_uuid.startswith("GPU-") else f"GPU-{gpu_uuid}")
-    sampler.start()
-    time.sleep(0.25)
-    graph.replay()  # under the clock sampler only
-    if world > 1:
-        dist.barrier()
-    torch.cuda.synchronize()
-    t_all0 = torch.cuda.Event(enable_timing=True)
-    t_all1 = torch.cuda.Event(enable_timing=True)
-    t_all0.record(stream)
-    graph.replay()
-    t_all1.record(stream)
-    torch.cuda.synchronize()
-    if world > 1:
-        dist.barrier()
-    clocks = sampler.stop()
-    status = f.device_status()
+    def replay():
+        t0.record(stream)
+        graph.replay()
+        t1.record(stream)
+        torch.cuda.synchronize()
 
+    (on_timed or (lambda r: r()))(replay)
     step_ms_list = []
     for (e0, e1), fls in zip(steps_ev, flush_ev):
         step_ms_list.append(e0.elapsed_time(e1) - sum(a.elapsed_time(b) for a, b in fls))
     in_step_ms = {i: float(np.mean([op_ev[s_i][i][0].elapsed_time(op_ev[s_i][i][1])
-                                    for s_i in range(args.steps)]))
+                                    for s_i in range(steps)]))
                   for i in range(len(step_ops)) if long_op[i]}
-    total_ms = float(np.sum(step_ms_list))
+    graph_ms = t0.elapsed_time(t1)
+    del graph
+    op_ms = [in_step_ms.get(i, alone_ms[i]) for i in range(len(step_ops))]
+    return {"op_ms": op_ms, "alone_spread": alone_spread, "long_op": long_op,
+            "total_ms": float(np.sum(step_ms_list)), "graph_ms": graph_ms}
+
+
+def roofline_peaks(peaks, timed_s, scaled_mm):
+    """Denominators for one timed region. The measured bf16 cuBLAS figure is
+    taken as a burst for regions under 2 s (the part stays near its boost
+    clock) and as sustained for longer ones; FP8 dense = 2 x bf16 (the nominal
+    ratio, 4.5 / 2.25 PF). Spec denominators beside them: 4.5 PF FP8 dense and
+    8 TB/s HBM3e."""
+    burst = timed_s < 2.0
+    bf16 = peaks["bf16"] if burst else peaks["bf16_sustained"]
+    return {
+        "fp8": bf16 * FP8_PER_BF16,
+        "fp8_note": (f"fp8 dense = 2 x {peaks['source']} {'burst' if burst else 'sustained'} bf16 cuBLAS "
+                     f"({bf16}); timed region {timed_s:.2f} s"),
+        "hbm": peaks["hbm_gbs"], "hbm_note": f"{peaks['source']} HBM copy",
+        "fp8_spec": SPEC_FP8_TFLOPS, "hbm_spec": SPEC_HBM_GBS,
+        "fp8_scaled_mm": scaled_mm,
+    }
+
+
+def kernel_rows(step_ops, t, pk, workload):
+    rows = []
+    for i, ((name, fn, fl, by, bound, pre, nl), ms) in enumerate(zip(step_ops, t["op_ms"])):
+        k = {"workload": workload, "op": name, "us": round(ms * 1e3, 2),
+             "gbs": round(by / (ms * 1e-3) / 1e9, 1), "tflops": round(fl / (ms * 1e-3) / 1e12, 1),
+             "bound": bound, "timed": "in step" if t["long_op"][i] else "alone, back to back (median of 5)"}
+        if not t["long_op"][i]:
+            k["us_range"] = [round(t["alone_spread"][i][0] * 1e3, 2), round(t["alone_spread"][i][1] * 1e3, 2)]
+        if bound == "tensor":
+            k["frac"] = round(k["tflops"] / pk["fp8"], 3)
+            k["frac_spec"] = round(k["tflops"] / pk["fp8_spec"], 3)
+            if pk["fp8_scaled_mm"]:
+                k["frac_scaled_mm"] = round(k["tflops"] / pk["fp8_scaled_mm"], 3)
+        elif bound == "hbm":
+            k["frac"] = round(k["gbs"] / pk["hbm"], 3)
+            k["frac_spec"] = round(k["gbs"] / pk["hbm_spec"], 3)
+        rows.append(k)
+    return rows
+
+
+def scaled_mm_ceiling(torch, dev):
+    """The box's FP8 GEMM ceiling through the library route: torch._scaled_mm
+    (e4m3 x e4m3 -> bf16 with row-wise fp32 scales) at 8192^3, best of 10
+    after warm-up. A timing-only measurement beside the product path; None
+    where the build has no row-wise FP8 scaled mm."""
+    n = 8192
+    try:
+        g = torch.Generator(device=dev).manual_seed(0)
+        a = torch.randn((n, n), device=dev, generator=g).to(torch.float8_e4m3fn)
+        b = torch.randn((n, n), device=dev, generator=g).to(torch.float8_e4m3fn).t()
+        sa = torch.ones((n, 1), device=dev, dtype=torch.float32)
+        sb = torch.ones((1, n), device=dev, dtype=torch.float32)
+        out = torch.empty((n, n), device=dev, dtype=torch.bfloat16)
+
+        def mm():
+            torch._scaled_mm(a, b, scale_a=sa, scale_b=sb, out_dtype=torch.bfloat16, out=out)
+
+        for _ in range(5):
+            mm()
+        torch.cuda.synchronize()
+        best = float("inf")
+        for _ in range(10):
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record()
+            mm()
+            e1.record()
+            torch.cuda.synchronize()
+            best = min(best, e0.elapsed_time(e1))
+        del a, b, out
+        return 2.0 * n ** 3 / (best * 1e-3) / 1e12
+    except Exception:
+        return None
+
+
+# The other workloads whose ops the default run also measures (rank 0 of a
+# single-GPU run), so that one bench line covers every configuration.
+EXTRA_WORKLOADS = ("decode", "prefill", "moe")
+
+
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+
+    import fp8_w8a8_linear_b200 as f
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    stream = torch.cuda.current_stream()
+
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    flush_rd = torch.ones(64 << 20, dtype=torch.float32, device=dev)   # 256 MiB
+    flush_sum = torch.empty((), dtype=torch.float32, device=dev)
+
+    def flush_l2():
+        # Write 256 MiB (evicts the cache), then read another 256 MiB so the
+        # write-back of those dirty lines happens here, not inside the next op.
+        flush.zero_()
+        torch.sum(flush_rd, dim=0, out=flush_sum)
+
+    def setup(name):
+        wl = WORKLOADS[name]
+        seed = wl["seed"] + 1000 * rank  # each rank has its own batch (weak scaling)
+        if wl.get("moe"):
+            return setup_moe(torch, f, wl, seed, dev)
+        return setup_dense(torch, f, wl, seed, dev, True)
+
+    wl = WORKLOADS[args.workload]
+    step_ops, h, D, outs, cfg = setup(args.workload)
+    n_launch_per_step = sum(o[6] for o in step_ops)
+
+    gpu_uuid = str(torch.cuda.get_device_properties(dev).uuid)
+    sampler = ClockSampler(gpu_uuid if gpu_uuid.startswith("GPU-") else f"GPU-{gpu_uuid}")
+    clocks = {}
+
+    def timed(replay):
+        sampler.start()
+        time.sleep(0.25)
+        replay()  # under the clock sampler only
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        replay()
+        if world > 1:
+            dist.barrier()
+        clocks.update(sampler.stop())
+
+    t = time_ops(torch, step_ops, args.steps, args.warmup, flush_l2, stream, on_timed=timed)
+    assert f.device_status() == 0, "device status set while timing"
+    status = 0
+    total_ms = t["total_ms"]
     step_ms = total_ms / args.steps
-    graph_ms = t_all0.elapsed_time(t_all1)
     if world > 1:
         total_ms = max_over_ranks([total_ms], world, dev)[0]
         step_ms = total_ms / args.steps
     flops_step = sum(o[2] for o in step_ops)
     value = job_tflops(world, flops_step, args.steps, total_ms)
-    op_ms = [in_step_ms.get(i, alone_ms[i]) for i in range(len(step_ops))]
+    op_ms = t["op_ms"]
 
     peaks = load_peaks()
-    fp8_sus = peaks["bf16_sustained"] * FP8_PER_BF16
-    kernels = []
-    for i, ((name, fn, fl, by, bound, pre, nl), ms) in enumerate(zip(step_ops, op_ms)):
-        k = {"op": name, "us": round(ms * 1e3, 2), "gbs": round(by / (ms * 1e-3) / 1e9, 1),
-             "tflops": round(fl / (ms * 1e-3) / 1e12, 1), "bound": bound,
-             "timed": "in step" if long_op[i] else "alone, back to back (median of 5)"}
-        if not long_op[i]:
-            k["us_range"] = [round(alone_spread[i][0] * 1e3, 2), round(alone_spread[i][1] * 1e3, 2)]
-        if bound == "tensor":
-            k["frac"] = round(k["tflops"] / fp8_sus, 3)
-        elif bound == "hbm":
-            k["frac"] = round(k["gbs"] / peaks["hbm_gbs"], 3)
-        kernels.append(k)
+    smm = scaled_mm_ceiling(torch, dev) if (rank == 0 and world == 1) else None
+    pk = roofline_peaks(peaks, t["graph_ms"] * 1e-3, smm)
+    kernels = kernel_rows(step_ops, t, pk, args.workload)
     dom = max(range(len(step_ops)), key=lambda i: op_ms[i])  # the longest op of the step
     dname, _, dfl, dby, dbound, _, _ = step_ops[dom]
     dms = op_ms[dom]
     if dbound == "tensor":
-        roof = {"kernel": dname, "bound": "tensor", "achieved": round(dfl / (dms * 1e-3) / 1e12, 1),
-                "peak": round(fp8_sus, 1), "unit": "TFLOP/s",
-                "peak_note": f"fp8 dense = 2 x {peaks['source']} sustained bf16 cuBLAS ({peaks['bf16_sustained']})"}
+        ach = round(dfl / (dms * 1e-3) / 1e12, 1)
+        roof = {"kernel": dname, "bound": "tensor", "achieved": ach, "peak": round(pk["fp8"], 1),
+                "unit": "TFLOP/s", "peak_note": pk["fp8_note"],
+                "peak_spec": pk["fp8_spec"], "frac_spec": round(ach / pk["fp8_spec"], 3)}
+        if smm:
+            roof["peak_scaled_mm"] = round(smm, 1)
+            roof["frac_scaled_mm"] = round(ach / smm, 3)
     else:
-        roof = {"kernel": dname, "bound": "hbm", "achieved": round(dby / (dms * 1e-3) / 1e9, 1),
-                "peak": peaks["hbm_gbs"], "unit": "GB/s", "peak_note": f"{peaks['source']} HBM copy"}
+        ach = round(dby / (dms * 1e-3) / 1e9, 1)
+        roof = {"kernel": dname, "bound": "hbm", "achieved": ach, "peak": pk["hbm"], "unit": "GB/s",
+                "peak_note": pk["hbm_note"], "peak_spec": pk["hbm_spec"],
+                "frac_spec": round(ach / pk["hbm_spec"], 3)}
     roof["frac"] = round(roof["achieved"] / roof["peak"], 3)
     roof["traffic"] = TRAFFIC.get((args.workload, dname))
 
@@ -473,7 +575,7 @@ def run_ours(args, rank, world, local_rank):
     # step's inputs are copied in and its results read back every step.
     e2e_steps = max(1, min(args.steps, 3))
     outs_host = [torch.empty(o.shape, dtype=o.dtype).pin_memory() for o in outs]
-    h2d = sum(t.numel() * t.element_size() for t in h.values())
+    h2d = sum(v.numel() * v.element_size() for v in h.values())
     d2h = sum(o.numel() * o.element_size() for o in outs_host)
 
     def e2e_step():
@@ -499,6 +601,34 @@ def run_ours(args, rank, world, local_rank):
         e2e_ms = max_over_ranks([e2e_ms], world, dev)[0]
     e2e_val = job_tflops(world, flops_step, e2e_steps, e2e_ms)
     status |= f.device_status()
+    del step_ops, h, D, outs
+
+    # ---- the other configurations' ops (single-GPU runs of the default
+    # workload): each workload's own step graph, ops timed as above.
+    others = {}
+    if world == 1 and args.workload == "large" and not args.no_extra:
+        for name in EXTRA_WORKLOADS:
+            ops_x, _, _, _, cfg_x = setup(name)
+            clk = {}
+
+            def timed_x(replay, clk=clk):
+                sampler.start()
+                time.sleep(0.25)
+                replay()
+                clk.update(sampler.stop())
+
+            steps_x = min(args.steps, 10)
+            tx = time_ops(torch, ops_x, steps_x, args.warmup, flush_l2, stream, on_timed=timed_x)
+            pkx = roofline_peaks(peaks, tx["graph_ms"] * 1e-3, smm)
+            kernels += kernel_rows(ops_x, tx, pkx, name)
+            fl_x = sum(o[2] for o in ops_x)
+            others[name] = {"config": cfg_x, "desc": WORKLOADS[name]["desc"], "steps": steps_x,
+                            "ms_per_step": round(tx["total_ms"] / steps_x, 4),
+                            "tflops": round(job_tflops(1, fl_x, steps_x, tx["total_ms"]), 2),
+                            "peak_note": pkx["fp8_note"], "clocks": clk}
+            status |= f.device_status()
+            del ops_x
+            torch.cuda.empty_cache()
 
     out = None
     if rank == 0:
@@ -513,11 +643,18 @@ def run_ours(args, rank, world, local_rank):
             "timing": {"method": "CUDA graph of all timed steps; event pair per step with the L2 flushes' "
                                  "own pairs subtracted; per-op times in step for ops >= 200 us, else "
                                  "from a back-to-back graph of that op alone",
-                       "graph_ms_incl_flushes": round(graph_ms, 3)},
+                       "graph_ms_incl_flushes": round(t["graph_ms"], 3)},
             "data": "synthetic (seeded q4_0-grid weights, bf16 N(0,1) activations with 1% x20 outlier channels)",
             "config": config,
             "kernels": kernels,
             "roofline": roof,
+            "denominators": {"fp8_tflops_measured": round(pk["fp8"], 1), "fp8_note": pk["fp8_note"],
+                             "fp8_tflops_spec": SPEC_FP8_TFLOPS,
+                             "fp8_tflops_scaled_mm": None if smm is None else round(smm, 1),
+                             "scaled_mm_how": "torch._scaled_mm e4m3, row-wise fp32 scales, bf16 out, "
+                                              "8192^3, best of 10 (library GEMM, off the product path)",
+                             "hbm_gbs_measured": pk["hbm"], "hbm_gbs_spec": SPEC_HBM_GBS},
+            "other_workloads": others,
             "gpu_launches": n_launch_per_step * args.steps,
             "clocks": clocks,
             "device_status": status,
@@ -648,6 +785,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="large", choices=sorted(WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extra", action="store_true",
+                    help="skip the other configurations' ops in a default single-GPU run")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         ap.error("--warmup must be >= 3")
