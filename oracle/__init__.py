@@ -10,7 +10,9 @@ arithmetic.
 The oracle is plain numpy, written for a reader to check against the pages by
 eye: FP8 decodes by table, quantization is fp32 IEEE round-to-nearest
 arithmetic with a table-search encoder, and the GEMM accumulates in fp64
-(exact for these formats and sizes).
+(exact for these formats and sizes). ``int8`` holds the int8 W8A8 build
+(exact integer GEMM), ``w4a16`` the 4-bit build over the exact QAT weights,
+``moe`` the mixture-of-experts layer.
 
 Pages cited (by title and section):
 
@@ -46,11 +48,13 @@ from .quantize import (
     qat_values,
 )
 from .gemm import rowwise_linear_ref, rowwise_linear_tolerance, check_linear, bf16_ulp
-from . import moe
+from .formats import bf16_rne_bits
+from . import int8, moe, w4a16
 
 __all__ = [
     "E4M3_MAX", "E4M3FNUZ_MAX", "dec_e4m3", "dec_e4m3fnuz", "enc_e4m3", "enc_e4m3fnuz",
     "QuantResult", "convert_fnuz_to_e4m3", "fnuz_copy_of_e4m3", "quant_act",
     "quantize_rows", "quantize_rows_fnuz", "repack_qat", "unpack_q4", "qat_values",
     "rowwise_linear_ref", "rowwise_linear_tolerance", "check_linear", "bf16_ulp", "moe",
+    "bf16_rne_bits", "int8", "w4a16",
 ]

@@ -114,3 +114,16 @@ def enc_e4m3(x) -> np.ndarray:
 def enc_e4m3fnuz(x) -> np.ndarray:
     """Encode values (exact in float64) to E4M3FNUZ bytes, RNE + saturation."""
     return _encode(x, _MAG_E4M3FNUZ, E4M3FNUZ_NAN)
+
+
+def bf16_rne_bits(v: np.ndarray) -> np.ndarray:
+    """fp64 values -> bf16 bit patterns (uint16), round to nearest even: bf16
+    keeps 8 significant bits, so the rounding quantum is 2^(e-8) for
+    v = m 2^e (0.5 <= |m| < 1), and 2^-133 in the subnormal range. Values past
+    the largest finite bf16 (after rounding) become Inf; NaN stays NaN."""
+    v = np.asarray(v, dtype=np.float64)
+    with np.errstate(invalid="ignore", over="ignore"):
+        _, e = np.frexp(v)
+        q = np.ldexp(1.0, np.maximum(e - 8, -133))
+        r = np.where(np.isfinite(v), np.round(v / q) * q, v)   # numpy rounds half to even
+        return (r.astype(np.float32).view(np.uint32) >> np.uint32(16)).astype(np.uint16)

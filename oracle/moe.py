@@ -34,6 +34,7 @@ from __future__ import annotations
 
 import numpy as np
 
+from .formats import bf16_rne_bits
 from .gemm import rowwise_linear_ref
 
 
@@ -96,24 +97,13 @@ def gelu_tanh(x: np.ndarray) -> np.ndarray:
         return x / (1.0 + np.exp(-2.0 * v))
 
 
-def _bf16_rne(v: np.ndarray) -> np.ndarray:
-    """fp64 -> bf16 bit patterns, round to nearest even: bf16 keeps 8
-    significant bits, so the rounding quantum is 2^(e-8) for v = m 2^e
-    (0.5 <= |m| < 1), and 2^-133 in the subnormal range."""
-    v = np.asarray(v, dtype=np.float64)
-    _, e = np.frexp(v)
-    q = np.ldexp(1.0, np.maximum(e - 8, -133))
-    r = np.round(v / q) * q                 # exact scaling; numpy rounds half to even
-    return (r.astype(np.float32).view(np.uint32) >> np.uint32(16)).astype(np.uint16)
-
-
 def geglu_bf16(gate_up_bits: np.ndarray, inter: int) -> np.ndarray:
     """h = bf16(gelu_tanh(gate) * up) from a [M, 2*inter] bf16 (uint16 bits)
     matrix holding gate in the first half and up in the second."""
     g = np.asarray(gate_up_bits, dtype=np.uint16)
     vals = (g.astype(np.uint32) << np.uint32(16)).view(np.float32).astype(np.float64)
     gate, up = vals[:, :inter], vals[:, inter:2 * inter]
-    return _bf16_rne(gelu_tanh(gate) * up)
+    return bf16_rne_bits(gelu_tanh(gate) * up)
 
 
 def combine(y_rows: np.ndarray, inv: np.ndarray, tokens: int, top_k: int,
