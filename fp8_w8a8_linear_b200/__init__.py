@@ -15,6 +15,8 @@ Functions mirror the C entry points:
 * :func:`cast_e4m3` - the element-wise encoder.
 * :func:`moe_route`, :func:`moe_gather`, :func:`grouped_linear`,
   :func:`moe_geglu_quant`, :func:`moe_combine` - the mixture-of-experts layer.
+* :func:`int8_repack_qat`, :func:`int8_quant_act`, :func:`int8_rowwise_linear`,
+  :func:`int8_linear` - the int8 W8A8 build.
 * :func:`device_status` - read and clear the device status word.
 """
 
@@ -58,6 +60,10 @@ _SIGS = {
     "fp8_grouped_linear_geglu": ([_P, _P, _P, ctypes.c_int32, _I64, _P, _P, _I64, _I64, _P, _P],
                                  ctypes.c_int),
     "fp8_moe_combine": ([_P, _P, _I64, ctypes.c_int32, _I64, _P, _P, _P], ctypes.c_int),
+    "int8_repack_qat": ([_P, _P, _I64, _I64, _P, _P, _P], ctypes.c_int),
+    "int8_quant_act": ([_P, _I64, _I64, _I64, _P, _P, _P], ctypes.c_int),
+    "int8_rowwise_linear": ([_P, _P, _P, _P, _I64, _I64, _I64, _P, _P], ctypes.c_int),
+    "int8_linear_bf16": ([_P, _P, _P, _I64, _I64, _I64, _P, _P, _P, _P], ctypes.c_int),
 }
 for _name, (_args, _ret) in _SIGS.items():
     _f = getattr(_lib, _name)
@@ -289,6 +295,63 @@ def moe_combine(rows: torch.Tensor, inv: torch.Tensor, tokens: int, top_k: int,
     return out
 
 
+# ------------------------------------------------------------------ int8 W8A8
+def int8_repack_qat(q4: torch.Tensor, d: torch.Tensor, w8: torch.Tensor | None = None,
+                    s_ch: torch.Tensor | None = None):
+    """q4 uint8 [N, K/2] and d float32 [N, K/32] -> (w8 int8 [N, K], s_ch float32 [N])."""
+    N, K2 = q4.shape
+    K = 2 * K2
+    w8 = torch.empty((N, K), dtype=torch.int8, device=q4.device) if w8 is None else w8
+    s_ch = torch.empty((N,), dtype=torch.float32, device=q4.device) if s_ch is None else s_ch
+    _check(_lib.int8_repack_qat(_dev(q4, torch.uint8, "q4"), _dev(d, torch.float32, "d", (N, K // 32)),
+                                N, K, _dev(w8, torch.int8, "w8", (N, K)),
+                                _dev(s_ch, torch.float32, "s_ch", (N,)), _stream()), "int8_repack_qat")
+    return w8, s_ch
+
+
+def int8_quant_act(x: torch.Tensor, x8: torch.Tensor | None = None, s_tok: torch.Tensor | None = None):
+    """x bf16 [M, K] -> (x8 int8 [M, K], s_tok float32 [M])."""
+    if x.dtype != torch.bfloat16 or x.dim() != 2 or x.stride(1) != 1 or not x.is_cuda:
+        raise ValueError("x must be a CUDA bf16 [M, K] tensor with unit inner stride")
+    M, K = x.shape
+    x8 = torch.empty((M, K), dtype=torch.int8, device=x.device) if x8 is None else x8
+    s_tok = torch.empty((M,), dtype=torch.float32, device=x.device) if s_tok is None else s_tok
+    _check(_lib.int8_quant_act(x.data_ptr(), M, K, x.stride(0), _dev(x8, torch.int8, "x8", (M, K)),
+                               _dev(s_tok, torch.float32, "s_tok", (M,)), _stream()), "int8_quant_act")
+    return x8, s_tok
+
+
+def int8_rowwise_linear(x8: torch.Tensor, s_tok: torch.Tensor, w8: torch.Tensor, s_ch: torch.Tensor,
+                        y: torch.Tensor | None = None):
+    """y bf16 [M, N] = (x8 . w8^T) * s_tok[:, None] * s_ch[None, :] with int8 operands."""
+    M, K = x8.shape
+    N = w8.shape[0]
+    y = torch.empty((M, N), dtype=torch.bfloat16, device=x8.device) if y is None else y
+    _check(_lib.int8_rowwise_linear(_dev(x8, torch.int8, "x8"), _dev(s_tok, torch.float32, "s_tok", (M,)),
+                                    _dev(w8, torch.int8, "w8", (N, K)),
+                                    _dev(s_ch, torch.float32, "s_ch", (N,)), M, N, K,
+                                    _dev(y, torch.bfloat16, "y", (M, N)), _stream()),
+           "int8_rowwise_linear")
+    return y
+
+
+def int8_linear(x: torch.Tensor, w8: torch.Tensor, s_ch: torch.Tensor, y: torch.Tensor | None = None,
+                x8: torch.Tensor | None = None, s_tok: torch.Tensor | None = None):
+    """The int8 W8A8 linear from bf16 activations: int8 quant per token, then GEMM."""
+    M, K = x.shape
+    N = w8.shape[0]
+    dev = x.device
+    y = torch.empty((M, N), dtype=torch.bfloat16, device=dev) if y is None else y
+    x8 = torch.empty((M, K), dtype=torch.int8, device=dev) if x8 is None else x8
+    s_tok = torch.empty((M,), dtype=torch.float32, device=dev) if s_tok is None else s_tok
+    _check(_lib.int8_linear_bf16(_dev(x, torch.bfloat16, "x"), _dev(w8, torch.int8, "w8", (N, K)),
+                                 _dev(s_ch, torch.float32, "s_ch", (N,)), M, N, K,
+                                 _dev(x8, torch.int8, "x8", (M, K)),
+                                 _dev(s_tok, torch.float32, "s_tok", (M,)),
+                                 _dev(y, torch.bfloat16, "y", (M, N)), _stream()), "int8_linear_bf16")
+    return y
+
+
 NOALLOC_SCRATCH_BYTES = 4 << 20
 
 
@@ -324,5 +387,6 @@ __all__ = [
     "convert_fnuz", "quant_act", "rowwise_linear", "linear", "linear_noalloc", "cast_e4m3",
     "moe_route", "moe_gather", "grouped_linear", "moe_geglu_quant", "moe_combine",
     "moe_interleave_gate_up", "grouped_linear_geglu",
+    "int8_repack_qat", "int8_quant_act", "int8_rowwise_linear", "int8_linear",
     "DEV_NONFINITE", "DEV_NAN_CODE", "DEV_INEXACT", "DEV_TIMEOUT", "LIB_PATH",
 ]

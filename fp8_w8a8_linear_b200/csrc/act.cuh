@@ -19,23 +19,28 @@ namespace fp8k {
 // With a = -2|v| <= 0 and e = exp(a) in (0, 1] (no overflow for any g):
 //   g >= 0:  sigmoid(2v) = 1 / (1 + e),   gelu = g / (1 + e);
 //   g <  0:  sigmoid(2v) = e / (1 + e),   gelu = g e / (1 + e).
-// On the common path -2|v| >= -86, so e >= 4e-38 is a normal number and
-// 1 + e lies in [1, 2]: the fast hardware exponential and division keep a
-// relative error below 1e-5 there (no flush to zero, no huge divisor), far
-// inside one bf16 ulp (2^-8), at a fraction of the accurate functions' cost -
-// this runs in the gate/up GEMM's epilogue for every element.
-// When g < 0 and -2v > 86 (g < -9.3), e is near or below the smallest normal
-// fp32 value and 1 + e == 1; the product g e up is then taken in the log
-// domain with the accurate functions, exp(2v + ln|g| + ln|up|), so that it
-// neither flushes through a subnormal intermediate nor depends on how small
-// e is (relative error below 1e-5).
+// On the common path -2|v| <= 86 (all g >= -9.3), e >= 4e-38 is a normal
+// number and 1 + e lies in [1, 2]: the hardware exponential and division
+// keep a relative error below 1e-5 there (no flush to zero, no huge divisor),
+// far inside one bf16 ulp (2^-8).
+// In the far negative tail (g < -9.3, -2v > 86) e is near or below the
+// smallest normal fp32 value and 1 + e == 1, so h = g e up, taken in the log
+// domain as exp(L), L = 2v + ln|g| + ln|up|: that neither flushes through a
+// subnormal intermediate nor depends on how small e is. exp(L) is evaluated
+// as exp(L + 64 ln 2) * 2^-64, so the hardware exponential always returns a
+// normal number (L >= -131.7) or underflows only where exp(L) < 1e-57, far
+// below the smallest bf16 subnormal; the multiply by 2^-64 is exact but for
+// one rounding onto the fp32 grid (2^-149). Relative error: below 2e-5.
+// Every step is a few hardware instructions: this runs for every element in
+// the gate/up GEMM's epilogue.
 __device__ __forceinline__ float geglu_f32(float g, float up) {
   constexpr float kA = -1.5957691216057308f;            // -2 sqrt(2/pi)
   constexpr float kB = -1.5957691216057308f * 0.044715f;
+  constexpr float k64Ln2 = 44.3614195558365f;           // 64 ln 2
   const float m2v = __fmul_rn(g, __fmaf_rn(kB, __fmul_rn(g, g), kA));  // -2v, sign opposite to g
   if (g < 0.0f && m2v > 86.0f) {
-    const float L = __fadd_rn(__fadd_rn(-m2v, logf(-g)), logf(fabsf(up)));
-    return copysignf(expf(L), -up);  // sign of g * up with g < 0
+    const float L = __fadd_rn(__fadd_rn(-m2v, __logf(-g)), __logf(fabsf(up)));
+    return copysignf(__fmul_rn(__expf(__fadd_rn(L, k64Ln2)), 0x1p-64f), -up);  // sign of g up
   }
   const float e = __expf(-fabsf(m2v));
   const float num = g < 0.0f ? __fmul_rn(g, e) : g;

@@ -109,10 +109,10 @@ fp8_status last_launch() {
 // ----------------------------------------------------------------- GEMM plans
 using namespace fp8k;
 
-template <int BN, int STAGES, bool GROUPED>
+template <int BN, int STAGES, bool GROUPED, int KD = kKindE4M3>
 fp8_status set_prefill_attr() {
   const size_t smem = PrefillCfg<BN, STAGES>::kSmem + (GROUPED ? grouped_smem_bytes(kMaxExperts) : 0);
-  return cudaFuncSetAttribute(gemm_prefill_kernel<BN, STAGES, GROUPED>,
+  return cudaFuncSetAttribute(gemm_prefill_kernel<BN, STAGES, GROUPED, KD>,
                               cudaFuncAttributeMaxDynamicSharedMemorySize,
                               static_cast<int>(smem)) == cudaSuccess
              ? FP8_OK
@@ -121,11 +121,11 @@ fp8_status set_prefill_attr() {
 
 // Deep-ring variants whose split-K layout would not fit are set up (and
 // launched) without a K split only.
-template <int BNT, int STAGES, int KBS>
+template <int BNT, int STAGES, int KBS, int KD = kKindE4M3>
 fp8_status set_decode_attr(int smem_optin) {
   using C = DecodeCfg<BNT, STAGES, KBS>;
   const size_t smem = C::kSmemSplit <= static_cast<size_t>(smem_optin) ? C::kSmemSplit : C::kSmemSingle;
-  return cudaFuncSetAttribute(gemm_decode_kernel<BNT, STAGES, KBS>,
+  return cudaFuncSetAttribute(gemm_decode_kernel<BNT, STAGES, KBS, KD>,
                               cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) ==
                  cudaSuccess
              ? FP8_OK
@@ -136,6 +136,12 @@ template <int STAGES>
 fp8_status set_pair_attr() {
   return cudaFuncSetAttribute(gemm_pair_kernel<STAGES>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                               static_cast<int>(PairCfg<STAGES>::kSmem)) == cudaSuccess &&
+                 cudaFuncSetAttribute(gemm_pair_kernel<STAGES, false, false, kKindS8>,
+                                      cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      static_cast<int>(PairCfg<STAGES>::kSmem)) == cudaSuccess &&
+                 cudaFuncSetAttribute(gemm_pair_kernel<STAGES, false, false, kKindBF16>,
+                                      cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      static_cast<int>(PairCfg<STAGES>::kSmem)) == cudaSuccess &&
                  cudaFuncSetAttribute(gemm_pair_kernel<STAGES, true>,
                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
                                       static_cast<int>(PairCfg<STAGES>::kSmem + grouped_smem_bytes(kMaxExperts))) ==
@@ -146,6 +152,23 @@ fp8_status set_pair_attr() {
                      cudaSuccess
              ? FP8_OK
              : FP8_ERR_CUDA;
+}
+
+// Every decode variant launch_linear can pick, for one operand kind.
+template <int KD>
+fp8_status set_decode_attrs(int so) {
+  fp8_status st = FP8_OK;
+  st = st != FP8_OK ? st : set_decode_attr<16, 2, 2, KD>(so);
+  st = st != FP8_OK ? st : set_decode_attr<16, 3, 2, KD>(so);
+  st = st != FP8_OK ? st : set_decode_attr<16, 6, 2, KD>(so);
+  st = st != FP8_OK ? st : set_decode_attr<32, 4, 1, KD>(so);
+  st = st != FP8_OK ? st : set_decode_attr<32, 3, 2, KD>(so);
+  st = st != FP8_OK ? st : set_decode_attr<64, 4, 1, KD>(so);
+  st = st != FP8_OK ? st : set_decode_attr<64, 4, 2, KD>(so);
+  st = st != FP8_OK ? st : set_decode_attr<128, 3, 1, KD>(so);
+  st = st != FP8_OK ? st : set_decode_attr<128, 4, 1, KD>(so);
+  st = st != FP8_OK ? st : set_decode_attr<128, 6, 1, KD>(so);
+  return st;
 }
 
 constexpr int kPairStages = 6;
@@ -168,6 +191,8 @@ fp8_status device_info(DeviceInfo** out) {
     if (!d.supported) return FP8_ERR_UNSUPPORTED;
     fp8_status st = FP8_OK;
     st = st != FP8_OK ? st : set_prefill_attr<kPrefillBN, kPrefillStages, false>();
+    st = st != FP8_OK ? st : set_prefill_attr<kPrefillBN, kPrefillStages, false, kKindS8>();
+    st = st != FP8_OK ? st : set_prefill_attr<kPrefillBN, kPrefillStages, false, kKindBF16>();
     st = st != FP8_OK ? st : set_prefill_attr<256, kPrefillStages, true>();
     st = st != FP8_OK ? st : set_pair_attr<kPairStages>();
     if (st == FP8_OK) {
@@ -190,21 +215,20 @@ fp8_status device_info(DeviceInfo** out) {
       d.pair_clusters = n;
     }
     const int so = d.smem_optin;
-    st = st != FP8_OK ? st : set_decode_attr<16, 2, 2>(so);
-    st = st != FP8_OK ? st : set_decode_attr<16, 3, 2>(so);
-    st = st != FP8_OK ? st : set_decode_attr<16, 6, 2>(so);
-    st = st != FP8_OK ? st : set_decode_attr<32, 4, 1>(so);
-    st = st != FP8_OK ? st : set_decode_attr<32, 3, 2>(so);
-    st = st != FP8_OK ? st : set_decode_attr<64, 4, 1>(so);
-    st = st != FP8_OK ? st : set_decode_attr<64, 4, 2>(so);
-    st = st != FP8_OK ? st : set_decode_attr<128, 3, 1>(so);
-    st = st != FP8_OK ? st : set_decode_attr<128, 4, 1>(so);
-    st = st != FP8_OK ? st : set_decode_attr<128, 6, 1>(so);
+    st = st != FP8_OK ? st : set_decode_attrs<kKindE4M3>(so);
+    st = st != FP8_OK ? st : set_decode_attrs<kKindS8>(so);
+    st = st != FP8_OK ? st : set_decode_attrs<kKindBF16>(so);
     if (st == FP8_OK &&
         (cudaFuncSetAttribute(quant_act_staged_kernel<false>,
                               cudaFuncAttributeMaxDynamicSharedMemorySize,
                               kStagedSmemBudget + 1024) != cudaSuccess ||
          cudaFuncSetAttribute(quant_act_staged_kernel<true>,
+                              cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              kStagedSmemBudget + 1024) != cudaSuccess ||
+         cudaFuncSetAttribute(quant_act_staged_kernel<false, kEncI8>,
+                              cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              kStagedSmemBudget + 1024) != cudaSuccess ||
+         cudaFuncSetAttribute(quant_act_staged_kernel<true, kEncI8>,
                               cudaFuncAttributeMaxDynamicSharedMemorySize,
                               kStagedSmemBudget + 1024) != cudaSuccess))
       st = FP8_ERR_CUDA;
@@ -213,8 +237,10 @@ fp8_status device_info(DeviceInfo** out) {
                              kStagedSmemBudget + 1024) != cudaSuccess)
       st = FP8_ERR_CUDA;
     if (st == FP8_OK &&
-        cudaFuncSetAttribute(repack_qat_staged_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             110 * 1024) != cudaSuccess)
+        (cudaFuncSetAttribute(repack_qat_staged_kernel<kEncE4M3>,
+                              cudaFuncAttributeMaxDynamicSharedMemorySize, 110 * 1024) != cudaSuccess ||
+         cudaFuncSetAttribute(repack_qat_staged_kernel<kEncI8>,
+                              cudaFuncAttributeMaxDynamicSharedMemorySize, 110 * 1024) != cudaSuccess))
       st = FP8_ERR_CUDA;
     if (st != FP8_OK) return st;
     d.attrs_set = true;
@@ -231,6 +257,9 @@ void set_pdl(cudaLaunchAttribute* a, int& n, bool pdl) {
   ++n;
 }
 
+// Operands are row-major [rows, K] arrays of 1-byte (E4M3, int8) or 2-byte
+// (bf16) elements; K here counts BYTES per row. A null scale means 1.
+template <int KD = kKindE4M3>
 fp8_status launch_prefill(const DeviceInfo& dev, const uint8_t* x8, const float* s_tok,
                           const uint8_t* w8, const float* s_ch, int M, int N, int K, uint16_t* y,
                           cudaStream_t stream, bool pdl) {
@@ -263,12 +292,13 @@ fp8_status launch_prefill(const DeviceInfo& dev, const uint8_t* x8, const float*
   g.group_m = group_m;
   CUtensorMap tmY;
   make_epilogue_store_map(&tmY, g, y, M, N);
-  if (cudaLaunchKernelEx(&cfg, gemm_prefill_kernel<BN, ST, false>, tmA, tmB, tmY, g) != cudaSuccess)
+  if (cudaLaunchKernelEx(&cfg, gemm_prefill_kernel<BN, ST, false, KD>, tmA, tmB, tmY, g) != cudaSuccess)
     return FP8_ERR_CUDA;
   return FP8_OK;
 }
 
 // Dense GEMM on 256 x 256 tiles per CTA pair (clusters of 2, persistent).
+template <int KD = kKindE4M3>
 fp8_status launch_pair(const DeviceInfo& dev, const uint8_t* x8, const float* s_tok,
                        const uint8_t* w8, const float* s_ch, int M, int N, int K, uint16_t* y,
                        cudaStream_t stream, bool pdl) {
@@ -309,7 +339,8 @@ fp8_status launch_pair(const DeviceInfo& dev, const uint8_t* x8, const float* s_
   g.group_m = std::min(tiles_m, 16);
   CUtensorMap tmY;
   make_epilogue_store_map(&tmY, g, y, M, N);
-  if (cudaLaunchKernelEx(&cfg, gemm_pair_kernel<kPairStages>, tmA, tmB, tmB, tmY, g) != cudaSuccess)
+  if (cudaLaunchKernelEx(&cfg, gemm_pair_kernel<kPairStages, false, false, KD>, tmA, tmB, tmB, tmY,
+                         g) != cudaSuccess)
     return FP8_ERR_CUDA;
   return FP8_OK;
 }
@@ -448,7 +479,7 @@ int decode_splits(const DeviceInfo& dev, int N, int K, int kbs) {
   return splits;
 }
 
-template <int BNT, int ST, int KBS>
+template <int BNT, int ST, int KBS, int KD = kKindE4M3>
 fp8_status launch_decode_t(const DeviceInfo& dev, const uint8_t* x8, const float* s_tok,
                            const uint8_t* w8, const float* s_ch, int M, int N, int K, uint16_t* y,
                            cudaStream_t stream, bool pdl, int force_splits = 0) {
@@ -481,12 +512,14 @@ fp8_status launch_decode_t(const DeviceInfo& dev, const uint8_t* x8, const float
   set_pdl(attrs, na, pdl);
   cfg.attrs = attrs;
   cfg.numAttrs = na;
-  if (cudaLaunchKernelEx(&cfg, gemm_decode_kernel<BNT, ST, KBS>, tmW, tmX, tmY, s_tok, s_ch, y, M,
+  if (cudaLaunchKernelEx(&cfg, gemm_decode_kernel<BNT, ST, KBS, KD>, tmW, tmX, tmY, s_tok, s_ch, y, M,
                          N, K, splits, steps_per_split, use_tma_store) != cudaSuccess)
     return FP8_ERR_CUDA;
   return FP8_OK;
 }
 
+// y = (a . b^T) * s_a * s_b for one operand kind; K counts bytes per row.
+template <int KD = kKindE4M3>
 fp8_status launch_linear(const DeviceInfo& dev, const uint8_t* x8, const float* s_tok,
                          const uint8_t* w8, const float* s_ch, int M, int N, int K, uint16_t* y,
                          cudaStream_t stream, bool pdl) {
@@ -506,22 +539,22 @@ fp8_status launch_linear(const DeviceInfo& dev, const uint8_t* x8, const float* 
     const int num_kb = (K + kBK - 1) / kBK;
     int s = 1;
     while (s < 8 && tiles * s * 2 <= 2 * dev.sm_count && s * 2 * 4 <= num_kb) s *= 2;
-    if (s >= 4) return launch_decode_t<16, 2, 2>(dev, x8, s_tok, w8, s_ch, M, N, K, y, stream, pdl, s);
+    if (s >= 4) return launch_decode_t<16, 2, 2, KD>(dev, x8, s_tok, w8, s_ch, M, N, K, y, stream, pdl, s);
     return one_per_sm && no_split
-               ? launch_decode_t<16, 6, 2>(dev, x8, s_tok, w8, s_ch, M, N, K, y, stream, pdl)
-               : launch_decode_t<16, 3, 2>(dev, x8, s_tok, w8, s_ch, M, N, K, y, stream, pdl);
+               ? launch_decode_t<16, 6, 2, KD>(dev, x8, s_tok, w8, s_ch, M, N, K, y, stream, pdl)
+               : launch_decode_t<16, 3, 2, KD>(dev, x8, s_tok, w8, s_ch, M, N, K, y, stream, pdl);
   }
   if (M <= 32)
-    return one_per_sm ? launch_decode_t<32, 3, 2>(dev, x8, s_tok, w8, s_ch, M, N, K, y, stream, pdl)
-                      : launch_decode_t<32, 4, 1>(dev, x8, s_tok, w8, s_ch, M, N, K, y, stream, pdl);
+    return one_per_sm ? launch_decode_t<32, 3, 2, KD>(dev, x8, s_tok, w8, s_ch, M, N, K, y, stream, pdl)
+                      : launch_decode_t<32, 4, 1, KD>(dev, x8, s_tok, w8, s_ch, M, N, K, y, stream, pdl);
   if (M <= 64)
-    return one_per_sm ? launch_decode_t<64, 4, 2>(dev, x8, s_tok, w8, s_ch, M, N, K, y, stream, pdl)
-                      : launch_decode_t<64, 4, 1>(dev, x8, s_tok, w8, s_ch, M, N, K, y, stream, pdl);
+    return one_per_sm ? launch_decode_t<64, 4, 2, KD>(dev, x8, s_tok, w8, s_ch, M, N, K, y, stream, pdl)
+                      : launch_decode_t<64, 4, 1, KD>(dev, x8, s_tok, w8, s_ch, M, N, K, y, stream, pdl);
   if (M <= 128) {
     if (!one_per_sm)
-      return launch_decode_t<128, 3, 1>(dev, x8, s_tok, w8, s_ch, M, N, K, y, stream, pdl);
-    return no_split ? launch_decode_t<128, 6, 1>(dev, x8, s_tok, w8, s_ch, M, N, K, y, stream, pdl)
-                    : launch_decode_t<128, 4, 1>(dev, x8, s_tok, w8, s_ch, M, N, K, y, stream, pdl);
+      return launch_decode_t<128, 3, 1, KD>(dev, x8, s_tok, w8, s_ch, M, N, K, y, stream, pdl);
+    return no_split ? launch_decode_t<128, 6, 1, KD>(dev, x8, s_tok, w8, s_ch, M, N, K, y, stream, pdl)
+                    : launch_decode_t<128, 4, 1, KD>(dev, x8, s_tok, w8, s_ch, M, N, K, y, stream, pdl);
   }
   // Prefill: 256 x 256 tiles on CTA pairs or 128 x 256 tiles on single SMs
   // (the same work per SM per tile). Pairs move a third less operand traffic
@@ -535,9 +568,9 @@ fp8_status launch_linear(const DeviceInfo& dev, const uint8_t* x8, const float* 
     const int64_t pair_waves = ((M + 255) / 256 * tiles_n + dev.pair_clusters - 1) / dev.pair_clusters;
     const int64_t sm_waves = ((M + kBM - 1) / kBM * tiles_n + dev.sm_count - 1) / dev.sm_count;
     if (pair_waves < sm_waves || (pair_waves == sm_waves && K >= 4096))
-      return launch_pair(dev, x8, s_tok, w8, s_ch, M, N, K, y, stream, pdl);
+      return launch_pair<KD>(dev, x8, s_tok, w8, s_ch, M, N, K, y, stream, pdl);
   }
-  return launch_prefill(dev, x8, s_tok, w8, s_ch, M, N, K, y, stream, pdl);
+  return launch_prefill<KD>(dev, x8, s_tok, w8, s_ch, M, N, K, y, stream, pdl);
 }
 
 // Blocks of a row-staged streaming kernel that fit on one SM at once (its
@@ -555,6 +588,7 @@ int64_t staged_blocks_per_sm(Kernel kernel, int threads, size_t smem) {
 // Every quantizer kernel waits for the preceding grid before it reads x and
 // writes nothing before that, so it is always launched as a programmatic
 // dependent: in a chain of linears it starts while the previous GEMM ends.
+template <int ENC = kEncE4M3>
 fp8_status launch_quant_act(const DeviceInfo& dev, const uint16_t* x, int64_t M, int64_t K,
                             int64_t ldx, uint8_t* x8, float* s_tok, cudaStream_t stream) {
   const int64_t nvec = K / 8;
@@ -566,11 +600,11 @@ fp8_status launch_quant_act(const DeviceInfo& dev, const uint16_t* x, int64_t M,
     // short rows still keep enough rows in flight.
     const int warps = static_cast<int>(staged_warps);
     const size_t smem = static_cast<size_t>(warps) * 2 * row_pad + 16 * warps;
-    const int64_t per_sm = staged_blocks_per_sm(quant_act_staged_kernel<false>, 32 * warps, smem);
+    const int64_t per_sm = staged_blocks_per_sm(quant_act_staged_kernel<false, ENC>, 32 * warps, smem);
     const int64_t blocks = std::min<int64_t>(per_sm * dev.sm_count, (M + warps - 1) / warps);
     // Short rows (16 or more warps per SM) are issue-bound: packed divisions.
-    const auto kernel = per_sm * warps >= 16 ? quant_act_staged_kernel<true>
-                                             : quant_act_staged_kernel<false>;
+    const auto kernel = per_sm * warps >= 16 ? quant_act_staged_kernel<true, ENC>
+                                             : quant_act_staged_kernel<false, ENC>;
     return launch_pdl_smem(kernel, dim3(static_cast<unsigned>(blocks)), dim3(32 * warps), smem,
                            stream, x, M, K, ldx, x8, s_tok, row_pad);
   }
@@ -579,19 +613,48 @@ fp8_status launch_quant_act(const DeviceInfo& dev, const uint16_t* x, int64_t M,
     // registers (one memory round trip for the amax, none for the quantize).
     const dim3 grid(static_cast<unsigned>(M));
     if (nvec <= 4 * 256)
-      return launch_pdl(quant_act_kernel<256, 4>, grid, dim3(256), stream, x, M, K, ldx, x8, s_tok);
-    return launch_pdl(quant_act_kernel<1024, 8, 1024>, grid, dim3(1024), stream, x, M, K, ldx, x8,
+      return launch_pdl(quant_act_kernel<256, 4, 256, ENC>, grid, dim3(256), stream, x, M, K, ldx, x8, s_tok);
+    return launch_pdl(quant_act_kernel<1024, 8, 1024, ENC>, grid, dim3(1024), stream, x, M, K, ldx, x8,
                       s_tok);
   }
   const dim3 grid(static_cast<unsigned>((M + 7) / 8));
   if (nvec <= 24 * 32)
-    return launch_pdl(quant_act_kernel<32, 24>, grid, dim3(256), stream, x, M, K, ldx, x8, s_tok);
-  return launch_pdl(quant_act_kernel<32, 0>, grid, dim3(256), stream, x, M, K, ldx, x8, s_tok);
+    return launch_pdl(quant_act_kernel<32, 24, 256, ENC>, grid, dim3(256), stream, x, M, K, ldx, x8, s_tok);
+  return launch_pdl(quant_act_kernel<32, 0, 256, ENC>, grid, dim3(256), stream, x, M, K, ldx, x8, s_tok);
 }
 
 bool dims_ok(int64_t v, int64_t lim) { return v >= 0 && v <= lim; }
 
 constexpr int64_t kMaxRows = (int64_t(1) << 31) - 1;
+
+// QAT q4_0 -> per-channel codes of one encoder (E4M3 or int8): checks, then
+// rows staged through shared memory (two blocks of 8 warps per SM) when K %
+// 128 == 0 and there are enough rows, else the register-cached kernel.
+template <int ENC>
+fp8_status repack_qat_checked(const uint8_t* q4, const float* d, int64_t N, int64_t K, uint8_t* w8,
+                              float* s_ch, cudaStream_t stream) {
+  if (!dims_ok(N, kMaxRows) || !dims_ok(K, int64_t(1) << 24)) return FP8_ERR_INVALID_ARG;
+  if (K % 32 != 0) return FP8_ERR_SHAPE;
+  if (N == 0) return FP8_OK;
+  if (!q4 || !d || !w8 || !s_ch) return FP8_ERR_INVALID_ARG;
+  if (!aligned16(q4) || !aligned16(w8) || !aligned4(d) || !aligned4(s_ch)) return FP8_ERR_ALIGNMENT;
+  DeviceInfo* dev;
+  if (fp8_status st = device_info(&dev)) return st;
+  const uint32_t rbuf = static_cast<uint32_t>((K / 2 + K / 8 + 127) / 128 * 128);
+  const size_t rsmem = size_t(8) * kRepackBufs * rbuf + 8 * 8 * kRepackBufs;
+  if (K % 128 == 0 && N >= 4 * dev->sm_count && rsmem <= 110 * 1024) {
+    const int64_t blocks = std::min<int64_t>(2 * dev->sm_count, (N + 7) / 8);
+    repack_qat_staged_kernel<ENC><<<static_cast<unsigned>(blocks), 256, rsmem, stream>>>(
+        q4, d, N, K, w8, s_ch, rbuf);
+    return last_launch();
+  }
+  const dim3 grid(static_cast<unsigned>((N + 7) / 8));
+  if (K / 32 <= 6 * 32)
+    repack_qat_kernel<32, 6, ENC><<<grid, 256, 0, stream>>>(q4, d, N, K, w8, s_ch);
+  else
+    repack_qat_kernel<32, 0, ENC><<<grid, 256, 0, stream>>>(q4, d, N, K, w8, s_ch);
+  return last_launch();
+}
 
 }  // namespace
 
@@ -631,30 +694,7 @@ fp8_status fp8_get_device_status(unsigned int* out) {
 
 fp8_status fp8_repack_qat(const uint8_t* q4, const float* d, int64_t N, int64_t K, uint8_t* w8,
                           float* s_ch, void* stream) {
-  if (!dims_ok(N, kMaxRows) || !dims_ok(K, int64_t(1) << 24)) return FP8_ERR_INVALID_ARG;
-  if (K % 32 != 0) return FP8_ERR_SHAPE;
-  if (N == 0) return FP8_OK;
-  if (!q4 || !d || !w8 || !s_ch) return FP8_ERR_INVALID_ARG;
-  if (!aligned16(q4) || !aligned16(w8) || !aligned4(d) || !aligned4(s_ch)) return FP8_ERR_ALIGNMENT;
-  DeviceInfo* dev;
-  if (fp8_status st = device_info(&dev)) return st;
-  const uint32_t rbuf = static_cast<uint32_t>((K / 2 + K / 8 + 127) / 128 * 128);
-  const size_t rsmem = size_t(8) * kRepackBufs * rbuf + 8 * 8 * kRepackBufs;
-  if (K % 128 == 0 && N >= 4 * dev->sm_count && rsmem <= 110 * 1024) {
-    // Rows staged through shared memory, two blocks of 8 warps per SM.
-    const uint32_t buf = rbuf;
-    const size_t smem = rsmem;
-    const int64_t blocks = std::min<int64_t>(2 * dev->sm_count, (N + 7) / 8);
-    repack_qat_staged_kernel<<<static_cast<unsigned>(blocks), 256, smem, as_stream(stream)>>>(
-        q4, d, N, K, w8, s_ch, buf);
-    return last_launch();
-  }
-  const dim3 grid(static_cast<unsigned>((N + 7) / 8));
-  if (K / 32 <= 6 * 32)
-    repack_qat_kernel<32, 6><<<grid, 256, 0, as_stream(stream)>>>(q4, d, N, K, w8, s_ch);
-  else
-    repack_qat_kernel<32, 0><<<grid, 256, 0, as_stream(stream)>>>(q4, d, N, K, w8, s_ch);
-  return last_launch();
+  return repack_qat_checked<kEncE4M3>(q4, d, N, K, w8, s_ch, as_stream(stream));
 }
 
 fp8_status fp8_convert_fnuz(const uint8_t* w8_fnuz, const float* s_fnuz, int64_t N, int64_t K,
@@ -901,6 +941,66 @@ fp8_status fp8_moe_combine(const uint16_t* rows, const int32_t* inv, int64_t tok
                       static_cast<int>(top_k), H, weights, out);
   return launch_pdl(moe_combine_kernel<kCombineMaxK>, grid, dim3(256), as_stream(stream), rows, inv,
                     tokens, static_cast<int>(top_k), H, weights, out);
+}
+
+// ------------------------------------------------------------ int8 W8A8 build
+fp8_status int8_repack_qat(const uint8_t* q4, const float* d, int64_t N, int64_t K, int8_t* w8,
+                           float* s_ch, void* stream) {
+  return repack_qat_checked<kEncI8>(q4, d, N, K, reinterpret_cast<uint8_t*>(w8), s_ch,
+                                    as_stream(stream));
+}
+
+fp8_status int8_quant_act(const uint16_t* x, int64_t M, int64_t K, int64_t ldx, int8_t* x8,
+                          float* s_tok, void* stream) {
+  if (!dims_ok(M, kMaxRows) || !dims_ok(K, int64_t(1) << 24) || ldx < K) return FP8_ERR_INVALID_ARG;
+  if (K % 16 != 0 || ldx % 8 != 0) return FP8_ERR_SHAPE;
+  if (M == 0 || K == 0) return FP8_OK;
+  if (!x || !x8 || !s_tok) return FP8_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(x8) || !aligned4(s_tok)) return FP8_ERR_ALIGNMENT;
+  DeviceInfo* dev;
+  if (fp8_status st = device_info(&dev)) return st;
+  return launch_quant_act<kEncI8>(*dev, x, M, K, ldx, reinterpret_cast<uint8_t*>(x8), s_tok,
+                                  as_stream(stream));
+}
+
+fp8_status int8_rowwise_linear(const int8_t* x8, const float* s_tok, const int8_t* w8,
+                               const float* s_ch, int64_t M, int64_t N, int64_t K, uint16_t* y,
+                               void* stream) {
+  if (fp8_status st = check_linear(x8, s_tok, reinterpret_cast<const uint8_t*>(w8), s_ch, M, N, K, y))
+    return st;
+  if (M == 0 || N == 0) return FP8_OK;
+  DeviceInfo* dev;
+  if (fp8_status st = device_info(&dev)) return st;
+  if (K == 0) {
+    if (cudaMemsetAsync(y, 0, static_cast<size_t>(M) * N * 2, as_stream(stream)) != cudaSuccess)
+      return FP8_ERR_CUDA;
+    return FP8_OK;
+  }
+  return launch_linear<kKindS8>(*dev, reinterpret_cast<const uint8_t*>(x8), s_tok,
+                                reinterpret_cast<const uint8_t*>(w8), s_ch, static_cast<int>(M),
+                                static_cast<int>(N), static_cast<int>(K), y, as_stream(stream), true);
+}
+
+fp8_status int8_linear_bf16(const uint16_t* x, const int8_t* w8, const float* s_ch, int64_t M,
+                            int64_t N, int64_t K, int8_t* x8, float* s_tok, uint16_t* y,
+                            void* stream) {
+  if (fp8_status st = check_linear(x, s_tok, reinterpret_cast<const uint8_t*>(w8), s_ch, M, N, K, y))
+    return st;
+  if (M == 0 || N == 0) return FP8_OK;
+  if (!x8) return FP8_ERR_INVALID_ARG;
+  if (!aligned16(x8)) return FP8_ERR_ALIGNMENT;
+  DeviceInfo* dev;
+  if (fp8_status st = device_info(&dev)) return st;
+  if (K == 0) {
+    if (cudaMemsetAsync(y, 0, static_cast<size_t>(M) * N * 2, as_stream(stream)) != cudaSuccess)
+      return FP8_ERR_CUDA;
+    return FP8_OK;
+  }
+  uint8_t* xq = reinterpret_cast<uint8_t*>(x8);
+  if (fp8_status st = launch_quant_act<kEncI8>(*dev, x, M, K, K, xq, s_tok, as_stream(stream))) return st;
+  return launch_linear<kKindS8>(*dev, xq, s_tok, reinterpret_cast<const uint8_t*>(w8), s_ch,
+                                static_cast<int>(M), static_cast<int>(N), static_cast<int>(K), y,
+                                as_stream(stream), true);
 }
 
 }  // extern "C"

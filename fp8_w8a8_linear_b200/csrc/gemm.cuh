@@ -139,7 +139,7 @@ __device__ __forceinline__ void epi_store_chunk(const uint4 (&pk)[4], uint8_t* s
 // this lane's row `row`), scaled by s_a of the row and the chunk's 32 column
 // scales (sb_chunk, staged in shared memory), rounded to bf16 and stored -
 // through store_chunk_coalesced when rows are 16-byte storable (warp-uniform
-// vec_ok), else element by element with the scales from global memory.
+// vec_ok), else element by element.
 //
 // With tma_ok (warp-uniform: a store tensor map over y exists and all 32
 // rows of the chunk belong to the tile's row range) the staged chunk leaves
@@ -147,7 +147,7 @@ __device__ __forceinline__ void epi_store_chunk(const uint4 (&pk)[4], uint8_t* s
 // the map clips columns at N); the buffer is reused only after the previous
 // store from it has read it.
 __device__ __forceinline__ void epi_chunk(const uint32_t (&r)[32], const float* sb_chunk,
-                                          const float* __restrict__ sb_glob, float sa, bool vec_ok,
+                                          float sa, bool vec_ok,
                                           uint8_t* stg, uint16_t* __restrict__ y, int row,
                                           int64_t row_end, int N, int n0, int lane,
                                           const CUtensorMap* tmY, bool tma_ok) {
@@ -174,7 +174,7 @@ __device__ __forceinline__ void epi_chunk(const uint32_t (&r)[32], const float* 
 #pragma unroll
     for (int j = 0; j < 32; ++j) {
       if (n0 + j < N) {
-        const float v = __fmul_rn(__fmul_rn(__uint_as_float(r[j]), sa), __ldg(sb_glob + n0 + j));
+        const float v = __fmul_rn(__fmul_rn(__uint_as_float(r[j]), sa), sb_chunk[j]);
         yrow[n0 + j] = f32_to_bf16_rn(v);
       }
     }
@@ -349,7 +349,7 @@ __device__ __forceinline__ Tile dense_tile(const GemmArgs& g, int t, int BN) {
 constexpr int kEpiWarps = 8;
 constexpr int kPrefillThreads = 64 + 32 * kEpiWarps;
 
-template <int BN, int STAGES, bool GROUPED>
+template <int BN, int STAGES, bool GROUPED, int KD = kKindE4M3>
 __global__ void __launch_bounds__(kPrefillThreads, 1)
     gemm_prefill_kernel(const __grid_constant__ CUtensorMap tmA,
                         const __grid_constant__ CUtensorMap tmB,
@@ -424,7 +424,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     }
   } else if (warp == 1) {
     if (lane == 0) {
-      constexpr uint32_t idesc = idesc_e4m3_f32(kBM, BN);
+      constexpr uint32_t idesc = idesc_kind<KD>(kBM, BN);
       int stage = 0;
       uint32_t phase = 0;
       int acc = 0;
@@ -442,8 +442,8 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
           const uint32_t b0 = smem_u32(sB + stage * C::kBBytes);
 #pragma unroll
           for (int k = k0; k < kBK / 32; ++k) {
-            umma_f8(d_tmem, sw128_kmajor_desc(a0 + 32 * k), sw128_kmajor_desc(b0 + 32 * k), idesc,
-                    (kb | k) != 0);
+            umma_kind<KD>(d_tmem, sw128_kmajor_desc(a0 + 32 * k), sw128_kmajor_desc(b0 + 32 * k),
+                          idesc, (kb | k) != 0);
           }
           umma_commit(empty0 + 8 * stage);
           if (++stage == STAGES) { stage = 0; phase ^= 1; }
@@ -477,7 +477,8 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         // epilogue thread (weight-side data, read before the tile is done;
         // every warp left the buffer's previous tile before the last barrier).
         const int col = T.col0 + (threadIdx.x - 64);
-        sb_tile[acc * 256 + (threadIdx.x - 64)] = col < N ? __ldg(g.s_b + T.sb_off + col) : 0.0f;
+        sb_tile[acc * 256 + (threadIdx.x - 64)] =
+            col < N ? (g.s_b ? __ldg(g.s_b + T.sb_off + col) : 1.0f) : 0.0f;
       }
       const bool got = mbar_wait(tfull0 + 8 * acc, acc_phase);
       // all epilogue warps: scales visible; leave together if any wait failed
@@ -485,8 +486,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       tc_fence_after();
       if (!waited) { pdl_wait(); waited = true; }
       const int row = T.a_row + quad * 32 + lane;
-      const float sa = row < T.row_end ? __ldg(g.s_a + row) : 0.0f;
-      const float* sb_base = g.s_b + T.sb_off;
+      const float sa = row < T.row_end ? (g.s_a ? __ldg(g.s_a + row) : 1.0f) : 0.0f;
       // whole 32-row chunk inside the tile's rows: one TMA store per chunk
       const bool tma_rows = g.use_tma_store && (row - lane) + 32 <= T.row_end;
       const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + acc * BN;
@@ -496,7 +496,8 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         uint32_t r[32];
         tmem_ld32(t_row + c * 32, r);
         tmem_ld_wait();
-        epi_chunk(r, sb_tile + acc * 256 + c * 32, sb_base, sa, vec_ok, stg, g.y, row, T.row_end, N,
+        acc_to_f32<KD>(r);
+        epi_chunk(r, sb_tile + acc * 256 + c * 32, sa, vec_ok, stg, g.y, row, T.row_end, N,
                   T.col0 + c * 32, lane, &tmY, tma_rows);
       }
       tc_fence_before();
@@ -556,13 +557,14 @@ struct PairCfg {
 // is half width: each CTA loads 64 B rows (through tmBh, a map with 64-row
 // boxes) and the MMAs run with N = 128, so the leader's gate rows fill
 // accumulator columns 0..63 and the peer's up rows columns 64..127.
-template <int STAGES, bool GROUPED = false, bool GEGLU = false>
+template <int STAGES, bool GROUPED = false, bool GEGLU = false, int KD = kKindE4M3>
 __global__ void __launch_bounds__(kPrefillThreads, 1)
     gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                      const __grid_constant__ CUtensorMap tmBh, const __grid_constant__ CUtensorMap tmY,
                      const GemmArgs g) {
   using C = PairCfg<STAGES>;
   static_assert(GROUPED || !GEGLU, "the GeGLU epilogue is for the grouped GEMM");
+  static_assert(!GEGLU || KD == kKindE4M3, "the GeGLU epilogue is for E4M3 operands");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
   uint8_t* sA = smem;
@@ -658,8 +660,8 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     }
   } else if (warp == 1) {
     if (lane == 0 && rank == 0) {
-      constexpr uint32_t kIdescFull = idesc_e4m3_f32(256, C::kBN);
-      constexpr uint32_t kIdescHalf = idesc_e4m3_f32(256, C::kBN / 2);
+      constexpr uint32_t kIdescFull = idesc_kind<KD>(256, C::kBN);
+      constexpr uint32_t kIdescHalf = idesc_kind<KD>(256, C::kBN / 2);
       int stage = 0;
       uint32_t phase = 0;
       int acc = 0;
@@ -678,8 +680,8 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
           const uint32_t b0 = smem_u32(sB + stage * C::kBBytes);
 #pragma unroll
           for (int k = k0; k < kBK / 32; ++k) {
-            umma_f8_pair(d_tmem, sw128_kmajor_desc(a0 + 32 * k), sw128_kmajor_desc(b0 + 32 * k), idesc,
-                         (kb | k) != 0);
+            umma_kind_pair<KD>(d_tmem, sw128_kmajor_desc(a0 + 32 * k), sw128_kmajor_desc(b0 + 32 * k),
+                               idesc, (kb | k) != 0);
           }
           umma_commit_pair(empty0 + 8 * stage, 0x3);
           if (++stage == STAGES) { stage = 0; phase ^= 1; }
@@ -721,7 +723,12 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     auto fetch_scales = [&](const Tile& Tt, float4& sbv, float& sav) {
       const int col = Tt.col0 + scol;
       const float* src = g.s_b + Tt.sb_off + col;
-      if (vec_ok) {  // N % 8 == 0: the lane's 4 columns are all inside N or all past it
+      if (!g.s_b) {  // unscaled columns
+        sbv.x = col < N ? 1.0f : 0.0f;
+        sbv.y = col + 1 < N ? 1.0f : 0.0f;
+        sbv.z = col + 2 < N ? 1.0f : 0.0f;
+        sbv.w = col + 3 < N ? 1.0f : 0.0f;
+      } else if (vec_ok) {  // N % 8 == 0: the lane's 4 columns are all inside N or all past it
         sbv = col < N ? __ldg(reinterpret_cast<const float4*>(src)) : make_float4(0.f, 0.f, 0.f, 0.f);
       } else {
         sbv.x = col < N ? __ldg(src) : 0.0f;
@@ -730,7 +737,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         sbv.w = col + 3 < N ? __ldg(src + 3) : 0.0f;
       }
       const int rr = Tt.a_row + rank * C::kHalf + quad * 32 + lane;
-      sav = rr < Tt.row_end ? __ldg(g.s_a + rr) : 0.0f;
+      sav = rr < Tt.row_end ? (g.s_a ? __ldg(g.s_a + rr) : 1.0f) : 0.0f;
     };
     Tile T = {}, T1 = {};
     float4 sb_v = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -754,7 +761,6 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       if (!__all_sync(0xFFFFFFFFu, got)) break;
       tc_fence_after();
       const int row = T.a_row + rank * C::kHalf + quad * 32 + lane;
-      const float* sb_base = g.s_b + T.sb_off;
       // whole 32-row chunk inside the tile's rows: one TMA store per chunk
       const bool tma_rows = g.use_tma_store && (row - lane) + 32 <= T.row_end;
       const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + acc * C::kBN;
@@ -805,8 +811,9 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
           uint32_t r[32];
           tmem_ld32(t_row + c * 32, r);
           tmem_ld_wait();
-          epi_chunk(r, sbw + (c - half * kCh) * 32, sb_base, sa, vec_ok, stg, g.y, row, T.row_end,
-                    N, T.col0 + c * 32, lane, &tmY, tma_rows);
+          acc_to_f32<KD>(r);
+          epi_chunk(r, sbw + (c - half * kCh) * 32, sa, vec_ok, stg, g.y, row, T.row_end, N,
+                    T.col0 + c * 32, lane, &tmY, tma_rows);
         }
       }
       tc_fence_before();
@@ -854,7 +861,7 @@ struct DecodeCfg {
 
 // y is written either by one TMA store per output tile (tmY valid, N % 8 == 0;
 // its box is {rows written per CTA, BNT}) or element by element.
-template <int BNT, int STAGES, int KBS>
+template <int BNT, int STAGES, int KBS, int KD = kKindE4M3>
 __global__ void __launch_bounds__(192)
     gemm_decode_kernel(const __grid_constant__ CUtensorMap tmW,
                        const __grid_constant__ CUtensorMap tmX,
@@ -953,7 +960,7 @@ __global__ void __launch_bounds__(192)
     }
   } else if (warp == 1) {
     if (lane == 0 && have_acc) {
-      constexpr uint32_t idesc = idesc_e4m3_f32(kBM, BNT);
+      constexpr uint32_t idesc = idesc_kind<KD>(kBM, BNT);
       int stage = 0;
       uint32_t phase = 0;
       for (int st = st0; st < st1; ++st) {
@@ -965,8 +972,8 @@ __global__ void __launch_bounds__(192)
           const uint32_t b0 = smem_u32(sX + (stage * KBS + j) * C::kXBytes);
 #pragma unroll
           for (int k = 0; k < kBK / 32; ++k) {
-            umma_f8(tmem_base, sw128_kmajor_desc(a0 + 32 * k), sw128_kmajor_desc(b0 + 32 * k),
-                    idesc, (st != st0) || (j != 0) || (k != 0));
+            umma_kind<KD>(tmem_base, sw128_kmajor_desc(a0 + 32 * k), sw128_kmajor_desc(b0 + 32 * k),
+                          idesc, (st != st0) || (j != 0) || (k != 0));
           }
         }
         umma_commit(empty0 + 8 * stage);
@@ -981,9 +988,9 @@ __global__ void __launch_bounds__(192)
     // Stage both scale vectors while the main loop runs.
     {
       const int n = tile_n * kBM + et;
-      sch_s[et] = n < N ? __ldg(s_ch + n) : 0.0f;
+      sch_s[et] = n < N ? (s_ch ? __ldg(s_ch + n) : 1.0f) : 0.0f;
       pdl_wait();  // per-token scales come from a preceding quantizer grid
-      if (et < BNT) stok_s[et] = et < M ? s_tok[et] : 0.0f;
+      if (et < BNT) stok_s[et] = et < M ? (s_tok ? s_tok[et] : 1.0f) : 0.0f;
       named_bar_sync(1, 128);
     }
     if (have_acc && !mbar_wait(tfull, 0)) have_acc = false;
@@ -1002,15 +1009,19 @@ __global__ void __launch_bounds__(192)
       uint32_t r[16];
       tmem_ld16(t_row + c * 16, r);
       tmem_ld_wait();
+      // split partials travel as raw accumulator words (int32 for kind::i8,
+      // summed exactly by the owner); a single CTA converts them here
+      if (!split) acc_to_f32<KD>(r);
 #pragma unroll
       for (int j = 0; j < 16; ++j) {
         const int tok = c * 16 + j;
-        const float acc = have_acc ? __uint_as_float(r[j]) : 0.0f;
+        const uint32_t word = have_acc ? r[j] : 0u;  // 0u is both 0.0f and int 0
         if (!split) {
-          ytile[tok * kBM + ch] = f32_to_bf16_rn(__fmul_rn(__fmul_rn(acc, stok_s[tok]), sc));
+          ytile[tok * kBM + ch] =
+              f32_to_bf16_rn(__fmul_rn(__fmul_rn(__uint_as_float(word), stok_s[tok]), sc));
         } else if (tok < M) {
           // owner's buffer [rank][token][row in slice]: lanes write consecutive words
-          st_shared_cluster_f32(dst + static_cast<uint32_t>(tok * rows * 4), acc);
+          st_shared_cluster_f32(dst + static_cast<uint32_t>(tok * rows * 4), __uint_as_float(word));
         }
       }
     }
@@ -1031,8 +1042,15 @@ __global__ void __launch_bounds__(192)
       for (int e = et; e < rows * BNT; e += 128) {
         const int tok = e / rows;
         const int rl = e % rows;
-        float sum = red[tok * rows + rl];
-        for (int j = 1; j < splits; ++j) sum = __fadd_rn(sum, red[(j * BNT + tok) * rows + rl]);
+        float sum;
+        if constexpr (KD == kKindS8) {  // exact int32 sum, one rounding to fp32
+          int isum = __float_as_int(red[tok * rows + rl]);
+          for (int j = 1; j < splits; ++j) isum += __float_as_int(red[(j * BNT + tok) * rows + rl]);
+          sum = __int2float_rn(isum);
+        } else {
+          sum = red[tok * rows + rl];
+          for (int j = 1; j < splits; ++j) sum = __fadd_rn(sum, red[(j * BNT + tok) * rows + rl]);
+        }
         ytile[tok * rows + rl] =
             f32_to_bf16_rn(__fmul_rn(__fmul_rn(sum, stok_s[tok]), sch_s[rank * rows + rl]));
       }

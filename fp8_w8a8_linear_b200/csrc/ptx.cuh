@@ -257,6 +257,59 @@ __host__ __device__ constexpr uint32_t idesc_e4m3_f32(int m, int n) {
   return (1u << 4) | (static_cast<uint32_t>(n >> 3) << 17) | (static_cast<uint32_t>(m >> 4) << 24);
 }
 
+// Operand kinds of the GEMM kernels: E4M3 x E4M3 -> fp32 (kind::f8f6f4),
+// signed int8 x int8 -> int32 (kind::i8, exact), bf16 x bf16 -> fp32
+// (kind::f16). Every kind takes 32 bytes of K per instruction, so the
+// 128-byte swizzled stages serve all three: 128 E4M3 / int8 values or 64 bf16
+// values per row.
+enum MmaKind : int { kKindE4M3 = 0, kKindS8 = 1, kKindBF16 = 2 };
+
+// Instruction descriptor of a kind: D format (bits [4,6)) fp32 = 1 or s32 =
+// 2; A and B formats (bits [7,10) and [10,13)) E4M3 = 0 for kind::f8f6f4,
+// signed = 1 for kind::i8, bf16 = 1 for kind::f16; both operands K-major;
+// N >> 3 at bits [17,23), M >> 4 at bits [24,29).
+template <int KD>
+__host__ __device__ constexpr uint32_t idesc_kind(int m, int n) {
+  return (static_cast<uint32_t>(KD == kKindS8 ? 2 : 1) << 4) |
+         (static_cast<uint32_t>(KD == kKindE4M3 ? 0 : 1) << 7) |
+         (static_cast<uint32_t>(KD == kKindE4M3 ? 0 : 1) << 10) |
+         (static_cast<uint32_t>(n >> 3) << 17) | (static_cast<uint32_t>(m >> 4) << 24);
+}
+static_assert(idesc_kind<kKindE4M3>(128, 256) == idesc_e4m3_f32(128, 256), "E4M3 descriptor");
+
+// D[tmem] (+)= A * B^T of the given kind, issued by one thread (cta_group::1).
+template <int KD>
+__device__ __forceinline__ void umma_kind(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                          uint32_t idesc, uint32_t accumulate) {
+  if constexpr (KD == kKindE4M3) {
+    umma_f8(d_tmem, a_desc, b_desc, idesc, accumulate);
+  } else if constexpr (KD == kKindS8) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+  } else {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+  }
+}
+
+// Accumulator words as fp32 values: kind::i8 accumulates exact int32, which
+// the epilogue converts with one IEEE rounding (cvt.rn.f32.s32).
+template <int KD, int N>
+__device__ __forceinline__ void acc_to_f32(uint32_t (&r)[N]) {
+  if constexpr (KD == kKindS8) {
+#pragma unroll
+    for (int j = 0; j < N; ++j) r[j] = __float_as_uint(__int2float_rn(static_cast<int>(r[j])));
+  }
+}
+
 // ------------------------------------------------- CTA-pair (cta_group::2)
 // The pair's TMEM allocation / release: one warp with the same warp index in
 // each CTA of the pair executes each of these; both pass the same holder.
@@ -283,6 +336,28 @@ __device__ __forceinline__ void umma_f8_pair(uint32_t d_tmem, uint64_t a_desc, u
       "tcgen05.mma.cta_group::2.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
       "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
       : "memory");
+}
+// The pair MMA of the given kind (see umma_f8_pair).
+template <int KD>
+__device__ __forceinline__ void umma_kind_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                               uint32_t idesc, uint32_t accumulate) {
+  if constexpr (KD == kKindE4M3) {
+    umma_f8_pair(d_tmem, a_desc, b_desc, idesc, accumulate);
+  } else if constexpr (KD == kKindS8) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::i8 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+  } else {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+  }
 }
 // Arrive once on the barrier at offset `bar` in every CTA of `cta_mask` when
 // the pair MMAs issued so far are done.

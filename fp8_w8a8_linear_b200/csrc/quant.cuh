@@ -29,6 +29,31 @@ namespace fp8k {
 
 constexpr float kE4M3Max = 448.0f;
 
+// Encoders of the per-row quantizers. E4M3: round to nearest even, saturating
+// at +-448, zero always +0 (the FP8 build). INT8: the int8 W8A8 build (sizes
+// article, "The Sizes and the Builds": int8 weights per channel and int8
+// activations per token; E2B article, "它们离训练权重有多近？": 255 levels per
+// row): scale amax / 127 and code = clamp(RNE(q), -127, 127) as a two's
+// complement byte. Both take the same correctly rounded quotient q = v / s.
+enum QuantEnc : int { kEncE4M3 = 0, kEncI8 = 1 };
+
+template <int ENC>
+__host__ __device__ constexpr float enc_max() { return ENC == kEncE4M3 ? kE4M3Max : 127.0f; }
+
+__device__ __forceinline__ uint32_t i8_code(float q) {
+  return static_cast<uint32_t>(max(-127, min(127, __float2int_rn(q)))) & 0xFFu;
+}
+
+// Four codes packed little-endian (value a in byte 0).
+template <int ENC>
+__device__ __forceinline__ uint32_t pack4_codes(float a, float b, float c, float d) {
+  if constexpr (ENC == kEncE4M3) {
+    return pack4_e4m3(a, b, c, d);
+  } else {
+    return i8_code(a) | (i8_code(b) << 8) | (i8_code(c) << 16) | (i8_code(d) << 24);
+  }
+}
+
 // Correctly rounded v / s for a fixed divisor s (one row's scale). With
 // r = RN(1/s) computed once (__frcp_rn), q0 = RN(v * r) is within 1.5 ulp of
 // v/s; one correction q1 = RN(q0 + RN(v - q0 s) r) brings it within one ulp,
@@ -117,7 +142,7 @@ __device__ __forceinline__ uint32_t row_max_u32(uint32_t v, uint32_t* red) {
 // x: [M, ldx] bf16, K % 8 == 0 (16-byte vectors of 8 values).
 // BLOCK threads per block, TPR threads per row, V cached 16-byte vectors per
 // thread (the row is read from memory once when K / 8 <= V * TPR).
-template <int TPR, int V, int BLOCK = 256>
+template <int TPR, int V, int BLOCK = 256, int ENC = kEncE4M3>
 __global__ void __launch_bounds__(BLOCK) quant_act_kernel(const uint16_t* __restrict__ x, int64_t M,
                                                            int64_t K, int64_t ldx,
                                                            uint8_t* __restrict__ x8,
@@ -164,7 +189,7 @@ __global__ void __launch_bounds__(BLOCK) quant_act_kernel(const uint16_t* __rest
     if (t == 0) report(FP8_DEV_NONFINITE);
   }
   const float amax = __uint_as_float(amax_bits << 16);
-  const float s = __fdiv_rn(amax, kE4M3Max);
+  const float s = __fdiv_rn(amax, enc_max<ENC>());
   if (t == 0) s_tok[row] = s;
   uint2* dst = reinterpret_cast<uint2*>(x8 + row * K);
   const RowDivisor dv = make_divisor(s, amax);
@@ -186,7 +211,7 @@ __global__ void __launch_bounds__(BLOCK) quant_act_kernel(const uint16_t* __rest
         f[2 * i + 1] = div_rn(dv, __uint_as_float(w[i] & 0xFFFF0000u));
       }
     }
-    return make_uint2(pack4_e4m3(f[0], f[1], f[2], f[3]), pack4_e4m3(f[4], f[5], f[6], f[7]));
+    return make_uint2(pack4_codes<ENC>(f[0], f[1], f[2], f[3]), pack4_codes<ENC>(f[4], f[5], f[6], f[7]));
   };
 
   if (V > 0 && nvec <= static_cast<int64_t>(V) * TPR) {
@@ -210,7 +235,7 @@ __global__ void __launch_bounds__(BLOCK) quant_act_kernel(const uint16_t* __rest
 // with many warps per SM, where issue slots are what limits short rows; with
 // few warps per SM (long rows) the scalar form's independent chains hide
 // latency better.
-template <bool PACKED>
+template <bool PACKED, int ENC = kEncE4M3>
 __global__ void __launch_bounds__(256) quant_act_staged_kernel(const uint16_t* __restrict__ x,
                                                                 int64_t M, int64_t K, int64_t ldx,
                                                                 uint8_t* __restrict__ x8,
@@ -263,7 +288,7 @@ __global__ void __launch_bounds__(256) quant_act_staged_kernel(const uint16_t* _
     const uint32_t amax_bits = __reduce_max_sync(0xFFFFFFFFu, mx);
     if (amax_bits >= 0x7F80u && lane == 0) report(FP8_DEV_NONFINITE);
     const float amax = __uint_as_float(amax_bits << 16);
-    const float s = __fdiv_rn(amax, kE4M3Max);
+    const float s = __fdiv_rn(amax, enc_max<ENC>());
     if (lane == 0) s_tok[row] = s;
     const RowDivisor dv = make_divisor(s, amax);
     uint2* dst = reinterpret_cast<uint2*>(x8 + row * K);
@@ -286,8 +311,7 @@ __global__ void __launch_bounds__(256) quant_act_staged_kernel(const uint16_t* _
             f[2 * i + 1] = div_rn(dv, __uint_as_float(wv[i] & 0xFFFF0000u));
           }
         }
-        dst[j] = make_uint2(canon_zero4(cvt_e4m3x2(f[1], f[0]) | (cvt_e4m3x2(f[3], f[2]) << 16)),
-                            canon_zero4(cvt_e4m3x2(f[5], f[4]) | (cvt_e4m3x2(f[7], f[6]) << 16)));
+        dst[j] = make_uint2(pack4_codes<ENC>(f[0], f[1], f[2], f[3]), pack4_codes<ENC>(f[4], f[5], f[6], f[7]));
       }
     } else {
       for (int64_t j = lane; j < nvec; j += 32) {
@@ -299,8 +323,7 @@ __global__ void __launch_bounds__(256) quant_act_staged_kernel(const uint16_t* _
           f[2 * i] = __fdiv_rn(__uint_as_float(wv[i] << 16), s);
           f[2 * i + 1] = __fdiv_rn(__uint_as_float(wv[i] & 0xFFFF0000u), s);
         }
-        dst[j] = make_uint2(canon_zero4(cvt_e4m3x2(f[1], f[0]) | (cvt_e4m3x2(f[3], f[2]) << 16)),
-                            canon_zero4(cvt_e4m3x2(f[5], f[4]) | (cvt_e4m3x2(f[7], f[6]) << 16)));
+        dst[j] = make_uint2(pack4_codes<ENC>(f[0], f[1], f[2], f[3]), pack4_codes<ENC>(f[4], f[5], f[6], f[7]));
       }
     }
     __syncwarp();  // every lane is done reading this buffer before it is refilled
@@ -322,13 +345,20 @@ struct GroupLUT {
 
 // Codes of q = 1..8 from their fp32 quotients f[q-1] (canonical zeros), and
 // the table built from them.
+template <int ENC = kEncE4M3>
 __device__ __forceinline__ GroupLUT group_lut_from(const float (&f)[8]) {
-  const uint32_t p0 = canon_zero4(cvt_e4m3x2(f[1], f[0]) | (cvt_e4m3x2(f[3], f[2]) << 16));
-  const uint32_t p1 = canon_zero4(cvt_e4m3x2(f[5], f[4]) | (cvt_e4m3x2(f[7], f[6]) << 16));
-  // Negation flips bit 7 of every nonzero code (d may be negative, so the
-  // codes of q = 1..8 can carry either sign); a code is zero only as 0x00.
+  const uint32_t p0 = pack4_codes<ENC>(f[0], f[1], f[2], f[3]);
+  const uint32_t p1 = pack4_codes<ENC>(f[4], f[5], f[6], f[7]);
+  // E4M3: negation flips bit 7 of every nonzero code (d may be negative, so
+  // the codes of q = 1..8 can carry either sign); a code is zero only as
+  // 0x00. INT8: two's complement negation of each byte (codes lie in
+  // -127..127, so it never overflows).
   auto negate4 = [](uint32_t p) {
-    return p ^ ((((p & 0x7F7F7F7Fu) + 0x7F7F7F7Fu) | p) & 0x80808080u);
+    if constexpr (ENC == kEncE4M3) {
+      return p ^ ((((p & 0x7F7F7F7Fu) + 0x7F7F7F7Fu) | p) & 0x80808080u);
+    } else {
+      return static_cast<uint32_t>(__vneg4(p));
+    }
   };
   const uint32_t n0 = negate4(p0);
   const uint32_t n1 = negate4(p1);
@@ -348,6 +378,7 @@ __device__ __forceinline__ GroupLUT group_lut_from(const float (&f)[8]) {
 // by 2 is exact, so fp32(d*2q) = 2 fp32(d*q) and fp32(2w/s) = 2 fp32(w/s);
 // the even q's quotients are therefore doublings, bit for bit. (Quotients
 // too small to be normal encode to 0 either way.)
+template <int ENC = kEncE4M3>
 __device__ __forceinline__ GroupLUT group_lut_fast(float d, const RowDivisor2& dv2) {
   float f[8];
   div2_rn(dv2, d, __fmul_rn(d, 3.0f), f[0], f[2]);
@@ -356,15 +387,16 @@ __device__ __forceinline__ GroupLUT group_lut_fast(float d, const RowDivisor2& d
   f[3] = __fmul_rn(f[1], 2.0f);
   f[5] = __fmul_rn(f[2], 2.0f);
   f[7] = __fmul_rn(f[3], 2.0f);
-  return group_lut_from(f);
+  return group_lut_from<ENC>(f);
 }
 
 // Same table with IEEE division for each q (rows with tiny amax).
+template <int ENC = kEncE4M3>
 __device__ __forceinline__ GroupLUT group_lut_slow(float d, float s) {
   float f[8];
 #pragma unroll
   for (int q = 1; q <= 8; ++q) f[q - 1] = __fdiv_rn(__fmul_rn(d, static_cast<float>(q)), s);
-  return group_lut_from(f);
+  return group_lut_from<ENC>(f);
 }
 
 // Four nibbles (the low 16 bits of `chunk`, nibble i -> output byte i): look
@@ -399,7 +431,7 @@ __device__ __forceinline__ uint32_t group_maxabs(const uint4& u) {
   return m;
 }
 
-template <int TPR, int V>
+template <int TPR, int V, int ENC = kEncE4M3>
 __global__ void __launch_bounds__(256) repack_qat_kernel(const uint8_t* __restrict__ q4,
                                                           const float* __restrict__ d, int64_t N,
                                                           int64_t K, uint8_t* __restrict__ w8,
@@ -445,7 +477,7 @@ __global__ void __launch_bounds__(256) repack_qat_kernel(const uint8_t* __restri
     if (t == 0) report(FP8_DEV_NONFINITE);
   }
   const float amax = __uint_as_float(amax_bits);
-  const float s = __fdiv_rn(amax, kE4M3Max);
+  const float s = __fdiv_rn(amax, enc_max<ENC>());
   if (t == 0) s_ch[row] = s;
   uint4* dst = reinterpret_cast<uint4*>(w8 + row * K);
   const RowDivisor dv = make_divisor(s, amax);
@@ -457,7 +489,7 @@ __global__ void __launch_bounds__(256) repack_qat_kernel(const uint8_t* __restri
       o0 = make_uint4(0, 0, 0, 0);
       o1 = o0;
     } else {
-      const GroupLUT L = dv.fast ? group_lut_fast(dg, dv2) : group_lut_slow(dg, s);
+      const GroupLUT L = dv.fast ? group_lut_fast<ENC>(dg, dv2) : group_lut_slow<ENC>(dg, s);
       o0.x = lut4(L, u.x);
       o0.y = lut4(L, u.x >> 16);
       o0.z = lut4(L, u.y);
@@ -502,6 +534,7 @@ __device__ __forceinline__ void emit_group(uint4* dst, const uint4& u, const Gro
 // so several rows per warp are in flight while one is encoded.
 constexpr int kRepackBufs = 3;
 
+template <int ENC = kEncE4M3>
 __global__ void __launch_bounds__(256) repack_qat_staged_kernel(const uint8_t* __restrict__ q4,
                                                                  const float* __restrict__ d,
                                                                  int64_t N, int64_t K,
@@ -549,7 +582,7 @@ __global__ void __launch_bounds__(256) repack_qat_staged_kernel(const uint8_t* _
     const uint32_t amax_bits = __reduce_max_sync(0xFFFFFFFFu, mbits);
     if (amax_bits >= 0x7F800000u && lane == 0) report(FP8_DEV_NONFINITE);
     const float amax = __uint_as_float(amax_bits);
-    const float s = __fdiv_rn(amax, kE4M3Max);
+    const float s = __fdiv_rn(amax, enc_max<ENC>());
     if (lane == 0) s_ch[row] = s;
     const RowDivisor dv = make_divisor(s, amax);
     uint4* dst = reinterpret_cast<uint4*>(w8 + row * K);
@@ -561,9 +594,9 @@ __global__ void __launch_bounds__(256) repack_qat_staged_kernel(const uint8_t* _
     } else if (dv.fast) {
       const RowDivisor2 dv2 = make_divisor2(dv);
 #pragma unroll 2
-      for (int64_t g = lane; g < ng; g += 32) emit_group(dst + 2 * g, qs[g], group_lut_fast(ds[g], dv2));
+      for (int64_t g = lane; g < ng; g += 32) emit_group(dst + 2 * g, qs[g], group_lut_fast<ENC>(ds[g], dv2));
     } else {
-      for (int64_t g = lane; g < ng; g += 32) emit_group(dst + 2 * g, qs[g], group_lut_slow(ds[g], s));
+      for (int64_t g = lane; g < ng; g += 32) emit_group(dst + 2 * g, qs[g], group_lut_slow<ENC>(ds[g], s));
     }
     __syncwarp();
     if (row + kRepackBufs * nw < N) issue(row + kRepackBufs * nw, b);

@@ -301,6 +301,61 @@ fp8_status fp8_moe_combine(const uint16_t* rows, const int32_t* inv, int64_t tok
                            int32_t top_k, int64_t H, const float* weights, uint16_t* out,
                            void* stream);
 
+/* ------------------------------------------------------------------------
+ * int8 W8A8 build. Source: dev.to "Gemma 4 From E2B to 31B on an AMD MI300X",
+ * section "The Sizes and the Builds" (format table: w8a8 = int8 weights per
+ * channel, int8 activations per token, from the same QAT release); E2B
+ * article, section "它们离训练权重有多近？" (the int8 build rounds every value
+ * to one of 255 levels per row) and section "第二步：测这张卡的矩阵乘法" (the
+ * int8 GEMM at M = 64; PyTorch's int8 matmul there refuses M < 17 - these
+ * calls accept every M >= 1).
+ *
+ * Quantization contract (bit-exact): per row, amax = max |v|,
+ * s = fp32(amax / 127) (IEEE division), code = clamp(RNE(fp32(v / s)), -127,
+ * 127) as int8 (round half to even); an all-zero row gets s = 0 and zero
+ * codes. GEMM contract (bit-exact): acc = the exact int32 sum of the int8
+ * products (tensor-core kind::i8), y = bf16_rn(fp32(fp32(fp32(acc) * s_tok)
+ * * s_ch)) with one IEEE rounding per step.
+ * ------------------------------------------------------------------------ */
+
+/*
+ * int8_repack_qat: QAT q4_0-grid weights -> per-output-channel int8.
+ *   q4 [N, K/2] uint8 and d [N, K/32] float32 as in fp8_repack_qat (values
+ *   w = fp32(d * q)); w8 [N, K] int8 out; s_ch [N] float32 out.
+ * Requires K % 32 == 0; q4, d, w8 16-byte aligned. Device status:
+ * FP8_DEV_NONFINITE when a row's d*q is not finite.
+ */
+fp8_status int8_repack_qat(const uint8_t* q4, const float* d, int64_t N, int64_t K, int8_t* w8,
+                           float* s_ch, void* stream);
+
+/*
+ * int8_quant_act: per-token int8 quantization of bf16 activations.
+ *   x [M, ldx] bf16 (pitch ldx >= K), x8 [M, K] int8 out, s_tok [M] fp32 out.
+ * Requires K % 16 == 0, ldx % 8 == 0, x and x8 16-byte aligned. Device
+ * status: FP8_DEV_NONFINITE when a token row holds NaN/Inf.
+ */
+fp8_status int8_quant_act(const uint16_t* x, int64_t M, int64_t K, int64_t ldx, int8_t* x8,
+                          float* s_tok, void* stream);
+
+/*
+ * int8_rowwise_linear: y = (x8 . w8^T) * s_tok * s_ch in bf16 (contract
+ * above). x8 [M, K] int8, s_tok [M], w8 [N, K] int8, s_ch [N], y [M, N] bf16.
+ * The same kernels, tiles and launch order as fp8_rowwise_linear (see its
+ * notes on programmatic dependent launch), with int8 operands and int32
+ * accumulators. Requires K % 16 == 0, K <= 65536; x8, w8, y 16-byte aligned.
+ */
+fp8_status int8_rowwise_linear(const int8_t* x8, const float* s_tok, const int8_t* w8,
+                               const float* s_ch, int64_t M, int64_t N, int64_t K, uint16_t* y,
+                               void* stream);
+
+/*
+ * int8_linear_bf16: int8_quant_act of x (pitch K) into the caller's x8 /
+ * s_tok, then int8_rowwise_linear; bit-identical to the two calls.
+ */
+fp8_status int8_linear_bf16(const uint16_t* x, const int8_t* w8, const float* s_ch, int64_t M,
+                            int64_t N, int64_t K, int8_t* x8, float* s_tok, uint16_t* y,
+                            void* stream);
+
 /*
  * fp8_linear_bf16_noalloc: the same computation as fp8_linear_bf16 (per-token
  * quantization of x, then the row-wise FP8 GEMM, with bit-identical results),

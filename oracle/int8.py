@@ -79,12 +79,19 @@ def quant_act_int8(x_bf16_bits: np.ndarray) -> QuantResult:
 
 
 def int8_gemm_acc(x8: np.ndarray, w8: np.ndarray) -> np.ndarray:
-    """Exact integer sums acc[m, n] = sum_k x8[m, k] * w8[n, k] (int64)."""
-    x = np.asarray(x8, dtype=np.int8).astype(np.int64)
-    w = np.asarray(w8, dtype=np.int8).astype(np.int64)
+    """Exact integer sums acc[m, n] = sum_k x8[m, k] * w8[n, k] (int64).
+
+    Computed as an fp64 matrix product (a library primitive): every product
+    is an integer of magnitude <= 127^2 and every partial sum an integer of
+    magnitude <= 127^2 K < 2^53 for K < 2^39, so fp64 holds each one exactly,
+    in any order and blocking."""
+    x = np.asarray(x8, dtype=np.int8).astype(np.float64)
+    w = np.asarray(w8, dtype=np.int8).astype(np.float64)
     if x.shape[1] != w.shape[1]:
         raise ValueError("K mismatch")
-    return x @ w.T
+    if x.shape[1] >= (1 << 39):
+        raise ValueError("K too large for exact fp64 integer sums")
+    return (x @ w.T).astype(np.int64)
 
 
 def int8_linear_ref(x8, s_tok, w8, s_ch) -> np.ndarray:
