@@ -17,7 +17,13 @@ Readings where the pages are silent (listed in the design notes):
   h = bf16(gelu_tanh(gate) * up), computed here in fp64 (relative accuracy
   near 1e-15 for every gate, the far negative tail included) and rounded once
   to bf16; h is quantized per row like any activation.
-* The combine weights are uniform, 1/k, and the sum runs in slot order.
+* The combine weights are uniform, 1/k, unless given (the router's), and the
+  sum runs in slot order.
+* The router (router.proj, bf16 in every build) is a bf16 linear: logits =
+  bf16(x . Wr^T) with the products summed exactly here in fp64; its expert
+  choice takes the top_k largest logits, ties to the lower expert index, and
+  the renormalized softmax over the chosen logits as weights (the pages give
+  no router weights).
 
 Pinned by tests/test_oracle_moe.py: a hand-worked routing example, the
 stable-order and counting invariants, gelu_tanh against torch's
@@ -27,7 +33,9 @@ definition (relative error, the far negative tail included) and its
 closed-form limits, the grouped GEMM against an exact-rational triple loop on a tiny
 two-expert case and against the dense GEMM when every token picks the same
 expert, and the combine against a direct per-token sum, an exact-rational
-weighted sum and a hand-worked weighted case.
+weighted sum and a hand-worked weighted case; the router GEMM against an
+exact-rational triple loop, the top-k choice against a hand-worked example
+with ties and the weights against the two-expert closed form (a logistic).
 """
 
 from __future__ import annotations
@@ -116,3 +124,37 @@ def combine(y_rows: np.ndarray, inv: np.ndarray, tokens: int, top_k: int,
     for j in range(top_k):
         out += w[:, j:j + 1] * y_rows[idx[:, j]]
     return out
+
+
+def bf16_linear_ref(x_bits, w_bits, return_abs: bool = False):
+    """y = x . w^T in fp64 from bf16 operands (uint16 patterns). Each product
+    of two bf16 values is exact in fp64 (16 significant bits); the sum is
+    fp64's, with relative error below K 2^-53. The contract for a GPU result
+    accumulated in fp32 (any order): |y - y_ref| <= K 2^-24 sum|x w| + 1 bf16
+    ulp (bf16_linear_tolerance)."""
+    X = (np.asarray(x_bits, np.uint16).astype(np.uint32) << np.uint32(16)).view(np.float32).astype(np.float64)
+    W = (np.asarray(w_bits, np.uint16).astype(np.uint32) << np.uint32(16)).view(np.float32).astype(np.float64)
+    y = X @ W.T
+    if not return_abs:
+        return y
+    return y, np.abs(X) @ np.abs(W).T
+
+
+def bf16_linear_tolerance(y_ref, abs_sum, K):
+    from .gemm import bf16_ulp
+    return K * 2.0 ** -24 * np.asarray(abs_sum) + bf16_ulp(y_ref)
+
+
+def topk_softmax(logits_bits, top_k: int):
+    """Router choice: per token the top_k largest logits (bf16 patterns
+    [T, E]), in descending order, ties to the lower expert index; weights =
+    exp(l_j - l_max) / sum_i exp(l_i - l_max) over the chosen ones, in fp64.
+    Returns (ids int32 [T, k], weights float64 [T, k])."""
+    L = (np.asarray(logits_bits, np.uint16).astype(np.uint32) << np.uint32(16)).view(np.float32).astype(np.float64)
+    T, E = L.shape
+    idx = np.broadcast_to(np.arange(E), (T, E))
+    order = np.lexsort((idx, -L), axis=1)[:, :top_k]     # key: -logit, then expert index
+    ids = order.astype(np.int32)
+    v = np.take_along_axis(L, order, axis=1)
+    ex = np.exp(v - v[:, :1])
+    return ids, ex / ex.sum(axis=1, keepdims=True)

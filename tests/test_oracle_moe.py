@@ -198,3 +198,51 @@ def test_combine_weighted_hand_worked():
     # token 0: 0.75 * [1, 2] + 0.25 * [4, -8] = [1.75, -0.5]
     # token 1: 0.5 * [2, 6] + 0.5 * [-2, 10] = [0, 8]
     assert out.tolist() == [[1.75, -0.5], [0.0, 8.0]]
+
+
+def test_router_gemm_exact_rational():
+    rng = np.random.default_rng(10)
+    M, N, K = 3, 4, 40
+    xb = (rng.standard_normal((M, K)).astype(np.float32).view(np.uint32) >> 16).astype(np.uint16)
+    wb = (rng.standard_normal((N, K)).astype(np.float32).view(np.uint32) >> 16).astype(np.uint16)
+    y, a = moe.bf16_linear_ref(xb, wb, return_abs=True)
+    xv = (xb.astype(np.uint32) << 16).view(np.float32)
+    wv = (wb.astype(np.uint32) << 16).view(np.float32)
+    for m in range(M):
+        for n in range(N):
+            exact = sum(Fraction(float(xv[m, k])) * Fraction(float(wv[n, k])) for k in range(K))
+            mag = sum(abs(Fraction(float(xv[m, k])) * Fraction(float(wv[n, k]))) for k in range(K))
+            assert abs(Fraction(float(y[m, n])) - exact) <= mag * Fraction(K, 2 ** 53)
+            assert abs(Fraction(float(a[m, n])) - mag) <= mag * Fraction(K, 2 ** 53)
+
+
+def _bf(vals):
+    return (np.asarray(vals, np.float32).view(np.uint32) >> 16).astype(np.uint16)
+
+
+def test_topk_hand_worked_with_ties():
+    # token 0: experts 1 and 4 tie at 3.0 (lower index first), then 2.0 at expert 0
+    # token 1: all equal -> experts 0, 1, 2
+    logits = _bf([[2.0, 3.0, -1.0, 0.5, 3.0, 1.0],
+                  [0.25] * 6])
+    ids, w = moe.topk_softmax(logits, 3)
+    assert ids.tolist() == [[1, 4, 0], [0, 1, 2]]
+    e = np.exp(-1.0)
+    assert np.allclose(w[0], [1 / (2 + e), 1 / (2 + e), e / (2 + e)], rtol=1e-15, atol=0)
+    assert np.allclose(w[1], [1 / 3] * 3, rtol=1e-15, atol=0)
+
+
+def test_topk_weights_two_expert_logistic():
+    """With top_k = 2 the weights are the logistic of the logit gap:
+    w_0 = 1 / (1 + exp(-(a - b))), w_1 = 1 - w_0."""
+    rng = np.random.default_rng(11)
+    L = rng.standard_normal((500, 16)).astype(np.float32) * 3
+    lb = _bf(L)
+    ids, w = moe.topk_softmax(lb, 2)
+    lv = (lb.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    for t in range(500):
+        srt = sorted(range(16), key=lambda e: (-lv[t, e], e))
+        assert ids[t].tolist() == srt[:2]
+        a, b = lv[t, srt[0]], lv[t, srt[1]]
+        assert abs(w[t, 0] - 1 / (1 + np.exp(-(a - b)))) <= 1e-15
+        assert abs(w[t, 0] + w[t, 1] - 1) <= 1e-15
