@@ -24,16 +24,22 @@ error <= 2^-9) and accumulates in fp32:
 ``|y - y_ref| <= 4e-3 * sum_k |x * w| + 1 ulp_bf16(y_ref)``, the same form
 as the FP8 GEMM's bound.
 
+The unpacked weight the GPU multiplies by is a plain definition too:
+``bf16_RN(fp32(d * q))``, the QAT value (as the FP8 repack reads it) rounded
+once to bf16 (``w4a16_unpacked_bits``); it is compared bit for bit.
+
 Pinned by tests/test_oracle_w4a16.py: an exact-rational triple loop on small
-shapes, one-hot activation rows (y = bf16 of one weight), and the linearity
-identities (negated x, doubled d).
+shapes, one-hot activation rows (y = bf16 of one weight), the linearity
+identities (negated x, doubled d), and the unpacked bf16 weights against
+exact-rational rounding.
 """
 
 from __future__ import annotations
 
 import numpy as np
 
-from .quantize import unpack_q4
+from .formats import bf16_rne_bits
+from .quantize import qat_values, unpack_q4
 
 
 def w4a16_weights(q4: np.ndarray, d: np.ndarray) -> np.ndarray:
@@ -56,3 +62,9 @@ def w4a16_linear_ref(x_bf16_bits, q4, d, return_abs: bool = False):
     if not return_abs:
         return y
     return y, np.abs(X) @ np.abs(W).T
+
+
+def w4a16_unpacked_bits(q4: np.ndarray, d: np.ndarray) -> np.ndarray:
+    """The bf16 weights the 4-bit build multiplies by: bf16_RN(fp32(d * q))
+    as bit patterns (uint16 [N, K])."""
+    return bf16_rne_bits(qat_values(q4, d).astype(np.float64))
