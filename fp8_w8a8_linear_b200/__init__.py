@@ -15,6 +15,10 @@ Functions mirror the C entry points:
 * :func:`cast_e4m3` - the element-wise encoder.
 * :func:`moe_route`, :func:`moe_gather`, :func:`grouped_linear`,
   :func:`moe_geglu_quant`, :func:`moe_combine` - the mixture-of-experts layer.
+* :func:`bf16_linear` - the bf16 GEMM (the router), :func:`moe_topk` - the
+  router's top-k choice and weights.
+* :func:`w4a16_dequant`, :func:`w4a16_linear` - the W4A16 build (int4 QAT
+  weights, bf16 activations).
 * :func:`int8_repack_qat`, :func:`int8_quant_act`, :func:`int8_rowwise_linear`,
   :func:`int8_linear` - the int8 W8A8 build.
 * :func:`device_status` - read and clear the device status word.
@@ -60,6 +64,11 @@ _SIGS = {
     "fp8_grouped_linear_geglu": ([_P, _P, _P, ctypes.c_int32, _I64, _P, _P, _I64, _I64, _P, _P],
                                  ctypes.c_int),
     "fp8_moe_combine": ([_P, _P, _I64, ctypes.c_int32, _I64, _P, _P, _P], ctypes.c_int),
+    "bf16_linear": ([_P, _P, _I64, _I64, _I64, _P, _P], ctypes.c_int),
+    "fp8_moe_topk": ([_P, _I64, ctypes.c_int32, ctypes.c_int32, _P, _P, _P], ctypes.c_int),
+    "w4a16_dequant": ([_P, _P, _I64, _I64, _P, _P], ctypes.c_int),
+    "w4a16_workspace_bytes": ([_I64, _I64, _I64], ctypes.c_size_t),
+    "w4a16_linear": ([_P, _P, _P, _I64, _I64, _I64, _P, _P, ctypes.c_size_t, _P], ctypes.c_int),
     "int8_repack_qat": ([_P, _P, _I64, _I64, _P, _P, _P], ctypes.c_int),
     "int8_quant_act": ([_P, _I64, _I64, _I64, _P, _P, _P], ctypes.c_int),
     "int8_rowwise_linear": ([_P, _P, _P, _P, _I64, _I64, _I64, _P, _P], ctypes.c_int),
@@ -295,6 +304,64 @@ def moe_combine(rows: torch.Tensor, inv: torch.Tensor, tokens: int, top_k: int,
     return out
 
 
+def bf16_linear(x: torch.Tensor, w: torch.Tensor, y: torch.Tensor | None = None):
+    """y bf16 [M, N] = x [M, K] . w [N, K]^T with bf16 operands (fp32 accumulation)."""
+    M, K = x.shape
+    N = w.shape[0]
+    y = torch.empty((M, N), dtype=torch.bfloat16, device=x.device) if y is None else y
+    _check(_lib.bf16_linear(_dev(x, torch.bfloat16, "x"), _dev(w, torch.bfloat16, "w", (N, K)), M, N, K,
+                            _dev(y, torch.bfloat16, "y", (M, N)), _stream()), "bf16_linear")
+    return y
+
+
+def moe_topk(logits: torch.Tensor, top_k: int, ids: torch.Tensor | None = None,
+             weights: torch.Tensor | None = None):
+    """Router logits bf16 [T, E] -> (ids int32 [T, k], weights fp32 [T, k])."""
+    T, E = logits.shape
+    dev = logits.device
+    ids = torch.empty((T, top_k), dtype=torch.int32, device=dev) if ids is None else ids
+    weights = torch.empty((T, top_k), dtype=torch.float32, device=dev) if weights is None else weights
+    _check(_lib.fp8_moe_topk(_dev(logits, torch.bfloat16, "logits"), T, E, top_k,
+                             _dev(ids, torch.int32, "ids", (T, top_k)),
+                             _dev(weights, torch.float32, "weights", (T, top_k)), _stream()),
+           "fp8_moe_topk")
+    return ids, weights
+
+
+# ------------------------------------------------------------------ W4A16
+def w4a16_dequant(q4: torch.Tensor, d: torch.Tensor, w: torch.Tensor | None = None):
+    """q4 uint8 [N, K/2] + d float32 [N, K/32] -> w bf16 [N, K] = bf16(fp32(d * q))."""
+    N, K2 = q4.shape
+    K = 2 * K2
+    w = torch.empty((N, K), dtype=torch.bfloat16, device=q4.device) if w is None else w
+    _check(_lib.w4a16_dequant(_dev(q4, torch.uint8, "q4"), _dev(d, torch.float32, "d", (N, K // 32)), N, K,
+                              _dev(w, torch.bfloat16, "w", (N, K)), _stream()), "w4a16_dequant")
+    return w
+
+
+def w4a16_workspace_bytes(M: int, N: int, K: int) -> int:
+    return int(_lib.w4a16_workspace_bytes(M, N, K))
+
+
+def w4a16_linear(x: torch.Tensor, q4: torch.Tensor, d: torch.Tensor, y: torch.Tensor | None = None,
+                 ws: torch.Tensor | None = None):
+    """y bf16 [M, N] = x bf16 [M, K] . w^T with w the int4 QAT weights unpacked
+    to bf16 (in the kernel for M <= 64, else into the workspace ws)."""
+    M, K = x.shape
+    N = q4.shape[0]
+    y = torch.empty((M, N), dtype=torch.bfloat16, device=x.device) if y is None else y
+    need = w4a16_workspace_bytes(M, N, K)
+    if need and ws is None:
+        ws = torch.empty((N, K), dtype=torch.bfloat16, device=x.device)
+    ws_ptr = None if ws is None else ws.data_ptr()
+    ws_bytes = 0 if ws is None else ws.numel() * ws.element_size()
+    _check(_lib.w4a16_linear(_dev(x, torch.bfloat16, "x"), _dev(q4, torch.uint8, "q4", (N, K // 2)),
+                             _dev(d, torch.float32, "d", (N, K // 32)), M, N, K,
+                             _dev(y, torch.bfloat16, "y", (M, N)), ws_ptr, ws_bytes, _stream()),
+           "w4a16_linear")
+    return y
+
+
 # ------------------------------------------------------------------ int8 W8A8
 def int8_repack_qat(q4: torch.Tensor, d: torch.Tensor, w8: torch.Tensor | None = None,
                     s_ch: torch.Tensor | None = None):
@@ -388,5 +455,6 @@ __all__ = [
     "moe_route", "moe_gather", "grouped_linear", "moe_geglu_quant", "moe_combine",
     "moe_interleave_gate_up", "grouped_linear_geglu",
     "int8_repack_qat", "int8_quant_act", "int8_rowwise_linear", "int8_linear",
+    "bf16_linear", "moe_topk", "w4a16_dequant", "w4a16_workspace_bytes", "w4a16_linear",
     "DEV_NONFINITE", "DEV_NAN_CODE", "DEV_INEXACT", "DEV_TIMEOUT", "LIB_PATH",
 ]

@@ -17,7 +17,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libfp8w8a8.so")
 SOURCES = ["fp8w8a8.cu"]
-DEPS = ["fp8w8a8.cu", "ptx.cuh", "quant.cuh", "gemm.cuh", "moe.cuh", "act.cuh"]
+DEPS = ["fp8w8a8.cu", "ptx.cuh", "quant.cuh", "gemm.cuh", "moe.cuh", "act.cuh", "w4a16.cuh"]
 HEADER = os.path.join(os.path.dirname(HERE), "include", "fp8w8a8.h")
 
 

@@ -15,6 +15,7 @@
 #include "moe.cuh"
 #include "ptx.cuh"
 #include "quant.cuh"
+#include "w4a16.cuh"
 
 namespace {
 
@@ -90,6 +91,23 @@ bool make_tmap_bf16_store(CUtensorMap* m, const void* base, uint64_t rows, uint6
   return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_NONE,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Row-major 2-D array [rows, cols] of `dtype` elements (row pitch
+// `pitch_bytes`, a multiple of 16), boxes of box_cols x box_rows, no
+// swizzle, out-of-range elements read as zero.
+bool make_tmap_plain(CUtensorMap* m, CUtensorMapDataType dtype, const void* base, uint64_t rows,
+                     uint64_t cols, uint64_t pitch_bytes, uint32_t box_cols, uint32_t box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {pitch_bytes};
+  cuuint32_t box[2] = {box_cols, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  std::memset(m, 0, sizeof(*m));
+  return fn(m, dtype, 2, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 // Store map of the prefill epilogues: y [rows, cols] bf16 in 32 x 32 boxes
@@ -171,6 +189,17 @@ fp8_status set_decode_attrs(int so) {
   return st;
 }
 
+template <int BNT, int RS, int AS>
+fp8_status set_w4_attr(int smem_optin) {
+  using C = W4DecodeCfg<BNT, RS, AS>;
+  const size_t smem = C::kSmemSplit <= static_cast<size_t>(smem_optin) ? C::kSmemSplit : C::kSmemSingle;
+  return cudaFuncSetAttribute(gemm_w4_decode_kernel<BNT, RS, AS>,
+                              cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) ==
+                 cudaSuccess
+             ? FP8_OK
+             : FP8_ERR_CUDA;
+}
+
 constexpr int kPairStages = 6;
 constexpr int kPrefillBN = 256;
 // Shared memory the staged quantizer may use per block (one block per SM).
@@ -218,6 +247,12 @@ fp8_status device_info(DeviceInfo** out) {
     st = st != FP8_OK ? st : set_decode_attrs<kKindE4M3>(so);
     st = st != FP8_OK ? st : set_decode_attrs<kKindS8>(so);
     st = st != FP8_OK ? st : set_decode_attrs<kKindBF16>(so);
+    st = st != FP8_OK ? st : set_w4_attr<16, 6, 4>(so);
+    st = st != FP8_OK ? st : set_w4_attr<16, 3, 2>(so);
+    st = st != FP8_OK ? st : set_w4_attr<32, 6, 3>(so);
+    st = st != FP8_OK ? st : set_w4_attr<32, 3, 2>(so);
+    st = st != FP8_OK ? st : set_w4_attr<64, 4, 3>(so);
+    st = st != FP8_OK ? st : set_w4_attr<64, 2, 2>(so);
     if (st == FP8_OK &&
         (cudaFuncSetAttribute(quant_act_staged_kernel<false>,
                               cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -571,6 +606,67 @@ fp8_status launch_linear(const DeviceInfo& dev, const uint8_t* x8, const float* 
       return launch_pair<KD>(dev, x8, s_tok, w8, s_ch, M, N, K, y, stream, pdl);
   }
   return launch_prefill<KD>(dev, x8, s_tok, w8, s_ch, M, N, K, y, stream, pdl);
+}
+
+// W4A16 decode, weights unpacked on chip (M <= 64, K % 128 == 0). K is split
+// over a cluster (powers of two up to 8) while the CTAs still fit one per SM
+// and each keeps two or more 128-value steps; the deep-ring variant (one CTA
+// per SM) when the grid fits the SMs, else a shallow one (two per SM).
+template <int BNT, int RS, int AS>
+fp8_status launch_w4_decode_t(const DeviceInfo& dev, const uint16_t* x, const uint8_t* q4,
+                              const float* d, int M, int N, int K, uint16_t* y, int splits,
+                              cudaStream_t stream, bool pdl) {
+  using C = W4DecodeCfg<BNT, RS, AS>;
+  CUtensorMap tmQ, tmD, tmX;
+  if (!make_tmap_plain(&tmQ, CU_TENSOR_MAP_DATA_TYPE_UINT8, q4, N, K / 2, K / 2, 64, kBM) ||
+      !make_tmap_plain(&tmD, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, d, N, K / 32, static_cast<uint64_t>(K / 32) * 4,
+                       4, kBM) ||
+      !make_tmap_u8(&tmX, x, M, static_cast<uint64_t>(2) * K, BNT))
+    return FP8_ERR_CUDA;
+  if (splits > 1 && C::kSmemSplit > static_cast<size_t>(dev.smem_optin)) return FP8_ERR_UNSUPPORTED;
+  const int tiles = (N + kBM - 1) / kBM;
+  const int num_st = (K + 127) / 128;
+  const int st_per_split = (num_st + splits - 1) / splits;
+  CUtensorMap tmY;
+  std::memset(&tmY, 0, sizeof(tmY));
+  const int use_tma_store =
+      (N % 8 == 0) && make_tmap_bf16_store(&tmY, y, M, N, kBM / splits, BNT) ? 1 : 0;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(tiles * splits);
+  cfg.blockDim = dim3(kW4Threads);
+  cfg.dynamicSmemBytes = splits > 1 ? C::kSmemSplit : C::kSmemSingle;
+  cfg.stream = stream;
+  cudaLaunchAttribute attrs[2];
+  int na = 0;
+  attrs[na].id = cudaLaunchAttributeClusterDimension;
+  attrs[na].val.clusterDim.x = splits;
+  attrs[na].val.clusterDim.y = 1;
+  attrs[na].val.clusterDim.z = 1;
+  ++na;
+  set_pdl(attrs, na, pdl);
+  cfg.attrs = attrs;
+  cfg.numAttrs = na;
+  return cudaLaunchKernelEx(&cfg, gemm_w4_decode_kernel<BNT, RS, AS>, tmQ, tmD, tmX, tmY, y, M, N, K,
+                            splits, st_per_split, use_tma_store) == cudaSuccess
+             ? FP8_OK
+             : FP8_ERR_CUDA;
+}
+
+fp8_status launch_w4_decode(const DeviceInfo& dev, const uint16_t* x, const uint8_t* q4,
+                            const float* d, int M, int N, int K, uint16_t* y, cudaStream_t stream) {
+  const int tiles = (N + kBM - 1) / kBM;
+  const int num_st = (K + 127) / 128;
+  int splits = 1;
+  while (splits < 8 && tiles * splits * 2 <= dev.sm_count && splits * 4 <= num_st) splits *= 2;
+  const bool deep = tiles * splits <= dev.sm_count;
+  if (M <= 16)
+    return deep ? launch_w4_decode_t<16, 6, 4>(dev, x, q4, d, M, N, K, y, splits, stream, true)
+                : launch_w4_decode_t<16, 3, 2>(dev, x, q4, d, M, N, K, y, splits, stream, true);
+  if (M <= 32)
+    return deep ? launch_w4_decode_t<32, 6, 3>(dev, x, q4, d, M, N, K, y, splits, stream, true)
+                : launch_w4_decode_t<32, 3, 2>(dev, x, q4, d, M, N, K, y, splits, stream, true);
+  return deep ? launch_w4_decode_t<64, 4, 3>(dev, x, q4, d, M, N, K, y, splits, stream, true)
+              : launch_w4_decode_t<64, 2, 2>(dev, x, q4, d, M, N, K, y, splits, stream, true);
 }
 
 // Blocks of a row-staged streaming kernel that fit on one SM at once (its
@@ -941,6 +1037,104 @@ fp8_status fp8_moe_combine(const uint16_t* rows, const int32_t* inv, int64_t tok
                       static_cast<int>(top_k), H, weights, out);
   return launch_pdl(moe_combine_kernel<kCombineMaxK>, grid, dim3(256), as_stream(stream), rows, inv,
                     tokens, static_cast<int>(top_k), H, weights, out);
+}
+
+// ------------------------------------------------------------ bf16 GEMM, router
+fp8_status bf16_linear(const uint16_t* x, const uint16_t* w, int64_t M, int64_t N, int64_t K,
+                       uint16_t* y, void* stream) {
+  if (!dims_ok(M, kMaxRows) || !dims_ok(N, kMaxRows) || !dims_ok(K, 32768)) return FP8_ERR_INVALID_ARG;
+  if (K % 8 != 0) return FP8_ERR_SHAPE;
+  if (M == 0 || N == 0) return FP8_OK;
+  if (!x || !w || !y) return FP8_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(w) || !aligned16(y)) return FP8_ERR_ALIGNMENT;
+  DeviceInfo* dev;
+  if (fp8_status st = device_info(&dev)) return st;
+  if (K == 0) {
+    if (cudaMemsetAsync(y, 0, static_cast<size_t>(M) * N * 2, as_stream(stream)) != cudaSuccess)
+      return FP8_ERR_CUDA;
+    return FP8_OK;
+  }
+  // bf16 rows are 2K bytes; no scales (y = bf16(acc)).
+  return launch_linear<kKindBF16>(*dev, reinterpret_cast<const uint8_t*>(x), nullptr,
+                                  reinterpret_cast<const uint8_t*>(w), nullptr, static_cast<int>(M),
+                                  static_cast<int>(N), static_cast<int>(2 * K), y, as_stream(stream),
+                                  true);
+}
+
+fp8_status fp8_moe_topk(const uint16_t* logits, int64_t tokens, int32_t num_experts, int32_t top_k,
+                        int32_t* ids, float* weights, void* stream) {
+  if (tokens < 0 || num_experts < 1 || num_experts > kTopkMaxE || top_k < 1 || top_k > kTopkMaxK ||
+      top_k > num_experts)
+    return FP8_ERR_INVALID_ARG;
+  if (tokens == 0) return FP8_OK;
+  if (!logits || !ids || !weights) return FP8_ERR_INVALID_ARG;
+  if (!aligned4(ids) || !aligned4(weights) || (reinterpret_cast<uintptr_t>(logits) & 1))
+    return FP8_ERR_ALIGNMENT;
+  DeviceInfo* dev;
+  if (fp8_status st = device_info(&dev)) return st;
+  const dim3 grid(static_cast<unsigned>((tokens + 7) / 8));
+  const cudaStream_t st = as_stream(stream);
+  if (num_experts <= 128)
+    return launch_pdl(moe_topk_kernel<4>, grid, dim3(256), st, logits, tokens, num_experts, top_k, ids, weights);
+  if (num_experts <= 256)
+    return launch_pdl(moe_topk_kernel<8>, grid, dim3(256), st, logits, tokens, num_experts, top_k, ids, weights);
+  return launch_pdl(moe_topk_kernel<32>, grid, dim3(256), st, logits, tokens, num_experts, top_k, ids, weights);
+}
+
+// ------------------------------------------------------------ W4A16 build
+static fp8_status w4a16_check(const uint8_t* q4, const float* d, int64_t N, int64_t K) {
+  if (!dims_ok(N, kMaxRows) || !dims_ok(K, 32768)) return FP8_ERR_INVALID_ARG;
+  if (K % 32 != 0) return FP8_ERR_SHAPE;
+  if (N > 0 && K > 0 && (!q4 || !d)) return FP8_ERR_INVALID_ARG;
+  if (!aligned16(q4) || !aligned4(d)) return FP8_ERR_ALIGNMENT;
+  return FP8_OK;
+}
+
+fp8_status w4a16_dequant(const uint8_t* q4, const float* d, int64_t N, int64_t K, uint16_t* w,
+                         void* stream) {
+  if (fp8_status st = w4a16_check(q4, d, N, K)) return st;
+  if (N == 0 || K == 0) return FP8_OK;
+  if (!w) return FP8_ERR_INVALID_ARG;
+  if (!aligned16(w)) return FP8_ERR_ALIGNMENT;
+  DeviceInfo* dev;
+  if (fp8_status st = device_info(&dev)) return st;
+  const int64_t groups = N * (K / 32);
+  const int64_t blocks = std::min<int64_t>((groups + 255) / 256, int64_t(dev->sm_count) * 8);
+  return launch_pdl(w4a16_dequant_kernel, dim3(static_cast<unsigned>(blocks)), dim3(256),
+                    as_stream(stream), q4, d, groups, w);
+}
+
+size_t w4a16_workspace_bytes(int64_t M, int64_t N, int64_t K) {
+  if (M <= 0 || N <= 0 || K <= 0) return 0;
+  if (M <= 64 && K % 128 == 0) return 0;
+  return static_cast<size_t>(N) * static_cast<size_t>(K) * 2;
+}
+
+fp8_status w4a16_linear(const uint16_t* x, const uint8_t* q4, const float* d, int64_t M, int64_t N,
+                        int64_t K, uint16_t* y, uint16_t* w_ws, size_t ws_bytes, void* stream) {
+  if (fp8_status st = w4a16_check(q4, d, N, K)) return st;
+  if (!dims_ok(M, kMaxRows)) return FP8_ERR_INVALID_ARG;
+  if (M == 0 || N == 0) return FP8_OK;
+  if (!x || !y) return FP8_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(y)) return FP8_ERR_ALIGNMENT;
+  DeviceInfo* dev;
+  if (fp8_status st = device_info(&dev)) return st;
+  if (K == 0) {
+    if (cudaMemsetAsync(y, 0, static_cast<size_t>(M) * N * 2, as_stream(stream)) != cudaSuccess)
+      return FP8_ERR_CUDA;
+    return FP8_OK;
+  }
+  const size_t need = w4a16_workspace_bytes(M, N, K);
+  if (need == 0)
+    return launch_w4_decode(*dev, x, q4, d, static_cast<int>(M), static_cast<int>(N),
+                            static_cast<int>(K), y, as_stream(stream));
+  if (!w_ws || ws_bytes < need) return FP8_ERR_INVALID_ARG;
+  if (!aligned16(w_ws)) return FP8_ERR_ALIGNMENT;
+  if (fp8_status st = w4a16_dequant(q4, d, N, K, w_ws, stream)) return st;
+  return launch_linear<kKindBF16>(*dev, reinterpret_cast<const uint8_t*>(x), nullptr,
+                                  reinterpret_cast<const uint8_t*>(w_ws), nullptr, static_cast<int>(M),
+                                  static_cast<int>(N), static_cast<int>(2 * K), y, as_stream(stream),
+                                  true);
 }
 
 // ------------------------------------------------------------ int8 W8A8 build

@@ -793,12 +793,13 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
               fmul2_rn(uv[i], uv[i + 1], __uint_as_float(ru[j]), __uint_as_float(ru[j + 1]), sa, sa);
               fmul2_rn(uv[i], uv[i + 1], uv[i], uv[i + 1], sbu[j], sbu[j + 1]);
             }
+            float gb[8], ub[8];
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
-              const float gb = __uint_as_float(static_cast<uint32_t>(f32_to_bf16_rn(gv[i])) << 16);
-              const float ub = __uint_as_float(static_cast<uint32_t>(f32_to_bf16_rn(uv[i])) << 16);
-              hv[i] = geglu_f32(gb, ub);
+              gb[i] = __uint_as_float(static_cast<uint32_t>(f32_to_bf16_rn(gv[i])) << 16);
+              ub[i] = __uint_as_float(static_cast<uint32_t>(f32_to_bf16_rn(uv[i])) << 16);
             }
+            geglu8_f32(gb, ub, hv);
             pk[q] = make_uint4(pack_bf16x2(hv[0], hv[1]), pack_bf16x2(hv[2], hv[3]),
                                pack_bf16x2(hv[4], hv[5]), pack_bf16x2(hv[6], hv[7]));
           }

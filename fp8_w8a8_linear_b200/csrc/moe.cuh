@@ -18,6 +18,85 @@
 
 namespace fp8k {
 
+// ------------------------------------------------------------------ router
+// Top-k expert choice from the bf16 router's logits (the router, router.proj,
+// stays bf16 in every build: sizes article, "Step 1 - Build the Larger
+// Repacks"). One warp per token: each lane holds the logits of experts lane,
+// lane + 32, ... (at most kTopkMaxE / 32 each); k rounds of a warp-wide
+// argmax pick the largest logits, ties to the lower expert index, so the
+// choice is unique. The weights are the softmax over the k chosen logits,
+// w_j = exp(l_j - l_max) / sum_i exp(l_i - l_max), in fp32 with IEEE
+// division (the pages give no router weights; the renormalized top-k softmax
+// is the reading). A NaN or infinite logit sets FP8_DEV_NONFINITE (a NaN
+// ranks lowest); that token's outputs are unspecified.
+constexpr int kTopkMaxE = 1024;
+constexpr int kTopkMaxK = 16;
+
+template <int PER_LANE>  // logits held per lane: E <= 32 * PER_LANE
+__global__ void __launch_bounds__(256) moe_topk_kernel(const uint16_t* __restrict__ logits,
+                                                        int64_t T, int E, int k,
+                                                        int32_t* __restrict__ ids,
+                                                        float* __restrict__ weights) {
+  pdl_launch_dependents();
+  pdl_wait();  // the logits come from the preceding router GEMM
+  const int lane = threadIdx.x & 31;
+  const int64_t t = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
+  if (t >= T) return;
+  const uint16_t* row = logits + t * E;
+  float v[PER_LANE];
+  bool nan = false;
+#pragma unroll
+  for (int i = 0; i < PER_LANE; ++i) {
+    const int e = lane + 32 * i;
+    v[i] = -INFINITY;
+    if (e < E) {
+      const float f = __uint_as_float(static_cast<uint32_t>(__ldg(row + e)) << 16);
+      nan |= !(fabsf(f) <= 3.4028235e38f);
+      v[i] = f != f ? -INFINITY : f;
+    }
+  }
+  if (__any_sync(0xFFFFFFFFu, nan) && lane == 0) report(FP8_DEV_NONFINITE);
+  int my_id = 0;
+  float my_val = 0.0f;
+  unsigned taken = 0u;  // bit i: v[i] already chosen
+  for (int r = 0; r < k; ++r) {
+    // this lane's best remaining logit (lowest index first on ties)
+    float bv = -INFINITY;
+    int bi = 0x7FFFFFFF;
+#pragma unroll
+    for (int i = 0; i < PER_LANE; ++i) {
+      const int e = lane + 32 * i;
+      if (e < E && !((taken >> i) & 1u) && (v[i] > bv || (v[i] == bv && e < bi))) {
+        bv = v[i];
+        bi = e;
+      }
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+      const float ov = __shfl_xor_sync(0xFFFFFFFFu, bv, off);
+      const int oi = __shfl_xor_sync(0xFFFFFFFFu, bi, off);
+      if (ov > bv || (ov == bv && oi < bi)) {
+        bv = ov;
+        bi = oi;
+      }
+    }
+    if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
+    if (lane == r) {
+      my_id = bi;
+      my_val = bv;
+    }
+  }
+  // softmax over the chosen logits: lane 0 holds the largest
+  const float vmax = __shfl_sync(0xFFFFFFFFu, my_val, 0);
+  const float ex = lane < k ? expf(__fsub_rn(my_val, vmax)) : 0.0f;
+  float sum = 0.0f;
+  for (int j = 0; j < k; ++j) sum = __fadd_rn(sum, __shfl_sync(0xFFFFFFFFu, ex, j));
+  if (lane < k) {
+    ids[t * k + lane] = my_id;
+    weights[t * k + lane] = __fdiv_rn(ex, sum);
+  }
+}
+
 // ------------------------------------------------------------------ routing
 // One block per expert e over the n = tokens * top_k flat ids:
 //   pass 1: base = #{ids < e}, cnt = #{ids == e}; offsets[e + 1] = base + cnt;
@@ -218,14 +297,20 @@ __global__ void __launch_bounds__(256) moe_gather_kernel(const uint8_t* __restri
 // Eight bf16 h values (packed) from eight gate and eight up values.
 __device__ __forceinline__ uint4 geglu8(const uint4& g, const uint4& u) {
   const uint32_t gw[4] = {g.x, g.y, g.z, g.w}, uw[4] = {u.x, u.y, u.z, u.w};
+  float gf[8], uf[8], hf[8];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    gf[2 * i] = __uint_as_float(gw[i] << 16);
+    gf[2 * i + 1] = __uint_as_float(gw[i] & 0xFFFF0000u);
+    uf[2 * i] = __uint_as_float(uw[i] << 16);
+    uf[2 * i + 1] = __uint_as_float(uw[i] & 0xFFFF0000u);
+  }
+  geglu8_f32(gf, uf, hf);
   uint32_t o[4];
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
-    const float g0 = __uint_as_float(gw[i] << 16), g1 = __uint_as_float(gw[i] & 0xFFFF0000u);
-    const float u0 = __uint_as_float(uw[i] << 16), u1 = __uint_as_float(uw[i] & 0xFFFF0000u);
-    const float h0 = geglu_f32(g0, u0), h1 = geglu_f32(g1, u1);
     uint32_t r;
-    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(h1), "f"(h0));
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hf[2 * i + 1]), "f"(hf[2 * i]));
     o[i] = r;
   }
   return make_uint4(o[0], o[1], o[2], o[3]);

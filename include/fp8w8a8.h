@@ -301,6 +301,74 @@ fp8_status fp8_moe_combine(const uint16_t* rows, const int32_t* inv, int64_t tok
                            int32_t top_k, int64_t H, const float* weights, uint16_t* out,
                            void* stream);
 
+/*
+ * bf16_linear: y = x . w^T with bf16 operands, fp32 tensor-core accumulation
+ * (kind::f16) and one rounding to bf16; no scales. The router of the
+ * mixture-of-experts layer, router.proj, stays bf16 in every build (sizes
+ * article, "Step 1 - Build the Larger Repacks"); the W4A16 build's long-M
+ * path multiplies by its weights unpacked to bf16 (w4a16_linear).
+ *   x [M, K] bf16, w [N, K] bf16, y [M, N] bf16 out; pitch K and N.
+ * The same kernels and launch order as fp8_rowwise_linear. Requires K % 8
+ * == 0 and K <= 32768; x, w, y 16-byte aligned.
+ */
+fp8_status bf16_linear(const uint16_t* x, const uint16_t* w, int64_t M, int64_t N, int64_t K,
+                       uint16_t* y, void* stream);
+
+/*
+ * fp8_moe_topk: the router's expert choice from its bf16 logits.
+ *   logits [tokens, num_experts] bf16; ids [tokens, top_k] int32 out: the
+ *   top_k largest logits' experts in descending order of logit, ties to the
+ *   lower expert index (unique); weights [tokens, top_k] fp32 out: the
+ *   softmax over the chosen logits, exp(l_j - l_max) / sum_i exp(l_i - l_max)
+ *   (fp32, sum in slot order, IEEE division). The pages give no router
+ *   weights; the renormalized top-k softmax is the reading used.
+ * Requires 1 <= top_k <= 16, top_k <= num_experts <= 1024. A NaN or infinite
+ * logit sets FP8_DEV_NONFINITE; that token's outputs are unspecified.
+ */
+fp8_status fp8_moe_topk(const uint16_t* logits, int64_t tokens, int32_t num_experts, int32_t top_k,
+                        int32_t* ids, float* weights, void* stream);
+
+/* ------------------------------------------------------------------------
+ * W4A16 build. Source: dev.to "Gemma 4 From E2B to 31B on an AMD MI300X",
+ * section "The Sizes and the Builds" (q4w4a16: int4 holding the QAT grid
+ * exactly, bf16 activations) and section "The 4-Bit Builds Stay Slow at
+ * Every Size" (the weights are unpacked to bf16 before each multiply); E2B
+ * article, section "十种构建" (the 4-bit repack stores the QAT values as int4
+ * with each group's trained step, without rounding again).
+ *
+ * The weights are the QAT q4_0 tensors themselves: q4 [N, K/2] packed int4
+ * and d [N, K/32] fp32, as fp8_repack_qat takes them. They are unpacked to
+ * w = bf16_rn(fp32(d * q)) and multiplied with bf16 tensor-core MMAs
+ * (fp32 accumulation): |y - y_exact| <= 4e-3 sum_k |x w| + 1 bf16 ulp,
+ * y_exact = sum_k x d q.
+ * ------------------------------------------------------------------------ */
+
+/*
+ * w4a16_dequant: w [N, K] bf16 out = bf16_rn(fp32(d[n, k/32] * q[n, k])),
+ * bit-exact. Requires K % 32 == 0, K <= 32768; q4 and w 16-byte aligned.
+ */
+fp8_status w4a16_dequant(const uint8_t* q4, const float* d, int64_t N, int64_t K, uint16_t* w,
+                         void* stream);
+
+/*
+ * w4a16_workspace_bytes: the workspace w4a16_linear needs for this shape:
+ * 0 when M <= 64 and K % 128 == 0 (the weights are unpacked on chip, inside
+ * the GEMM), else N * K * 2 bytes (the unpacked bf16 weights).
+ */
+size_t w4a16_workspace_bytes(int64_t M, int64_t N, int64_t K);
+
+/*
+ * w4a16_linear: y = x . w^T, x [M, K] bf16 (pitch K), y [M, N] bf16 out.
+ * M <= 64 with K % 128 == 0: one kernel streams q4 and d (0.625 bytes per
+ * weight) and unpacks them in shared memory for the MMA (swap-AB, K split
+ * over a cluster for narrow layers). Otherwise w4a16_dequant into w_ws
+ * (ws_bytes >= w4a16_workspace_bytes; caller-owned) followed by
+ * bf16_linear. Requires K % 32 == 0, K <= 32768; x, y, w_ws 16-byte aligned.
+ * FP8_ERR_INVALID_ARG when a needed workspace is missing or too small.
+ */
+fp8_status w4a16_linear(const uint16_t* x, const uint8_t* q4, const float* d, int64_t M, int64_t N,
+                        int64_t K, uint16_t* y, uint16_t* w_ws, size_t ws_bytes, void* stream);
+
 /* ------------------------------------------------------------------------
  * int8 W8A8 build. Source: dev.to "Gemma 4 From E2B to 31B on an AMD MI300X",
  * section "The Sizes and the Builds" (format table: w8a8 = int8 weights per
