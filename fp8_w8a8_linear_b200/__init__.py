@@ -12,6 +12,7 @@ Functions mirror the C entry points:
 * :func:`quant_act` - per-token E4M3 activation quantization.
 * :func:`rowwise_linear` - ``y = (x8 . w8^T) * s_tok * s_ch`` in bf16.
 * :func:`linear` - bf16 activations in, bf16 out (quantizer + GEMM).
+* :func:`linear_siblings` - several linears of the same x, quantized once.
 * :func:`cast_e4m3` - the element-wise encoder.
 * :func:`moe_route`, :func:`moe_gather`, :func:`grouped_linear`,
   :func:`moe_geglu_quant`, :func:`moe_combine` - the mixture-of-experts layer.
@@ -48,12 +49,15 @@ _SIGS = {
     "fp8_status_string": ([ctypes.c_int], ctypes.c_char_p),
     "fp8_device_supported": ([ctypes.c_int], ctypes.c_int),
     "fp8_get_device_status": ([ctypes.POINTER(ctypes.c_uint)], ctypes.c_int),
+    "fp8_test_set_fault": ([_I64, ctypes.c_int32], ctypes.c_int),
     "fp8_repack_qat": ([_P, _P, _I64, _I64, _P, _P, _P], ctypes.c_int),
     "fp8_convert_fnuz": ([_P, _P, _I64, _I64, _P, _P, _P], ctypes.c_int),
     "fp8_quant_act": ([_P, _I64, _I64, _I64, _P, _P, _P], ctypes.c_int),
     "fp8_rowwise_linear": ([_P, _P, _P, _P, _I64, _I64, _I64, _P, _P], ctypes.c_int),
     "fp8_linear_bf16": ([_P, _P, _P, _I64, _I64, _I64, _P, _P, _P, _P], ctypes.c_int),
     "fp8_cast_e4m3": ([_P, _I64, _P, _P], ctypes.c_int),
+    "fp8_linear_bf16_siblings": ([_P, _I64, _I64, ctypes.c_int32, _P, _P, _P, _P, _P, _P, _P],
+                                 ctypes.c_int),
     "fp8_linear_bf16_noalloc": ([_P, _P, _P, _I64, _I64, _I64, _P, _P], ctypes.c_int),
     "fp8_moe_route": ([_P, _I64, ctypes.c_int32, ctypes.c_int32, _P, _P, _P, _P], ctypes.c_int),
     "fp8_moe_gather": ([_P, _P, _P, _I64, _I64, ctypes.c_int32, _P, _P, _P], ctypes.c_int),
@@ -131,6 +135,12 @@ def device_status() -> int:
     return v.value
 
 
+def test_set_fault(wait_cycles: int = 0, drop_step: int = -1):
+    """Test hook: in-kernel wait limit (0 = default) and the decode GEMM's
+    dropped pipeline step (-1 = none); see fp8_test_set_fault."""
+    _check(_lib.fp8_test_set_fault(wait_cycles, drop_step), "fp8_test_set_fault")
+
+
 def repack_qat(q4: torch.Tensor, d: torch.Tensor, w8: torch.Tensor | None = None,
                s_ch: torch.Tensor | None = None):
     """q4 uint8 [N, K/2] (packed int4) and d float32 [N, K/32] -> (w8 uint8 [N, K], s_ch float32 [N])."""
@@ -201,6 +211,29 @@ def linear(x: torch.Tensor, w8: torch.Tensor, s_ch: torch.Tensor, y: torch.Tenso
                                 _dev(s_tok, torch.float32, "s_tok", (M,)),
                                 _dev(y, torch.bfloat16, "y", (M, N)), _stream()), "fp8_linear_bf16")
     return y
+
+
+def linear_siblings(x: torch.Tensor, weights, ys=None, x8: torch.Tensor | None = None,
+                    s_tok: torch.Tensor | None = None):
+    """Several W8A8 linears of the same bf16 activations (q/k/v, gate/up):
+    x is quantized once. ``weights`` is a list of (w8 [N_i, K], s_ch [N_i])."""
+    M, K = x.shape
+    dev = x.device
+    n = len(weights)
+    ys = [torch.empty((M, w.shape[0]), dtype=torch.bfloat16, device=dev) for w, _ in weights] if ys is None else ys
+    x8 = torch.empty((M, K), dtype=torch.uint8, device=dev) if x8 is None else x8
+    s_tok = torch.empty((M,), dtype=torch.float32, device=dev) if s_tok is None else s_tok
+    P = ctypes.c_void_p * n
+    w_arr = P(*[_dev(w, torch.uint8, "w8", (w.shape[0], K)) for w, _ in weights])
+    s_arr = P(*[_dev(sc, torch.float32, "s_ch", (w.shape[0],)) for w, sc in weights])
+    n_arr = (ctypes.c_int64 * n)(*[w.shape[0] for w, _ in weights])
+    y_arr = P(*[_dev(yy, torch.bfloat16, "y", (M, w.shape[0])) for yy, (w, _) in zip(ys, weights)])
+    _check(_lib.fp8_linear_bf16_siblings(_dev(x, torch.bfloat16, "x"), M, K, n, ctypes.cast(w_arr, _P),
+                                         ctypes.cast(s_arr, _P), ctypes.cast(n_arr, _P),
+                                         _dev(x8, torch.uint8, "x8", (M, K)),
+                                         _dev(s_tok, torch.float32, "s_tok", (M,)),
+                                         ctypes.cast(y_arr, _P), _stream()), "fp8_linear_bf16_siblings")
+    return ys
 
 
 # ------------------------------------------------------------------ MoE
@@ -452,6 +485,7 @@ def cast_e4m3(x: torch.Tensor, out: torch.Tensor | None = None):
 __all__ = [
     "Fp8Error", "raw", "version", "device_supported", "device_status", "repack_qat",
     "convert_fnuz", "quant_act", "rowwise_linear", "linear", "linear_noalloc", "cast_e4m3",
+    "linear_siblings", "test_set_fault",
     "moe_route", "moe_gather", "grouped_linear", "moe_geglu_quant", "moe_combine",
     "moe_interleave_gate_up", "grouped_linear_geglu",
     "int8_repack_qat", "int8_quant_act", "int8_rowwise_linear", "int8_linear",

@@ -778,6 +778,17 @@ int fp8_device_supported(int device) {
   return prop.major == 10 && prop.minor == 0;
 }
 
+fp8_status fp8_test_set_fault(int64_t wait_cycles, int32_t drop_step) {
+  if (wait_cycles < 0 || drop_step < -1) return FP8_ERR_INVALID_ARG;
+  const long long lim = wait_cycles == 0 ? fp8k::kWaitCycles : static_cast<long long>(wait_cycles);
+  const int drop = drop_step;
+  if (cudaDeviceSynchronize() != cudaSuccess) return FP8_ERR_CUDA;
+  if (cudaMemcpyToSymbol(fp8k::g_wait_limit, &lim, sizeof(lim)) != cudaSuccess ||
+      cudaMemcpyToSymbol(fp8k::g_fault_drop_step, &drop, sizeof(drop)) != cudaSuccess)
+    return FP8_ERR_CUDA;
+  return cudaDeviceSynchronize() == cudaSuccess ? FP8_OK : FP8_ERR_CUDA;
+}
+
 fp8_status fp8_get_device_status(unsigned int* out) {
   if (!out) return FP8_ERR_INVALID_ARG;
   if (cudaDeviceSynchronize() != cudaSuccess) return FP8_ERR_CUDA;
@@ -882,6 +893,37 @@ fp8_status fp8_linear_bf16(const uint16_t* x, const uint8_t* w8, const float* s_
   if (fp8_status st = launch_quant_act(*dev, x, M, K, K, x8, s_tok, as_stream(stream))) return st;
   return launch_linear(*dev, x8, s_tok, w8, s_ch, static_cast<int>(M), static_cast<int>(N),
                        static_cast<int>(K), y, as_stream(stream), true);
+}
+
+fp8_status fp8_linear_bf16_siblings(const uint16_t* x, int64_t M, int64_t K, int32_t count,
+                                    const uint8_t* const* w8, const float* const* s_ch,
+                                    const int64_t* N, uint8_t* x8, float* s_tok,
+                                    uint16_t* const* y, void* stream) {
+  if (count < 1 || count > 16 || !w8 || !s_ch || !N || !y) return FP8_ERR_INVALID_ARG;
+  for (int i = 0; i < count; ++i)
+    if (fp8_status st = check_linear(x, s_tok, w8[i], s_ch[i], M, N[i], K, y[i])) return st;
+  if (M == 0) return FP8_OK;
+  if (!x8) return FP8_ERR_INVALID_ARG;
+  if (!aligned16(x8)) return FP8_ERR_ALIGNMENT;
+  DeviceInfo* dev;
+  if (fp8_status st = device_info(&dev)) return st;
+  const cudaStream_t stream_ = as_stream(stream);
+  if (K == 0) {
+    for (int i = 0; i < count; ++i)
+      if (N[i] > 0 && cudaMemsetAsync(y[i], 0, static_cast<size_t>(M) * N[i] * 2, stream_) != cudaSuccess)
+        return FP8_ERR_CUDA;
+    return FP8_OK;
+  }
+  // One quantization of x, then every GEMM as a programmatic dependent of the
+  // one before (each reads only w8 / s_ch before its grid-dependency wait).
+  if (fp8_status st = launch_quant_act(*dev, x, M, K, K, x8, s_tok, stream_)) return st;
+  for (int i = 0; i < count; ++i) {
+    if (N[i] == 0) continue;
+    if (fp8_status st = launch_linear(*dev, x8, s_tok, w8[i], s_ch[i], static_cast<int>(M),
+                                      static_cast<int>(N[i]), static_cast<int>(K), y[i], stream_, true))
+      return st;
+  }
+  return FP8_OK;
 }
 
 fp8_status fp8_cast_e4m3(const float* x, int64_t n, uint8_t* out, void* stream) {

@@ -883,6 +883,9 @@ __global__ void __launch_bounds__(192)
   const uint32_t full0 = smem_u32(bars);
   const uint32_t empty0 = smem_u32(bars + STAGES);
   const uint32_t tfull = smem_u32(bars + 2 * STAGES);
+  // Abort word shared by the producer and MMA roles (mbar_wait_ab): the
+  // first whose wait runs out makes the other leave at once.
+  const uint32_t abort_w = smem_u32(tmem_holder + 1);
 
   const int warp = warp_id(), lane = lane_id();
   const int tile_n = blockIdx.x / splits;
@@ -897,7 +900,12 @@ __global__ void __launch_bounds__(192)
   const int pre = have_acc ? min(STAGES, st1 - st0) : 0;
 
   if (split) cluster_arrive_relaxed();  // this CTA has started (waited on before any DSMEM store)
+  // Test hook: CTA 0 skips one pipeline step's stage (no arrive, no loads).
+  const int drop = blockIdx.x == 0 ? *const_cast<volatile int*>(&g_fault_drop_step) : -1;
+  // The stages the producer armed and the phase parity each last arm fills.
+  uint32_t armed = 0u, armed_par = 0u;
   if (warp == 0 && lane == 0) {
+    st_shared_volatile_u32(abort_w, 0u);
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(full0 + 8 * s, 1);
       mbar_init(empty0 + 8 * s, 1);
@@ -910,8 +918,10 @@ __global__ void __launch_bounds__(192)
     // preceding quantizer grid: start the first ring of weight boxes now.
     const uint64_t pol_w = l2_policy_evict_first();
     for (int i = 0; i < pre; ++i) {
+      if (i == drop) continue;
       const uint32_t fb = full0 + 8 * i;
       mbar_arrive_expect_tx(fb, C::kStageBytes);
+      armed |= 1u << i;
 #pragma unroll
       for (int j = 0; j < KBS; ++j)
         tma_load_2d(smem_u32(sW + (i * KBS + j) * C::kWBytes), &tmW, fb,
@@ -938,26 +948,38 @@ __global__ void __launch_bounds__(192)
       const uint64_t pol_w = l2_policy_evict_first();
       const uint64_t pol_x = l2_policy_evict_last();
       pdl_wait();  // activations come from a preceding quantizer grid
-      for (int i = 0; i < pre; ++i)
+      for (int i = 0; i < pre; ++i) {
+        if (i == drop) continue;
 #pragma unroll
         for (int j = 0; j < KBS; ++j)
           tma_load_2d(smem_u32(sX + (i * KBS + j) * C::kXBytes), &tmX, full0 + 8 * i,
                       ((st0 + i) * KBS + j) * kBK, 0, pol_x);
+      }
       int stage = pre % STAGES;
       uint32_t phase = pre == STAGES ? 1u : 0u;
       for (int st = st0 + pre; st < st1; ++st) {
-        if (!mbar_wait(empty0 + 8 * stage, phase ^ 1)) break;
-        const uint32_t fb = full0 + 8 * stage;
-        mbar_arrive_expect_tx(fb, C::kStageBytes);
+        if (!mbar_wait_ab(empty0 + 8 * stage, phase ^ 1, abort_w)) break;
+        if (st - st0 != drop) {
+          const uint32_t fb = full0 + 8 * stage;
+          mbar_arrive_expect_tx(fb, C::kStageBytes);
+          armed |= 1u << stage;
+          armed_par = (armed_par & ~(1u << stage)) | (phase << stage);
 #pragma unroll
-        for (int j = 0; j < KBS; ++j) {
-          tma_load_2d(smem_u32(sW + (stage * KBS + j) * C::kWBytes), &tmW, fb, (st * KBS + j) * kBK,
-                      tile_n * kBM, pol_w);
-          tma_load_2d(smem_u32(sX + (stage * KBS + j) * C::kXBytes), &tmX, fb, (st * KBS + j) * kBK,
-                      0, pol_x);
+          for (int j = 0; j < KBS; ++j) {
+            tma_load_2d(smem_u32(sW + (stage * KBS + j) * C::kWBytes), &tmW, fb, (st * KBS + j) * kBK,
+                        tile_n * kBM, pol_w);
+            tma_load_2d(smem_u32(sX + (stage * KBS + j) * C::kXBytes), &tmX, fb, (st * KBS + j) * kBK,
+                        0, pol_x);
+          }
         }
         if (++stage == STAGES) { stage = 0; phase ^= 1; }
       }
+      // Let every copy this thread started land (each wait bounded) before
+      // the CTA can leave, also after an abort: a stage's last arm fills the
+      // phase with the recorded parity, which completes once its bytes have
+      // arrived (at once if the MMA already consumed it).
+      for (int s2 = 0; s2 < STAGES; ++s2)
+        if ((armed >> s2) & 1u) mbar_wait(full0 + 8 * s2, (armed_par >> s2) & 1u);
     }
   } else if (warp == 1) {
     if (lane == 0 && have_acc) {
@@ -965,7 +987,7 @@ __global__ void __launch_bounds__(192)
       int stage = 0;
       uint32_t phase = 0;
       for (int st = st0; st < st1; ++st) {
-        if (!mbar_wait(full0 + 8 * stage, phase)) break;
+        if (!mbar_wait_ab(full0 + 8 * stage, phase, abort_w)) break;
         tc_fence_after();
 #pragma unroll
         for (int j = 0; j < KBS; ++j) {
@@ -981,6 +1003,9 @@ __global__ void __launch_bounds__(192)
         if (++stage == STAGES) { stage = 0; phase ^= 1; }
       }
       umma_commit(tfull);
+      // the issued MMAs have finished before this thread can reach the TMEM
+      // release (also when the loop above was left by an abort)
+      mbar_wait(tfull, 0);
     }
   } else {
     const int et = threadIdx.x - 64;                 // 0..127

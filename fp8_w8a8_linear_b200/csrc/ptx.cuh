@@ -55,16 +55,53 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Bound on a single wait: ~2^31 SM cycles (about a second at B200 clocks).
+// Bound on a single wait, in SM clock cycles (clock64): 2^31 by default,
+// about 1.1 s at the 1965 MHz boost clock. fp8_test_set_fault can lower it
+// for one device (a test that makes a wait run out).
 constexpr long long kWaitCycles = 1ll << 31;
+__device__ long long g_wait_limit = kWaitCycles;
+
+// Test hook (fp8_test_set_fault): when >= 0, CTA 0 of the decode GEMM skips
+// this pipeline step's stage (no arrive, no loads), so the MMA's wait on it
+// can only end by its time limit.
+__device__ int g_fault_drop_step = -1;
 
 // Waits for the phase with the given parity to complete. Returns false (and
-// records FP8_DEV_TIMEOUT) if that does not happen within kWaitCycles.
+// records FP8_DEV_TIMEOUT) if that does not happen within the wait limit.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
   if (mbar_try_wait(bar, parity)) return true;
+  const long long lim = *const_cast<volatile long long*>(&g_wait_limit);
   const long long t0 = clock64();
   while (!mbar_try_wait(bar, parity)) {
-    if (clock64() - t0 > kWaitCycles) {
+    if (clock64() - t0 > lim) {
+      report(FP8_DEV_TIMEOUT);
+      return false;
+    }
+  }
+  return true;
+}
+
+__device__ __forceinline__ uint32_t ld_shared_volatile_u32(uint32_t addr) {
+  uint32_t v;
+  asm volatile("ld.volatile.shared.u32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
+  return v;
+}
+__device__ __forceinline__ void st_shared_volatile_u32(uint32_t addr, uint32_t v) {
+  asm volatile("st.volatile.shared.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+}
+
+// mbar_wait for kernels whose roles share an abort word in shared memory:
+// the first role whose wait runs out sets it (and FP8_DEV_TIMEOUT), and
+// every other role then leaves its own wait at once instead of waiting out
+// its own limit.
+__device__ __forceinline__ bool mbar_wait_ab(uint32_t bar, uint32_t parity, uint32_t abort_word) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const long long lim = *const_cast<volatile long long*>(&g_wait_limit);
+  const long long t0 = clock64();
+  while (!mbar_try_wait(bar, parity)) {
+    if (ld_shared_volatile_u32(abort_word) != 0u) return false;
+    if (clock64() - t0 > lim) {
+      st_shared_volatile_u32(abort_word, 1u);
       report(FP8_DEV_TIMEOUT);
       return false;
     }

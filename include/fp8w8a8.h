@@ -94,6 +94,21 @@ int fp8_device_supported(int device);
 fp8_status fp8_get_device_status(unsigned int* out);
 
 /*
+ * fp8_test_set_fault: test hook for the bounded waits (no counterpart on the
+ * pages). Sets, for the current device, the limit of every in-kernel wait to
+ * `wait_cycles` SM clock cycles (0 restores the default, 2^31 cycles, about
+ * 1.1 s at 1965 MHz), and when `drop_step` >= 0 makes CTA 0 of every decode
+ * GEMM launch (fp8_rowwise_linear with M <= 128) skip that pipeline step of
+ * its K range: no arrive, no copies, so the MMA's wait for it can end only by
+ * the limit. The kernel then records FP8_DEV_TIMEOUT, the producer and MMA
+ * roles leave their pipelines, the producer waits for its copies in flight,
+ * and the kernel returns (its output is undefined). -1 turns the drop off.
+ * Synchronizes the device before and after; not for use while other work of
+ * this library runs.
+ */
+fp8_status fp8_test_set_fault(int64_t wait_cycles, int32_t drop_step);
+
+/*
  * fp8_repack_qat: QAT q4_0-grid weights -> per-output-channel E4M3.
  * Source: model card above, "QAT trained the weights onto a 4-bit grid with
  * one scale per group of 32 values"; header paragraph (one float32 scale per
@@ -184,6 +199,25 @@ fp8_status fp8_rowwise_linear(const uint8_t* x8, const float* s_tok, const uint8
 fp8_status fp8_linear_bf16(const uint16_t* x, const uint8_t* w8, const float* s_ch, int64_t M,
                            int64_t N, int64_t K, uint8_t* x8, float* s_tok, uint16_t* y,
                            void* stream);
+
+/*
+ * fp8_linear_bf16_siblings: several linears that read the same activations
+ * (q, k and v of an attention block; gate and up of an MLP), with x
+ * quantized once. Source: E2B article, section "第二步：测这张卡的矩阵乘法"
+ * (the whole per-token GEMM set of the model, timed inside one graph).
+ *   x [M, K] bf16 (pitch K), quantized once into the caller's x8 [M, K] and
+ *   s_tok [M] (as fp8_quant_act); then for i < count: y[i] [M, N[i]] =
+ *   fp8_rowwise_linear(x8, s_tok, w8[i], s_ch[i]), each GEMM launched as a
+ *   programmatic dependent of the one before, so its prologue and weight
+ *   stream start while the previous one ends. Bit-identical to
+ *   fp8_linear_bf16 called once per weight.
+ *   w8, s_ch, N, y: HOST arrays of `count` (1..16) device pointers / sizes.
+ * Requirements per linear as fp8_rowwise_linear.
+ */
+fp8_status fp8_linear_bf16_siblings(const uint16_t* x, int64_t M, int64_t K, int32_t count,
+                                    const uint8_t* const* w8, const float* const* s_ch,
+                                    const int64_t* N, uint8_t* x8, float* s_tok,
+                                    uint16_t* const* y, void* stream);
 
 /*
  * fp8_cast_e4m3: element-wise fp32 -> E4M3 with the library's encoder

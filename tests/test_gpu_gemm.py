@@ -266,3 +266,28 @@ def test_bf16_weights_quantized_per_channel_online(lib):
     ok, worst = oracle.check_linear(bf16_values(y), y_ref, abs_s)
     assert ok, worst
     assert lib.device_status() == 0
+
+
+@pytest.mark.parametrize("M,K,Ns", [(1, 2048, (8192, 8192, 8192)), (8, 2048, (4096, 1024, 1024)),
+                                    (64, 5376, (21504, 21504)), (300, 1024, (1000, 520, 4096))])
+def test_sibling_linears_quantize_once(lib, M, K, Ns):
+    """q/k/v- or gate/up-like siblings of one activation: x quantized once into
+    x8 / s_tok (bit-exact against the oracle), every output within the bound
+    of the oracle's GEMM and bit-identical to fp8_linear_bf16 per weight."""
+    xb = activations_bf16(M, K, seed=M + K, outlier_frac=0.01)
+    a = oracle.quant_act(xb)
+    ws, wds = [], []
+    for i, N in enumerate(Ns):
+        q4, d = q4_weights(N, K, seed=100 + i)
+        w = oracle.repack_qat(q4, d)
+        ws.append(w)
+        wds.append((to_dev(w.codes), to_dev(w.scales)))
+    x = to_dev(xb)
+    x8 = torch.empty((M, K), dtype=torch.uint8, device="cuda")
+    st = torch.empty((M,), dtype=torch.float32, device="cuda")
+    ys = lib.linear_siblings(x, wds, x8=x8, s_tok=st)
+    assert np.array_equal(u8(x8), a.codes) and same_bits_f32(f32(st), a.scales)
+    for y, w, (w8, sc) in zip(ys, ws, wds):
+        _check(y, a, w)
+        assert torch.equal(y.view(torch.int16), lib.linear(x, w8, sc).view(torch.int16))
+    assert lib.device_status() == 0
