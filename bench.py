@@ -72,6 +72,7 @@ FALLBACK_BF16_TFLOPS_SUSTAINED = 1400.0
 FP8_PER_BF16 = 2.0  # nominal dense ratio, 4.5 PF fp8 / 2.25 PF bf16
 SPEC_FP8_TFLOPS = 4500.0  # B200 dense FP8, vendor spec
 SPEC_HBM_GBS = 8000.0     # B200 HBM3e, about 8 TB/s
+SPEC_BF16_TFLOPS = 2250.0  # B200 dense bf16, vendor spec
 
 
 def load_peaks():
@@ -91,9 +92,13 @@ WORKLOADS = {
     "large8k": dict(K=5376, N=21504, Ms=(8192, 1, 64), seed=3, outl=0.01, repack=True, fnuz=True,
                     desc="large dense layer K=5376 N=21504 at M in {8192,1,64} (profiling size), repack + FNUZ"),
     "decode": dict(K=2048, N=8192, Ms=(1, 8, 64), seed=1, outl=0.01, repack=False, fnuz=False,
-                   desc="decode GEMM sweep K=2048 N=8192, M in {1,8,64}"),
+                   builds=True, siblings=3,
+                   desc="decode GEMM sweep K=2048 N=8192, M in {1,8,64}; int8 W8A8 and W4A16 builds; "
+                        "three sibling linears sharing one quantized x"),
     "prefill": dict(K=4096, N=14336, Ms=(8192, 1024, 128), seed=2, outl=0.01, repack=False, fnuz=True,
-                    desc="prefill GEMM K=4096 N=14336, M in {8192,1024,128}, FNUZ load conversion"),
+                    builds=True,
+                    desc="prefill GEMM K=4096 N=14336, M in {8192,1024,128}, FNUZ load conversion; "
+                         "int8 W8A8 and W4A16 builds"),
     "tiny": dict(K=256, N=128, Ms=(4,), seed=0, outl=0.0, repack=True, fnuz=False,
                  desc="tiny W8A8 linear M=4 K=256 N=128"),
     "moe": dict(moe=True, tokens=8192, hidden=2048, inter=704, experts=128, top_k=8, seed=4, outl=0.01,
@@ -234,6 +239,54 @@ def setup_dense(torch, f, wl, seed, dev, flushable):
                       lambda i, x=D[f"x{M}"], x8=x8, st=st, y=y: f.linear(
                           x, wcopies[i % ncopies], wsrc[1], y, x8, st),
                       fl, qb + gb, "hbm", flushable, 2))
+    if wl.get("siblings"):
+        # q/k/v-like siblings of one activation at M = 1: x quantized once, then
+        # the GEMMs as a chain of dependents (fp8_linear_bf16_siblings)
+        ns = wl["siblings"]
+        M = 1
+        x8, st, _ = bufs[M]
+        sib_y = [torch.empty((M, N), dtype=torch.bfloat16, device=dev) for _ in range(ns)]
+        qb, gb = linear_bytes(M, N, K)
+        L.append((f"linear_siblings_x{ns}[M={M}]",
+                  lambda i, x=D[f"x{M}"], x8=x8, st=st: f.linear_siblings(
+                      x, [(wcopies[(i * ns + j) % ncopies], wsrc[1]) for j in range(ns)], sib_y, x8, st),
+                  ns * gemm_flops(M, N, K), qb + ns * gb - (ns - 1) * (M * K + 4 * M), "hbm", flushable,
+                  1 + ns))
+    if wl.get("builds"):
+        # the int8 W8A8 build (int8 weights per channel, int8 activations per
+        # token) and the W4A16 build (the QAT int4 weights, bf16 activations)
+        # of the same layer, at every M
+        w8i, s8i = f.int8_repack_qat(D["q4"], D["d"])
+        i8copies = [w8i] + [w8i.clone() for _ in range(ncopies - 1)]
+        ncq = max(2, -(-int(2.5 * 126e6) // int(N * K * 0.625)))
+        q4copies = [(D["q4"], D["d"])] + [(D["q4"].clone(), D["d"].clone()) for _ in range(ncq - 1)]
+        ws = torch.empty((N, K), dtype=torch.bfloat16, device=dev)
+        for M in Ms:
+            x8, st, y = bufs[M]
+            x8i = torch.empty((M, K), dtype=torch.int8, device=dev)
+            qb, gb = linear_bytes(M, N, K)
+            fl = gemm_flops(M, N, K)
+            if M > 128:
+                L.append((f"int8_quant_act[M={M}]", lambda i, x=D[f"x{M}"], x8i=x8i, st=st: f.int8_quant_act(x, x8i, st),
+                          0.0, qb, "hbm", False, 1))
+                L.append((f"int8_gemm[M={M}]",
+                          lambda i, x8i=x8i, st=st, y=y: f.int8_rowwise_linear(x8i, st, w8i, s8i, y),
+                          fl, gb, "tensor", False, 1))
+                # unpack to the workspace (0.625 B in, 2 B out per weight), then the bf16 GEMM
+                L.append((f"w4a16_unpack[N={N}]", lambda i: f.w4a16_dequant(D["q4"], D["d"], ws), 0.0,
+                          N * K * 2.625, "hbm", False, 1))
+                L.append((f"w4a16_bf16_gemm[M={M}]", lambda i, x=D[f"x{M}"], y=y: f.bf16_linear(x, ws, y),
+                          fl, 2.0 * M * K + 2.0 * N * K + 2.0 * M * N, "tensor_bf16", False, 1))
+            else:
+                L.append((f"int8_linear_decode[M={M}]",
+                          lambda i, x=D[f"x{M}"], x8i=x8i, st=st, y=y: f.int8_linear(
+                              x, i8copies[i % ncopies], s8i, y, x8i, st),
+                          fl, qb + gb, "hbm", flushable, 2))
+                wsb = None if f.w4a16_workspace_bytes(M, N, K) == 0 else ws
+                L.append((f"w4a16_linear_decode[M={M}]",
+                          lambda i, x=D[f"x{M}"], y=y, wsb=wsb: f.w4a16_linear(
+                              x, q4copies[i % ncq][0], q4copies[i % ncq][1], y, wsb),
+                          fl, N * K * 0.625 + 2.0 * M * K + 2.0 * M * N, "hbm", flushable, 1))
     outs = [bufs[M][2] for M in Ms]
     cfg = {"K": K, "N": N, "M": list(Ms)}
     return L, h, D, outs, cfg
@@ -244,7 +297,7 @@ def setup_moe(torch, f, wl, seed, dev):
     unit in its epilogue, quantization of h, down GEMM, combine. Expert
     weights are resident (repacked, and the gate/up rows interleaved, at
     setup)."""
-    from workloads import activations_bf16, moe_routing, q4_weights
+    from workloads import activations_bf16, f32_to_bf16_bits, moe_routing, q4_weights
 
     T, Hd, I, E, k = wl["tokens"], wl["hidden"], wl["inter"], wl["experts"], wl["top_k"]
     R = T * k
@@ -269,6 +322,17 @@ def setup_moe(torch, f, wl, seed, dev):
     out = torch.empty((T, Hd), dtype=torch.bfloat16, device=dev)
     ids = D["ids"]
 
+    # the bf16 router (router.proj stays bf16 in every build) and its top-k
+    # choice with softmax weights: computed as the layer does; the expert path
+    # below routes by the workload's seeded uniform ids, so that every expert
+    # gets its binomial share of the 65,536 rows as the configuration fixes
+    w_router = torch.from_numpy(f32_to_bf16_bits(
+        (np.random.default_rng(seed + 3).standard_normal((E, Hd)) * Hd ** -0.5).astype(np.float32)).view(np.int16)
+    ).to(dev).view(torch.bfloat16)
+    logits = torch.empty((T, E), dtype=torch.bfloat16, device=dev)
+    r_ids = torch.empty((T, k), dtype=torch.int32, device=dev)
+    r_w = torch.empty((T, k), dtype=torch.float32, device=dev)
+
     def route(i):
         f.raw.fp8_moe_route(ids.data_ptr(), T, k, E, perm.data_ptr(), inv.data_ptr(), off.data_ptr(),
                             torch.cuda.current_stream().cuda_stream)
@@ -276,6 +340,10 @@ def setup_moe(torch, f, wl, seed, dev):
     fl_gu = gemm_flops(R, 2 * I, Hd)
     fl_dn = gemm_flops(R, Hd, I)
     L = [
+        ("router_bf16_gemm", lambda i: f.bf16_linear(D["x"], w_router, logits), gemm_flops(T, E, Hd),
+         2.0 * T * Hd + 2.0 * E * Hd + 2.0 * T * E, "hbm", False, 1),
+        ("router_topk", lambda i: f.moe_topk(logits, k, r_ids, r_w), 0.0, 2.0 * T * E + 8.0 * T * k,
+         "hbm", False, 1),
         ("moe_route", route, 0.0, 4.0 * R * 3 + 4 * (E + 1), "latency", False, 3),
         ("quant_act", lambda i: f.quant_act(D["x"], x8, st), 0.0, 3.0 * T * Hd + 4 * T, "hbm", False, 1),
         ("moe_gather", lambda i: f.moe_gather(x8, st, perm, k, xr, sr), 0.0,
@@ -420,7 +488,7 @@ def roofline_peaks(peaks, timed_s, scaled_mm):
     burst = timed_s < 2.0
     bf16 = peaks["bf16"] if burst else peaks["bf16_sustained"]
     return {
-        "fp8": bf16 * FP8_PER_BF16,
+        "fp8": bf16 * FP8_PER_BF16, "bf16": bf16,
         "fp8_note": (f"fp8 dense = 2 x {peaks['source']} {'burst' if burst else 'sustained'} bf16 cuBLAS "
                      f"({bf16}); timed region {timed_s:.2f} s"),
         "hbm": peaks["hbm_gbs"], "hbm_note": f"{peaks['source']} HBM copy",
@@ -442,6 +510,9 @@ def kernel_rows(step_ops, t, pk, workload):
             k["frac_spec"] = round(k["tflops"] / pk["fp8_spec"], 3)
             if pk["fp8_scaled_mm"]:
                 k["frac_scaled_mm"] = round(k["tflops"] / pk["fp8_scaled_mm"], 3)
+        elif bound == "tensor_bf16":  # bf16 MMAs: the measured bf16 cuBLAS figure, 2.25 PF spec
+            k["frac"] = round(k["tflops"] / pk["bf16"], 3)
+            k["frac_spec"] = round(k["tflops"] / SPEC_BF16_TFLOPS, 3)
         elif bound == "hbm":
             k["frac"] = round(k["gbs"] / pk["hbm"], 3)
             k["frac_spec"] = round(k["gbs"] / pk["hbm_spec"], 3)
