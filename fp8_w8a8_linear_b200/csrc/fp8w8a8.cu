@@ -253,6 +253,7 @@ fp8_status device_info(DeviceInfo** out) {
     st = st != FP8_OK ? st : set_w4_attr<32, 3, 2>(so);
     st = st != FP8_OK ? st : set_w4_attr<64, 4, 3>(so);
     st = st != FP8_OK ? st : set_w4_attr<64, 2, 2>(so);
+    st = st != FP8_OK ? st : set_w4_attr<128, 4, 2>(so);
     if (st == FP8_OK &&
         (cudaFuncSetAttribute(quant_act_staged_kernel<false>,
                               cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -608,10 +609,11 @@ fp8_status launch_linear(const DeviceInfo& dev, const uint8_t* x8, const float* 
   return launch_prefill<KD>(dev, x8, s_tok, w8, s_ch, M, N, K, y, stream, pdl);
 }
 
-// W4A16 decode, weights unpacked on chip (M <= 64, K % 128 == 0). K is split
+// W4A16 decode, weights unpacked on chip (M <= 128, K % 128 == 0). K is split
 // over a cluster (powers of two up to 8) while the CTAs still fit one per SM
-// and each keeps two or more 128-value steps; the deep-ring variant (one CTA
-// per SM) when the grid fits the SMs, else a shallow one (two per SM).
+// and each keeps four or more 128-value steps; the deep-ring variant (one CTA
+// per SM) when the grid fits the SMs, else a shallow one (two per SM). Up to
+// 128 tokens: one CTA per SM and no split (the token tiles take the room).
 template <int BNT, int RS, int AS>
 fp8_status launch_w4_decode_t(const DeviceInfo& dev, const uint16_t* x, const uint8_t* q4,
                               const float* d, int M, int N, int K, uint16_t* y, int splits,
@@ -665,8 +667,10 @@ fp8_status launch_w4_decode(const DeviceInfo& dev, const uint16_t* x, const uint
   if (M <= 32)
     return deep ? launch_w4_decode_t<32, 6, 3>(dev, x, q4, d, M, N, K, y, splits, stream, true)
                 : launch_w4_decode_t<32, 3, 2>(dev, x, q4, d, M, N, K, y, splits, stream, true);
-  return deep ? launch_w4_decode_t<64, 4, 3>(dev, x, q4, d, M, N, K, y, splits, stream, true)
-              : launch_w4_decode_t<64, 2, 2>(dev, x, q4, d, M, N, K, y, splits, stream, true);
+  if (M <= 64)
+    return deep ? launch_w4_decode_t<64, 4, 3>(dev, x, q4, d, M, N, K, y, splits, stream, true)
+                : launch_w4_decode_t<64, 2, 2>(dev, x, q4, d, M, N, K, y, splits, stream, true);
+  return launch_w4_decode_t<128, 4, 2>(dev, x, q4, d, M, N, K, y, 1, stream, true);
 }
 
 // Blocks of a row-staged streaming kernel that fit on one SM at once (its
@@ -1148,7 +1152,7 @@ fp8_status w4a16_dequant(const uint8_t* q4, const float* d, int64_t N, int64_t K
 
 size_t w4a16_workspace_bytes(int64_t M, int64_t N, int64_t K) {
   if (M <= 0 || N <= 0 || K <= 0) return 0;
-  if (M <= 64 && K % 128 == 0) return 0;
+  if (M <= 128 && K % 128 == 0) return 0;
   return static_cast<size_t>(N) * static_cast<size_t>(K) * 2;
 }
 

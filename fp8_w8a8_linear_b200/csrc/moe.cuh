@@ -23,7 +23,7 @@ namespace fp8k {
 // stays bf16 in every build: sizes article, "Step 1 - Build the Larger
 // Repacks"). One warp per token: each lane holds the logits of experts lane,
 // lane + 32, ... (at most kTopkMaxE / 32 each); k rounds of a warp-wide
-// argmax pick the largest logits, ties to the lower expert index, so the
+// maximum pick the largest logits, ties to the lower expert index, so the
 // choice is unique. The weights are the softmax over the k chosen logits,
 // w_j = exp(l_j - l_max) / sum_i exp(l_i - l_max), in fp32 with IEEE
 // division (the pages give no router weights; the renormalized top-k softmax
@@ -31,6 +31,25 @@ namespace fp8k {
 // ranks lowest); that token's outputs are unspecified.
 constexpr int kTopkMaxE = 1024;
 constexpr int kTopkMaxK = 16;
+
+// Each logit travels as one 32-bit key whose unsigned order is the choice
+// order: the bf16 pattern made order-preserving (negative values bit-flipped,
+// positive ones with the sign bit set; -0 taken as +0; NaN mapped to 0,
+// below -inf) in the
+// high half and 0xFFFF - expert in the low half (ties go to the lower
+// expert). A round is then one warp-wide unsigned max (redux.sync); a chosen
+// key is replaced by 0.
+__device__ __forceinline__ uint32_t topk_key(uint16_t b, int e) {
+  if ((b & 0x7FFFu) == 0u) b = 0u;  // -0 ranks as +0 (equal values tie by index)
+  const uint32_t ord = (b & 0x7FFFu) > 0x7F80u ? 0u : ((b & 0x8000u) ? (~b & 0xFFFFu) : (b | 0x8000u));
+  return (ord << 16) | (0xFFFFu - static_cast<uint32_t>(e));
+}
+
+__device__ __forceinline__ float topk_key_value(uint32_t key) {
+  const uint32_t ord = key >> 16;
+  const uint32_t b = (ord & 0x8000u) ? (ord & 0x7FFFu) : (~ord & 0xFFFFu);
+  return __uint_as_float(b << 16);
+}
 
 template <int PER_LANE>  // logits held per lane: E <= 32 * PER_LANE
 __global__ void __launch_bounds__(256) moe_topk_kernel(const uint16_t* __restrict__ logits,
@@ -43,47 +62,35 @@ __global__ void __launch_bounds__(256) moe_topk_kernel(const uint16_t* __restric
   const int64_t t = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
   if (t >= T) return;
   const uint16_t* row = logits + t * E;
-  float v[PER_LANE];
-  bool nan = false;
+  uint32_t key[PER_LANE];
+  bool bad = false;
 #pragma unroll
   for (int i = 0; i < PER_LANE; ++i) {
     const int e = lane + 32 * i;
-    v[i] = -INFINITY;
+    key[i] = 0u;
     if (e < E) {
-      const float f = __uint_as_float(static_cast<uint32_t>(__ldg(row + e)) << 16);
-      nan |= !(fabsf(f) <= 3.4028235e38f);
-      v[i] = f != f ? -INFINITY : f;
+      const uint16_t bits = __ldg(row + e);
+      bad |= (bits & 0x7FFFu) >= 0x7F80u;  // NaN or +-inf
+      key[i] = topk_key(bits, e);
     }
   }
-  if (__any_sync(0xFFFFFFFFu, nan) && lane == 0) report(FP8_DEV_NONFINITE);
+  if (__any_sync(0xFFFFFFFFu, bad) && lane == 0) report(FP8_DEV_NONFINITE);
   int my_id = 0;
   float my_val = 0.0f;
-  unsigned taken = 0u;  // bit i: v[i] already chosen
   for (int r = 0; r < k; ++r) {
-    // this lane's best remaining logit (lowest index first on ties)
-    float bv = -INFINITY;
-    int bi = 0x7FFFFFFF;
+    uint32_t best = 0u;
 #pragma unroll
-    for (int i = 0; i < PER_LANE; ++i) {
-      const int e = lane + 32 * i;
-      if (e < E && !((taken >> i) & 1u) && (v[i] > bv || (v[i] == bv && e < bi))) {
-        bv = v[i];
-        bi = e;
-      }
-    }
+    for (int i = 0; i < PER_LANE; ++i) best = max(best, key[i]);
+    const uint32_t win = __reduce_max_sync(0xFFFFFFFFu, best);
+    const int e = static_cast<int>(0xFFFFu - (win & 0xFFFFu));
+    if ((e & 31) == lane) {
 #pragma unroll
-    for (int off = 16; off > 0; off >>= 1) {
-      const float ov = __shfl_xor_sync(0xFFFFFFFFu, bv, off);
-      const int oi = __shfl_xor_sync(0xFFFFFFFFu, bi, off);
-      if (ov > bv || (ov == bv && oi < bi)) {
-        bv = ov;
-        bi = oi;
-      }
+      for (int i = 0; i < PER_LANE; ++i)
+        if (i == (e >> 5)) key[i] = 0u;
     }
-    if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
     if (lane == r) {
-      my_id = bi;
-      my_val = bv;
+      my_id = e;
+      my_val = topk_key_value(win);
     }
   }
   // softmax over the chosen logits: lane 0 holds the largest

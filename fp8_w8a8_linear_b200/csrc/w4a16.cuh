@@ -14,13 +14,14 @@
 //
 // * w4a16_dequant_kernel: q4 [N, K/2] + d [N, K/32] -> w [N, K] bf16, an HBM
 //   streaming kernel (one 32-value group per thread: 16 + 4 bytes in, 64 out).
-// * gemm_w4_decode_kernel (M <= 64): swap-AB like the FP8 decode GEMM, with
+// * gemm_w4_decode_kernel (M <= 128): swap-AB like the FP8 decode GEMM, with
 //   the weight operand unpacked on chip. Warp 0 streams the packed weights
-//   and scales (0.625 bytes per weight) into a ring of raw stages with TMA,
-//   and the token tiles with TMA into the operand ring; warps 2..9 unpack each
-//   raw stage into two 128-row x 64-value bf16 operand blocks in the 128-byte
-//   swizzled K-major layout the MMA reads; warp 1 issues tcgen05.mma.kind::f16
-//   into a TMEM accumulator. K may be split across a thread-block cluster with
+//   and scales (0.625 bytes per weight) into a ring of raw stages with TMA;
+//   warp 10 streams the token tiles into the operand ring (a thread of its
+//   own, so that no token-tile load waits behind a raw-stage refill); warps
+//   2..9 unpack each raw stage into two 128-row x 64-value bf16 operand blocks
+//   in the 128-byte swizzled K-major layout the MMA reads; warp 1 issues
+//   tcgen05.mma.kind::f16 into a TMEM accumulator. K may be split across a thread-block cluster with
 //   the partial tiles summed in rank order through distributed shared memory,
 //   as in the FP8 decode GEMM. The epilogue stores y = bf16(acc).
 #pragma once
@@ -110,13 +111,14 @@ struct W4DecodeCfg {
   static constexpr int kFixed = kOpRing + kRawRing + kBarBytes;
   static constexpr size_t kSmemSingle = 1024 + static_cast<size_t>(kFixed);
   static constexpr size_t kSmemSplit = kSmemSingle + kRedBytes;
-  static_assert(BNT % 16 == 0 && BNT >= 16 && BNT <= 64, "BNT");
+  static_assert(BNT % 16 == 0 && BNT >= 16 && BNT <= 128, "BNT");
   static_assert(kXBlock % 1024 == 0 && kRawBytes % 1024 == 0, "1024-byte alignment of blocks");
   static_assert(kYBytes <= kOpRing, "output tile must fit in the operand ring");
 };
 
 constexpr int kW4DequantWarps = 8;
-constexpr int kW4Threads = 64 + 32 * kW4DequantWarps;
+constexpr int kW4XWarp = 2 + kW4DequantWarps;  // the token-tile producer
+constexpr int kW4Threads = 32 * (kW4XWarp + 1);
 
 template <int BNT, int RS, int AS>
 __global__ void __launch_bounds__(kW4Threads, 1)
@@ -190,7 +192,20 @@ __global__ void __launch_bounds__(kW4Threads, 1)
 
   if (warp == 0) {
     if (lane == 0 && have_acc) {
+      // refill the raw stage step i used with step i + RS, once it is unpacked
       const uint64_t pol_w = l2_policy_evict_first();
+      for (int i = 0; i + RS < nst; ++i) {
+        const int rs = i % RS;
+        if (!mbar_wait(rempty0 + 8 * rs, (i / RS) & 1)) break;
+        const uint32_t rb = rfull0 + 8 * rs;
+        uint8_t* r = raws + rs * C::kRawBytes;
+        mbar_arrive_expect_tx(rb, C::kRawBytes);
+        tma_load_2d(smem_u32(r), &tmQ, rb, (st0 + i + RS) * 64, tile_n * kBM, pol_w);
+        tma_load_2d(smem_u32(r + C::kQBytes), &tmD, rb, (st0 + i + RS) * 4, tile_n * kBM, pol_w);
+      }
+    }
+  } else if (warp == kW4XWarp) {
+    if (lane == 0 && have_acc) {
       const uint64_t pol_x = l2_policy_evict_last();
       pdl_wait();  // the activations may come from the preceding grid
       for (int i = 0; i < nst; ++i) {
@@ -202,17 +217,6 @@ __global__ void __launch_bounds__(kW4Threads, 1)
         mbar_arrive_expect_tx(fb, 2 * C::kXBlock);
         tma_load_2d(smem_u32(x0), &tmX, fb, (st0 + i) * 256, 0, pol_x);
         tma_load_2d(smem_u32(x0 + C::kXBlock), &tmX, fb, (st0 + i) * 256 + 128, 0, pol_x);
-        // refill the raw stage step i used with step i + RS, once it is unpacked
-        const int nxt = i + RS;
-        if (nxt < nst) {
-          const int rs = i % RS;
-          if (!mbar_wait(rempty0 + 8 * rs, (i / RS) & 1)) break;
-          const uint32_t rb = rfull0 + 8 * rs;
-          uint8_t* r = raws + rs * C::kRawBytes;
-          mbar_arrive_expect_tx(rb, C::kRawBytes);
-          tma_load_2d(smem_u32(r), &tmQ, rb, (st0 + nxt) * 64, tile_n * kBM, pol_w);
-          tma_load_2d(smem_u32(r + C::kQBytes), &tmD, rb, (st0 + nxt) * 4, tile_n * kBM, pol_w);
-        }
       }
     }
   } else if (warp == 1) {

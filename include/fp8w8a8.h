@@ -386,14 +386,14 @@ fp8_status w4a16_dequant(const uint8_t* q4, const float* d, int64_t N, int64_t K
 
 /*
  * w4a16_workspace_bytes: the workspace w4a16_linear needs for this shape:
- * 0 when M <= 64 and K % 128 == 0 (the weights are unpacked on chip, inside
+ * 0 when M <= 128 and K % 128 == 0 (the weights are unpacked on chip, inside
  * the GEMM), else N * K * 2 bytes (the unpacked bf16 weights).
  */
 size_t w4a16_workspace_bytes(int64_t M, int64_t N, int64_t K);
 
 /*
  * w4a16_linear: y = x . w^T, x [M, K] bf16 (pitch K), y [M, N] bf16 out.
- * M <= 64 with K % 128 == 0: one kernel streams q4 and d (0.625 bytes per
+ * M <= 128 with K % 128 == 0: one kernel streams q4 and d (0.625 bytes per
  * weight) and unpacks them in shared memory for the MMA (swap-AB, K split
  * over a cluster for narrow layers). Otherwise w4a16_dequant into w_ws
  * (ws_bytes >= w4a16_workspace_bytes; caller-owned) followed by

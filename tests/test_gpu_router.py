@@ -38,6 +38,8 @@ def test_bf16_linear_within_bound(lib, M, N, K):
 def test_topk_matches_oracle_on_gpu_logits(lib, T, E, k):
     logits = _bf16_normal((T, E), seed=T + E, scale=2.0)
     logits[: T // 4, :E // 2] = logits[: T // 4, E // 2: 2 * (E // 2)]   # many exact ties
+    logits[T // 4: T // 2, ::3] = 0x0000                                 # +0 ...
+    logits[T // 4: T // 2, 1::3] = 0x8000                                # ... and -0 tie by index
     ids, w = lib.moe_topk(to_dev(logits), k)
     rid, rw = moe.topk_softmax(logits, k)
     assert np.array_equal(ids.cpu().numpy(), rid)

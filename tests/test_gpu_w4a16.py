@@ -1,6 +1,6 @@
 """GPU parity of the W4A16 build against the CPU oracle: the unpacked bf16
 weights bf16(fp32(d q)) bit for bit, and the GEMM - with the weights unpacked
-on chip (M <= 64) or into the workspace (longer M) - within
+on chip (M <= 128) or into the workspace (longer M) - within
 |y - y_exact| <= 4e-3 sum_k |x w| + 1 bf16 ulp of the exact sum over the QAT
 weights, element by element."""
 
@@ -32,11 +32,12 @@ def _check(y, xb, q4, d, rows=None):
 
 
 W4_SHAPES = [
-    # on-chip unpacking (M <= 64, K % 128 == 0): splits, variants, ragged N
+    # on-chip unpacking (M <= 128, K % 128 == 0): splits, variants, ragged N
     (1, 128, 256), (1, 8192, 2048), (8, 8192, 2048), (64, 8192, 2048), (16, 256, 4096),
     (17, 1000, 2048), (33, 130, 1024), (3, 21504, 5376), (64, 21504, 5376), (5, 520, 32768),
-    # workspace path: M > 64, or K % 128 != 0
-    (65, 1024, 2048), (300, 4096, 4096), (1000, 1000, 2048), (4, 256, 96), (200, 1001, 224),
+    (65, 1024, 2048), (128, 14336, 4096), (100, 21504, 5376),
+    # workspace path: M > 128, or K % 128 != 0
+    (129, 1024, 2048), (300, 4096, 4096), (1000, 1000, 2048), (4, 256, 96), (200, 1001, 224),
 ]
 
 
@@ -50,8 +51,8 @@ def test_w4a16_linear_within_bound(lib, M, N, K):
 
 
 def test_w4a16_workspace_is_required_and_sized(lib):
-    assert lib.w4a16_workspace_bytes(64, 1024, 2048) == 0
-    assert lib.w4a16_workspace_bytes(65, 1024, 2048) == 1024 * 2048 * 2
+    assert lib.w4a16_workspace_bytes(128, 1024, 2048) == 0
+    assert lib.w4a16_workspace_bytes(129, 1024, 2048) == 1024 * 2048 * 2
     assert lib.w4a16_workspace_bytes(8, 1024, 96) == 1024 * 96 * 2
     q4, d = q4_weights(256, 512, seed=1)
     x = to_dev(activations_bf16(200, 512, seed=1))
