@@ -17,10 +17,13 @@
 // * gemm_w4_decode_kernel (M <= 128): swap-AB like the FP8 decode GEMM, with
 //   the weight operand unpacked on chip. Warp 0 streams the packed weights
 //   and scales (0.625 bytes per weight) into a ring of raw stages with TMA;
-//   warp 10 streams the token tiles into the operand ring (a thread of its
+//   warp 18 streams the token tiles into the operand ring (a thread of its
 //   own, so that no token-tile load waits behind a raw-stage refill); warps
-//   2..9 unpack each raw stage into two 128-row x 64-value bf16 operand blocks
-//   in the 128-byte swizzled K-major layout the MMA reads; warp 1 issues
+//   2..17 unpack each raw stage into two 128-row x 64-value bf16 operand
+//   blocks in the 128-byte swizzled K-major layout the MMA reads (sixteen
+//   warps, four per scheduler, one 32-value group per thread: the unpacking
+//   is a chain of dependent integer and fp32 steps whose latency the other
+//   warps hide); warp 1 issues
 //   tcgen05.mma.kind::f16 into a TMEM accumulator. K may be split across a thread-block cluster with
 //   the partial tiles summed in rank order through distributed shared memory,
 //   as in the FP8 decode GEMM. The epilogue stores y = bf16(acc).
@@ -116,7 +119,7 @@ struct W4DecodeCfg {
   static_assert(kYBytes <= kOpRing, "output tile must fit in the operand ring");
 };
 
-constexpr int kW4DequantWarps = 8;
+constexpr int kW4DequantWarps = 16;
 constexpr int kW4XWarp = 2 + kW4DequantWarps;  // the token-tile producer
 constexpr int kW4Threads = 32 * (kW4XWarp + 1);
 
@@ -241,25 +244,33 @@ __global__ void __launch_bounds__(kW4Threads, 1)
       umma_commit(tfull);
     }
   } else {
-    // Warps 2..9 unpack: thread (r, j) turns row r's 64 packed values of
-    // k-block j (32 bytes, two groups) into the 128-byte swizzled row r of
-    // weight block j (16-byte piece c at position c ^ (r & 7)).
+    // Warps 2..17 unpack: thread (r, c) turns 16-byte piece c of row r's
+    // packed step (32 values, one group; k-block j = c / 2) into four
+    // 16-byte pieces of row r of weight block j, piece p of a row stored at
+    // p ^ (r & 7) (the 128-byte swizzle). Explicit shared-memory accesses.
     const int t = threadIdx.x - 64;
-    const int r = t & 127, j = t >> 7;
+    const int r = t & 127, c = t >> 7;
+    const int j = c >> 1, p0 = (c & 1) * 4;
     for (int i = 0; have_acc && i < nst; ++i) {
       const int rs = i % RS, os = i % AS;
       const bool ok = mbar_wait(rfull0 + 8 * rs, (i / RS) & 1) &&
                       mbar_wait(oempty0 + 8 * os, ((i / AS) & 1) ^ 1);
       if (!__all_sync(0xFFFFFFFFu, ok)) break;
-      const uint8_t* raw = raws + rs * C::kRawBytes;
-      const uint4 q0 = *reinterpret_cast<const uint4*>(raw + r * 64 + j * 32);
-      const uint4 q1 = *reinterpret_cast<const uint4*>(raw + r * 64 + j * 32 + 16);
-      const float2 dd = *reinterpret_cast<const float2*>(raw + C::kQBytes + r * 16 + j * 8);
-      uint8_t* arow = ops + os * C::kStageBytes + j * C::kABlock + r * 128;
-      const uint32_t wq[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
+      const uint32_t raw = smem_u32(raws + rs * C::kRawBytes);
+      uint32_t q[4];
+      float dg;
+      asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                   : "=r"(q[0]), "=r"(q[1]), "=r"(q[2]), "=r"(q[3])
+                   : "r"(raw + r * 64 + c * 16));
+      asm volatile("ld.shared.f32 %0, [%1];" : "=f"(dg) : "r"(raw + C::kQBytes + r * 16 + c * 4));
+      const uint32_t arow = smem_u32(ops + os * C::kStageBytes + j * C::kABlock + r * 128);
 #pragma unroll
-      for (int c = 0; c < 8; ++c)
-        *reinterpret_cast<uint4*>(arow + ((c ^ (r & 7)) << 4)) = unpack8_bf16(wq[c], c < 4 ? dd.x : dd.y);
+      for (int w = 0; w < 4; ++w) {
+        const uint4 v = unpack8_bf16(q[w], dg);
+        asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(arow + (((p0 + w) ^ (r & 7)) << 4)),
+                     "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
+                     : "memory");
+      }
       fence_proxy_async_shared();  // the generic writes -> visible to the tensor core
       __syncwarp();
       if (lane == 0) {
