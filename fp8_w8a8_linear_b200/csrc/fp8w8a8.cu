@@ -635,7 +635,7 @@ fp8_status launch_w4_decode_t(const DeviceInfo& dev, const uint16_t* x, const ui
       (N % 8 == 0) && make_tmap_bf16_store(&tmY, y, M, N, kBM / splits, BNT) ? 1 : 0;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(tiles * splits);
-  cfg.blockDim = dim3(kW4Threads);
+  cfg.blockDim = dim3(w4_threads(RS));
   cfg.dynamicSmemBytes = splits > 1 ? C::kSmemSplit : C::kSmemSingle;
   cfg.stream = stream;
   cudaLaunchAttribute attrs[2];

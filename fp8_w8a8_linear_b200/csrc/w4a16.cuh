@@ -112,25 +112,30 @@ struct W4DecodeCfg {
   static constexpr int kBarBytes = 8 * (2 * RS + 2 * AS + 1) + 16;
   static constexpr int kRedBytes = BNT * kBM * 4;
   static constexpr int kFixed = kOpRing + kRawRing + kBarBytes;
+  static constexpr int kRedOff = (kFixed + 127) / 128 * 128;  // 16-byte vector accesses
   static constexpr size_t kSmemSingle = 1024 + static_cast<size_t>(kFixed);
-  static constexpr size_t kSmemSplit = kSmemSingle + kRedBytes;
+  static constexpr size_t kSmemSplit = 1024 + static_cast<size_t>(kRedOff) + kRedBytes;
   static_assert(BNT % 16 == 0 && BNT >= 16 && BNT <= 128, "BNT");
   static_assert(kXBlock % 1024 == 0 && kRawBytes % 1024 == 0, "1024-byte alignment of blocks");
   static_assert(kYBytes <= kOpRing, "output tile must fit in the operand ring");
 };
 
-constexpr int kW4DequantWarps = 16;
-constexpr int kW4XWarp = 2 + kW4DequantWarps;  // the token-tile producer
-constexpr int kW4Threads = 32 * (kW4XWarp + 1);
+// Unpacking warps: 16 in the deep-ring variants (one CTA per SM), 8 in the
+// shallow ones, which must leave room - registers included - for a second
+// CTA on the SM.
+__host__ __device__ constexpr int w4_unpack_warps(int rs) { return rs >= 4 ? 16 : 8; }
+__host__ __device__ constexpr int w4_threads(int rs) { return 32 * (3 + w4_unpack_warps(rs)); }
 
 template <int BNT, int RS, int AS>
-__global__ void __launch_bounds__(kW4Threads, 1)
+__global__ void __launch_bounds__(w4_threads(RS), RS >= 4 ? 1 : 2)
     gemm_w4_decode_kernel(const __grid_constant__ CUtensorMap tmQ,
                           const __grid_constant__ CUtensorMap tmD,
                           const __grid_constant__ CUtensorMap tmX,
                           const __grid_constant__ CUtensorMap tmY, uint16_t* __restrict__ y, int M,
                           int N, int K, int splits, int st_per_split, int use_tma_store) {
   using C = W4DecodeCfg<BNT, RS, AS>;
+  constexpr int kW4DequantWarps = w4_unpack_warps(RS);
+  constexpr int kW4XWarp = 2 + kW4DequantWarps;  // the token-tile producer
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
   uint8_t* ops = smem;                          // AS operand stages
@@ -138,7 +143,7 @@ __global__ void __launch_bounds__(kW4Threads, 1)
   uint16_t* ytile = reinterpret_cast<uint16_t*>(smem);
   uint64_t* bars = reinterpret_cast<uint64_t*>(raws + C::kRawRing);
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 2 * RS + 2 * AS + 1);
-  float* red = reinterpret_cast<float*>(smem + C::kFixed);  // split only
+  float* red = reinterpret_cast<float*>(smem + C::kRedOff);  // split only
   const uint32_t rfull0 = smem_u32(bars);
   const uint32_t rempty0 = smem_u32(bars + RS);
   const uint32_t ofull0 = smem_u32(bars + 2 * RS);
@@ -244,32 +249,36 @@ __global__ void __launch_bounds__(kW4Threads, 1)
       umma_commit(tfull);
     }
   } else {
-    // Warps 2..17 unpack: thread (r, c) turns 16-byte piece c of row r's
+    // The unpacking warps: unit (r, c) turns 16-byte piece c of row r's
     // packed step (32 values, one group; k-block j = c / 2) into four
     // 16-byte pieces of row r of weight block j, piece p of a row stored at
-    // p ^ (r & 7) (the 128-byte swizzle). Explicit shared-memory accesses.
+    // p ^ (r & 7) (the 128-byte swizzle). 512 units per step, one or two per
+    // thread. Explicit shared-memory accesses.
     const int t = threadIdx.x - 64;
-    const int r = t & 127, c = t >> 7;
-    const int j = c >> 1, p0 = (c & 1) * 4;
     for (int i = 0; have_acc && i < nst; ++i) {
       const int rs = i % RS, os = i % AS;
       const bool ok = mbar_wait(rfull0 + 8 * rs, (i / RS) & 1) &&
                       mbar_wait(oempty0 + 8 * os, ((i / AS) & 1) ^ 1);
       if (!__all_sync(0xFFFFFFFFu, ok)) break;
       const uint32_t raw = smem_u32(raws + rs * C::kRawBytes);
-      uint32_t q[4];
-      float dg;
-      asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
-                   : "=r"(q[0]), "=r"(q[1]), "=r"(q[2]), "=r"(q[3])
-                   : "r"(raw + r * 64 + c * 16));
-      asm volatile("ld.shared.f32 %0, [%1];" : "=f"(dg) : "r"(raw + C::kQBytes + r * 16 + c * 4));
-      const uint32_t arow = smem_u32(ops + os * C::kStageBytes + j * C::kABlock + r * 128);
 #pragma unroll
-      for (int w = 0; w < 4; ++w) {
-        const uint4 v = unpack8_bf16(q[w], dg);
-        asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(arow + (((p0 + w) ^ (r & 7)) << 4)),
-                     "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
-                     : "memory");
+      for (int u = t; u < 512; u += 32 * kW4DequantWarps) {
+        const int r = u & 127, c = u >> 7;
+        const int j = c >> 1, p0 = (c & 1) * 4;
+        uint32_t q[4];
+        float dg;
+        asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                     : "=r"(q[0]), "=r"(q[1]), "=r"(q[2]), "=r"(q[3])
+                     : "r"(raw + r * 64 + c * 16));
+        asm volatile("ld.shared.f32 %0, [%1];" : "=f"(dg) : "r"(raw + C::kQBytes + r * 16 + c * 4));
+        const uint32_t arow = smem_u32(ops + os * C::kStageBytes + j * C::kABlock + r * 128);
+#pragma unroll
+        for (int w = 0; w < 4; ++w) {
+          const uint4 v = unpack8_bf16(q[w], dg);
+          asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(arow + (((p0 + w) ^ (r & 7)) << 4)),
+                       "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
+                       : "memory");
+        }
       }
       fence_proxy_async_shared();  // the generic writes -> visible to the tensor core
       __syncwarp();
@@ -280,7 +289,7 @@ __global__ void __launch_bounds__(kW4Threads, 1)
     }
   }
 
-  // ---- epilogue: warps 2..5 (TMEM lane quadrants); warps 6..9 only wait
+  // ---- epilogue: warps 2..5 (TMEM lane quadrants); the other warps only wait
   const bool epi = warp >= 2 && warp < 6;
   if (epi) {
     const int et = threadIdx.x - 64;  // 0..127
@@ -293,7 +302,8 @@ __global__ void __launch_bounds__(kW4Threads, 1)
     uint32_t dst = 0;
     if (split) {
       cluster_wait_acquire();  // every CTA of the cluster has started
-      dst = mapa_shared(smem_u32(red) + static_cast<uint32_t>((rank * BNT * rows + ch % rows) * 4),
+      // owner's buffer [rank][channel in slice][token], 16-byte stores
+      dst = mapa_shared(smem_u32(red) + static_cast<uint32_t>(((rank * rows + ch % rows) * BNT) * 4),
                         ch / rows);
     }
     (void)et;
@@ -302,15 +312,20 @@ __global__ void __launch_bounds__(kW4Threads, 1)
       uint32_t rr[16];
       tmem_ld16(t_row + c * 16, rr);
       tmem_ld_wait();
+      float acc[16];
 #pragma unroll
-      for (int jj = 0; jj < 16; ++jj) {
-        const int tok = c * 16 + jj;
-        const float acc = have_acc ? __uint_as_float(rr[jj]) : 0.0f;
-        if (!split) {
-          ytile[tok * kBM + ch] = f32_to_bf16_rn(acc);
-        } else if (tok < M) {
-          st_shared_cluster_f32(dst + static_cast<uint32_t>(tok * rows * 4), acc);
-        }
+      for (int jj = 0; jj < 16; ++jj) acc[jj] = have_acc ? __uint_as_float(rr[jj]) : 0.0f;
+      if (!split) {
+#pragma unroll
+        for (int jj = 0; jj < 16; ++jj) ytile[(c * 16 + jj) * kBM + ch] = f32_to_bf16_rn(acc[jj]);
+      } else {
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+          if (c * 16 + 4 * q < M)
+            asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(
+                             dst + static_cast<uint32_t>((c * 16 + 4 * q) * 4)),
+                         "f"(acc[4 * q]), "f"(acc[4 * q + 1]), "f"(acc[4 * q + 2]), "f"(acc[4 * q + 3])
+                         : "memory");
       }
     }
   }
@@ -326,13 +341,32 @@ __global__ void __launch_bounds__(kW4Threads, 1)
     cluster_arrive_release();          // this CTA's partials are in their owners' buffers
     cluster_wait_acquire();
     if (epi) {
+      // four tokens of one channel per thread and step, summed over the ranks
+      // in rank order (tokens past M are left out: the store clips them)
       const int et = threadIdx.x - 64;
-      for (int e = et; e < rows * BNT; e += 128) {
-        const int tok = e / rows;
-        const int rl = e % rows;
-        float sum = red[tok * rows + rl];
-        for (int s = 1; s < splits; ++s) sum = __fadd_rn(sum, red[(s * BNT + tok) * rows + rl]);
-        ytile[tok * rows + rl] = f32_to_bf16_rn(sum);
+      constexpr int kTG = BNT / 4;
+      const uint32_t red_s = smem_u32(red);
+      for (int e = et; e < rows * kTG; e += 128) {
+        const int rl = e / kTG, tg = e % kTG;
+        if (4 * tg >= M) continue;
+        float4 sum;
+        asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
+                     : "=f"(sum.x), "=f"(sum.y), "=f"(sum.z), "=f"(sum.w)
+                     : "r"(red_s + static_cast<uint32_t>((rl * BNT + 4 * tg) * 4)));
+        for (int s = 1; s < splits; ++s) {
+          float4 v;
+          asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
+                       : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+                       : "r"(red_s + static_cast<uint32_t>(((s * rows + rl) * BNT + 4 * tg) * 4)));
+          sum.x = __fadd_rn(sum.x, v.x);
+          sum.y = __fadd_rn(sum.y, v.y);
+          sum.z = __fadd_rn(sum.z, v.z);
+          sum.w = __fadd_rn(sum.w, v.w);
+        }
+        ytile[(4 * tg) * rows + rl] = f32_to_bf16_rn(sum.x);
+        ytile[(4 * tg + 1) * rows + rl] = f32_to_bf16_rn(sum.y);
+        ytile[(4 * tg + 2) * rows + rl] = f32_to_bf16_rn(sum.z);
+        ytile[(4 * tg + 3) * rows + rl] = f32_to_bf16_rn(sum.w);
       }
     }
   }
