@@ -150,7 +150,13 @@ fp8_status set_decode_attr(int smem_optin) {
              : FP8_ERR_CUDA;
 }
 
+// Shared memory of a grouped pair launch with E experts.
 template <int STAGES>
+size_t grouped_pair_smem(int E) {
+  return PairCfg<STAGES, pair_stg_bufs<true>()>::kSmem + grouped_smem_bytes(E);
+}
+
+template <int STAGES, int GSTAGES>
 fp8_status set_pair_attr() {
   return cudaFuncSetAttribute(gemm_pair_kernel<STAGES>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                               static_cast<int>(PairCfg<STAGES>::kSmem)) == cudaSuccess &&
@@ -160,13 +166,13 @@ fp8_status set_pair_attr() {
                  cudaFuncSetAttribute(gemm_pair_kernel<STAGES, false, false, kKindBF16>,
                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
                                       static_cast<int>(PairCfg<STAGES>::kSmem)) == cudaSuccess &&
-                 cudaFuncSetAttribute(gemm_pair_kernel<STAGES, true>,
+                 cudaFuncSetAttribute(gemm_pair_kernel<GSTAGES, true>,
                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                      static_cast<int>(PairCfg<STAGES>::kSmem + grouped_smem_bytes(kMaxExperts))) ==
+                                      static_cast<int>(grouped_pair_smem<GSTAGES>(kMaxExperts))) ==
                      cudaSuccess &&
-                 cudaFuncSetAttribute(gemm_pair_kernel<STAGES, true, true>,
+                 cudaFuncSetAttribute(gemm_pair_kernel<GSTAGES, true, true>,
                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                      static_cast<int>(PairCfg<STAGES>::kSmem + grouped_smem_bytes(kMaxExperts))) ==
+                                      static_cast<int>(grouped_pair_smem<GSTAGES>(kMaxExperts))) ==
                      cudaSuccess
              ? FP8_OK
              : FP8_ERR_CUDA;
@@ -201,6 +207,9 @@ fp8_status set_w4_attr(int smem_optin) {
 }
 
 constexpr int kPairStages = 6;
+// Grouped pair launches: five stages, which leaves room for the epilogue's
+// second staging buffer per warp.
+constexpr int kGroupedPairStages = 5;
 constexpr int kPrefillBN = 256;
 // Shared memory the staged quantizer may use per block (one block per SM).
 constexpr int kStagedSmemBudget = 200 * 1024;
@@ -223,7 +232,7 @@ fp8_status device_info(DeviceInfo** out) {
     st = st != FP8_OK ? st : set_prefill_attr<kPrefillBN, kPrefillStages, false, kKindS8>();
     st = st != FP8_OK ? st : set_prefill_attr<kPrefillBN, kPrefillStages, false, kKindBF16>();
     st = st != FP8_OK ? st : set_prefill_attr<256, kPrefillStages, true>();
-    st = st != FP8_OK ? st : set_pair_attr<kPairStages>();
+    st = st != FP8_OK ? st : set_pair_attr<kPairStages, kGroupedPairStages>();
     if (st == FP8_OK) {
       // A persistent grid must fit at once: count the 2-CTA clusters that can
       // be resident together (an SM left over in a GPC cannot host a pair).
@@ -432,7 +441,7 @@ fp8_status launch_grouped_pair(const DeviceInfo& dev, const uint8_t* x8, const f
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2 * dev.pair_clusters);
   cfg.blockDim = dim3(kPrefillThreads);
-  cfg.dynamicSmemBytes = PairCfg<kPairStages>::kSmem + grouped_smem_bytes(E);
+  cfg.dynamicSmemBytes = grouped_pair_smem<kGroupedPairStages>(E);
   cfg.stream = stream;
   cudaLaunchAttribute attrs[2];
   int na = 0;
@@ -460,8 +469,8 @@ fp8_status launch_grouped_pair(const DeviceInfo& dev, const uint8_t* x8, const f
   // GeGLU: half-width last feature tiles load 64 B rows per CTA through tmBh
   CUtensorMap tmBh = tmB;
   if (n_out > 0 && !make_tmap_u8(&tmBh, w8, static_cast<uint64_t>(E) * N, K, 64)) return FP8_ERR_CUDA;
-  const auto kernel = n_out > 0 ? gemm_pair_kernel<kPairStages, true, true>
-                                : gemm_pair_kernel<kPairStages, true, false>;
+  const auto kernel = n_out > 0 ? gemm_pair_kernel<kGroupedPairStages, true, true>
+                                : gemm_pair_kernel<kGroupedPairStages, true, false>;
   if (cudaLaunchKernelEx(&cfg, kernel, tmA, tmB, tmBh, tmY, g) != cudaSuccess) return FP8_ERR_CUDA;
   return FP8_OK;
 }

@@ -108,17 +108,36 @@ __device__ __forceinline__ void store_chunk_coalesced(uint8_t* stg, const uint4 
   __syncwarp();  // the buffer is rewritten by the next chunk
 }
 
+// A warp's epilogue staging buffers (one, or two used in turn): `last` is
+// the buffer the most recently committed TMA store reads (-1: none yet).
+struct StgRing {
+  uint8_t* base;
+  int nbuf;
+  int turn;
+  int last;
+  __device__ __forceinline__ uint8_t* buf(int b) const { return base + b * kStageChunkBytes; }
+};
+
 // Store of one 32 x 32 bf16 chunk a warp holds one row per lane (pk = the
 // lane's 64 bytes; `row` = this lane's row): one TMA store of the swizzled
 // staging buffer when tma_ok (warp-uniform: the map covers y and all 32 rows
 // belong to the tile's rows; the map clips columns at N), else through
-// store_chunk_coalesced. The buffer is rewritten only after the previous
-// store from it has read it.
-__device__ __forceinline__ void epi_store_chunk(const uint4 (&pk)[4], uint8_t* stg,
+// store_chunk_coalesced. A buffer is rewritten only after every store that
+// reads it has done so: with two buffers, when the latest store reads the
+// other one, every store but that latest one - so staging a chunk overlaps
+// the previous chunk's store.
+__device__ __forceinline__ void epi_store_chunk(const uint4 (&pk)[4], StgRing& ring,
                                                 uint16_t* __restrict__ y, int row, int64_t row_end,
                                                 int N, int n0, int lane, const CUtensorMap* tmY,
                                                 bool tma_ok) {
-  if (lane == 0) bulk_wait_group_read_all();  // the previous store from stg has read it
+  const int b = ring.turn;
+  uint8_t* stg = ring.buf(b);
+  if (lane == 0) {
+    if (ring.nbuf > 1 && ring.last != b)
+      bulk_wait_group_read_but_last();
+    else
+      bulk_wait_group_read_all();
+  }
   __syncwarp();
   if (tma_ok) {
 #pragma unroll
@@ -130,6 +149,8 @@ __device__ __forceinline__ void epi_store_chunk(const uint4 (&pk)[4], uint8_t* s
       tma_store_2d(tmY, smem_u32(stg), n0, row - lane);
       bulk_commit_group();
     }
+    ring.last = b;
+    if (ring.nbuf > 1) ring.turn ^= 1;
   } else {
     store_chunk_coalesced(stg, pk, y, row - lane, row_end, N, n0, lane);
   }
@@ -148,7 +169,7 @@ __device__ __forceinline__ void epi_store_chunk(const uint4 (&pk)[4], uint8_t* s
 // store from it has read it.
 __device__ __forceinline__ void epi_chunk(const uint32_t (&r)[32], const float* sb_chunk,
                                           float sa, bool vec_ok,
-                                          uint8_t* stg, uint16_t* __restrict__ y, int row,
+                                          StgRing& stg, uint16_t* __restrict__ y, int row,
                                           int64_t row_end, int N, int n0, int lane,
                                           const CUtensorMap* tmY, bool tma_ok) {
   if (n0 >= N) return;
@@ -462,7 +483,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     // and warps w and w+4 share a quadrant, splitting its column chunks.
     const int quad = warp & 3;
     const int half = (warp - 2) >> 2;
-    uint8_t* stg = stg_all + (warp - 2) * kStageChunkBytes;  // this warp's staging chunk
+    StgRing stg = {stg_all + (warp - 2) * kStageChunkBytes, 1, 0, -1};  // this warp's staging chunk
     float* sb_tile = reinterpret_cast<float*>(stg_all + 8 * kStageChunkBytes);  // [2][256]
     const int N = g.N;
     // 16-byte stores of y rows and 16-byte loads of the column scales
@@ -527,7 +548,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
 // multicast to the stage's empty barrier (or the accumulator's full barrier)
 // in both CTAs; each CTA drains its own 128 TMEM lanes (its 128 rows), and the
 // even CTA's accumulator-empty barrier counts the epilogue warps of both.
-template <int STAGES>
+template <int STAGES, int STG_BUFS = 1>
 struct PairCfg {
   static constexpr int kHalf = 128;                  // rows of A and of B per CTA
   static constexpr int kBN = 256;                    // tile columns
@@ -536,8 +557,9 @@ struct PairCfg {
   static constexpr int kStageBytes = kABytes + kBBytes;
   static constexpr int kTmemCols = 512;              // two 256-column accumulators
   static constexpr int kBarBytes = 8 * (2 * STAGES + 4) + 16;
-  // epilogue staging: one 2 KB chunk and 128 column scales per epilogue warp
-  static constexpr int kStgBytes = kEpiWarps * (kStageChunkBytes + 128 * 4);
+  // epilogue staging: STG_BUFS 2 KB chunks and 128 column scales per epilogue
+  // warp
+  static constexpr int kStgBytes = kEpiWarps * (STG_BUFS * kStageChunkBytes + 128 * 4);
   static constexpr size_t kSmem =
       1024 + static_cast<size_t>(STAGES) * kStageBytes + kStgBytes + kBarBytes;
 };
@@ -557,12 +579,18 @@ struct PairCfg {
 // is half width: each CTA loads 64 B rows (through tmBh, a map with 64-row
 // boxes) and the MMAs run with N = 128, so the leader's gate rows fill
 // accumulator columns 0..63 and the peer's up rows columns 64..127.
+// Grouped launches (short K per expert tile, so the epilogue sets the pace)
+// give each epilogue warp two staging buffers.
+template <bool GROUPED>
+__host__ __device__ constexpr int pair_stg_bufs() { return GROUPED ? 2 : 1; }
+
 template <int STAGES, bool GROUPED = false, bool GEGLU = false, int KD = kKindE4M3>
 __global__ void __launch_bounds__(kPrefillThreads, 1)
     gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                      const __grid_constant__ CUtensorMap tmBh, const __grid_constant__ CUtensorMap tmY,
                      const GemmArgs g) {
-  using C = PairCfg<STAGES>;
+  constexpr int kStgBufs = pair_stg_bufs<GROUPED>();
+  using C = PairCfg<STAGES, kStgBufs>;
   static_assert(GROUPED || !GEGLU, "the GeGLU epilogue is for the grouped GEMM");
   static_assert(!GEGLU || KD == kKindE4M3, "the GeGLU epilogue is for E4M3 operands");
   extern __shared__ uint8_t smem_raw[];
@@ -703,8 +731,10 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     // another: a tile is a TMEM-full wait, the warp's chunks and an arrive.
     const int quad = warp & 3;
     const int half = (warp - 2) >> 2;
-    uint8_t* stg = stg_all + (warp - 2) * kStageChunkBytes;  // this warp's staging chunk
-    float* sbw = reinterpret_cast<float*>(stg_all + kEpiWarps * kStageChunkBytes) + (warp - 2) * 128;
+    // this warp's staging chunk(s), used in turn
+    StgRing stg = {stg_all + (warp - 2) * kStgBufs * kStageChunkBytes, kStgBufs, 0, -1};
+    float* sbw =
+        reinterpret_cast<float*>(stg_all + kEpiWarps * kStgBufs * kStageChunkBytes) + (warp - 2) * 128;
     const int N = g.N;
     // 16-byte stores of y rows and 16-byte loads of the column scales
     const bool vec_ok = (N % 8) == 0 && (reinterpret_cast<uintptr_t>(g.s_b) & 15) == 0;

@@ -165,6 +165,11 @@ __device__ __forceinline__ void bulk_wait_group_all() {
 __device__ __forceinline__ void bulk_wait_group_read_all() {
   asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
 }
+// As above, except for the most recently committed group (which may still be
+// reading its own, other buffer).
+__device__ __forceinline__ void bulk_wait_group_read_but_last() {
+  asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
+}
 
 // Named barrier among `count` threads (a multiple of 32), id 1..15.
 __device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t count) {
