@@ -139,11 +139,11 @@ fp8_status set_prefill_attr() {
 
 // Deep-ring variants whose split-K layout would not fit are set up (and
 // launched) without a K split only.
-template <int BNT, int STAGES, int KBS, int KD = kKindE4M3, bool FQ = false>
+template <int BNT, int STAGES, int KBS, int KD = kKindE4M3>
 fp8_status set_decode_attr(int smem_optin) {
   using C = DecodeCfg<BNT, STAGES, KBS>;
   const size_t smem = C::kSmemSplit <= static_cast<size_t>(smem_optin) ? C::kSmemSplit : C::kSmemSingle;
-  return cudaFuncSetAttribute(gemm_decode_kernel<BNT, STAGES, KBS, KD, FQ>,
+  return cudaFuncSetAttribute(gemm_decode_kernel<BNT, STAGES, KBS, KD>,
                               cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) ==
                  cudaSuccess
              ? FP8_OK
@@ -192,11 +192,6 @@ fp8_status set_decode_attrs(int so) {
   st = st != FP8_OK ? st : set_decode_attr<128, 3, 1, KD>(so);
   st = st != FP8_OK ? st : set_decode_attr<128, 4, 1, KD>(so);
   st = st != FP8_OK ? st : set_decode_attr<128, 6, 1, KD>(so);
-  if (KD == kKindE4M3) {  // the fused-quantization variants (up to 16 tokens)
-    st = st != FP8_OK ? st : set_decode_attr<16, 2, 2, kKindE4M3, true>(so);
-    st = st != FP8_OK ? st : set_decode_attr<16, 3, 2, kKindE4M3, true>(so);
-    st = st != FP8_OK ? st : set_decode_attr<16, 6, 2, kKindE4M3, true>(so);
-  }
   return st;
 }
 
@@ -529,11 +524,10 @@ int decode_splits(const DeviceInfo& dev, int N, int K, int kbs) {
   return splits;
 }
 
-template <int BNT, int ST, int KBS, int KD = kKindE4M3, bool FQ = false>
+template <int BNT, int ST, int KBS, int KD = kKindE4M3>
 fp8_status launch_decode_t(const DeviceInfo& dev, const uint8_t* x8, const float* s_tok,
                            const uint8_t* w8, const float* s_ch, int M, int N, int K, uint16_t* y,
-                           cudaStream_t stream, bool pdl, int force_splits = 0,
-                           const DecodeFQ fq = DecodeFQ{nullptr, nullptr, nullptr}) {
+                           cudaStream_t stream, bool pdl, int force_splits = 0) {
   using C = DecodeCfg<BNT, ST, KBS>;
   CUtensorMap tmW, tmX;
   if (!make_tmap_u8(&tmW, w8, N, K, kBM) || !make_tmap_u8(&tmX, x8, M, K, BNT))
@@ -563,8 +557,8 @@ fp8_status launch_decode_t(const DeviceInfo& dev, const uint8_t* x8, const float
   set_pdl(attrs, na, pdl);
   cfg.attrs = attrs;
   cfg.numAttrs = na;
-  if (cudaLaunchKernelEx(&cfg, gemm_decode_kernel<BNT, ST, KBS, KD, FQ>, tmW, tmX, tmY, s_tok, s_ch, y,
-                         M, N, K, splits, steps_per_split, use_tma_store, fq) != cudaSuccess)
+  if (cudaLaunchKernelEx(&cfg, gemm_decode_kernel<BNT, ST, KBS, KD>, tmW, tmX, tmY, s_tok, s_ch, y, M,
+                         N, K, splits, steps_per_split, use_tma_store) != cudaSuccess)
     return FP8_ERR_CUDA;
   return FP8_OK;
 }
@@ -622,42 +616,6 @@ fp8_status launch_linear(const DeviceInfo& dev, const uint8_t* x8, const float* 
       return launch_pair<KD>(dev, x8, s_tok, w8, s_ch, M, N, K, y, stream, pdl);
   }
   return launch_prefill<KD>(dev, x8, s_tok, w8, s_ch, M, N, K, y, stream, pdl);
-}
-
-// The whole W8A8 linear from bf16 in one decode launch (quantization fused,
-// bit-identical to launch_quant_act + launch_linear), when it applies: up to
-// 16 tokens, and the decode variant launch_linear would pick keeps every CTA's
-// K range inside its token-tile ring. Returns FP8_ERR_UNSUPPORTED (nothing
-// launched) otherwise.
-fp8_status launch_linear_fused(const DeviceInfo& dev, const uint16_t* x, const uint8_t* w8,
-                               const float* s_ch, int M, int N, int K, uint8_t* x8, float* s_tok,
-                               uint16_t* y, cudaStream_t stream) {
-  if (M > 16) return FP8_ERR_UNSUPPORTED;
-  const DecodeFQ fq{x, x8, s_tok};
-  const int tiles = (N + kBM - 1) / kBM;
-  const bool one_per_sm = tiles <= dev.sm_count;
-  const bool no_split = 4 * tiles >= dev.sm_count;
-  const int num_kb = (K + kBK - 1) / kBK;
-  // the same variant choice as launch_linear for M <= 16
-  int s = 1;
-  while (s < 8 && tiles * s * 2 <= 2 * dev.sm_count && s * 2 * 4 <= num_kb) s *= 2;
-  auto fits = [&](int stages, int kbs, int splits) {
-    const int num_steps = (num_kb + kbs - 1) / kbs;
-    return (num_steps + splits - 1) / splits <= stages;
-  };
-  if (s >= 4) {
-    if (!fits(2, 2, s)) return FP8_ERR_UNSUPPORTED;
-    return launch_decode_t<16, 2, 2, kKindE4M3, true>(dev, x8, s_tok, w8, s_ch, M, N, K, y, stream,
-                                                       true, s, fq);
-  }
-  if (one_per_sm && no_split) {
-    if (!fits(6, 2, decode_splits(dev, N, K, 2))) return FP8_ERR_UNSUPPORTED;
-    return launch_decode_t<16, 6, 2, kKindE4M3, true>(dev, x8, s_tok, w8, s_ch, M, N, K, y, stream,
-                                                       true, 0, fq);
-  }
-  if (!fits(3, 2, decode_splits(dev, N, K, 2))) return FP8_ERR_UNSUPPORTED;
-  return launch_decode_t<16, 3, 2, kKindE4M3, true>(dev, x8, s_tok, w8, s_ch, M, N, K, y, stream,
-                                                     true, 0, fq);
 }
 
 // W4A16 decode, weights unpacked on chip (M <= 128, K % 128 == 0). K is split
@@ -941,17 +899,10 @@ fp8_status fp8_linear_bf16(const uint16_t* x, const uint8_t* w8, const float* s_
       return FP8_ERR_CUDA;
     return FP8_OK;
   }
-  // Up to 16 tokens, when every decode CTA's K range fits its token tiles:
-  // one launch, the quantization inside the GEMM (each CTA computes the
-  // tokens' scales from their whole rows and the codes of its own K range).
-  // Otherwise two launches, the GEMM a programmatic dependent of the
-  // quantizer, so its weight stream starts while the quantizer runs.
-  {
-    const fp8_status st = launch_linear_fused(*dev, x, w8, s_ch, static_cast<int>(M),
-                                              static_cast<int>(N), static_cast<int>(K), x8, s_tok,
-                                              y, as_stream(stream));
-    if (st != FP8_ERR_UNSUPPORTED) return st;
-  }
+  // Two launches: the GEMM is a programmatic dependent of the quantizer, so
+  // its weight stream starts while the quantizer runs. (Quantizing inside the
+  // decode GEMM was measured slower on B200: every CTA must quantize the whole
+  // token block, and staging it costs the second CTA per SM.)
   if (fp8_status st = launch_quant_act(*dev, x, M, K, K, x8, s_tok, as_stream(stream))) return st;
   return launch_linear(*dev, x8, s_tok, w8, s_ch, static_cast<int>(M), static_cast<int>(N),
                        static_cast<int>(K), y, as_stream(stream), true);

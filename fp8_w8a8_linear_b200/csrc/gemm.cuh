@@ -41,7 +41,6 @@
 
 #include "act.cuh"
 #include "ptx.cuh"
-#include "quant.cuh"
 
 namespace fp8k {
 
@@ -879,7 +878,7 @@ struct DecodeCfg {
   static constexpr int kTmemCols = tmem_cols_for(BNT);
   static constexpr int kPipeBytes = STAGES * kStageBytes;
   static constexpr int kYBytes = BNT * kBM * 2;    // bf16 output tile, reuses the pipeline
-  static constexpr int kBarBytes = 8 * (2 * STAGES + 2) + 16;
+  static constexpr int kBarBytes = 8 * (2 * STAGES + 1) + 16;
   static constexpr int kScaleBytes = (kBM + BNT) * 4;  // s_ch of the tile, s_tok
   static constexpr int kRedBytes = BNT * kBM * 4;  // fp32 partials [rank][token][row in slice]
   static constexpr int kFixed = kPipeBytes + kBarBytes + kScaleBytes;
@@ -893,116 +892,30 @@ struct DecodeCfg {
 
 // y is written either by one TMA store per output tile (tmY valid, N % 8 == 0;
 // its box is {rows written per CTA, BNT}) or element by element.
-// Per-token quantization of x for one decode CTA (FQ mode), bit for bit the
-// quantizer kernels' arithmetic: amax over the whole row as the integer max
-// of |bf16| patterns, s = fp32(amax / 448), each code RNE(fp32(v / s)) by the
-// same correctly rounded division; codes of the CTA's k-blocks [st0 * KBS,
-// st1 * KBS) go to its token tiles sX (tile kb: BNT rows of 128 bytes, 16-byte
-// piece p of row r at p ^ (r & 7)), bytes past K as zeros. Warp w of the four
-// takes tokens w, w + 4, ...; CTAs of column tile 0 also write x8 and (rank
-// 0) s_tok.
-struct DecodeFQ;
-template <int BNT, int KBS>
-__device__ __forceinline__ void decode_fused_quant(const DecodeFQ& fq, int M, int K, int st0, int st1,
-                                                   int tile_n, int rank, uint8_t* sX, float* stok_s,
-                                                   int w, int lane);
-
-// Arguments of the decode GEMM's fused-quantization mode (FQ): the bf16
-// activations x [M, K] (pitch K) are quantized per token inside the GEMM,
-// bit for bit as fp8_quant_act does it, and the codes and scales are also
-// written to x8 / s_tok (by the CTAs of column tile 0).
-struct DecodeFQ {
-  const uint16_t* x;
-  uint8_t* x8;
-  float* s_tok;
-};
-
-template <int BNT, int KBS>
-__device__ __forceinline__ void decode_fused_quant(const DecodeFQ& fq, int M, int K, int st0, int st1,
-                                                   int tile_n, int rank, uint8_t* sX, float* stok_s,
-                                                   int w, int lane) {
-  constexpr int kXBytes = BNT * kBK;
-  const int64_t nvec = K / 8;                       // 16-byte vectors of 8 bf16 per row
-  const int kb0 = st0 * KBS, nkb = (st1 - st0) * KBS;
-  const int v0 = kb0 * (kBK / 8), v1 = v0 + nkb * (kBK / 8);  // the CTA's vectors (may pass K)
-  for (int m = w; m < M; m += 4) {
-    const uint4* row = reinterpret_cast<const uint4*>(fq.x + static_cast<int64_t>(m) * K);
-    uint32_t mx = 0;
-    for (int64_t j = lane; j < nvec; j += 32) {
-      const uint4 u = __ldg(row + j);
-      mx = __vmaxu2(mx, u.x & 0x7FFF7FFFu);
-      mx = __vmaxu2(mx, u.y & 0x7FFF7FFFu);
-      mx = __vmaxu2(mx, u.z & 0x7FFF7FFFu);
-      mx = __vmaxu2(mx, u.w & 0x7FFF7FFFu);
-    }
-    mx = max(mx & 0xFFFFu, mx >> 16);
-    const uint32_t amax_bits = __reduce_max_sync(0xFFFFFFFFu, mx);
-    if (amax_bits >= 0x7F80u && lane == 0 && tile_n == 0 && rank == 0) report(FP8_DEV_NONFINITE);
-    const float amax = __uint_as_float(amax_bits << 16);
-    const float s = __fdiv_rn(amax, kE4M3Max);
-    if (lane == 0) {
-      stok_s[m] = s;
-      if (tile_n == 0 && rank == 0) fq.s_tok[m] = s;
-    }
-    const RowDivisor dv = make_divisor(s, amax);
-    for (int v = v0 + lane; v < v1; v += 32) {
-      uint2 codes = make_uint2(0u, 0u);
-      if (v < nvec && s != 0.0f) {
-        const uint4 u = __ldg(row + v);
-        const uint32_t wv[4] = {u.x, u.y, u.z, u.w};
-        float f[8];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          f[2 * i] = div_rn(dv, __uint_as_float(wv[i] << 16));
-          f[2 * i + 1] = div_rn(dv, __uint_as_float(wv[i] & 0xFFFF0000u));
-        }
-        codes = make_uint2(pack4_e4m3(f[0], f[1], f[2], f[3]), pack4_e4m3(f[4], f[5], f[6], f[7]));
-      }
-      const int off = (v - v0) * 8;  // byte offset of the vector within the CTA's k-blocks
-      const int kb = off / kBK, ob = off % kBK;
-      uint8_t* dst = sX + kb * kXBytes + m * kBK + ((((ob >> 4) ^ (m & 7))) << 4) + (ob & 15);
-      *reinterpret_cast<uint2*>(dst) = codes;
-      if (tile_n == 0 && v < nvec)
-        *reinterpret_cast<uint2*>(fq.x8 + static_cast<int64_t>(m) * K + static_cast<int64_t>(v) * 8) = codes;
-    }
-  }
-}
-
-// FQ: every CTA computes each token's scale from the whole row (the amax is
-// over all of K) and the codes of its own K range only, straight into its
-// token tiles in shared memory (the 128-byte swizzled layout the MMA reads);
-// this needs the CTA's K range to fit its token-tile ring (STAGES * KBS
-// k-blocks). The producer then streams weights only; the four epilogue warps,
-// idle during the main loop, do the quantization (warp w takes tokens w,
-// w + 4, ...) and release the tiles to the MMA thread with one barrier.
-template <int BNT, int STAGES, int KBS, int KD = kKindE4M3, bool FQ = false>
+template <int BNT, int STAGES, int KBS, int KD = kKindE4M3>
 __global__ void __launch_bounds__(192)
     gemm_decode_kernel(const __grid_constant__ CUtensorMap tmW,
                        const __grid_constant__ CUtensorMap tmX,
                        const __grid_constant__ CUtensorMap tmY, const float* __restrict__ s_tok,
                        const float* __restrict__ s_ch, uint16_t* __restrict__ y, int M, int N,
-                       int K, int splits, int kb_per_split, int use_tma_store, const DecodeFQ fq) {
+                       int K, int splits, int kb_per_split, int use_tma_store) {
   using C = DecodeCfg<BNT, STAGES, KBS>;
-  static_assert(!FQ || KD == kKindE4M3, "fused quantization produces E4M3 codes");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
   uint8_t* sW = smem;                                   // STAGES x KBS weight boxes
   uint8_t* sX = smem + STAGES * KBS * C::kWBytes;       // STAGES x KBS token boxes
   uint16_t* ytile = reinterpret_cast<uint16_t*>(smem);  // after the MMAs: bf16 [token][row]
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kPipeBytes);
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 2);
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 1);
   float* sch_s = reinterpret_cast<float*>(smem + C::kPipeBytes + C::kBarBytes);
   float* stok_s = sch_s + kBM;
   float* red = reinterpret_cast<float*>(smem + C::kFixed);  // split only
   const uint32_t full0 = smem_u32(bars);
   const uint32_t empty0 = smem_u32(bars + STAGES);
   const uint32_t tfull = smem_u32(bars + 2 * STAGES);
-  const uint32_t xfull = smem_u32(bars + 2 * STAGES + 1);  // FQ: the token tiles are written
   // Abort word shared by the producer and MMA roles (mbar_wait_ab): the
   // first whose wait runs out makes the other leave at once.
   const uint32_t abort_w = smem_u32(tmem_holder + 1);
-  // FQ: a stage's transaction bytes are its weight boxes only.
-  constexpr uint32_t kStageTx = FQ ? KBS * C::kWBytes : C::kStageBytes;
 
   const int warp = warp_id(), lane = lane_id();
   const int tile_n = blockIdx.x / splits;
@@ -1028,17 +941,16 @@ __global__ void __launch_bounds__(192)
       mbar_init(empty0 + 8 * s, 1);
     }
     mbar_init(tfull, 1);
-    mbar_init(xfull, 1);
     fence_barrier_init();
     tma_prefetch_desc(&tmW);
-    if (!FQ) tma_prefetch_desc(&tmX);
+    tma_prefetch_desc(&tmX);
     // The weight stream depends neither on the TMEM allocation nor on a
     // preceding quantizer grid: start the first ring of weight boxes now.
     const uint64_t pol_w = l2_policy_evict_first();
     for (int i = 0; i < pre; ++i) {
       if (i == drop) continue;
       const uint32_t fb = full0 + 8 * i;
-      mbar_arrive_expect_tx(fb, kStageTx);
+      mbar_arrive_expect_tx(fb, C::kStageBytes);
       armed |= 1u << i;
 #pragma unroll
       for (int j = 0; j < KBS; ++j)
@@ -1065,15 +977,13 @@ __global__ void __launch_bounds__(192)
     if (lane == 0 && have_acc) {
       const uint64_t pol_w = l2_policy_evict_first();
       const uint64_t pol_x = l2_policy_evict_last();
-      if (!FQ) {
-        pdl_wait();  // activations come from a preceding quantizer grid
-        for (int i = 0; i < pre; ++i) {
-          if (i == drop) continue;
+      pdl_wait();  // activations come from a preceding quantizer grid
+      for (int i = 0; i < pre; ++i) {
+        if (i == drop) continue;
 #pragma unroll
-          for (int j = 0; j < KBS; ++j)
-            tma_load_2d(smem_u32(sX + (i * KBS + j) * C::kXBytes), &tmX, full0 + 8 * i,
-                        ((st0 + i) * KBS + j) * kBK, 0, pol_x);
-        }
+        for (int j = 0; j < KBS; ++j)
+          tma_load_2d(smem_u32(sX + (i * KBS + j) * C::kXBytes), &tmX, full0 + 8 * i,
+                      ((st0 + i) * KBS + j) * kBK, 0, pol_x);
       }
       int stage = pre % STAGES;
       uint32_t phase = pre == STAGES ? 1u : 0u;
@@ -1081,16 +991,15 @@ __global__ void __launch_bounds__(192)
         if (!mbar_wait_ab(empty0 + 8 * stage, phase ^ 1, abort_w)) break;
         if (st - st0 != drop) {
           const uint32_t fb = full0 + 8 * stage;
-          mbar_arrive_expect_tx(fb, kStageTx);
+          mbar_arrive_expect_tx(fb, C::kStageBytes);
           armed |= 1u << stage;
           armed_par = (armed_par & ~(1u << stage)) | (phase << stage);
 #pragma unroll
           for (int j = 0; j < KBS; ++j) {
             tma_load_2d(smem_u32(sW + (stage * KBS + j) * C::kWBytes), &tmW, fb, (st * KBS + j) * kBK,
                         tile_n * kBM, pol_w);
-            if (!FQ)
-              tma_load_2d(smem_u32(sX + (stage * KBS + j) * C::kXBytes), &tmX, fb,
-                          (st * KBS + j) * kBK, 0, pol_x);
+            tma_load_2d(smem_u32(sX + (stage * KBS + j) * C::kXBytes), &tmX, fb, (st * KBS + j) * kBK,
+                        0, pol_x);
           }
         }
         if (++stage == STAGES) { stage = 0; phase ^= 1; }
@@ -1107,17 +1016,13 @@ __global__ void __launch_bounds__(192)
       constexpr uint32_t idesc = idesc_kind<KD>(kBM, BNT);
       int stage = 0;
       uint32_t phase = 0;
-      // FQ: the token tiles of the whole K range, written by the epilogue warps
-      const bool x_ok = !FQ || mbar_wait_ab(xfull, 0, abort_w);
-      for (int st = st0; x_ok && st < st1; ++st) {
+      for (int st = st0; st < st1; ++st) {
         if (!mbar_wait_ab(full0 + 8 * stage, phase, abort_w)) break;
         tc_fence_after();
 #pragma unroll
         for (int j = 0; j < KBS; ++j) {
           const uint32_t a0 = smem_u32(sW + (stage * KBS + j) * C::kWBytes);
-          // FQ: the range's token tiles sit in order, one per k-block
-          const uint32_t b0 =
-              smem_u32(sX + ((FQ ? st - st0 : stage) * KBS + j) * C::kXBytes);
+          const uint32_t b0 = smem_u32(sX + (stage * KBS + j) * C::kXBytes);
 #pragma unroll
           for (int k = 0; k < kBK / 32; ++k) {
             umma_kind<KD>(tmem_base, sw128_kmajor_desc(a0 + 32 * k), sw128_kmajor_desc(b0 + 32 * k),
@@ -1140,19 +1045,9 @@ __global__ void __launch_bounds__(192)
     {
       const int n = tile_n * kBM + et;
       sch_s[et] = n < N ? (s_ch ? __ldg(s_ch + n) : 1.0f) : 0.0f;
-      pdl_wait();  // x, or the per-token scales, come from the preceding grid
-      if constexpr (FQ) {
-        if (et < BNT) stok_s[et] = 0.0f;  // tokens past M
-        named_bar_sync(1, 128);
-        if (have_acc) decode_fused_quant<BNT, KBS>(fq, M, K, st0, st1, tile_n, rank, sX, stok_s,
-                                                   quad, lane);
-        fence_proxy_async_shared();  // the generic writes of the tiles -> visible to the MMA
-        named_bar_sync(1, 128);
-        if (et == 0) mbar_arrive(xfull);
-      } else {
-        if (et < BNT) stok_s[et] = et < M ? (s_tok ? s_tok[et] : 1.0f) : 0.0f;
-        named_bar_sync(1, 128);
-      }
+      pdl_wait();  // per-token scales come from a preceding quantizer grid
+      if (et < BNT) stok_s[et] = et < M ? (s_tok ? s_tok[et] : 1.0f) : 0.0f;
+      named_bar_sync(1, 128);
     }
     if (have_acc && !mbar_wait(tfull, 0)) have_acc = false;
     __syncwarp();
