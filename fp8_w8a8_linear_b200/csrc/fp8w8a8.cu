@@ -80,12 +80,11 @@ bool make_tmap_u8(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols
 // not written. Requires cols % 8 == 0 (16-byte pitch).
 bool make_tmap_bf16_store(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols,
                           uint32_t box_cols, uint32_t box_rows,
-                          CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_NONE,
-                          uint64_t pitch = 0) {
+                          CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_NONE) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
   cuuint64_t dims[2] = {cols, rows};
-  cuuint64_t strides[1] = {(pitch ? pitch : cols) * 2};
+  cuuint64_t strides[1] = {cols * 2};
   cuuint32_t box[2] = {box_cols, box_rows};
   cuuint32_t estr[2] = {1, 1};
   std::memset(m, 0, sizeof(*m));
@@ -343,11 +342,6 @@ fp8_status launch_prefill(const DeviceInfo& dev, const uint8_t* x8, const float*
   return FP8_OK;
 }
 
-template <int BNT, int ST, int KBS, int KD>
-fp8_status launch_decode_t(const DeviceInfo& dev, const uint8_t* x8, const float* s_tok,
-                           const uint8_t* w8, const float* s_ch, int M, int N, int K, uint16_t* y,
-                           cudaStream_t stream, bool pdl, int force_splits, int ldy);
-
 // Dense GEMM on 256 x 256 tiles per CTA pair (clusters of 2, persistent).
 template <int KD = kKindE4M3>
 fp8_status launch_pair(const DeviceInfo& dev, const uint8_t* x8, const float* s_tok,
@@ -388,34 +382,12 @@ fp8_status launch_pair(const DeviceInfo& dev, const uint8_t* x8, const float* s_
   // (measured on B200 at M = 65536, K = 5376, N = 21504: 8 -> 16 pairs,
   // 6.4 -> 5.7 ms per GEMM under the power cap; 32 pairs: 5.8 ms).
   g.group_m = std::min(tiles_m, 16);
-  // A last, partial wave of at most a quarter of the pairs would leave the
-  // others idle for a whole tile time. Those tiles are the last ones of the
-  // raster - the trailing row tiles of the last column tile, a rectangle when
-  // they are no more than the last group's rows - and go to the decode
-  // kernel instead, as token blocks of 128 rows with K split over clusters
-  // (partials summed in rank order through distributed shared memory, so
-  // still deterministic), launched after this grid.
-  const int rem = num_tiles > pairs ? num_tiles % pairs : 0;
-  const int first_m_last = (tiles_m - 1) / g.group_m * g.group_m;
-  const int gm_last = tiles_m - first_m_last;
-  const bool tail = rem > 0 && 4 * rem <= pairs && rem <= gm_last && N % 8 == 0;
-  g.tile_end = tail ? num_tiles - rem : 0;
   CUtensorMap tmY;
   make_epilogue_store_map(&tmY, g, y, M, N);
   if (cudaLaunchKernelEx(&cfg, gemm_pair_kernel<kPairStages, false, false, KD>, tmA, tmB, tmB, tmY,
                          g) != cudaSuccess)
     return FP8_ERR_CUDA;
-  if (!tail) return FP8_OK;
-  const int row0 = (first_m_last + gm_last - rem) * 256;
-  const int col0 = (tiles_n - 1) * 256;
-  const int Mt = M - row0, Nt = N - col0;
-  const int blocks = (Mt + 127) / 128, ctiles = (Nt + kBM - 1) / kBM;
-  const int steps = (K + kBK - 1) / kBK;
-  int splits = 1;
-  while (splits < 8 && ctiles * blocks * splits * 2 <= dev.sm_count && splits * 8 <= steps) splits *= 2;
-  return launch_decode_t<128, 3, 1, KD>(dev, x8 + static_cast<int64_t>(row0) * K, s_tok ? s_tok + row0 : nullptr,
-                                        w8 + static_cast<int64_t>(col0) * K, s_ch ? s_ch + col0 : nullptr, Mt, Nt,
-                                        K, y + static_cast<int64_t>(row0) * N + col0, stream, true, splits, N);
+  return FP8_OK;
 }
 
 // Per-expert GEMM: persistent grid, tiles decoded on the GPU from offsets.
@@ -552,13 +524,10 @@ int decode_splits(const DeviceInfo& dev, int N, int K, int kbs) {
   return splits;
 }
 
-// M may exceed BNT (blocks of BNT tokens on the grid's y dimension); y has
-// row pitch ldy (0: N).
-template <int BNT, int ST, int KBS, int KD>
+template <int BNT, int ST, int KBS, int KD = kKindE4M3>
 fp8_status launch_decode_t(const DeviceInfo& dev, const uint8_t* x8, const float* s_tok,
                            const uint8_t* w8, const float* s_ch, int M, int N, int K, uint16_t* y,
-                           cudaStream_t stream, bool pdl, int force_splits, int ldy) {
-  if (ldy == 0) ldy = N;
+                           cudaStream_t stream, bool pdl, int force_splits = 0) {
   using C = DecodeCfg<BNT, ST, KBS>;
   CUtensorMap tmW, tmX;
   if (!make_tmap_u8(&tmW, w8, N, K, kBM) || !make_tmap_u8(&tmX, x8, M, K, BNT))
@@ -572,13 +541,9 @@ fp8_status launch_decode_t(const DeviceInfo& dev, const uint8_t* x8, const float
   CUtensorMap tmY;
   std::memset(&tmY, 0, sizeof(tmY));
   const int use_tma_store =
-      (N % 8 == 0) && (ldy % 8 == 0) &&
-              (reinterpret_cast<uintptr_t>(y) & 15) == 0 &&
-              make_tmap_bf16_store(&tmY, y, M, N, kBM / splits, BNT, CU_TENSOR_MAP_SWIZZLE_NONE, ldy)
-          ? 1
-          : 0;
+      (N % 8 == 0) && make_tmap_bf16_store(&tmY, y, M, N, kBM / splits, BNT) ? 1 : 0;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(tiles * splits, (M + BNT - 1) / BNT);
+  cfg.gridDim = dim3(tiles * splits);
   cfg.blockDim = dim3(192);
   cfg.dynamicSmemBytes = splits > 1 ? C::kSmemSplit : C::kSmemSingle;
   cfg.stream = stream;
@@ -593,7 +558,7 @@ fp8_status launch_decode_t(const DeviceInfo& dev, const uint8_t* x8, const float
   cfg.attrs = attrs;
   cfg.numAttrs = na;
   if (cudaLaunchKernelEx(&cfg, gemm_decode_kernel<BNT, ST, KBS, KD>, tmW, tmX, tmY, s_tok, s_ch, y, M,
-                         N, K, splits, steps_per_split, use_tma_store, ldy) != cudaSuccess)
+                         N, K, splits, steps_per_split, use_tma_store) != cudaSuccess)
     return FP8_ERR_CUDA;
   return FP8_OK;
 }
@@ -619,22 +584,22 @@ fp8_status launch_linear(const DeviceInfo& dev, const uint8_t* x8, const float* 
     const int num_kb = (K + kBK - 1) / kBK;
     int s = 1;
     while (s < 8 && tiles * s * 2 <= 2 * dev.sm_count && s * 2 * 4 <= num_kb) s *= 2;
-    if (s >= 4) return launch_decode_t<16, 2, 2, KD>(dev, x8, s_tok, w8, s_ch, M, N, K, y, stream, pdl, s, 0);
+    if (s >= 4) return launch_decode_t<16, 2, 2, KD>(dev, x8, s_tok, w8, s_ch, M, N, K, y, stream, pdl, s);
     return one_per_sm && no_split
-               ? launch_decode_t<16, 6, 2, KD>(dev, x8, s_tok, w8, s_ch, M, N, K, y, stream, pdl, 0, 0)
-               : launch_decode_t<16, 3, 2, KD>(dev, x8, s_tok, w8, s_ch, M, N, K, y, stream, pdl, 0, 0);
+               ? launch_decode_t<16, 6, 2, KD>(dev, x8, s_tok, w8, s_ch, M, N, K, y, stream, pdl)
+               : launch_decode_t<16, 3, 2, KD>(dev, x8, s_tok, w8, s_ch, M, N, K, y, stream, pdl);
   }
   if (M <= 32)
-    return one_per_sm ? launch_decode_t<32, 3, 2, KD>(dev, x8, s_tok, w8, s_ch, M, N, K, y, stream, pdl, 0, 0)
-                      : launch_decode_t<32, 4, 1, KD>(dev, x8, s_tok, w8, s_ch, M, N, K, y, stream, pdl, 0, 0);
+    return one_per_sm ? launch_decode_t<32, 3, 2, KD>(dev, x8, s_tok, w8, s_ch, M, N, K, y, stream, pdl)
+                      : launch_decode_t<32, 4, 1, KD>(dev, x8, s_tok, w8, s_ch, M, N, K, y, stream, pdl);
   if (M <= 64)
-    return one_per_sm ? launch_decode_t<64, 4, 2, KD>(dev, x8, s_tok, w8, s_ch, M, N, K, y, stream, pdl, 0, 0)
-                      : launch_decode_t<64, 4, 1, KD>(dev, x8, s_tok, w8, s_ch, M, N, K, y, stream, pdl, 0, 0);
+    return one_per_sm ? launch_decode_t<64, 4, 2, KD>(dev, x8, s_tok, w8, s_ch, M, N, K, y, stream, pdl)
+                      : launch_decode_t<64, 4, 1, KD>(dev, x8, s_tok, w8, s_ch, M, N, K, y, stream, pdl);
   if (M <= 128) {
     if (!one_per_sm)
-      return launch_decode_t<128, 3, 1, KD>(dev, x8, s_tok, w8, s_ch, M, N, K, y, stream, pdl, 0, 0);
-    return no_split ? launch_decode_t<128, 6, 1, KD>(dev, x8, s_tok, w8, s_ch, M, N, K, y, stream, pdl, 0, 0)
-                    : launch_decode_t<128, 4, 1, KD>(dev, x8, s_tok, w8, s_ch, M, N, K, y, stream, pdl, 0, 0);
+      return launch_decode_t<128, 3, 1, KD>(dev, x8, s_tok, w8, s_ch, M, N, K, y, stream, pdl);
+    return no_split ? launch_decode_t<128, 6, 1, KD>(dev, x8, s_tok, w8, s_ch, M, N, K, y, stream, pdl)
+                    : launch_decode_t<128, 4, 1, KD>(dev, x8, s_tok, w8, s_ch, M, N, K, y, stream, pdl);
   }
   // Prefill: 256 x 256 tiles on CTA pairs or 128 x 256 tiles on single SMs
   // (the same work per SM per tile). Pairs move a third less operand traffic

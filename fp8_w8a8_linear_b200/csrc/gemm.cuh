@@ -278,7 +278,6 @@ struct GemmArgs {
   int num_experts;     // grouped only
   int use_tma_store;   // tmY is a 32 x 32 bf16 store map over y (64-byte swizzle)
   int n_out;           // GeGLU epilogue only: columns of h (the features)
-  int tile_end;        // dense pair GEMM: tiles >= tile_end are left to another launch (0: none)
 };
 
 struct Tile {
@@ -641,8 +640,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
   const uint32_t tmem_base = *tmem_holder;
   // tiles of 256 x 256; the fields of a Tile here are the pair's (row 0 of
   // the tile, column 0), each CTA adding rank * 128 to its A and B rows
-  const int num_tiles = GROUPED ? mt_off[g.num_experts] * g.tiles_n
-                                : (g.tile_end > 0 ? g.tile_end : g.tiles_m * g.tiles_n);
+  const int num_tiles = GROUPED ? mt_off[g.num_experts] * g.tiles_n : g.tiles_m * g.tiles_n;
   // GeGLU: the last feature tile holds at most 64 features (tiles are
   // numbered m-tile major, so tile % tiles_n is the feature tile)
   auto half_width = [&](int t) { return GEGLU && g.n_out - 128 * (t % g.tiles_n) <= 64; };
@@ -877,12 +875,7 @@ struct DecodeCfg {
   static constexpr int kWBytes = kBM * kBK;   // one weight box: 128 channels x 128 K bytes
   static constexpr int kXBytes = BNT * kBK;   // one token box
   static constexpr int kStageBytes = KBS * (kWBytes + kXBytes);
-  // Independent accumulators the k-steps rotate over when the token tile is
-  // narrow (each MMA is then short, and consecutive MMAs into one
-  // accumulator wait for each other); the epilogue sums them in a fixed
-  // order, so results stay bit-reproducible.
-  static constexpr int kNAcc = BNT <= 32 ? 4 : 1;
-  static constexpr int kTmemCols = tmem_cols_for(kNAcc * BNT);
+  static constexpr int kTmemCols = tmem_cols_for(BNT);
   static constexpr int kPipeBytes = STAGES * kStageBytes;
   static constexpr int kYBytes = BNT * kBM * 2;    // bf16 output tile, reuses the pipeline
   static constexpr int kBarBytes = 8 * (2 * STAGES + 1) + 16;
@@ -905,7 +898,7 @@ __global__ void __launch_bounds__(192)
                        const __grid_constant__ CUtensorMap tmX,
                        const __grid_constant__ CUtensorMap tmY, const float* __restrict__ s_tok,
                        const float* __restrict__ s_ch, uint16_t* __restrict__ y, int M, int N,
-                       int K, int splits, int kb_per_split, int use_tma_store, int ldy) {
+                       int K, int splits, int kb_per_split, int use_tma_store) {
   using C = DecodeCfg<BNT, STAGES, KBS>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
@@ -925,11 +918,6 @@ __global__ void __launch_bounds__(192)
   const uint32_t abort_w = smem_u32(tmem_holder + 1);
 
   const int warp = warp_id(), lane = lane_id();
-  // Token block blockIdx.y: rows m0 .. m0 + Mb - 1 of x and y (one block for
-  // decode batches; several when the kernel computes a prefill GEMM's last,
-  // partial wave of tiles).
-  const int m0 = blockIdx.y * BNT;
-  const int Mb = min(BNT, M - m0);
   const int tile_n = blockIdx.x / splits;
   const int rank = blockIdx.x % splits;  // == %cluster_ctarank for cluster dims (splits,1,1)
   const int num_kb = (K + kBK - 1) / kBK;
@@ -943,8 +931,7 @@ __global__ void __launch_bounds__(192)
 
   if (split) cluster_arrive_relaxed();  // this CTA has started (waited on before any DSMEM store)
   // Test hook: CTA 0 skips one pipeline step's stage (no arrive, no loads).
-  const int drop =
-      (blockIdx.x == 0 && blockIdx.y == 0) ? *const_cast<volatile int*>(&g_fault_drop_step) : -1;
+  const int drop = blockIdx.x == 0 ? *const_cast<volatile int*>(&g_fault_drop_step) : -1;
   // The stages the producer armed and the phase parity each last arm fills.
   uint32_t armed = 0u, armed_par = 0u;
   if (warp == 0 && lane == 0) {
@@ -996,7 +983,7 @@ __global__ void __launch_bounds__(192)
 #pragma unroll
         for (int j = 0; j < KBS; ++j)
           tma_load_2d(smem_u32(sX + (i * KBS + j) * C::kXBytes), &tmX, full0 + 8 * i,
-                      ((st0 + i) * KBS + j) * kBK, m0, pol_x);
+                      ((st0 + i) * KBS + j) * kBK, 0, pol_x);
       }
       int stage = pre % STAGES;
       uint32_t phase = pre == STAGES ? 1u : 0u;
@@ -1012,7 +999,7 @@ __global__ void __launch_bounds__(192)
             tma_load_2d(smem_u32(sW + (stage * KBS + j) * C::kWBytes), &tmW, fb, (st * KBS + j) * kBK,
                         tile_n * kBM, pol_w);
             tma_load_2d(smem_u32(sX + (stage * KBS + j) * C::kXBytes), &tmX, fb, (st * KBS + j) * kBK,
-                        m0, pol_x);
+                        0, pol_x);
           }
         }
         if (++stage == STAGES) { stage = 0; phase ^= 1; }
@@ -1038,9 +1025,8 @@ __global__ void __launch_bounds__(192)
           const uint32_t b0 = smem_u32(sX + (stage * KBS + j) * C::kXBytes);
 #pragma unroll
           for (int k = 0; k < kBK / 32; ++k) {
-            const int kk = ((st - st0) * KBS + j) * (kBK / 32) + k;  // this CTA's k-step
-            umma_kind<KD>(tmem_base + (kk % C::kNAcc) * BNT, sw128_kmajor_desc(a0 + 32 * k),
-                          sw128_kmajor_desc(b0 + 32 * k), idesc, kk >= C::kNAcc);
+            umma_kind<KD>(tmem_base, sw128_kmajor_desc(a0 + 32 * k), sw128_kmajor_desc(b0 + 32 * k),
+                          idesc, (st != st0) || (j != 0) || (k != 0));
           }
         }
         umma_commit(empty0 + 8 * stage);
@@ -1060,7 +1046,7 @@ __global__ void __launch_bounds__(192)
       const int n = tile_n * kBM + et;
       sch_s[et] = n < N ? (s_ch ? __ldg(s_ch + n) : 1.0f) : 0.0f;
       pdl_wait();  // per-token scales come from a preceding quantizer grid
-      if (et < BNT) stok_s[et] = et < Mb ? (s_tok ? s_tok[m0 + et] : 1.0f) : 0.0f;
+      if (et < BNT) stok_s[et] = et < M ? (s_tok ? s_tok[et] : 1.0f) : 0.0f;
       named_bar_sync(1, 128);
     }
     if (have_acc && !mbar_wait(tfull, 0)) have_acc = false;
@@ -1079,22 +1065,6 @@ __global__ void __launch_bounds__(192)
       uint32_t r[16];
       tmem_ld16(t_row + c * 16, r);
       tmem_ld_wait();
-      // the other accumulators, added in order (int32 for kind::i8: exact;
-      // an accumulator that no k-step reached holds no value and is skipped)
-#pragma unroll 1
-      for (int a = 1; a < C::kNAcc; ++a) {
-        if (a >= (st1 - st0) * KBS * (kBK / 32)) break;
-        uint32_t r2[16];
-        tmem_ld16(t_row + a * BNT + c * 16, r2);
-        tmem_ld_wait();
-#pragma unroll
-        for (int jj = 0; jj < 16; ++jj) {
-          if constexpr (KD == kKindS8)
-            r[jj] = static_cast<uint32_t>(static_cast<int>(r[jj]) + static_cast<int>(r2[jj]));
-          else
-            r[jj] = __float_as_uint(__fadd_rn(__uint_as_float(r[jj]), __uint_as_float(r2[jj])));
-        }
-      }
       // split partials travel as raw accumulator words (int32 for kind::i8,
       // summed exactly by the owner); a single CTA converts them here
       if (!split) acc_to_f32<KD>(r);
@@ -1105,7 +1075,7 @@ __global__ void __launch_bounds__(192)
         if (!split) {
           ytile[tok * kBM + ch] =
               f32_to_bf16_rn(__fmul_rn(__fmul_rn(__uint_as_float(word), stok_s[tok]), sc));
-        } else if (tok < Mb) {
+        } else if (tok < M) {
           // owner's buffer [rank][token][row in slice]: lanes write consecutive words
           st_shared_cluster_f32(dst + static_cast<uint32_t>(tok * rows * 4), __uint_as_float(word));
         }
@@ -1150,7 +1120,7 @@ __global__ void __launch_bounds__(192)
       fence_proxy_async_shared();  // generic writes of the tile -> visible to the TMA store
       named_bar_sync(1, 128);
       if (threadIdx.x == 64) {
-        tma_store_2d(&tmY, smem_u32(ytile), n0, m0);
+        tma_store_2d(&tmY, smem_u32(ytile), n0, 0);
         bulk_commit_group();
         bulk_wait_group_all();
       }
@@ -1160,8 +1130,7 @@ __global__ void __launch_bounds__(192)
     const int et = threadIdx.x - 64;
     for (int e = et; e < rows_out * BNT; e += 128) {
       const int tok = e / rows_out, rl = e % rows_out;
-      if (tok < Mb && n0 + rl < N)
-        y[static_cast<int64_t>(m0 + tok) * ldy + n0 + rl] = ytile[tok * rows_out + rl];
+      if (tok < M && n0 + rl < N) y[static_cast<int64_t>(tok) * N + n0 + rl] = ytile[tok * rows_out + rl];
     }
   }
 }
