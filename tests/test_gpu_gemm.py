@@ -68,8 +68,7 @@ GEMM_SHAPES = [
     (600, 768, 224),
     (129, 256, 160),
     (1024, 2048, 4160),
-    # more pair tiles than pairs, with a last partial wave of at most a quarter
-    # of them: that wave runs as token blocks on the split-K decode kernel
+    # more pair tiles than pairs, with a last partial wave of a few tiles
     (2048, 2560, 1024),
     (2000, 2504, 1040),
 ]

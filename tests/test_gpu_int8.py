@@ -72,7 +72,7 @@ INT8_GEMM_SHAPES = [
     (600, 1003, 4096), (700, 2056, 4096), (300, 520, 704), (1000, 1024, 416),
     (1, 8192, 2048), (8, 8192, 2048), (64, 8192, 2048),
     (1, 256, 65536), (16, 256, 65536), (300, 256, 65536),
-    (2048, 2560, 1024), (2000, 2504, 1040),   # a last partial wave on the decode kernel
+    (2048, 2560, 1024), (2000, 2504, 1040),   # more pair tiles than pairs, ragged
 ]
 
 
