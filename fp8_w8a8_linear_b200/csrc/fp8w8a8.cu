@@ -191,7 +191,7 @@ fp8_status set_decode_attrs(int so) {
   st = st != FP8_OK ? st : set_decode_attr<64, 4, 2, KD>(so);
   st = st != FP8_OK ? st : set_decode_attr<128, 3, 1, KD>(so);
   st = st != FP8_OK ? st : set_decode_attr<128, 4, 1, KD>(so);
-  st = st != FP8_OK ? st : set_decode_attr<128, 6, 1, KD>(so);
+  st = st != FP8_OK ? st : set_decode_attr<128, 3, 2, KD>(so);
   return st;
 }
 
@@ -596,9 +596,13 @@ fp8_status launch_linear(const DeviceInfo& dev, const uint8_t* x8, const float* 
     return one_per_sm ? launch_decode_t<64, 4, 2, KD>(dev, x8, s_tok, w8, s_ch, M, N, K, y, stream, pdl)
                       : launch_decode_t<64, 4, 1, KD>(dev, x8, s_tok, w8, s_ch, M, N, K, y, stream, pdl);
   if (M <= 128) {
+    // One CTA per SM with no split: two 128-byte k-blocks per stage, so each
+    // weight row is read 256 contiguous bytes at a time (measured on B200 at
+    // 14336 x 4096, M = 128: 19.8 -> 19.3 us per linear against one k-block
+    // per stage in a ring of the same size).
     if (!one_per_sm)
       return launch_decode_t<128, 3, 1, KD>(dev, x8, s_tok, w8, s_ch, M, N, K, y, stream, pdl);
-    return no_split ? launch_decode_t<128, 6, 1, KD>(dev, x8, s_tok, w8, s_ch, M, N, K, y, stream, pdl)
+    return no_split ? launch_decode_t<128, 3, 2, KD>(dev, x8, s_tok, w8, s_ch, M, N, K, y, stream, pdl)
                     : launch_decode_t<128, 4, 1, KD>(dev, x8, s_tok, w8, s_ch, M, N, K, y, stream, pdl);
   }
   // Prefill: 256 x 256 tiles on CTA pairs or 128 x 256 tiles on single SMs
