@@ -217,6 +217,9 @@ def setup_dense(torch, f, wl, seed, dev, flushable):
     ncopies = max(2, -(-int(2.5 * 126e6) // (N * K)))
     wcopies = [wsrc[0]] + [wsrc[0].clone() for _ in range(ncopies - 1)]
 
+    # the GEMM workspace that lets a partial last wave of pair tiles be split
+    # by k-blocks (zero-filled once; every call leaves its flags zero)
+    gws = f.linear_workspace(dev)
     L = []  # (name, fn(rotation), flops, bytes, bound, flushed_before, launches)
     if wl["repack"]:
         L.append(("repack_qat", lambda i: f.repack_qat(D["q4"], D["d"], w8, s_ch), 0.0,
@@ -232,7 +235,7 @@ def setup_dense(torch, f, wl, seed, dev, flushable):
             L.append((f"quant_act[M={M}]", lambda i, x=D[f"x{M}"], x8=x8, st=st: f.quant_act(x, x8, st),
                       0.0, qb, "hbm", False, 1))
             L.append((f"gemm_prefill[M={M}]",
-                      lambda i, x8=x8, st=st, y=y: f.rowwise_linear(x8, st, wsrc[0], wsrc[1], y),
+                      lambda i, x8=x8, st=st, y=y: f.rowwise_linear_ws(x8, st, wsrc[0], wsrc[1], gws, y),
                       fl, gb, "tensor", False, 1))
         else:
             L.append((f"linear_decode[M={M}]",

@@ -10,7 +10,8 @@ Functions mirror the C entry points:
 * :func:`repack_qat` - QAT q4_0 grid -> per-channel E4M3 weight + scales.
 * :func:`convert_fnuz` - E4M3FNUZ-stored weight -> E4M3 weight + scales.
 * :func:`quant_act` - per-token E4M3 activation quantization.
-* :func:`rowwise_linear` - ``y = (x8 . w8^T) * s_tok * s_ch`` in bf16.
+* :func:`rowwise_linear` - ``y = (x8 . w8^T) * s_tok * s_ch`` in bf16;
+  :func:`rowwise_linear_ws` with a workspace (:func:`linear_workspace`).
 * :func:`linear` - bf16 activations in, bf16 out (quantizer + GEMM).
 * :func:`linear_siblings` - several linears of the same x, quantized once.
 * :func:`cast_e4m3` - the element-wise encoder.
@@ -54,6 +55,8 @@ _SIGS = {
     "fp8_convert_fnuz": ([_P, _P, _I64, _I64, _P, _P, _P], ctypes.c_int),
     "fp8_quant_act": ([_P, _I64, _I64, _I64, _P, _P, _P], ctypes.c_int),
     "fp8_rowwise_linear": ([_P, _P, _P, _P, _I64, _I64, _I64, _P, _P], ctypes.c_int),
+    "fp8_linear_workspace_bytes": ([], ctypes.c_size_t),
+    "fp8_rowwise_linear_ws": ([_P, _P, _P, _P, _I64, _I64, _I64, _P, _P, ctypes.c_size_t, _P], ctypes.c_int),
     "fp8_linear_bf16": ([_P, _P, _P, _I64, _I64, _I64, _P, _P, _P, _P], ctypes.c_int),
     "fp8_cast_e4m3": ([_P, _I64, _P, _P], ctypes.c_int),
     "fp8_linear_bf16_siblings": ([_P, _I64, _I64, ctypes.c_int32, _P, _P, _P, _P, _P, _P, _P],
@@ -193,6 +196,29 @@ def rowwise_linear(x8: torch.Tensor, s_tok: torch.Tensor, w8: torch.Tensor, s_ch
                                    _dev(s_ch, torch.float32, "s_ch", (N,)), M, N, K,
                                    _dev(y, torch.bfloat16, "y", (M, N)), _stream()),
            "fp8_rowwise_linear")
+    return y
+
+
+def linear_workspace(device=None) -> torch.Tensor:
+    """A zero-filled workspace for rowwise_linear_ws on the current device
+    (uint8, fp8_linear_workspace_bytes() bytes; at least 16)."""
+    n = int(_lib.fp8_linear_workspace_bytes())
+    return torch.zeros(max(n, 16), dtype=torch.uint8, device=device or "cuda")
+
+
+def rowwise_linear_ws(x8: torch.Tensor, s_tok: torch.Tensor, w8: torch.Tensor, s_ch: torch.Tensor,
+                      ws: torch.Tensor, y: torch.Tensor | None = None):
+    """rowwise_linear with a workspace (from linear_workspace) that lets a
+    partial last wave of tiles be split by k-blocks over all SM pairs."""
+    M, K = x8.shape
+    N = w8.shape[0]
+    y = torch.empty((M, N), dtype=torch.bfloat16, device=x8.device) if y is None else y
+    _check(_lib.fp8_rowwise_linear_ws(_dev(x8, torch.uint8, "x8"), _dev(s_tok, torch.float32, "s_tok", (M,)),
+                                      _dev(w8, torch.uint8, "w8", (N, K)),
+                                      _dev(s_ch, torch.float32, "s_ch", (N,)), M, N, K,
+                                      _dev(y, torch.bfloat16, "y", (M, N)), _dev(ws, torch.uint8, "ws"),
+                                      ws.numel(), _stream()),
+           "fp8_rowwise_linear_ws")
     return y
 
 
@@ -484,7 +510,8 @@ def cast_e4m3(x: torch.Tensor, out: torch.Tensor | None = None):
 
 __all__ = [
     "Fp8Error", "raw", "version", "device_supported", "device_status", "repack_qat",
-    "convert_fnuz", "quant_act", "rowwise_linear", "linear", "linear_noalloc", "cast_e4m3",
+    "convert_fnuz", "quant_act", "rowwise_linear", "rowwise_linear_ws", "linear_workspace", "linear",
+    "linear_noalloc", "cast_e4m3",
     "linear_siblings", "test_set_fault",
     "moe_route", "moe_gather", "grouped_linear", "moe_geglu_quant", "moe_combine",
     "moe_interleave_gate_up", "grouped_linear_geglu",

@@ -160,6 +160,10 @@ template <int STAGES, int GSTAGES>
 fp8_status set_pair_attr() {
   return cudaFuncSetAttribute(gemm_pair_kernel<STAGES>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                               static_cast<int>(PairCfg<STAGES>::kSmem)) == cudaSuccess &&
+                 cudaFuncSetAttribute(gemm_pair_kernel<STAGES, false, false, kKindE4M3, true>,
+                                      cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      static_cast<int>(PairCfg<STAGES>::kSmem)) == cudaSuccess &&
+
                  cudaFuncSetAttribute(gemm_pair_kernel<STAGES, false, false, kKindS8>,
                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
                                       static_cast<int>(PairCfg<STAGES>::kSmem)) == cudaSuccess &&
@@ -346,7 +350,7 @@ fp8_status launch_prefill(const DeviceInfo& dev, const uint8_t* x8, const float*
 template <int KD = kKindE4M3>
 fp8_status launch_pair(const DeviceInfo& dev, const uint8_t* x8, const float* s_tok,
                        const uint8_t* w8, const float* s_ch, int M, int N, int K, uint16_t* y,
-                       cudaStream_t stream, bool pdl) {
+                       cudaStream_t stream, bool pdl, void* ws = nullptr, size_t ws_bytes = 0) {
   CUtensorMap tmA, tmB;
   if (!make_tmap_u8(&tmA, x8, M, K, 128) || !make_tmap_u8(&tmB, w8, N, K, 128)) return FP8_ERR_CUDA;
   const int tiles_m = (M + 255) / 256;
@@ -384,6 +388,22 @@ fp8_status launch_pair(const DeviceInfo& dev, const uint8_t* x8, const float* s_
   g.group_m = std::min(tiles_m, 16);
   CUtensorMap tmY;
   make_epilogue_store_map(&tmY, g, y, M, N);
+  // A partial last wave of tiles (fewer than 8 waves, so that it costs a
+  // noticeable share) is evened out by the k-block split when the caller
+  // gave a workspace: the last full wave and the partial one are shared
+  // out by k-blocks over all pairs.
+  if constexpr (KD == kKindE4M3) {
+    if (ws && ws_bytes >= split_ws_bytes(pairs) && num_tiles > pairs && num_tiles % pairs != 0 &&
+        num_tiles < 8 * pairs) {
+      g.sk_tiles = pairs + num_tiles % pairs;
+      g.ws_flag = static_cast<int*>(ws);
+      g.ws_part = reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(ws) + split_flag_bytes(pairs));
+      if (cudaLaunchKernelEx(&cfg, gemm_pair_kernel<kPairStages, false, false, KD, true>, tmA, tmB, tmB,
+                             tmY, g) != cudaSuccess)
+        return FP8_ERR_CUDA;
+      return FP8_OK;
+    }
+  }
   if (cudaLaunchKernelEx(&cfg, gemm_pair_kernel<kPairStages, false, false, KD>, tmA, tmB, tmB, tmY,
                          g) != cudaSuccess)
     return FP8_ERR_CUDA;
@@ -567,7 +587,7 @@ fp8_status launch_decode_t(const DeviceInfo& dev, const uint8_t* x8, const float
 template <int KD = kKindE4M3>
 fp8_status launch_linear(const DeviceInfo& dev, const uint8_t* x8, const float* s_tok,
                          const uint8_t* w8, const float* s_ch, int M, int N, int K, uint16_t* y,
-                         cudaStream_t stream, bool pdl) {
+                         cudaStream_t stream, bool pdl, void* ws = nullptr, size_t ws_bytes = 0) {
   // Decode-sized M: swap-AB kernel. Pipeline depth is chosen so that every
   // CTA is resident at once: with more 128-channel tiles than SMs, two CTAs
   // share an SM (<= ~110 KB of stages each), otherwise one CTA gets ~200 KB.
@@ -617,7 +637,7 @@ fp8_status launch_linear(const DeviceInfo& dev, const uint8_t* x8, const float* 
     const int64_t pair_waves = ((M + 255) / 256 * tiles_n + dev.pair_clusters - 1) / dev.pair_clusters;
     const int64_t sm_waves = ((M + kBM - 1) / kBM * tiles_n + dev.sm_count - 1) / dev.sm_count;
     if (pair_waves < sm_waves || (pair_waves == sm_waves && K >= 4096))
-      return launch_pair<KD>(dev, x8, s_tok, w8, s_ch, M, N, K, y, stream, pdl);
+      return launch_pair<KD>(dev, x8, s_tok, w8, s_ch, M, N, K, y, stream, pdl, ws, ws_bytes);
   }
   return launch_prefill<KD>(dev, x8, s_tok, w8, s_ch, M, N, K, y, stream, pdl);
 }
@@ -887,6 +907,29 @@ fp8_status fp8_rowwise_linear(const uint8_t* x8, const float* s_tok, const uint8
   }
   return launch_linear(*dev, x8, s_tok, w8, s_ch, static_cast<int>(M), static_cast<int>(N),
                        static_cast<int>(K), y, as_stream(stream), true);
+}
+
+size_t fp8_linear_workspace_bytes(void) {
+  DeviceInfo* dev;
+  if (device_info(&dev) != FP8_OK || dev->pair_clusters <= 0) return 0;
+  return split_ws_bytes(dev->pair_clusters);
+}
+
+fp8_status fp8_rowwise_linear_ws(const uint8_t* x8, const float* s_tok, const uint8_t* w8,
+                                 const float* s_ch, int64_t M, int64_t N, int64_t K, uint16_t* y,
+                                 void* ws, size_t ws_bytes, void* stream) {
+  if (fp8_status st = check_linear(x8, s_tok, w8, s_ch, M, N, K, y)) return st;
+  if (ws && !aligned16(ws)) return FP8_ERR_ALIGNMENT;
+  if (M == 0 || N == 0) return FP8_OK;
+  DeviceInfo* dev;
+  if (fp8_status st = device_info(&dev)) return st;
+  if (K == 0) {
+    if (cudaMemsetAsync(y, 0, static_cast<size_t>(M) * N * 2, as_stream(stream)) != cudaSuccess)
+      return FP8_ERR_CUDA;
+    return FP8_OK;
+  }
+  return launch_linear(*dev, x8, s_tok, w8, s_ch, static_cast<int>(M), static_cast<int>(N),
+                       static_cast<int>(K), y, as_stream(stream), true, ws, ws_bytes);
 }
 
 fp8_status fp8_linear_bf16(const uint16_t* x, const uint8_t* w8, const float* s_ch, int64_t M,

@@ -278,6 +278,12 @@ struct GemmArgs {
   int num_experts;     // grouped only
   int use_tma_store;   // tmY is a 32 x 32 bf16 store map over y (64-byte swizzle)
   int n_out;           // GeGLU epilogue only: columns of h (the features)
+  // Split (stream-K) launches of the dense pair GEMM only: the last
+  // sk_tiles tiles are shared out by k-blocks (see PairItems), partial
+  // accumulators passing through ws_part with per-warp flags ws_flag.
+  int sk_tiles;
+  uint32_t* ws_part;
+  int* ws_flag;
 };
 
 struct Tile {
@@ -548,6 +554,91 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
 // multicast to the stage's empty barrier (or the accumulator's full barrier)
 // in both CTAs; each CTA drains its own 128 TMEM lanes (its 128 rows), and the
 // even CTA's accumulator-empty barrier counts the epilogue warps of both.
+// Work items of one CTA pair of a persistent pair GEMM, in the order the
+// pair takes them. Tiles [0, T_dp) are whole tiles dealt round-robin (tile
+// p, p + P, ...). With a split, the last T - T_dp tiles (a full wave and
+// the partial last one) are cut into k-blocks, U in all, and pair p takes
+// the run [U p / P, U (p + 1) / P) of them in tile order, so every pair
+// does the same number of k-blocks (to one) instead of the last wave
+// leaving most pairs idle. A run of at least one tile's k-blocks (T - T_dp
+// >= P) starts with the end of one tile (a part: its fp32 or int32
+// accumulator goes to the workspace), then whole tiles, then the start of
+// another tile (owned: this pair adds the parts of the later k-blocks,
+// written by the next pair(s), and stores the tile). The owned piece is
+// the pair's last item and a part its first, so an owner's parts have
+// usually been written by the time it needs them.
+struct WorkItem {
+  int tile, kb0, kb1;  // k-blocks [kb0, kb1) of the tile
+  int role;            // kWhole, kOwned or kPart
+};
+constexpr int kWhole = 0, kOwned = 1, kPart = 2;
+
+struct PairItems {
+  int P, T_dp, nkb, U;
+  int dp, u, u_end;
+  __device__ __forceinline__ int u_lo(int q) const {
+    return static_cast<int>((static_cast<long long>(U) * q) / P);
+  }
+  __device__ __forceinline__ void init(int p, int P_, int T, int sk_tiles, int nkb_) {
+    P = P_;
+    nkb = nkb_;
+    T_dp = T - sk_tiles;
+    U = sk_tiles * nkb;
+    dp = p;
+    u = u_lo(p);
+    u_end = u_lo(p + 1);
+  }
+  __device__ __forceinline__ bool next(WorkItem& w) {
+    if (dp < T_dp) {
+      w.tile = dp;
+      w.kb0 = 0;
+      w.kb1 = nkb;
+      w.role = kWhole;
+      dp += P;
+      return true;
+    }
+    if (u >= u_end) return false;
+    const int ts = u / nkb;
+    w.tile = T_dp + ts;
+    w.kb0 = u - ts * nkb;
+    w.kb1 = min(nkb, w.kb0 + (u_end - u));
+    w.role = w.kb0 > 0 ? kPart : (w.kb1 == nkb ? kWhole : kOwned);
+    u += w.kb1 - w.kb0;
+    return true;
+  }
+};
+
+// Workspace of a split launch: per pair q, CTA rank r and epilogue warp w
+// one flag, and per (q, r) a 128 x 256 word accumulator part (16 KB per
+// epilogue warp, laid out so that the warp's accesses are contiguous).
+__host__ __device__ constexpr size_t split_flag_bytes(int pairs) {
+  return (static_cast<size_t>(pairs) * 2 * 8 * 4 + 255) / 256 * 256;
+}
+__host__ __device__ constexpr size_t split_ws_bytes(int pairs) {
+  return split_flag_bytes(pairs) + static_cast<size_t>(pairs) * 2 * 128 * 256 * 4;
+}
+
+// Bounded wait for a flag another CTA sets with release semantics (acquire
+// load); false (and FP8_DEV_TIMEOUT) when the limit runs out.
+__device__ __forceinline__ bool wait_flag_set(const int* flag) {
+  int v;
+  asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(flag) : "memory");
+  if (v != 0) return true;
+  const long long lim = *const_cast<volatile long long*>(&g_wait_limit);
+  const long long t0 = clock64();
+  for (;;) {
+    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(flag) : "memory");
+    if (v != 0) return true;
+    if (clock64() - t0 > lim) {
+      report(FP8_DEV_TIMEOUT);
+      return false;
+    }
+  }
+}
+__device__ __forceinline__ void set_flag_release(int* flag, int v) {
+  asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(flag), "r"(v) : "memory");
+}
+
 template <int STAGES, int STG_BUFS = 1>
 struct PairCfg {
   static constexpr int kHalf = 128;                  // rows of A and of B per CTA
@@ -584,7 +675,7 @@ struct PairCfg {
 template <bool GROUPED>
 __host__ __device__ constexpr int pair_stg_bufs() { return GROUPED ? 2 : 1; }
 
-template <int STAGES, bool GROUPED = false, bool GEGLU = false, int KD = kKindE4M3>
+template <int STAGES, bool GROUPED = false, bool GEGLU = false, int KD = kKindE4M3, bool SPLIT = false>
 __global__ void __launch_bounds__(kPrefillThreads, 1)
     gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                      const __grid_constant__ CUtensorMap tmBh, const __grid_constant__ CUtensorMap tmY,
@@ -593,6 +684,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
   using C = PairCfg<STAGES, kStgBufs>;
   static_assert(GROUPED || !GEGLU, "the GeGLU epilogue is for the grouped GEMM");
   static_assert(!GEGLU || KD == kKindE4M3, "the GeGLU epilogue is for E4M3 operands");
+  static_assert(!SPLIT || !GROUPED, "the k-block split is for the dense GEMM");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
   uint8_t* sA = smem;
@@ -667,14 +759,18 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
-      for (int tile = pair; ok && tile < num_tiles; tile += npairs) {
+      PairItems items;
+      items.init(pair, npairs, num_tiles, SPLIT ? g.sk_tiles : 0, num_kb);
+      WorkItem w;
+      while (ok && items.next(w)) {
+        const int tile = w.tile;
         const Tile T = tile_of(tile);
         const int a_row = T.a_row + rank * C::kHalf;
         const int b_row = T.b_row + rank * C::kHalf;
         const bool half = half_width(tile);  // 64 B rows per CTA
         const CUtensorMap* mapB = half ? &tmBh : &tmB;
         const uint32_t stage_tx = 2 * (C::kABytes + (half ? C::kBBytes / 2 : C::kBBytes));
-        for (int kb = 0; kb < num_kb; ++kb) {
+        for (int kb = w.kb0; kb < w.kb1; ++kb) {
           if (!mbar_wait(empty0 + 8 * stage, phase ^ 1)) { ok = false; break; }
           const uint32_t fb_local = full0 + 8 * stage;
           const uint32_t fb_leader = mapa_shared(fb_local, 0);
@@ -695,12 +791,17 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       int acc = 0;
       uint32_t acc_phase = 0;
       bool ok = true;
-      for (int tile = pair; ok && tile < num_tiles; tile += npairs) {
+      PairItems items;
+      items.init(pair, npairs, num_tiles, SPLIT ? g.sk_tiles : 0, num_kb);
+      WorkItem w;
+      while (ok && items.next(w)) {
+        const int tile = w.tile;
         if (!mbar_wait(tempty0 + 8 * acc, acc_phase ^ 1)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * C::kBN;
         const uint32_t idesc = half_width(tile) ? kIdescHalf : kIdescFull;
-        // one k-block's MMAs from k-step k0 on (k0 > 0 only for a shifted last block)
+        // one k-block's MMAs from k-step k0 on (k0 > 0 only for a shifted
+        // last block); the item's first MMA overwrites the accumulator
         auto kblock = [&](int kb, int k0) {
           if (!mbar_wait(full0 + 8 * stage, phase)) return false;
           tc_fence_after();
@@ -709,16 +810,16 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
 #pragma unroll
           for (int k = k0; k < kBK / 32; ++k) {
             umma_kind_pair<KD>(d_tmem, sw128_kmajor_desc(a0 + 32 * k), sw128_kmajor_desc(b0 + 32 * k),
-                               idesc, (kb | k) != 0);
+                               idesc, kb != w.kb0 || k != k0);
           }
           umma_commit_pair(empty0 + 8 * stage, 0x3);
           if (++stage == STAGES) { stage = 0; phase ^= 1; }
           return true;
         };
         // the hot loop keeps constant k-steps; a shifted last block is peeled off
-        const int kb_full = kblk.last_k0 != 0 ? num_kb - 1 : num_kb;
-        for (int kb = 0; ok && kb < kb_full; ++kb) ok = kblock(kb, 0);
-        if (ok && kb_full < num_kb) ok = kblock(num_kb - 1, kblk.last_k0);
+        const int kb_full = (w.kb1 == num_kb && kblk.last_k0 != 0) ? num_kb - 1 : w.kb1;
+        for (int kb = w.kb0; ok && kb < kb_full; ++kb) ok = kblock(kb, 0);
+        if (ok && kb_full < w.kb1) ok = kblock(num_kb - 1, kblk.last_k0);
         umma_commit_pair(tfull0 + 8 * acc, 0x3);
         if (++acc == 2) { acc = 0; acc_phase ^= 1; }
       }
@@ -769,20 +870,26 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       const int rr = Tt.a_row + rank * C::kHalf + quad * 32 + lane;
       sav = rr < Tt.row_end ? (g.s_a ? __ldg(g.s_a + rr) : 1.0f) : 0.0f;
     };
+    PairItems ahead;  // this pair's items, decoded two ahead of the one drained
+    ahead.init(pair, npairs, num_tiles, SPLIT ? g.sk_tiles : 0, num_kb);
+    WorkItem w = {}, w1 = {}, w2 = {};
+    bool has = ahead.next(w);
+    bool has1 = has && ahead.next(w1);
     Tile T = {}, T1 = {};
     float4 sb_v = make_float4(0.f, 0.f, 0.f, 0.f);
     float sa = 0.0f;
-    if (pair < num_tiles) {
-      T = tile_of(pair);
+    if (has) {
+      T = tile_of(w.tile);
       fetch_scales(T, sb_v, sa);
     }
-    if (pair + npairs < num_tiles) T1 = tile_of(pair + npairs);
-    for (int tile = pair; tile < num_tiles; tile += npairs) {
-      const int tile1 = tile + npairs, tile2 = tile + 2 * npairs;
+    if (has1) T1 = tile_of(w1.tile);
+    while (has) {
+      const int tile = w.tile;
       float4 sb_v1 = make_float4(0.f, 0.f, 0.f, 0.f);
       float sa1 = 0.0f;
-      if (tile1 < num_tiles) fetch_scales(T1, sb_v1, sa1);
-      const Tile T2 = tile2 < num_tiles ? tile_of(tile2) : T1;
+      if (has1) fetch_scales(T1, sb_v1, sa1);
+      const bool has2 = has1 && ahead.next(w2);
+      const Tile T2 = has2 ? tile_of(w2.tile) : T1;
       // this tile's column scales into the warp's buffer (its lanes finished
       // reading the previous tile's before the last __syncwarp)
       *reinterpret_cast<float4*>(sbw + 4 * lane) = sb_v;
@@ -837,14 +944,76 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         }
       } else {
         constexpr int kCh = 4;  // 32-column chunks per warp
+        // split items: this warp's flag and its rows of a pair's part
+        const int wslot = (warp - 2);
+        // a warp's part: its 4 chunks x 8 16-byte vectors x 32 lanes, the
+        // lanes of one vector contiguous (each warp access is 512 bytes)
+        auto part_at = [&](int q, int c) {
+          return reinterpret_cast<uint4*>(g.ws_part) +
+                 (((static_cast<size_t>(q) * 2 + rank) * 8 + wslot) * kCh + (c - half * kCh)) * 8 * 32 + lane;
+        };
+        auto flag_at = [&](int q) { return g.ws_flag + (q * 2 + static_cast<int>(rank)) * 8 + wslot; };
+        // an owned piece's parts: pairs pair+1 .. q_end-1 (the later k-blocks, in order)
+        int q_end = pair + 1;
+        if constexpr (SPLIT) {
+          if (w.role == kOwned) {
+            const int tile_end_u = (tile - ahead.T_dp + 1) * ahead.nkb;
+            while (q_end < npairs && ahead.u_lo(q_end) < tile_end_u) ++q_end;
+            if (lane == 0)
+              for (int q = pair + 1; q < q_end; ++q) wait_flag_set(flag_at(q));
+            __syncwarp();
+          }
+        }
 #pragma unroll 1
         for (int c = half * kCh; c < (half + 1) * kCh; ++c) {
+          if (SPLIT && T.col0 + c * 32 >= N) continue;  // warp-uniform; no part either
           uint32_t r[32];
           tmem_ld32(t_row + c * 32, r);
           tmem_ld_wait();
+          if constexpr (SPLIT) {
+            if (w.role == kPart) {  // raw accumulator words to the workspace
+              uint4* dst = part_at(pair, c);
+#pragma unroll
+              for (int v = 0; v < 8; ++v)
+                __stcg(dst + 32 * v, make_uint4(r[4 * v], r[4 * v + 1], r[4 * v + 2], r[4 * v + 3]));
+              continue;
+            }
+            // owned: add the later k-blocks' parts in pair order (int32
+            // sums for kind::i8, exact; fp32 otherwise)
+            for (int q = pair + 1; q < q_end; ++q) {
+              const uint4* src = part_at(q, c);
+              uint4 pvs[8];
+#pragma unroll
+              for (int v = 0; v < 8; ++v) pvs[v] = __ldcg(src + 32 * v);
+#pragma unroll
+              for (int v = 0; v < 8; ++v) {
+                const uint4 pv = pvs[v];
+                const uint32_t pw[4] = {pv.x, pv.y, pv.z, pv.w};
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                  uint32_t& x = r[4 * v + j];
+                  if constexpr (KD == kKindS8)
+                    x = static_cast<uint32_t>(static_cast<int>(x) + static_cast<int>(pw[j]));
+                  else
+                    x = __float_as_uint(__fadd_rn(__uint_as_float(x), __uint_as_float(pw[j])));
+                }
+              }
+            }
+          }
           acc_to_f32<KD>(r);
           epi_chunk(r, sbw + (c - half * kCh) * 32, sa, vec_ok, stg, g.y, row, T.row_end, N,
                     T.col0 + c * 32, lane, &tmY, tma_rows);
+        }
+        if constexpr (SPLIT) {
+          if (w.role == kPart) {  // this warp's rows of the part are written
+            __threadfence();
+            __syncwarp();
+            if (lane == 0) set_flag_release(flag_at(pair), 1);
+          } else if (w.role == kOwned) {  // parts read: their flags back to 0 for the next call
+            __syncwarp();
+            if (lane == 0)
+              for (int q = pair + 1; q < q_end; ++q) *flag_at(q) = 0;
+          }
         }
       }
       tc_fence_before();
@@ -855,6 +1024,10 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       sb_v = sb_v1;
       sa = sa1;
       T1 = T2;
+      w = w1;
+      w1 = w2;
+      has = has1;
+      has1 = has2;
     }
     if (lane == 0) bulk_wait_group_all();  // this warp's TMA stores of y are complete
   }

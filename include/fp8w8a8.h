@@ -186,6 +186,38 @@ fp8_status fp8_rowwise_linear(const uint8_t* x8, const float* s_tok, const uint8
                               uint16_t* y, void* stream);
 
 /*
+ * fp8_linear_workspace_bytes: size of the workspace fp8_rowwise_linear_ws
+ * can use on the current device (0 where the split below is not available).
+ * Per pair of SMs of the persistent GEMM grid one 256 x 256 fp32 tile and
+ * 16 flags.
+ */
+size_t fp8_linear_workspace_bytes(void);
+
+/*
+ * fp8_rowwise_linear_ws: fp8_rowwise_linear with a workspace ws of ws_bytes
+ * bytes (device memory, 16-byte aligned, zero-filled before its first use;
+ * every completed call leaves its flags zero again). When the prefill GEMM's
+ * tiles make fewer than eight waves over the SM pairs and the last wave is
+ * partial, ws_bytes >= fp8_linear_workspace_bytes() lets the last full wave
+ * and the partial one be shared out by k-blocks over all pairs (a stream-K
+ * split): a tile cut between two pairs has the accumulator of its later
+ * k-blocks written to ws by one pair and added, in k order, by the pair that
+ * computed its first k-blocks, which then stores the tile (its waits on the
+ * other pair are bounded, FP8_DEV_TIMEOUT after about a second). y has the
+ * same contract and bound as fp8_rowwise_linear; the sum order of a split
+ * tile differs from the unsplit one, but is fixed per shape and device, so
+ * results stay bit-reproducible. With ws NULL, too small, or a shape that
+ * does not split, it is fp8_rowwise_linear. Calls that may run at the same
+ * time (other streams) need workspaces of their own, and a call that ended
+ * with FP8_DEV_TIMEOUT may leave flags set: zero the workspace again before
+ * reusing it. No counterpart on the pages: a scheduling choice of this
+ * library's GEMM.
+ */
+fp8_status fp8_rowwise_linear_ws(const uint8_t* x8, const float* s_tok, const uint8_t* w8,
+                                 const float* s_ch, int64_t M, int64_t N, int64_t K, uint16_t* y,
+                                 void* ws, size_t ws_bytes, void* stream);
+
+/*
  * fp8_linear_bf16: the whole W8A8 linear from bf16 activations: per-token
  * quantization of x (exactly fp8_quant_act) followed by the row-wise GEMM
  * (exactly fp8_rowwise_linear), bit-identical to calling the two. Both are

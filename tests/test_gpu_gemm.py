@@ -106,6 +106,45 @@ def test_long_k_within_bound(lib, M, N, K):
     assert lib.device_status() == 0
 
 
+# Prefill shapes that run on CTA pairs whose tiles make a few waves with a
+# partial last one (148 SMs: 74 pairs), so fp8_rowwise_linear_ws shares the
+# last full wave and the partial one out by k-blocks: ragged N (N % 8 != 0),
+# a shifted last k-block (K % 128 = 64), a zero-filled one (K % 128 = 16),
+# every tile split (fewer than two waves), six waves and a partial seventh.
+SPLIT_SHAPES = [
+    (1024, 14336, 4096),
+    (700, 20001, 4096),
+    (768, 19000, 4160),
+    (1000, 12800, 4112),
+    (400, 12000, 8192),
+    (2048, 14336, 4096),
+]
+
+
+@pytest.mark.parametrize("M,N,K", SPLIT_SHAPES)
+def test_split_within_bound_and_reproducible(lib, M, N, K):
+    """The k-block split (stream-K over the CTA pairs) stays within the
+    row-wise GEMM bound, gives the same bits on a second call with the same
+    workspace (whose flags every call leaves zero), and equals the plain call
+    when the workspace is too small to split."""
+    xb, a, w = _operands(M, N, K, seed=M + N + K + 7)
+    x8, st, w8, sw = to_dev(a.codes), to_dev(a.scales), to_dev(w.codes), to_dev(w.scales)
+    ws = lib.linear_workspace()
+    y1 = lib.rowwise_linear_ws(x8, st, w8, sw, ws)
+    y2 = lib.rowwise_linear_ws(x8, st, w8, sw, ws)
+    assert lib.device_status() == 0
+    rows = None if M * N * K <= 4e9 else np.unique(np.concatenate([
+        np.arange(8), np.arange(M - 8, M), np.random.default_rng(M).choice(M, 48, replace=False)]))
+    _check(y1, a, w, rows)
+    assert np.array_equal(bf16_to_np_bits(y1), bf16_to_np_bits(y2))
+    # the flags: what precedes the pairs' 256 KB parts
+    nflag = int(lib.raw.fp8_linear_workspace_bytes()) % (2 * 128 * 256 * 4)
+    assert not u8(ws)[:nflag].any()
+    y0 = lib.rowwise_linear(x8, st, w8, sw)
+    small = torch.zeros(16, dtype=torch.uint8, device="cuda")
+    assert np.array_equal(bf16_to_np_bits(lib.rowwise_linear_ws(x8, st, w8, sw, small)), bf16_to_np_bits(y0))
+
+
 def test_k_beyond_the_limit_is_refused(lib):
     x8 = torch.zeros((1, 65552), dtype=torch.uint8, device="cuda")
     w8 = torch.zeros((128, 65552), dtype=torch.uint8, device="cuda")
