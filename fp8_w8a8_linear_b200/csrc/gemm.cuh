@@ -955,6 +955,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         auto flag_at = [&](int q) { return g.ws_flag + (q * 2 + static_cast<int>(rank)) * 8 + wslot; };
         // an owned piece's parts: pairs pair+1 .. q_end-1 (the later k-blocks, in order)
         int q_end = pair + 1;
+        const bool is_part = SPLIT && w.role == kPart;
         if constexpr (SPLIT) {
           if (w.role == kOwned) {
             const int tile_end_u = (tile - ahead.T_dp + 1) * ahead.nkb;
@@ -967,11 +968,21 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
 #pragma unroll 1
         for (int c = half * kCh; c < (half + 1) * kCh; ++c) {
           if (SPLIT && T.col0 + c * 32 >= N) continue;  // warp-uniform; no part either
+          // owned: the next pair's part of this chunk is requested before the
+          // TMEM load, so that the two latencies overlap (usually one part)
+          uint4 pv0[8];
+          if constexpr (SPLIT) {
+            if (w.role == kOwned && q_end > pair + 1) {
+              const uint4* src = part_at(pair + 1, c);
+#pragma unroll
+              for (int v = 0; v < 8; ++v) pv0[v] = __ldcg(src + 32 * v);
+            }
+          }
           uint32_t r[32];
           tmem_ld32(t_row + c * 32, r);
           tmem_ld_wait();
           if constexpr (SPLIT) {
-            if (w.role == kPart) {  // raw accumulator words to the workspace
+            if (is_part) {  // raw accumulator words to the workspace
               uint4* dst = part_at(pair, c);
 #pragma unroll
               for (int v = 0; v < 8; ++v)
@@ -981,10 +992,15 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
             // owned: add the later k-blocks' parts in pair order (int32
             // sums for kind::i8, exact; fp32 otherwise)
             for (int q = pair + 1; q < q_end; ++q) {
-              const uint4* src = part_at(q, c);
               uint4 pvs[8];
+              if (q == pair + 1) {
 #pragma unroll
-              for (int v = 0; v < 8; ++v) pvs[v] = __ldcg(src + 32 * v);
+                for (int v = 0; v < 8; ++v) pvs[v] = pv0[v];
+              } else {
+                const uint4* src = part_at(q, c);
+#pragma unroll
+                for (int v = 0; v < 8; ++v) pvs[v] = __ldcg(src + 32 * v);
+              }
 #pragma unroll
               for (int v = 0; v < 8; ++v) {
                 const uint4 pv = pvs[v];
