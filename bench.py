@@ -273,7 +273,7 @@ def setup_dense(torch, f, wl, seed, dev, flushable):
                 L.append((f"int8_quant_act[M={M}]", lambda i, x=D[f"x{M}"], x8i=x8i, st=st: f.int8_quant_act(x, x8i, st),
                           0.0, qb, "hbm", False, 1))
                 L.append((f"int8_gemm[M={M}]",
-                          lambda i, x8i=x8i, st=st, y=y: f.int8_rowwise_linear(x8i, st, w8i, s8i, y),
+                          lambda i, x8i=x8i, st=st, y=y: f.int8_rowwise_linear_ws(x8i, st, w8i, s8i, gws, y),
                           fl, gb, "tensor", False, 1))
                 # unpack to the workspace (0.625 B in, 2 B out per weight), then the bf16 GEMM
                 L.append((f"w4a16_unpack[N={N}]", lambda i: f.w4a16_dequant(D["q4"], D["d"], ws), 0.0,

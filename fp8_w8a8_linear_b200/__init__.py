@@ -21,7 +21,8 @@ Functions mirror the C entry points:
   router's top-k choice and weights.
 * :func:`w4a16_dequant`, :func:`w4a16_linear` - the W4A16 build (int4 QAT
   weights, bf16 activations).
-* :func:`int8_repack_qat`, :func:`int8_quant_act`, :func:`int8_rowwise_linear`,
+* :func:`int8_repack_qat`, :func:`int8_quant_act`, :func:`int8_rowwise_linear`
+  (:func:`int8_rowwise_linear_ws` with a workspace),
   :func:`int8_linear` - the int8 W8A8 build.
 * :func:`device_status` - read and clear the device status word.
 """
@@ -79,6 +80,7 @@ _SIGS = {
     "int8_repack_qat": ([_P, _P, _I64, _I64, _P, _P, _P], ctypes.c_int),
     "int8_quant_act": ([_P, _I64, _I64, _I64, _P, _P, _P], ctypes.c_int),
     "int8_rowwise_linear": ([_P, _P, _P, _P, _I64, _I64, _I64, _P, _P], ctypes.c_int),
+    "int8_rowwise_linear_ws": ([_P, _P, _P, _P, _I64, _I64, _I64, _P, _P, ctypes.c_size_t, _P], ctypes.c_int),
     "int8_linear_bf16": ([_P, _P, _P, _I64, _I64, _I64, _P, _P, _P, _P], ctypes.c_int),
 }
 for _name, (_args, _ret) in _SIGS.items():
@@ -461,6 +463,22 @@ def int8_rowwise_linear(x8: torch.Tensor, s_tok: torch.Tensor, w8: torch.Tensor,
     return y
 
 
+def int8_rowwise_linear_ws(x8: torch.Tensor, s_tok: torch.Tensor, w8: torch.Tensor, s_ch: torch.Tensor,
+                           ws: torch.Tensor, y: torch.Tensor | None = None):
+    """int8_rowwise_linear with a workspace (from linear_workspace) for the
+    k-block split; bit-identical to int8_rowwise_linear."""
+    M, K = x8.shape
+    N = w8.shape[0]
+    y = torch.empty((M, N), dtype=torch.bfloat16, device=x8.device) if y is None else y
+    _check(_lib.int8_rowwise_linear_ws(_dev(x8, torch.int8, "x8"), _dev(s_tok, torch.float32, "s_tok", (M,)),
+                                       _dev(w8, torch.int8, "w8", (N, K)),
+                                       _dev(s_ch, torch.float32, "s_ch", (N,)), M, N, K,
+                                       _dev(y, torch.bfloat16, "y", (M, N)), _dev(ws, torch.uint8, "ws"),
+                                       ws.numel(), _stream()),
+           "int8_rowwise_linear_ws")
+    return y
+
+
 def int8_linear(x: torch.Tensor, w8: torch.Tensor, s_ch: torch.Tensor, y: torch.Tensor | None = None,
                 x8: torch.Tensor | None = None, s_tok: torch.Tensor | None = None):
     """The int8 W8A8 linear from bf16 activations: int8 quant per token, then GEMM."""
@@ -515,7 +533,7 @@ __all__ = [
     "linear_siblings", "test_set_fault",
     "moe_route", "moe_gather", "grouped_linear", "moe_geglu_quant", "moe_combine",
     "moe_interleave_gate_up", "grouped_linear_geglu",
-    "int8_repack_qat", "int8_quant_act", "int8_rowwise_linear", "int8_linear",
+    "int8_repack_qat", "int8_quant_act", "int8_rowwise_linear", "int8_rowwise_linear_ws", "int8_linear",
     "bf16_linear", "moe_topk", "w4a16_dequant", "w4a16_workspace_bytes", "w4a16_linear",
     "DEV_NONFINITE", "DEV_NAN_CODE", "DEV_INEXACT", "DEV_TIMEOUT", "LIB_PATH",
 ]

@@ -163,6 +163,9 @@ fp8_status set_pair_attr() {
                  cudaFuncSetAttribute(gemm_pair_kernel<STAGES, false, false, kKindE4M3, true>,
                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
                                       static_cast<int>(PairCfg<STAGES>::kSmem)) == cudaSuccess &&
+                 cudaFuncSetAttribute(gemm_pair_kernel<STAGES, false, false, kKindS8, true>,
+                                      cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      static_cast<int>(PairCfg<STAGES>::kSmem)) == cudaSuccess &&
 
                  cudaFuncSetAttribute(gemm_pair_kernel<STAGES, false, false, kKindS8>,
                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -392,7 +395,7 @@ fp8_status launch_pair(const DeviceInfo& dev, const uint8_t* x8, const float* s_
   // noticeable share) is evened out by the k-block split when the caller
   // gave a workspace: the last full wave and the partial one are shared
   // out by k-blocks over all pairs.
-  if constexpr (KD == kKindE4M3) {
+  if constexpr (KD == kKindE4M3 || KD == kKindS8) {
     if (ws && ws_bytes >= split_ws_bytes(pairs) && num_tiles > pairs && num_tiles % pairs != 0 &&
         num_tiles < 8 * pairs) {
       g.sk_tiles = pairs + num_tiles % pairs;
@@ -1275,6 +1278,26 @@ fp8_status int8_rowwise_linear(const int8_t* x8, const float* s_tok, const int8_
   return launch_linear<kKindS8>(*dev, reinterpret_cast<const uint8_t*>(x8), s_tok,
                                 reinterpret_cast<const uint8_t*>(w8), s_ch, static_cast<int>(M),
                                 static_cast<int>(N), static_cast<int>(K), y, as_stream(stream), true);
+}
+
+fp8_status int8_rowwise_linear_ws(const int8_t* x8, const float* s_tok, const int8_t* w8,
+                                  const float* s_ch, int64_t M, int64_t N, int64_t K, uint16_t* y,
+                                  void* ws, size_t ws_bytes, void* stream) {
+  if (fp8_status st = check_linear(x8, s_tok, reinterpret_cast<const uint8_t*>(w8), s_ch, M, N, K, y))
+    return st;
+  if (ws && !aligned16(ws)) return FP8_ERR_ALIGNMENT;
+  if (M == 0 || N == 0) return FP8_OK;
+  DeviceInfo* dev;
+  if (fp8_status st = device_info(&dev)) return st;
+  if (K == 0) {
+    if (cudaMemsetAsync(y, 0, static_cast<size_t>(M) * N * 2, as_stream(stream)) != cudaSuccess)
+      return FP8_ERR_CUDA;
+    return FP8_OK;
+  }
+  return launch_linear<kKindS8>(*dev, reinterpret_cast<const uint8_t*>(x8), s_tok,
+                                reinterpret_cast<const uint8_t*>(w8), s_ch, static_cast<int>(M),
+                                static_cast<int>(N), static_cast<int>(K), y, as_stream(stream), true, ws,
+                                ws_bytes);
 }
 
 fp8_status int8_linear_bf16(const uint16_t* x, const int8_t* w8, const float* s_ch, int64_t M,

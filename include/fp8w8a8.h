@@ -483,6 +483,16 @@ fp8_status int8_rowwise_linear(const int8_t* x8, const float* s_tok, const int8_
                                void* stream);
 
 /*
+ * int8_rowwise_linear_ws: int8_rowwise_linear with the workspace and the
+ * k-block split of fp8_rowwise_linear_ws (same workspace contract). The
+ * parts are int32 sums, added exactly, so y is bit for bit that of
+ * int8_rowwise_linear.
+ */
+fp8_status int8_rowwise_linear_ws(const int8_t* x8, const float* s_tok, const int8_t* w8,
+                                  const float* s_ch, int64_t M, int64_t N, int64_t K, uint16_t* y,
+                                  void* ws, size_t ws_bytes, void* stream);
+
+/*
  * int8_linear_bf16: int8_quant_act of x (pitch K) into the caller's x8 /
  * s_tok, then int8_rowwise_linear; bit-identical to the two calls.
  */

@@ -87,6 +87,32 @@ def test_int8_gemm_bit_exact(lib, M, N, K):
     assert lib.device_status() == 0
 
 
+# Shapes on CTA pairs with a partial last wave (148 SMs: 74 pairs), split
+# by k-blocks when a workspace is given: ragged N, shifted and zero-filled
+# last k-blocks, every tile split, six waves and a partial seventh.
+INT8_SPLIT_SHAPES = [(1024, 14336, 4096), (700, 20001, 4096), (768, 19000, 4160),
+                     (1000, 12800, 4112), (400, 12000, 8192), (2048, 14336, 4096)]
+
+
+@pytest.mark.parametrize("M,N,K", INT8_SPLIT_SHAPES)
+def test_int8_split_bit_exact(lib, M, N, K):
+    """int8_rowwise_linear_ws: the k-block split's int32 parts add exactly,
+    so every output bit is still the oracle's (all rows up to M = 1024, 96
+    sampled rows above), on two calls with the same workspace."""
+    xb, a, wc, sc = _operands(M, N, K, seed=M + 3 * N + K)
+    x8, st, w8, s8 = to_dev(a.codes), to_dev(a.scales), to_dev(wc), to_dev(sc)
+    ws = lib.linear_workspace()
+    y1 = lib.int8_rowwise_linear_ws(x8, st, w8, s8, ws)
+    y2 = lib.int8_rowwise_linear_ws(x8, st, w8, s8, ws)
+    assert lib.device_status() == 0
+    rows = np.arange(M) if M <= 1024 else np.random.default_rng(M).choice(M, 96, replace=False)
+    ref = I8.int8_linear_ref(a.codes[rows], a.scales[rows], wc, sc)
+    got = bf16_to_np_bits(y1)[rows]
+    bad = got != ref
+    assert not bad.any(), (int(bad.sum()), np.argwhere(bad)[:4])
+    assert np.array_equal(bf16_to_np_bits(y2), bf16_to_np_bits(y1))
+
+
 @pytest.mark.parametrize("M", [1, 64, 8192])
 def test_int8_full_layer_sampled(lib, M):
     """The prefill layer K=4096, N=14336 at M = 1 / 64 / 8192: weights from the
