@@ -272,7 +272,8 @@ __global__ void __launch_bounds__(256) quant_act_staged_kernel(const uint16_t* _
   uint32_t phases = 0u;  // bit b: parity to wait for on buffer b
   int b = 0;
   for (int64_t row = gw; row < M; row += nw, b ^= 1) {
-    if (!mbar_wait(bar0 + 8 * b, (phases >> b) & 1u)) return;
+    // the warp leaves together (its lanes' bounded waits may end differently)
+    if (!__all_sync(0xFFFFFFFFu, mbar_wait(bar0 + 8 * b, (phases >> b) & 1u))) return;
     phases ^= 1u << b;
     const uint4* src = reinterpret_cast<const uint4*>(buf0 + b * row_bytes_padded);
     uint32_t mx = 0;
@@ -570,7 +571,8 @@ __global__ void __launch_bounds__(256) repack_qat_staged_kernel(const uint8_t* _
   uint32_t phases = 0u;
   int b = 0;
   for (int64_t row = gw; row < N; row += nw) {
-    if (!mbar_wait(bar0 + 8 * b, (phases >> b) & 1u)) return;
+    // the warp leaves together (its lanes' bounded waits may end differently)
+    if (!__all_sync(0xFFFFFFFFu, mbar_wait(bar0 + 8 * b, (phases >> b) & 1u))) return;
     phases ^= 1u << b;
     const uint4* qs = reinterpret_cast<const uint4*>(bufs + b * buf_bytes);
     const float* ds = reinterpret_cast<const float*>(bufs + b * buf_bytes + qbytes);
@@ -725,7 +727,8 @@ __global__ void __launch_bounds__(256) convert_fnuz_staged_kernel(const uint8_t*
   uint32_t phases = 0u;  // bit b: parity to wait for on buffer b
   int b = 0;
   for (int64_t row = gw; row < N; row += nw, b ^= 1) {
-    if (!mbar_wait(bar0 + 8 * b, (phases >> b) & 1u)) return;
+    // the warp leaves together (its lanes' bounded waits may end differently)
+    if (!__all_sync(0xFFFFFFFFu, mbar_wait(bar0 + 8 * b, (phases >> b) & 1u))) return;
     phases ^= 1u << b;
     const uint4* in = reinterpret_cast<const uint4*>(buf0 + b * row_bytes_padded);
     const float s_in = s_src[row];

@@ -13,7 +13,7 @@
 // tensor-core MMA (kind::f16) against the bf16 activations.
 //
 // * w4a16_dequant_kernel: q4 [N, K/2] + d [N, K/32] -> w [N, K] bf16, an HBM
-//   streaming kernel (one 32-value group per thread: 16 + 4 bytes in, 64 out).
+//   streaming kernel (32 groups per warp: 16 + 4 bytes in, 64 out per group).
 // * gemm_w4_decode_kernel (M <= 128): swap-AB like the FP8 decode GEMM, with
 //   the weight operand unpacked on chip. Warp 0 streams the packed weights
 //   and scales (0.625 bytes per weight) into a ring of raw stages with TMA;
@@ -72,23 +72,38 @@ __device__ __forceinline__ uint4 unpack8_bf16(uint32_t word, float d) {
   return make_uint4(out[0], out[1], out[2], out[3]);
 }
 
-// w [N, K] bf16 from q4 [N, K/2] and d [N, K/32]; K % 32 == 0. Thread g
-// handles group g of the row-major group order (consecutive threads read
-// consecutive 16-byte q4 vectors and write consecutive 64-byte pieces).
+// w [N, K] bf16 from q4 [N, K/2] and d [N, K/32]; K % 32 == 0. A warp takes
+// 32 consecutive groups (2 KB of output) at a time: in step j lane l unpacks
+// 16-byte piece l % 4 of group 8j + l / 4, so that each store instruction of
+// the warp writes 512 contiguous bytes and each load reads 128 contiguous
+// bytes of q4 (one whole-line store per lane and piece, not four partial
+// ones per 64-byte group).
 __global__ void __launch_bounds__(256) w4a16_dequant_kernel(const uint8_t* __restrict__ q4,
                                                              const float* __restrict__ d,
                                                              int64_t groups,
                                                              uint16_t* __restrict__ w) {
   pdl_launch_dependents();
-  for (int64_t g = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; g < groups;
-       g += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const uint4 q = __ldg(reinterpret_cast<const uint4*>(q4) + g);
-    const float dg = __ldg(d + g);
-    uint4* dst = reinterpret_cast<uint4*>(w) + 4 * g;
-    dst[0] = unpack8_bf16(q.x, dg);
-    dst[1] = unpack8_bf16(q.y, dg);
-    dst[2] = unpack8_bf16(q.z, dg);
-    dst[3] = unpack8_bf16(q.w, dg);
+  const int lane = threadIdx.x & 31;
+  const int64_t chunks = (groups + 31) / 32;
+  const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+  const uint32_t* qw = reinterpret_cast<const uint32_t*>(q4);
+  uint4* dst = reinterpret_cast<uint4*>(w);
+  for (int64_t c = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5; c < chunks;
+       c += nwarps) {
+    const int64_t g0 = 32 * c;
+    uint32_t qv[4];
+    float dv[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int64_t g = g0 + 8 * j + (lane >> 2);
+      qv[j] = g < groups ? __ldg(qw + 4 * g + (lane & 3)) : 0u;
+      dv[j] = g < groups ? __ldg(d + g) : 0.0f;
+    }
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int64_t g = g0 + 8 * j + (lane >> 2);
+      if (g < groups) dst[4 * g0 + 32 * j + lane] = unpack8_bf16(qv[j], dv[j]);
+    }
   }
 }
 
