@@ -282,6 +282,12 @@ fp8_status device_info(DeviceInfo** out) {
                               kStagedSmemBudget + 1024) != cudaSuccess ||
          cudaFuncSetAttribute(quant_act_staged_kernel<true, kEncI8>,
                               cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              kStagedSmemBudget + 1024) != cudaSuccess ||
+         cudaFuncSetAttribute(quant_act_staged_kernel<true, kEncE4M3, 2>,
+                              cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              kStagedSmemBudget + 1024) != cudaSuccess ||
+         cudaFuncSetAttribute(quant_act_staged_kernel<true, kEncI8, 2>,
+                              cudaFuncAttributeMaxDynamicSharedMemorySize,
                               kStagedSmemBudget + 1024) != cudaSuccess))
       st = FP8_ERR_CUDA;
     if (st == FP8_OK &&
@@ -737,6 +743,21 @@ fp8_status launch_quant_act(const DeviceInfo& dev, const uint16_t* x, int64_t M,
     const int warps = static_cast<int>(staged_warps);
     const size_t smem = static_cast<size_t>(warps) * 2 * row_pad + 16 * warps;
     const int64_t per_sm = staged_blocks_per_sm(quant_act_staged_kernel<false, ENC>, 32 * warps, smem);
+    // Long rows that leave fewer than 16 warps per SM: a warp pair per row,
+    // each warp staging half of it, where that gives 24 or more warps per SM
+    // (measured on B200: 8192 x 4096 20.4 -> 17.7 us with 24 warps per SM;
+    // 65536 x 5376, where pairs give 16, 169 -> 177 us, so not there).
+    const uint32_t half_pad = static_cast<uint32_t>((K + 127) / 128 * 128);
+    const int64_t pair_warps = std::min<int64_t>(8, kStagedSmemBudget / (2 * int64_t(half_pad) + 24)) & ~int64_t(1);
+    const int pw = static_cast<int>(pair_warps);
+    const size_t psmem = static_cast<size_t>(pw) * 2 * half_pad + 24 * pw;
+    const int64_t pper_sm =
+        pw >= 2 ? staged_blocks_per_sm(quant_act_staged_kernel<true, ENC, 2>, 32 * pw, psmem) : 0;
+    if (per_sm * warps < 16 && pper_sm * pw >= 24) {  // many warps per SM: packed divisions
+      const int64_t pblocks = std::min<int64_t>(pper_sm * dev.sm_count, (M + pw / 2 - 1) / (pw / 2));
+      return launch_pdl_smem(quant_act_staged_kernel<true, ENC, 2>, dim3(static_cast<unsigned>(pblocks)),
+                             dim3(32 * pw), psmem, stream, x, M, K, ldx, x8, s_tok, half_pad);
+    }
     const int64_t blocks = std::min<int64_t>(per_sm * dev.sm_count, (M + warps - 1) / warps);
     // Short rows (16 or more warps per SM) are issue-bound: packed divisions.
     const auto kernel = per_sm * warps >= 16 ? quant_act_staged_kernel<true, ENC>

@@ -235,25 +235,37 @@ __global__ void __launch_bounds__(BLOCK) quant_act_kernel(const uint16_t* __rest
 // with many warps per SM, where issue slots are what limits short rows; with
 // few warps per SM (long rows) the scalar form's independent chains hide
 // latency better.
-template <bool PACKED, int ENC = kEncE4M3>
+// RW = 2: a pair of warps per row, each staging and quantizing one half
+// (K % 16 == 0, so each half is a whole number of 16-byte vectors); the two
+// half-row maxima meet in shared memory at a 64-thread named barrier (which
+// also ORs the two warps' wait failures, so that they leave together). Long
+// rows fit twice as many warps per SM this way. Dynamic shared memory:
+// warps * 2 * row_bytes_padded (half rows for RW = 2), 2 barriers per warp,
+// then (RW = 2) two exchange words per warp.
+template <bool PACKED, int ENC = kEncE4M3, int RW = 1>
 __global__ void __launch_bounds__(256) quant_act_staged_kernel(const uint16_t* __restrict__ x,
                                                                 int64_t M, int64_t K, int64_t ldx,
                                                                 uint8_t* __restrict__ x8,
                                                                 float* __restrict__ s_tok,
                                                                 uint32_t row_bytes_padded) {
+  static_assert(RW == 1 || RW == 2, "one or two warps per row");
   pdl_launch_dependents();
   pdl_wait();  // x may come from the preceding grid (a no-op without programmatic launch)
   extern __shared__ __align__(128) uint8_t qsm[];
   const int warps = blockDim.x >> 5;
   const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int h = w % RW;   // this warp's part of the row
+  const int pw = w / RW;  // the row group (warp pair) within the block
   uint8_t* buf0 = qsm + static_cast<size_t>(w) * 2 * row_bytes_padded;
   uint64_t* bars =
       reinterpret_cast<uint64_t*>(qsm + static_cast<size_t>(warps) * 2 * row_bytes_padded);
+  volatile uint32_t* xch = reinterpret_cast<volatile uint32_t*>(bars + 2 * warps);
   const uint32_t bar0 = smem_u32(bars + 2 * w);
-  const uint32_t row_bytes = static_cast<uint32_t>(K) * 2;
-  const int64_t nvec = K / 8;
-  const int64_t gw = static_cast<int64_t>(blockIdx.x) * warps + w;
-  const int64_t nw = static_cast<int64_t>(gridDim.x) * warps;
+  const int64_t Kp = K / RW;  // values of the row this warp handles
+  const uint32_t row_bytes = static_cast<uint32_t>(Kp) * 2;
+  const int64_t nvec = Kp / 8;
+  const int64_t gw = static_cast<int64_t>(blockIdx.x) * (warps / RW) + pw;
+  const int64_t nw = static_cast<int64_t>(gridDim.x) * (warps / RW);
   if (lane == 0) {
     mbar_init(bar0, 1);
     mbar_init(bar0 + 8, 1);
@@ -264,7 +276,7 @@ __global__ void __launch_bounds__(256) quant_act_staged_kernel(const uint16_t* _
     if (lane == 0) {
       fence_proxy_async_shared();
       mbar_arrive_expect_tx(bar0 + 8 * b, row_bytes);
-      bulk_load(smem_u32(buf0 + b * row_bytes_padded), x + row * ldx, row_bytes, bar0 + 8 * b);
+      bulk_load(smem_u32(buf0 + b * row_bytes_padded), x + row * ldx + h * Kp, row_bytes, bar0 + 8 * b);
     }
   };
   if (gw < M) issue(gw, 0);
@@ -273,12 +285,13 @@ __global__ void __launch_bounds__(256) quant_act_staged_kernel(const uint16_t* _
   int b = 0;
   for (int64_t row = gw; row < M; row += nw, b ^= 1) {
     // the warp leaves together (its lanes' bounded waits may end differently)
-    if (!__all_sync(0xFFFFFFFFu, mbar_wait(bar0 + 8 * b, (phases >> b) & 1u))) return;
+    const bool ok = __all_sync(0xFFFFFFFFu, mbar_wait(bar0 + 8 * b, (phases >> b) & 1u));
+    if (RW == 1 && !ok) return;
     phases ^= 1u << b;
     const uint4* src = reinterpret_cast<const uint4*>(buf0 + b * row_bytes_padded);
     uint32_t mx = 0;
 #pragma unroll 4
-    for (int64_t j = lane; j < nvec; j += 32) {
+    for (int64_t j = lane; ok && j < nvec; j += 32) {
       const uint4 u = src[j];
       mx = __vmaxu2(mx, u.x & 0x7FFF7FFFu);
       mx = __vmaxu2(mx, u.y & 0x7FFF7FFFu);
@@ -286,13 +299,20 @@ __global__ void __launch_bounds__(256) quant_act_staged_kernel(const uint16_t* _
       mx = __vmaxu2(mx, u.w & 0x7FFF7FFFu);
     }
     mx = max(mx & 0xFFFFu, mx >> 16);
-    const uint32_t amax_bits = __reduce_max_sync(0xFFFFFFFFu, mx);
-    if (amax_bits >= 0x7F80u && lane == 0) report(FP8_DEV_NONFINITE);
+    uint32_t amax_bits = __reduce_max_sync(0xFFFFFFFFu, mx);
+    if constexpr (RW == 2) {
+      // the other half's maximum (exchange words alternate with the buffers,
+      // so a word is rewritten only after the next barrier)
+      if (lane == 0) xch[2 * w + b] = amax_bits;
+      if (named_bar_or(1 + pw, 64, !ok)) return;
+      amax_bits = max(amax_bits, xch[2 * (w ^ 1) + b]);
+    }
+    if (amax_bits >= 0x7F80u && lane == 0 && h == 0) report(FP8_DEV_NONFINITE);
     const float amax = __uint_as_float(amax_bits << 16);
     const float s = __fdiv_rn(amax, enc_max<ENC>());
-    if (lane == 0) s_tok[row] = s;
+    if (lane == 0 && h == 0) s_tok[row] = s;
     const RowDivisor dv = make_divisor(s, amax);
-    uint2* dst = reinterpret_cast<uint2*>(x8 + row * K);
+    uint2* dst = reinterpret_cast<uint2*>(x8 + row * K + h * Kp);
     if (s == 0.0f) {
       for (int64_t j = lane; j < nvec; j += 32) dst[j] = make_uint2(0, 0);
     } else if (dv.fast) {

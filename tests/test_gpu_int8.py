@@ -19,7 +19,8 @@ def _i8(t):
 
 
 @pytest.mark.parametrize("M,K", [(1, 2048), (4, 256), (64, 5376), (300, 4096), (1000, 16),
-                                 (1025, 2048), (4096, 704), (16384, 5376), (3000, 65536)])
+                                 (1025, 2048), (4096, 704), (16384, 5376), (3000, 65536),
+                                 (2049, 4096)])
 def test_int8_quant_act_bit_exact(lib, M, K):
     xb = activations_bf16(M, K, seed=M + K, outlier_frac=0.01)
     ref = I8.quant_act_int8(xb)

@@ -69,6 +69,8 @@ ACT_SHAPES = [
     (2, 21504, 11, 0.01),
     (1100, 6160, 9, 0.01),   # warp-per-row path, re-read from cache
     (7, 65536, 10, 0.01),
+    (4097, 4096, 13, 0.01),  # warp pair per row (each warp stages half of it)
+    (1500, 4608, 14, 0.01),
 ]
 
 
@@ -145,6 +147,33 @@ def test_quant_act_pitched_input(lib):
     assert st == 0
     assert np.array_equal(u8(x8), ref.codes)
     assert same_bits_f32(f32(s), ref.scales)
+
+
+def test_quant_act_warp_pair_rows(lib):
+    """Rows split over a warp pair (M > 1024, K = 4096): the row maximum only
+    in the first or only in the second half, zero halves, a NaN in the
+    second half (flagged), a pitched input - bytes and scales bit-exact."""
+    M, K, ldx = 2048, 4096, 4160
+    xb = activations_bf16(M, ldx, seed=15, outlier_frac=0.01)
+    xb[1, :K // 2] = 0                        # first half zero
+    xb[2, K // 2:K] = 0                       # second half zero
+    xb[3, :K] = 0                             # zero row: s = 0, codes 0
+    xb[4, K // 2 + 7] = 0x4780                # 65536 in the second half only
+    xb[5, 3] = 0xC780                         # -65536 in the first half only
+    xb[6, K - 1] = 0x7FC0                     # NaN in the second half
+    ref = oracle.quant_act(xb[:, :K])
+    x8 = torch.empty((M, K), dtype=torch.uint8, device="cuda")
+    s = torch.empty((M,), dtype=torch.float32, device="cuda")
+    lib.device_status()
+    st = lib.raw.fp8_quant_act(to_dev(xb).data_ptr(), M, K, ldx, x8.data_ptr(), s.data_ptr(),
+                               torch.cuda.current_stream().cuda_stream)
+    assert st == 0
+    assert lib.device_status() & lib.DEV_NONFINITE
+    ok = np.ones(M, bool)
+    ok[6] = False
+    assert np.array_equal(u8(x8)[ok], ref.codes[ok])
+    assert same_bits_f32(f32(s)[ok], ref.scales[ok])
+    assert f32(s)[3] == 0 and not u8(x8)[3].any()
 
 
 def test_quant_act_nonfinite_rows_are_reported(lib):
