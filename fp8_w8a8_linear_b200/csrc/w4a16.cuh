@@ -17,13 +17,13 @@
 // * gemm_w4_decode_kernel (M <= 128): swap-AB like the FP8 decode GEMM, with
 //   the weight operand unpacked on chip. Warp 0 streams the packed weights
 //   and scales (0.625 bytes per weight) into a ring of raw stages with TMA;
-//   warp 18 streams the token tiles into the operand ring (a thread of its
-//   own, so that no token-tile load waits behind a raw-stage refill); warps
-//   2..17 unpack each raw stage into two 128-row x 64-value bf16 operand
-//   blocks in the 128-byte swizzled K-major layout the MMA reads (sixteen
-//   warps, four per scheduler, one 32-value group per thread: the unpacking
-//   is a chain of dependent integer and fp32 steps whose latency the other
-//   warps hide); warp 1 issues
+//   the last warp streams the token tiles into the operand ring (a thread of
+//   its own, so that no token-tile load waits behind a raw-stage refill);
+//   the warps from 2 on - sixteen with the deep rings (one CTA per SM), eight
+//   with the shallow ones - unpack each raw stage into two 128-row x 64-value
+//   bf16 operand blocks in the 128-byte swizzled K-major layout the MMA reads
+//   (one 32-value group per thread: the unpacking is a chain of dependent
+//   integer and fp32 steps whose latency the other warps hide); warp 1 issues
 //   tcgen05.mma.kind::f16 into a TMEM accumulator. K may be split across a thread-block cluster with
 //   the partial tiles summed in rank order through distributed shared memory,
 //   as in the FP8 decode GEMM. The epilogue stores y = bf16(acc).
