@@ -166,7 +166,6 @@ fp8_status set_pair_attr() {
                  cudaFuncSetAttribute(gemm_pair_kernel<STAGES, false, false, kKindS8, true>,
                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
                                       static_cast<int>(PairCfg<STAGES>::kSmem)) == cudaSuccess &&
-
                  cudaFuncSetAttribute(gemm_pair_kernel<STAGES, false, false, kKindS8>,
                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
                                       static_cast<int>(PairCfg<STAGES>::kSmem)) == cudaSuccess &&

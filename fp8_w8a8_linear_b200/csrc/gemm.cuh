@@ -543,17 +543,6 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
   }
 }
 
-// ============================================================== prefill, CTA pair
-// Dense GEMM on 256 x 256 output tiles computed by a cluster of two CTAs on
-// two SMs with tcgen05.mma.cta_group::2: each CTA stages 128 rows of A (its
-// half of the tile's rows) and 128 rows of B (its half of the tile's
-// columns), so every SM moves 32 KB per 128-deep k-block for a 256 x 256 x
-// 128 product - two thirds of the operand traffic of a 128 x 256 single-SM
-// tile per unit of work. The even CTA's MMA thread issues the pair MMAs; both
-// CTAs' TMA loads complete on the even CTA's full barrier; each MMA commit is
-// multicast to the stage's empty barrier (or the accumulator's full barrier)
-// in both CTAs; each CTA drains its own 128 TMEM lanes (its 128 rows), and the
-// even CTA's accumulator-empty barrier counts the epilogue warps of both.
 // Work items of one CTA pair of a persistent pair GEMM, in the order the
 // pair takes them. Tiles [0, T_dp) are whole tiles dealt round-robin (tile
 // p, p + P, ...). With a split, the last T - T_dp tiles (a full wave and
@@ -639,6 +628,17 @@ __device__ __forceinline__ void set_flag_release(int* flag, int v) {
   asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(flag), "r"(v) : "memory");
 }
 
+// ============================================================== prefill, CTA pair
+// Dense GEMM on 256 x 256 output tiles computed by a cluster of two CTAs on
+// two SMs with tcgen05.mma.cta_group::2: each CTA stages 128 rows of A (its
+// half of the tile's rows) and 128 rows of B (its half of the tile's
+// columns), so every SM moves 32 KB per 128-deep k-block for a 256 x 256 x
+// 128 product - two thirds of the operand traffic of a 128 x 256 single-SM
+// tile per unit of work. The even CTA's MMA thread issues the pair MMAs; both
+// CTAs' TMA loads complete on the even CTA's full barrier; each MMA commit is
+// multicast to the stage's empty barrier (or the accumulator's full barrier)
+// in both CTAs; each CTA drains its own 128 TMEM lanes (its 128 rows), and the
+// even CTA's accumulator-empty barrier counts the epilogue warps of both.
 template <int STAGES, int STG_BUFS = 1>
 struct PairCfg {
   static constexpr int kHalf = 128;                  // rows of A and of B per CTA
