@@ -18,7 +18,11 @@ M = 128/1024/8192 with the FNUZ load conversion), ``moe`` (8192 tokens,
 top-8 of 128 experts, hidden 2048, intermediate 704: routing, quantization,
 gather, grouped gate/up GEMM, GeGLU + quantization, grouped down GEMM,
 combine), ``tiny`` (K=256, N=128, M=4) and ``large8k`` (the large layer at
-M=8192, for profiling).
+M=8192, for profiling). Prefill GEMMs (M > 128, FP8 and int8) go through the
+workspace entry points (``fp8_rowwise_linear_ws`` / ``int8_rowwise_linear_ws``,
+one zero-filled workspace per workload), so that a partial last wave of CTA
+pair tiles is split by k-blocks; at M = 65536 and 8192 there are too many waves
+for the split and the GEMM is the plain one.
 
 Timing: the step is one CUDA graph replayed K times after W warm-up steps,
 with CUDA events on the launching stream; ops of at least 200 us are timed
