@@ -210,8 +210,9 @@ size_t fp8_linear_workspace_bytes(void);
  * does not split, it is fp8_rowwise_linear. Calls that may run at the same
  * time (other streams) need workspaces of their own, and a call that ended
  * with FP8_DEV_TIMEOUT may leave flags set: zero the workspace again before
- * reusing it. No counterpart on the pages: a scheduling choice of this
- * library's GEMM.
+ * reusing it. Errors: those of fp8_rowwise_linear, and FP8_ERR_ALIGNMENT for a
+ * ws that is not 16-byte aligned. No counterpart on the pages: a scheduling
+ * choice of this library's GEMM.
  */
 fp8_status fp8_rowwise_linear_ws(const uint8_t* x8, const float* s_tok, const uint8_t* w8,
                                  const float* s_ch, int64_t M, int64_t N, int64_t K, uint16_t* y,
