@@ -145,6 +145,39 @@ def test_split_within_bound_and_reproducible(lib, M, N, K):
     assert np.array_equal(bf16_to_np_bits(lib.rowwise_linear_ws(x8, st, w8, sw, small)), bf16_to_np_bits(y0))
 
 
+def test_split_entry_edge_cases(lib):
+    """fp8_rowwise_linear_ws: M = 0 and N = 0 do nothing, K = 0 gives zeros, a
+    workspace that is not 16-byte aligned is refused, and a null workspace
+    is the plain call (the same bits)."""
+    raw, st_ = lib.raw, torch.cuda.current_stream().cuda_stream
+    ws = lib.linear_workspace()
+    nb = ws.numel()
+    w8 = torch.zeros((256, 64), dtype=torch.uint8, device="cuda")
+    s = torch.ones(256, dtype=torch.float32, device="cuda")
+    x8 = torch.zeros((300, 64), dtype=torch.uint8, device="cuda")
+    y = torch.full((300, 256), 7.0, dtype=torch.bfloat16, device="cuda")
+    assert raw.fp8_rowwise_linear_ws(x8.data_ptr(), s.data_ptr(), w8.data_ptr(), s.data_ptr(), 0, 256, 64,
+                                     y.data_ptr(), ws.data_ptr(), nb, st_) == 0
+    assert raw.fp8_rowwise_linear_ws(x8.data_ptr(), s.data_ptr(), w8.data_ptr(), s.data_ptr(), 300, 0, 64,
+                                     y.data_ptr(), ws.data_ptr(), nb, st_) == 0
+    torch.cuda.synchronize()
+    assert bool((y == 7.0).all())
+    assert raw.fp8_rowwise_linear_ws(x8.data_ptr(), s.data_ptr(), w8.data_ptr(), s.data_ptr(), 300, 256, 0,
+                                     y.data_ptr(), ws.data_ptr(), nb, st_) == 0
+    torch.cuda.synchronize()
+    assert not bf16_to_np_bits(y).any()
+    assert raw.fp8_rowwise_linear_ws(x8.data_ptr(), s.data_ptr(), w8.data_ptr(), s.data_ptr(), 300, 256, 64,
+                                     y.data_ptr(), ws.data_ptr() + 8, nb - 8, st_) != 0
+    xb, a, w = _operands(1024, 14336, 4096, seed=5)
+    xd, sd, wd, swd = to_dev(a.codes), to_dev(a.scales), to_dev(w.codes), to_dev(w.scales)
+    yn = torch.empty((1024, 14336), dtype=torch.bfloat16, device="cuda")
+    assert raw.fp8_rowwise_linear_ws(xd.data_ptr(), sd.data_ptr(), wd.data_ptr(), swd.data_ptr(), 1024, 14336,
+                                     4096, yn.data_ptr(), None, 0, st_) == 0
+    y0 = lib.rowwise_linear(xd, sd, wd, swd)
+    assert np.array_equal(bf16_to_np_bits(yn), bf16_to_np_bits(y0))
+    assert lib.device_status() == 0
+
+
 def test_k_beyond_the_limit_is_refused(lib):
     x8 = torch.zeros((1, 65552), dtype=torch.uint8, device="cuda")
     w8 = torch.zeros((128, 65552), dtype=torch.uint8, device="cuda")
